@@ -1,0 +1,162 @@
+"""Asymmetric b-bit grid, the column-wise OBS solver and the layer loss.
+
+Sources:
+  * KronQ summary (hyper.ai), "Method": the Kronecker-factored objective
+    tr(H_G dW H_X dW^T), dW = W - W_hat; under the column-wise OBS update the
+    compensation after quantizing column p uses only H_X's inverse factor,
+    H_G cancels (Proposition 1).
+  * KronQ review (pith.science), appendix, Algorithm 2: damping, inverse
+    Cholesky, then a loop over columns in blocks of B with an error buffer E.
+    Blocking is a reassociation of the same column loop; the oracle runs the
+    plain unblocked loop: after column j, every later column k is updated at
+    once.
+  * KronQ README (GitHub), "Reproduce from scratch": --w_asym, --w_groupsize
+    -1 (per-channel) or 128, 2/3/4 bits; --w_clip and --act_order are left
+    off (the pages do not define them).
+
+Readings:
+  * grid: lo = min(0, min w), hi = max(0, max w), scale = (hi - lo)/(2^b - 1),
+    zero = round(-lo / scale); a row or group that is all zero gets
+    scale = 1, zero = 0.
+  * code: q = clamp(round(w / scale) + zero, 0, 2^b - 1), w_hat = scale (q - zero);
+    round = half to even.
+  * The decisions that produce integers (scale, zero, q) are taken in fp32,
+    the precision the CUDA kernels take them in: w is cast to fp32, then the
+    fp32 operations above are applied in that order.
+  * per-channel parameters come from the whole row of W' before the loop;
+    group parameters at column j = 0 mod g from the current (already
+    error-updated) columns j .. j+g-1.
+  * column update: e = (w_j - w_hat_j) / U[j, j]; W[:, k] -= e U[j, k], k > j.
+"""
+
+from __future__ import annotations
+
+from concurrent.futures import ThreadPoolExecutor
+import os
+
+import numpy as np
+
+F32 = np.float32
+
+
+def grid_params(w: np.ndarray, bits: int):
+    """Per-row (scale fp32, zero int) of the asymmetric grid for each row of w."""
+    w32 = np.asarray(w, dtype=np.float64).astype(F32)
+    if w32.ndim == 1:
+        w32 = w32[None, :]
+    maxq = F32(2 ** bits - 1)
+    lo = np.minimum(w32.min(axis=1), F32(0))
+    hi = np.maximum(w32.max(axis=1), F32(0))
+    zero_row = (lo == 0) & (hi == 0)
+    span = (hi - lo).astype(F32)
+    span[zero_row] = maxq
+    scale = (span / maxq).astype(F32)
+    zero = np.rint((-lo).astype(F32) / scale).astype(F32)
+    zero = np.clip(zero, F32(0), maxq)
+    scale[zero_row] = F32(1)
+    zero[zero_row] = F32(0)
+    return scale, zero.astype(np.int64)
+
+
+def quantize(w: np.ndarray, scale: np.ndarray, zero: np.ndarray, bits: int) -> np.ndarray:
+    """Integer codes, decided in fp32 (reading in the module docstring)."""
+    maxq = 2 ** bits - 1
+    w32 = np.asarray(w, dtype=np.float64).astype(F32)
+    r = np.rint(w32 / np.asarray(scale, dtype=F32)).astype(np.int64)
+    return np.clip(r + np.asarray(zero, dtype=np.int64), 0, maxq)
+
+
+def dequantize(q, scale, zero) -> np.ndarray:
+    return np.asarray(scale, dtype=np.float64) * (np.asarray(q, dtype=np.int64)
+                                                 - np.asarray(zero, dtype=np.int64))
+
+
+def _check(n: int, group: int, bits: int):
+    if bits not in (2, 3, 4, 8):
+        raise ValueError("bits must be 2, 3, 4 or 8")
+    if group != -1 and (group <= 0 or n % group):
+        raise ValueError("group must be -1 or divide n")
+
+
+def obs_quantize(W: np.ndarray, U: np.ndarray, bits: int, group: int = -1):
+    """Unblocked column-wise OBS loop on the rows of W (rows are independent).
+
+    W: m x n (the rotated weights, widened to fp64).  U: n x n upper inverse
+    Cholesky factor of the damped H_X.  Returns a dict with codes (m x n),
+    scale and zero (m x n_groups), W_hat (m x n) and the scaled errors E."""
+    W = np.array(W, dtype=np.float64)
+    U = np.asarray(U, dtype=np.float64)
+    m, n = W.shape
+    _check(n, group, bits)
+    ng = 1 if group == -1 else n // group
+    codes = np.zeros((m, n), dtype=np.uint8)
+    scales = np.zeros((m, ng), dtype=F32)
+    zeros = np.zeros((m, ng), dtype=np.uint8)
+    What = np.zeros((m, n))
+    E = np.zeros((m, n))
+    if group == -1:
+        scale, zero = grid_params(W, bits)
+        scales[:, 0], zeros[:, 0] = scale, zero
+    for j in range(n):
+        if group != -1 and j % group == 0:
+            scale, zero = grid_params(W[:, j:j + group], bits)
+            scales[:, j // group], zeros[:, j // group] = scale, zero
+        w = W[:, j]
+        q = quantize(w, scale, zero, bits)
+        wh = dequantize(q, scale, zero)
+        e = (w - wh) / U[j, j]
+        W[:, j + 1:] -= np.outer(e, U[j, j + 1:])
+        codes[:, j] = q
+        What[:, j] = wh
+        E[:, j] = e
+    return {"codes": codes, "scale": scales, "zero": zeros, "W_hat": What, "E": E}
+
+
+def obs_quantize_rows(W: np.ndarray, U: np.ndarray, bits: int, group: int = -1,
+                      rows=None, chunk: int = 64, threads: int | None = None):
+    """obs_quantize on a subset of rows, in row chunks on a thread pool.
+
+    Each row's arithmetic is exactly that of obs_quantize: the rows of the
+    loop never interact, so splitting them changes no operation."""
+    W = np.asarray(W)
+    rows = np.arange(W.shape[0]) if rows is None else np.asarray(rows)
+    parts = [rows[i:i + chunk] for i in range(0, len(rows), chunk)]
+    threads = threads or min(32, os.cpu_count() or 1)
+    with ThreadPoolExecutor(threads) as ex:
+        res = list(ex.map(lambda r: obs_quantize(W[r], U, bits, group), parts))
+    if not res:
+        return obs_quantize(W[:0], U, bits, group)
+    return {k: np.concatenate([r[k] for r in res], axis=0) for k in res[0]}
+
+
+def rtn_quantize(W: np.ndarray, bits: int, group: int = -1):
+    """Round-to-nearest on the same grid (no error propagation)."""
+    W = np.asarray(W, dtype=np.float64)
+    m, n = W.shape
+    _check(n, group, bits)
+    g = n if group == -1 else group
+    codes = np.zeros((m, n), dtype=np.uint8)
+    What = np.zeros((m, n))
+    scales = np.zeros((m, n // g), dtype=F32)
+    zeros = np.zeros((m, n // g), dtype=np.uint8)
+    for b in range(n // g):
+        sl = slice(b * g, (b + 1) * g)
+        scale, zero = grid_params(W[:, sl], bits)
+        q = quantize(W[:, sl], scale[:, None], zero[:, None], bits)
+        codes[:, sl] = q
+        What[:, sl] = dequantize(q, scale[:, None], zero[:, None])
+        scales[:, b], zeros[:, b] = scale, zero
+    return {"codes": codes, "scale": scales, "zero": zeros, "W_hat": What}
+
+
+def layer_loss(dW: np.ndarray, HX: np.ndarray, HG: np.ndarray) -> float:
+    """tr(H_G dW H_X dW^T), fp64."""
+    dW = np.asarray(dW, dtype=np.float64)
+    M = np.asarray(HG, dtype=np.float64) @ dW @ np.asarray(HX, dtype=np.float64)
+    return float(np.sum(M * dW))
+
+
+def row_losses(dW: np.ndarray, HX: np.ndarray) -> np.ndarray:
+    """dW_i H_X dW_i^T for each row (the part of the loss the solver sees)."""
+    dW = np.asarray(dW, dtype=np.float64)
+    return np.einsum("ij,ij->i", dW @ np.asarray(HX, dtype=np.float64), dW)
