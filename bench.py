@@ -1,0 +1,542 @@
+#!/usr/bin/env python
+"""KronQ per-layer quantization throughput on B200.
+
+One step = the whole per-layer path over one synthetic layer's calibration
+batch: H_X = X^T X / N and H_G = G^T G / N (tensor cores), BiIP (rescale +
+randomized Hadamard on both sides of W, H_X, H_G), s = tr(H_G) tr(H_X),
+damped inverse Cholesky, column-wise OBS quantization, packing.
+
+Prints one JSON line (rank 0).  `value` is whole-job Mweights/s with X, G, W
+resident in HBM; `e2e` is the same metric through the public Python API with
+pinned host buffers (H2D of X, G, W and D2H of the packed result inside the
+timed region).  `--impl reference` times the fp64 CPU oracle on a bounded
+sample of the same workload instead.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import pathlib
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = pathlib.Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+METRIC = "layer quantize Mweights/s end-to-end; H_X/H_G GEMM % of bf16 tensor peak"
+UNIT = "Mweights/s"
+DEFAULT_CONFIG = "llama2-7b-q_proj"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default=DEFAULT_CONFIG)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    return ap.parse_args()
+
+
+def workload_desc(cfg) -> str:
+    subs = ", ".join(f"{s.name} {s.m}x{s.n}" for s in cfg.sublayers)
+    g = "per-channel" if cfg.sublayers[0].group == -1 else f"group-{cfg.sublayers[0].group}"
+    bits = "mixed 2/3/4 at 3.0 avg" if cfg.mixed_avg_bits else f"W{cfg.sublayers[0].bits}"
+    return (f"{cfg.name}: {subs}; X/G {cfg.tokens} tokens bf16 ({cfg.x_dist} X with outlier "
+            f"channels x{cfg.x_outlier_scale:g}, G scales over {cfg.g_decades:g} decades); "
+            f"{bits} asymmetric {g}; BiIP alpha {cfg.alpha}, damp {cfg.damp}")
+
+
+# ------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples every 200 ms while running (clocks and throttle reasons)."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str | None):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+        if self.gpu_id:
+            cmd += ["-i", self.gpu_id]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            if self.thread:
+                self.thread.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            p = [x.strip() for x in ln.split(",")]
+            if len(p) < 8:
+                continue
+            try:
+                sm.append(float(p[0]))
+                mx = float(p[1])
+            except ValueError:
+                continue
+            for nm, v in zip(names, p[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def gpu_id_for(dev_index: int) -> str | None:
+    import torch
+    try:
+        u = torch.cuda.get_device_properties(dev_index).uuid
+        s = str(u)
+        return s if s.startswith("GPU-") else f"GPU-{s}"
+    except Exception:
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+        return vis.split(",")[dev_index] if vis else None
+
+
+# -------------------------------------------------------- peaks / traffic
+def load_peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        return d, "MEASURED_PEAKS.json"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for f in ("covariance.cu", "common.cuh"):
+        h.update((ROOT / "post_quantization_02_b200" / "csrc" / f).read_bytes())
+    return h.hexdigest()[:16]
+
+
+def load_traffic(workload: str):
+    """DRAM bytes per launch of the covariance kernel from a committed ncu
+    summary, only while the kernel source is the one that was profiled."""
+    p = ROOT / "profiles" / "cov_tc_kernel.traffic.json"
+    if not p.exists():
+        return None
+    d = json.loads(p.read_text())
+    if d.get("source_sha") != kernel_source_sha() or d.get("workload") != workload:
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------- oracle side
+def oracle_sample(cfg, budget_s: float = 20.0):
+    """Time the fp64 oracle, as it stands, on a bounded sample of the workload
+    and extrapolate to the whole job.  Returns (seconds_full, sample_text)."""
+    import numpy as np
+    import synth
+    from oracle import biip as obiip, cholesky as ochol, quantizer as oq, pack as opack
+    from oracle import transform as otr
+
+    f = max(0.1, min(1.0, budget_s / 20.0))
+    tok = max(256, int(1024 * f)) // 256 * 256
+    rows_rot = max(32, int(256 * f))
+    rows_obs = max(4, int(16 * f))
+    total = 0.0
+    parts = []
+    for sub in cfg.sublayers:
+        site = cfg.site(sub.site)
+        m, n = sub.m, sub.n
+        # covariances: tok tokens of X and G, scaled to all tokens
+        xb = synth.x_chunk(cfg, site, 0, tokens=tok)
+        gb = synth.g_chunk(cfg, sub, 0, tokens=tok)
+        from oracle import covariance as ocov
+        t0 = time.perf_counter()
+        ocov.covariance(synth.bf16_bits_to_f32(xb).astype(np.float64))
+        ocov.covariance(synth.bf16_bits_to_f32(gb).astype(np.float64))
+        t_cov = (time.perf_counter() - t0) * cfg.tokens / tok
+        # BiIP: the row transform on rows_rot rows of each matrix, scaled to the
+        # row and column passes of W (m x n), H_X (n x n), H_G (m x m)
+        r = np.random.default_rng(0)
+        su, sv = synth.make_signs(cfg, sub)
+        t0 = time.perf_counter()
+        otr.apply(r.standard_normal((rows_rot, n)), sv)
+        t_rn = (time.perf_counter() - t0) / rows_rot
+        t0 = time.perf_counter()
+        otr.apply(r.standard_normal((rows_rot, m)), su)
+        t_rm = (time.perf_counter() - t0) / rows_rot
+        t_rot = t_rn * (m + 2 * n) + t_rm * (n + 2 * m)
+        # damped inverse Cholesky, n x n (on a smaller n if large, scaled n^3)
+        nc = min(n, 2048)
+        A = r.standard_normal((nc, nc))
+        H = A @ A.T / nc + np.eye(nc)
+        t0 = time.perf_counter()
+        ochol.inverse_cholesky(ochol.damp(H, cfg.damp))
+        t_chol = (time.perf_counter() - t0) * (n / nc) ** 3
+        # column loop: one wave of the oracle's threaded 64-row chunks, at the
+        # layer's width up to 4096 columns (scaled by rows, and by cols^2 beyond)
+        nn = min(n, 4096)
+        # the loop's cost does not depend on the factor's values: any upper
+        # triangular matrix with a positive diagonal serves for timing
+        U = np.triu(r.standard_normal((nn, nn)) * 0.01) + np.eye(nn)
+        bits = sub.bits or 3
+        grp = sub.group if sub.group == -1 or nn % sub.group == 0 else -1
+        rows_obs = min(m, 16 * max(1, min(32, os.cpu_count() or 1)))
+        rows_obs = max(4, int(rows_obs * f))
+        Wr = r.standard_normal((rows_obs, nn)) * 0.02
+        t0 = time.perf_counter()
+        res = oq.obs_quantize_rows(Wr, U, bits, grp)
+        t_obs = (time.perf_counter() - t0) * (m / rows_obs) * (n / nn) ** 2
+        t0 = time.perf_counter()
+        if bits in (2, 4):
+            opack.pack(res["codes"], bits)
+        t_pack = (time.perf_counter() - t0) * (m / rows_obs) * (n / nn)
+        total += t_cov + t_rot + t_chol + t_obs + t_pack
+        parts.append(f"{sub.name}: cov {tok} of {cfg.tokens} tokens, rotation {rows_rot} rows, "
+                     f"inverse Cholesky n={nc}, OBS {rows_obs} of {m} rows x {nn} cols")
+    sample = ("fp64 oracle stages timed on samples and scaled to the whole layer (covariance x tokens, "
+              "rotation x rows, inverse Cholesky x n^3, OBS x rows, x cols^2 above 4096): " + "; ".join(parts))
+    return total, sample
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max([i.get("num_threads", 1) for i in info if i.get("user_api") == "blas"] or [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, rank, world):
+    import synth
+    if rank != 0:
+        return
+    cfg = synth.get_config(args.config)
+    weights = cfg.weights
+    per_step = max(3.0, min(30.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(cfg, per_step)
+    t0 = time.perf_counter()
+    ests = []
+    sample = ""
+    for _ in range(args.steps):
+        est, sample = oracle_sample(cfg, per_step)
+        ests.append(est)
+    wall = time.perf_counter() - t0
+    full = statistics.mean(ests)
+    value = weights / full / 1e6
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": full * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded generator)",
+        "config": {"workload": workload_desc(cfg), "sample_wall_s_per_step": wall / max(1, args.steps)},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------- GPU side
+class Layer:
+    """Device buffers of one sublayer for the timed steps (allocated once)."""
+
+    def __init__(self, cfg, sub, dev, seed_offset, host):
+        import numpy as np
+        import torch
+        import synth
+        from post_quantization_02_b200 import abi
+        self.sub = sub
+        m, n = sub.m, sub.n
+        self.W0 = torch.from_numpy(synth.make_w(cfg, sub)).to(dev)
+        su, sv = synth.make_signs(cfg, sub)
+        self.su = torch.from_numpy(su).to(dev)
+        self.sv = torch.from_numpy(sv).to(dev)
+        self.G_host = host["G"][sub.name]
+        self.G = torch.from_numpy(self.G_host.view(np.int16)).to(dev).view(torch.bfloat16)
+        self.W = torch.empty_like(self.W0)
+        self.HX = torch.empty((n, n), dtype=torch.float32, device=dev)
+        self.HG = torch.empty((m, m), dtype=torch.float32, device=dev)
+        self.SX = torch.empty(n, dtype=torch.float32, device=dev)
+        self.SG = torch.empty(m, dtype=torch.float32, device=dev)
+        self.U = torch.empty((n, n), dtype=torch.float32, device=dev)
+        self.sens = torch.zeros(3, dtype=torch.float64, device=dev)
+        self.info = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.codes = torch.empty((m, n), dtype=torch.uint8, device=dev)
+        G = 1 if sub.group == -1 else n // sub.group
+        self.scales = torch.empty((m, G), dtype=torch.float32, device=dev)
+        self.zeros = torch.empty((m, G), dtype=torch.uint8, device=dev)
+        self.packed = torch.empty((m, abi.packed_words(n, 4)), dtype=torch.int32, device=dev)
+        self.bits = sub.bits
+
+
+def gpu_step(cfg, layers, X, ws, stream, cov_events=None):
+    """One pass of the whole path over every sublayer of the config."""
+    import torch
+    from post_quantization_02_b200 import abi, alloc
+    N = cfg.tokens
+    ev = iter(cov_events) if cov_events is not None else None
+
+    def cov(A, H):
+        if ev is not None:
+            next(ev).record(stream)
+        abi.kronq_covariance(A, H, 1.0 / N, 0.0, stream=stream)
+        if ev is not None:
+            next(ev).record(stream)
+
+    hx_site = {}
+    for L in layers:
+        site = L.sub.site
+        if site not in hx_site:
+            cov(X[site], layers[[l.sub.site for l in layers].index(site)].HX)
+            hx_site[site] = layers[[l.sub.site for l in layers].index(site)].HX
+        cov(L.G, L.HG)
+    for L in layers:
+        if L.HX is not hx_site[L.sub.site]:
+            L.HX.copy_(hx_site[L.sub.site])
+    for L in layers:
+        L.W.copy_(L.W0)
+    # H_X of a shared site is rotated per sublayer: rotate copies, the site's own last
+    for L in layers:
+        abi.kronq_biip_rotate(L.W, L.HX, L.HG, L.su, L.sv, cfg.alpha, cfg.mode, 0, L.SX, L.SG, ws,
+                              stream=stream)
+        abi.kronq_sensitivity(L.HX, L.HG, L.sens, stream=stream)
+    if cfg.mixed_avg_bits:
+        scores = torch.stack([L.sens[0] for L in layers]).cpu().tolist()
+        bits = alloc.allocate_bits(scores, [L.sub.m * L.sub.n for L in layers], cfg.mixed_avg_bits)
+        for L, b in zip(layers, bits):
+            L.bits = b
+    for L in layers:
+        abi.kronq_cholesky_inv(L.HX, cfg.damp, L.U, L.info, ws, stream=stream)
+        abi.kronq_quantize_layer(L.W, L.U, L.bits, L.sub.group, cfg.block, L.codes, L.scales,
+                                 L.zeros, None, L.info, ws, stream=stream)
+        if L.bits in (2, 4):
+            pk = L.packed[:, : abi.packed_words(L.sub.n, L.bits)]
+            abi.kronq_pack(L.codes, L.bits, pk.contiguous() if not pk.is_contiguous() else pk,
+                           stream=stream)
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    import synth
+    from post_quantization_02_b200 import abi
+    from post_quantization_02_b200 import pipeline as gpipe
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    abi.lib()
+    cfg0 = synth.get_config(args.config)
+    import dataclasses
+    cfg = dataclasses.replace(cfg0, seed=cfg0.seed + rank)   # each rank: its own layer (weak scaling)
+
+    # ---- seeded inputs on the host (pinned for the end-to-end leg), then HBM
+    t_gen = time.perf_counter()
+    host = {"X": {}, "G": {}}
+    for site in cfg.sites:
+        host["X"][site.name] = synth.make_x(cfg, site)
+    for sub in cfg.sublayers:
+        host["G"][sub.name] = synth.make_g(cfg, sub)
+    t_gen = time.perf_counter() - t_gen
+    X = {s: torch.from_numpy(v.view(np.int16)).to(dev).view(torch.bfloat16) for s, v in host["X"].items()}
+    layers = [Layer(cfg, sub, dev, rank, host) for sub in cfg.sublayers]
+    mmax = max(s.m for s in cfg.sublayers)
+    nmax = max(s.n for s in cfg.sublayers)
+    ws = abi.workspace(mmax, nmax, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    weights = cfg.weights
+
+    ncov = len(cfg.sites) + len(cfg.sublayers)
+    for _ in range(args.warmup):
+        gpu_step(cfg, layers, X, ws, stream)
+    torch.cuda.synchronize()
+    for L in layers:
+        if L.info.item() != 0:
+            raise RuntimeError(f"device status {L.info.item()} in warm-up")
+
+    sampler = ClockSampler(gpu_id_for(local))
+    sampler.start()
+    time.sleep(0.3)
+    cov_events = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * ncov)] for _ in range(args.steps)]
+    launches0 = abi.kronq_launch_count()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for k in range(args.steps):
+        gpu_step(cfg, layers, X, ws, stream, cov_events[k])
+    end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    launches = abi.kronq_launch_count() - launches0
+    ms = start.elapsed_time(end)
+    ms_t = torch.tensor([ms], device=dev)
+    if world > 1:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms = float(ms_t.item())
+    cov_ms = [ev[2 * i].elapsed_time(ev[2 * i + 1]) for ev in cov_events for i in range(ncov)]
+
+    # ---- end to end through the public API with pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        pin = {"X": {s: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).pin_memory()
+                     for s, v in host["X"].items()},
+               "G": {s: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).pin_memory()
+                     for s, v in host["G"].items()},
+               "W": {L.sub.name: L.W0.cpu().pin_memory() for L in layers}}
+        outs = {L.sub.name: (torch.empty(L.packed.shape, dtype=torch.int32).pin_memory(),
+                             torch.empty(L.scales.shape).pin_memory(),
+                             torch.empty(L.zeros.shape, dtype=torch.uint8).pin_memory()) for L in layers}
+        copy_stream = torch.cuda.Stream(dev)
+        staging = {}
+
+        def cov_host(A_host, H, width):
+            if width not in staging:
+                staging[width] = [torch.empty((16384, width), dtype=torch.bfloat16, device=dev)
+                                  for _ in range(2)]
+            return gpipe.covariance_from_host(A_host, H, copy_stream=copy_stream, stream=stream,
+                                              staging=staging[width])
+
+        def e2e_step():
+            h2d = 0
+            Hs = {}
+            for site in cfg.sites:
+                L0 = next(L for L in layers if L.sub.site == site.name)
+                h2d += cov_host(pin["X"][site.name], L0.HX, site.width)
+                Hs[site.name] = L0.HX
+            for L in layers:
+                h2d += cov_host(pin["G"][L.sub.name], L.HG, L.sub.m)
+                if L.HX is not Hs[L.sub.site]:
+                    L.HX.copy_(Hs[L.sub.site])
+                L.W.copy_(pin["W"][L.sub.name], non_blocking=True)
+                h2d += L.W.numel() * 4 + L.su.numel() + L.sv.numel()
+            d2h = 0
+            for L in layers:
+                abi.kronq_biip_rotate(L.W, L.HX, L.HG, L.su, L.sv, cfg.alpha, cfg.mode, 0, L.SX, L.SG,
+                                      ws, stream=stream)
+                abi.kronq_sensitivity(L.HX, L.HG, L.sens, stream=stream)
+            for L in layers:
+                abi.kronq_cholesky_inv(L.HX, cfg.damp, L.U, L.info, ws, stream=stream)
+                abi.kronq_quantize_layer(L.W, L.U, L.bits, L.sub.group, cfg.block, L.codes, L.scales,
+                                         L.zeros, None, L.info, ws, stream=stream)
+                pk, sc, zr = outs[L.sub.name]
+                if L.bits in (2, 4):
+                    words = abi.packed_words(L.sub.n, L.bits)
+                    abi.kronq_pack(L.codes, L.bits, L.packed[:, :words].contiguous()
+                                   if words != L.packed.shape[1] else L.packed, stream=stream)
+                    pk.copy_(L.packed, non_blocking=True)
+                    d2h += L.packed.numel() * 4
+                sc.copy_(L.scales, non_blocking=True)
+                zr.copy_(L.zeros, non_blocking=True)
+                d2h += L.scales.numel() * 4 + L.zeros.numel()
+            return h2d, d2h
+
+        e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(args.e2e_steps):
+            h2d, d2h = e2e_step()
+        s1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = s0.elapsed_time(s1)
+        et = torch.tensor([e_ms], device=dev)
+        if world > 1:
+            dist.all_reduce(et, op=dist.ReduceOp.MAX)
+        e_ms = float(et.item())
+        e2e = {"value": weights * world * args.e2e_steps / (e_ms / 1e3) / 1e6, "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": e_ms / args.e2e_steps}
+    time.sleep(0.3)
+    sampler.stop()
+    clocks = sampler.summary()
+
+    value = weights * world * args.steps / (ms / 1e3) / 1e6
+    peaks, peak_src = load_peaks()
+    timed_s = ms / 1e3
+    peak_kind = "bf16_tflops_sustained" if timed_s >= 1.0 else "bf16_tflops"
+    peak = float(peaks.get(peak_kind, peaks.get("bf16_tflops")))
+    cov_flops = []
+    for s in cfg.sites:
+        cov_flops.append(cfg.tokens * s.width ** 2)
+    for sub in cfg.sublayers:
+        cov_flops.append(cfg.tokens * sub.m ** 2)
+    avg_ms = statistics.mean(cov_ms)
+    achieved = statistics.mean(cov_flops) / (avg_ms / 1e3) / 1e12
+    workload = workload_desc(cfg0)
+    roofline = {"bound": "tensor", "kernel": "cov_tc_kernel (kronq_covariance)",
+                "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "traffic": load_traffic(workload),
+                "peak_source": f"{peak_src} {peak_kind}",
+                "flops_per_launch": statistics.mean(cov_flops), "avg_launch_ms": avg_ms,
+                "launches_timed": len(cov_ms)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        est, sample = oracle_sample(cfg0, 20.0)
+        cpu = {"value": cfg0.weights / est / 1e6, "unit": UNIT, "cores": blas_threads(),
+               "kind": "oracle", "sample": sample, "host_cpus": os.cpu_count()}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded generator; stands in for WikiText-2 activations and LLaMA weights)",
+            "config": {"workload": workload, "parallelism": f"replicas x{world} (one layer per GPU)",
+                       "l2": "inputs larger than L2 (X and G are 2 GiB each at 262144 x 4096 bf16)",
+                       "solver_dtype": "fp32", "input_gen_s": round(t_gen, 1)},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

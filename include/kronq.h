@@ -1,0 +1,221 @@
+/*
+ * kronq.h -- C ABI of libkronq, the sm_100a (B200) implementation of the
+ * KronQ per-layer quantization path.
+ *
+ * The path, in the order the KronQ pages run it:
+ *   1. kronq_covariance     H_X = X^T X / N, H_G = G^T G / N
+ *   2. kronq_biip_rotate    bidirectional incoherence processing of W, H_X, H_G
+ *   3. kronq_sensitivity    s = tr(H_G) tr(H_X)
+ *   4. kronq_cholesky_inv   damping and the inverse Cholesky factor of H_X
+ *   5. kronq_quantize_layer column-wise OBS quantization with lazy block updates
+ *   6. kronq_pack           2/4-bit codes packed into 32-bit words
+ * plus kronq_unpack and kronq_layer_loss (a measurement helper).
+ *
+ * Conventions shared by every call
+ *   - Matrices are row-major and contiguous unless a leading dimension is
+ *     passed.  W is m x n (m = d_out rows, n = d_in columns).
+ *   - Every data pointer is a DEVICE pointer owned by the caller; the library
+ *     keeps no pointer after the call returns and allocates no device memory.
+ *     Scratch memory comes from the caller's workspace (ws, ws_bytes), at
+ *     least kronq_workspace_size() bytes, 256-byte aligned.
+ *   - Calls are asynchronous and ordered on `stream` (a cudaStream_t; NULL is
+ *     the legacy default stream).  Argument errors are detected on the host
+ *     and returned before anything is launched.
+ *   - Numerical failures found on the device (a non-positive pivot, a wait
+ *     that timed out) are written to the optional device word `info`
+ *     (0 = fine, otherwise a negative KRONQ_ERR_* code; the first error
+ *     wins).  Read it after synchronising the stream.
+ *   - Return value: KRONQ_OK or a negative KRONQ_ERR_* code.
+ */
+#ifndef KRONQ_H
+#define KRONQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum kronq_status {
+  KRONQ_OK = 0,
+  KRONQ_ERR_INVALID_ARG = -1,  /* null pointer, bad shape, misalignment, group not dividing n */
+  KRONQ_ERR_UNSUPPORTED = -2,  /* valid request this build does not handle (3-bit packing, a width with no transform) */
+  KRONQ_ERR_NOT_PD = -3,       /* damped H_X not positive definite (device-side, via info) */
+  KRONQ_ERR_CUDA = -4,         /* a CUDA runtime call failed */
+  KRONQ_ERR_TIMEOUT = -5,      /* a bounded wait inside a kernel gave up (device-side, via info) */
+  KRONQ_ERR_WORKSPACE = -6     /* workspace missing or smaller than kronq_workspace_size() */
+};
+
+/* --incoh_mode of the pages (KronQ README (GitHub), "Mapping paper results to flags"). */
+enum kronq_incoh_mode {
+  KRONQ_MODE_FULL = 0,        /* both rescales, both rotations */
+  KRONQ_MODE_NO_RESCALE = 1,  /* both rotations, no diagonal rescale */
+  KRONQ_MODE_SU_ONLY = 2,     /* output side only: S_G and U */
+  KRONQ_MODE_SV_ONLY = 3      /* input side only: S_X and V */
+};
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* kronq_status_string(int status);
+
+/* ABI version of this header (major * 100 + minor). */
+int kronq_abi_version(void);
+
+/* Number of kernels this library has launched in this process (all devices,
+ * all streams; a host-side counter, for measurement). */
+uint64_t kronq_launch_count(void);
+
+/*
+ * Workspace, in bytes, that kronq_biip_rotate, kronq_cholesky_inv,
+ * kronq_quantize_layer and kronq_layer_loss need for a layer of m x n.
+ * Returns 0 for invalid sizes.
+ */
+size_t kronq_workspace_size(int64_t m, int64_t n, int bits, int group, int block);
+
+/*
+ * H = alpha * A^T A + beta * H   (d x d, fp32, full symmetric matrix written)
+ *
+ * KronQ summary (hyper.ai), "Method" (Eq. 7): H_X = E[x x^T] over the
+ * calibration activations and H_G = E[g g^T] over the output gradients.
+ * With alpha = 1/N over N rows this is the mean; calling it once per chunk of
+ * rows with alpha = 1/N_total and beta = 0 for the first chunk and 1 after
+ * streams the sum.
+ *
+ * A     : N x d bf16 (raw bf16 bits), row-major with leading dimension lda
+ *         (elements); lda >= d, lda % 8 == 0, A 16-byte aligned.
+ * H     : d x d fp32, leading dimension ldh >= d, ldh % 4 == 0, 16-byte aligned.
+ *         When beta == 0, H is write-only (its old contents may be NaN).
+ * N = 0 : H = beta * H.   d = 0 : no-op.   0 < d < 64: KRONQ_ERR_UNSUPPORTED.
+ * info  : optional device int32 (KRONQ_ERR_TIMEOUT on a stuck pipeline).
+ * Tensor cores (tcgen05, TMEM accumulators, TMA-fed); only tiles on or above
+ * the diagonal are computed; each writes its elements and their mirror
+ * images.  When beta != 0 the old H must be symmetric (its upper triangle is
+ * read).
+ */
+int kronq_covariance(const uint16_t* A, int64_t N, int64_t d, int64_t lda,
+                     float* H, int64_t ldh, float alpha, float beta,
+                     int32_t* info, void* stream);
+
+/*
+ * s = tr(H_G) * tr(H_X)   (fp64 sums of the diagonals)
+ *
+ * KronQ summary (hyper.ai), "Method" (Eq. 14): the sublayer sensitivity,
+ * taken after BiIP; sublayers with a larger s receive more bits.
+ * H_X: n x n fp32 (leading dim n), H_G: m x m fp32 (leading dim m).
+ * out  : DEVICE pointer to 3 doubles: {s, tr(H_X), tr(H_G)}.
+ */
+int kronq_sensitivity(const float* H_X, int64_t n, const float* H_G, int64_t m,
+                      double* out, void* stream);
+
+/*
+ * Bidirectional incoherence processing, in place.
+ *
+ * KronQ summary (hyper.ai), "Method", Eqs. 11-12: diagonal rescale on both
+ * sides, then W' = U W V^T, H_X' = V H_X V^T, H_G' = U H_G U^T with
+ * randomized Hadamard transforms U = T_m D_u, V = T_n D_v.
+ * Rescale: S_X[j] = (H_X[j,j] / ||W[:,j]||^2)^alpha first, then
+ * S_G[i] = (H_G[i,i] / ||(W S_X)[i,:]||^2)^alpha; W <- S_G W S_X,
+ * H_X <- S_X^-1 H_X S_X^-1, H_G <- S_G^-1 H_G S_G^-1 (a zero diagonal or norm
+ * gives a scale of 1).  T_d = C_q (x) H_{2^k}/sqrt(2^k) for d = q 2^k, q odd,
+ * C_q the orthonormal DCT-II.
+ *
+ * W      : m x n fp32, overwritten by W'.   H_X: n x n fp32.   H_G: m x m fp32.
+ * sign_u : m int8 (+1/-1), sign_v: n int8.
+ * mode   : enum kronq_incoh_mode.
+ * S_X, S_G : outputs (n and m fp32) when inverse == 0.
+ * inverse = 1 : apply the exact inverse to W only (W = S_G^-1 U^T W' V S_X^-1,
+ *          S_X and S_G are then inputs; H_X and H_G may be NULL).
+ * Widths: m, n multiples of 16 (KRONQ_ERR_INVALID_ARG otherwise); for
+ *         d = q 2^k (q odd) the transform runs as (C_q (x) H_{2^(k-k2)})
+ *         (x) H_{2^k2} with 2^k2 = min(2^k, 4096): q <= 63 and
+ *         q 2^(k-k2) <= 64 are required (KRONQ_ERR_UNSUPPORTED otherwise;
+ *         4096, 8192, 11008, 14336 and 28672 are all covered).
+ */
+int kronq_biip_rotate(float* W, int64_t m, int64_t n, float* H_X, float* H_G,
+                      const int8_t* sign_u, const int8_t* sign_v,
+                      float alpha, int mode, int inverse,
+                      float* S_X, float* S_G, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Damping and the inverse Cholesky factor.
+ *
+ * KronQ review (pith.science), appendix, Algorithm 2, steps 1-2:
+ * H_d = H + damp_rel * mean(diag(H)) * I, then U_c upper triangular with
+ * H_d^-1 = U_c^T U_c and a positive diagonal.  Computed as a reverse-order
+ * Cholesky factorisation of H_d followed by a triangular inverse (fp32).
+ *
+ * H    : n x n fp32 symmetric (not modified).  U_c: n x n fp32 output
+ *        (strictly lower part set to 0).  May not alias H.
+ * info : optional device int32, KRONQ_ERR_NOT_PD if a pivot is <= 0 (U_c is
+ *        then undefined).
+ */
+int kronq_cholesky_inv(const float* H, int64_t n, float damp_rel, float* U_c,
+                       int32_t* info, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Column-wise OBS quantization (GPTQ-style) of the rotated weights.
+ *
+ * KronQ summary (hyper.ai), "Method", Prop. 1: H_G cancels in the column
+ * update, so each row is solved with H_X's factor alone.  KronQ review
+ * (pith.science), appendix, Algorithm 2: blocks of B columns with an error
+ * buffer E and lazy updates of the trailing columns.
+ * Grid (asymmetric, b bits): lo = min(0, min w), hi = max(0, max w),
+ * scale = (hi - lo)/(2^b - 1), zero = round(-lo/scale); per-channel from the
+ * whole row before the loop, per group at the group's first column from the
+ * error-updated weights.  q = clamp(round(w/scale) + zero, 0, 2^b - 1)
+ * (round half to even, in fp32); e = (w - scale (q - zero)) / U_c[j,j];
+ * W[:, k] -= e U_c[j, k] for k > j.
+ *
+ * W      : m x n fp32, the rotated weights; overwritten (scratch).
+ * U_c    : n x n fp32 upper factor from kronq_cholesky_inv.
+ * bits   : 2, 3, 4 or 8.  group: -1 (per-channel), 32, 64 or 128.  block: 128.
+ * codes  : m x n uint8 output.   scales: m x G fp32, zeros: m x G uint8
+ *          (G = 1 per-channel, n/group otherwise).
+ * W_hat  : optional m x n fp32 output of the dequantized weights (NULL: skip).
+ * n must be a multiple of 128.
+ */
+int kronq_quantize_layer(float* W, int64_t m, int64_t n, const float* U_c,
+                         int bits, int group, int block,
+                         uint8_t* codes, float* scales, uint8_t* zeros, float* W_hat,
+                         int32_t* info, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Pack b-bit codes into 32-bit words (b = 2 or 4).
+ *
+ * KronQ README (GitHub), "Model zoo": W4 / W2 stored as packed int4 / int2;
+ * 3-bit is not packable (KRONQ_ERR_UNSUPPORTED).  Code (i, j) goes to word
+ * (i, floor(j b / 32)), bits [(j mod 32/b) b, +b).  Rows take
+ * ceil(n b / 32) words; spare high bits are 0.  Codes must be < 2^b.
+ * codes: m x n uint8.  packed: m x ceil(n b/32) uint32, 4-byte aligned.
+ */
+int kronq_pack(const uint8_t* codes, int64_t m, int64_t n, int bits,
+               uint32_t* packed, void* stream);
+
+/* Exact inverse of kronq_pack. */
+int kronq_unpack(const uint32_t* packed, int64_t m, int64_t n, int bits,
+                 uint8_t* codes, void* stream);
+
+/*
+ * Layer loss tr(H_G dW H_X dW^T), dW = W_ref - W_hat (a measurement helper,
+ * not on the quantization path).  KronQ summary (hyper.ai), "Method": the
+ * Kronecker-factored objective.  All inputs fp32 device; loss_out: DEVICE
+ * double.  Workspace: kronq_workspace_size(m, n, ...) bytes.
+ */
+int kronq_layer_loss(const float* W_ref, const float* W_hat, int64_t m, int64_t n,
+                     const float* H_X, const float* H_G, double* loss_out,
+                     void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Failure-detection self test: one CTA waits on an mbarrier that nothing
+ * arrives on, through the same bounded wait the pipelined kernels use, with
+ * a limit of limit_ns (1 .. 2e9).  Expected outcome: *info (device int32,
+ * caller-zeroed) becomes KRONQ_ERR_TIMEOUT and the kernel returns; the
+ * context stays usable.  Not part of the quantization path.
+ */
+int kronq_selftest_wait(int32_t* info, int64_t limit_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KRONQ_H */

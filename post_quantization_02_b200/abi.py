@@ -1,0 +1,220 @@
+"""Python binding of libkronq: the C ABI of include/kronq.h, one function per
+entry point, same names.  Argument marshalling only (device pointers, sizes,
+the current CUDA stream); every computation runs in the CUDA library.
+
+There is no fallback: if libkronq.so is missing or fails to load, every call
+raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import pathlib
+
+import torch
+
+HERE = pathlib.Path(__file__).resolve().parent
+LIB_PATH = HERE / "libkronq.so"
+
+KRONQ_OK = 0
+STATUS = {
+    0: "ok", -1: "invalid argument", -2: "unsupported", -3: "matrix not positive definite",
+    -4: "CUDA error", -5: "device wait timed out", -6: "workspace missing or too small",
+}
+MODES = {"full": 0, "no_rescale": 1, "su_only": 2, "sv_only": 3}
+
+_lib = None
+
+
+class KronqError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn}: {STATUS.get(code, 'unknown status')} ({code})")
+        self.code = code
+
+
+def lib() -> ctypes.CDLL:
+    """Load libkronq.so (built in-tree by post_quantization_02_b200.build)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not LIB_PATH.exists():
+        raise RuntimeError(f"{LIB_PATH} is not built; run `python -m post_quantization_02_b200.build`")
+    L = ctypes.CDLL(str(LIB_PATH))
+    P, I64, I32, F32, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    sig = {
+        "kronq_status_string": ([I32], ctypes.c_char_p),
+        "kronq_abi_version": ([], I32),
+        "kronq_launch_count": ([], ctypes.c_uint64),
+        "kronq_workspace_size": ([I64, I64, I32, I32, I32], SZ),
+        "kronq_covariance": ([P, I64, I64, I64, P, I64, F32, F32, P, P], I32),
+        "kronq_sensitivity": ([P, I64, P, I64, P, P], I32),
+        "kronq_biip_rotate": ([P, I64, I64, P, P, P, P, F32, I32, I32, P, P, P, SZ, P], I32),
+        "kronq_cholesky_inv": ([P, I64, F32, P, P, P, SZ, P], I32),
+        "kronq_quantize_layer": ([P, I64, I64, P, I32, I32, I32, P, P, P, P, P, P, SZ, P], I32),
+        "kronq_pack": ([P, I64, I64, I32, P, P], I32),
+        "kronq_unpack": ([P, I64, I64, I32, P, P], I32),
+        "kronq_layer_loss": ([P, P, I64, I64, P, P, P, P, SZ, P], I32),
+        "kronq_selftest_wait": ([P, I64, P], I32),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(L, name)
+        f.argtypes = args
+        f.restype = res
+    _lib = L
+    return L
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _s(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(fn: str, code: int):
+    if code != KRONQ_OK:
+        raise KronqError(fn, code)
+
+
+def _dev(t, dtype, name, ndim=None):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims")
+
+
+def _contig(t, name):
+    if t is not None and not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def kronq_status_string(code: int) -> str:
+    return lib().kronq_status_string(code).decode()
+
+
+def kronq_abi_version() -> int:
+    return lib().kronq_abi_version()
+
+
+def kronq_launch_count() -> int:
+    return int(lib().kronq_launch_count())
+
+
+def kronq_workspace_size(m: int, n: int, bits: int = 4, group: int = -1, block: int = 128) -> int:
+    return int(lib().kronq_workspace_size(m, n, bits, group, block))
+
+
+def workspace(m: int, n: int, bits: int = 4, group: int = -1, block: int = 128, device=None):
+    """A caller-owned workspace tensor of kronq_workspace_size bytes."""
+    nbytes = kronq_workspace_size(m, n, bits, group, block)
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device or "cuda")
+
+
+def kronq_covariance(A, H, alpha: float, beta: float = 0.0, info=None, stream=None):
+    """H = alpha A^T A + beta H.  A: (N, d) bf16 (row stride lda, unit column
+    stride); H: (d, d) fp32 with unit column stride."""
+    _dev(A, (torch.bfloat16, torch.int16, torch.uint16), "A", 2)
+    _dev(H, torch.float32, "H", 2)
+    if A.stride(1) != 1 or H.stride(1) != 1:
+        raise ValueError("A and H need unit stride along their last dimension")
+    N, d = A.shape
+    if H.shape != (d, d):
+        raise ValueError("H must be d x d")
+    _check("kronq_covariance", lib().kronq_covariance(
+        _p(A), N, d, A.stride(0) if N > 0 else d, _p(H), H.stride(0), alpha, beta, _p(info), _s(stream)))
+
+
+def kronq_sensitivity(HX, HG, out, stream=None):
+    """out (3 fp64, device) = {tr(H_G) tr(H_X), tr(H_X), tr(H_G)}."""
+    _dev(HX, torch.float32, "H_X", 2)
+    _dev(HG, torch.float32, "H_G", 2)
+    _dev(out, torch.float64, "out")
+    _contig(HX, "H_X"); _contig(HG, "H_G")
+    _check("kronq_sensitivity", lib().kronq_sensitivity(
+        _p(HX), HX.shape[0], _p(HG), HG.shape[0], _p(out), _s(stream)))
+
+
+def kronq_biip_rotate(W, HX, HG, sign_u, sign_v, alpha: float, mode, inverse: int, SX, SG, ws,
+                      stream=None):
+    _dev(W, torch.float32, "W", 2)
+    _dev(HX, torch.float32, "H_X", 2)
+    _dev(HG, torch.float32, "H_G", 2)
+    _dev(sign_u, torch.int8, "sign_u")
+    _dev(sign_v, torch.int8, "sign_v")
+    _dev(SX, torch.float32, "S_X")
+    _dev(SG, torch.float32, "S_G")
+    for t, nm in ((W, "W"), (HX, "H_X"), (HG, "H_G"), (ws, "ws")):
+        _contig(t, nm)
+    m, n = W.shape
+    mode = MODES[mode] if isinstance(mode, str) else int(mode)
+    _check("kronq_biip_rotate", lib().kronq_biip_rotate(
+        _p(W), m, n, _p(HX), _p(HG), _p(sign_u), _p(sign_v), alpha, mode, int(inverse),
+        _p(SX), _p(SG), _p(ws), ws.numel() * ws.element_size(), _s(stream)))
+
+
+def kronq_cholesky_inv(H, damp_rel: float, U, info, ws, stream=None):
+    _dev(H, torch.float32, "H", 2)
+    _dev(U, torch.float32, "U_c", 2)
+    _contig(H, "H"); _contig(U, "U_c")
+    _check("kronq_cholesky_inv", lib().kronq_cholesky_inv(
+        _p(H), H.shape[0], damp_rel, _p(U), _p(info), _p(ws), ws.numel() * ws.element_size(),
+        _s(stream)))
+
+
+def kronq_quantize_layer(W, U, bits: int, group: int, block: int, codes, scales, zeros,
+                         W_hat=None, info=None, ws=None, stream=None):
+    _dev(W, torch.float32, "W", 2)
+    _dev(U, torch.float32, "U_c", 2)
+    _dev(codes, torch.uint8, "codes", 2)
+    _dev(scales, torch.float32, "scales")
+    _dev(zeros, torch.uint8, "zeros")
+    _dev(W_hat, torch.float32, "W_hat", 2)
+    for t, nm in ((W, "W"), (U, "U_c"), (codes, "codes"), (scales, "scales"), (zeros, "zeros"),
+                  (W_hat, "W_hat")):
+        _contig(t, nm)
+    m, n = W.shape
+    _check("kronq_quantize_layer", lib().kronq_quantize_layer(
+        _p(W), m, n, _p(U), bits, group, block, _p(codes), _p(scales), _p(zeros), _p(W_hat),
+        _p(info), _p(ws), 0 if ws is None else ws.numel() * ws.element_size(), _s(stream)))
+
+
+def kronq_pack(codes, bits: int, packed, stream=None):
+    _dev(codes, torch.uint8, "codes", 2)
+    _dev(packed, (torch.int32, torch.uint32), "packed", 2)
+    _contig(codes, "codes"); _contig(packed, "packed")
+    m, n = codes.shape
+    _check("kronq_pack", lib().kronq_pack(_p(codes), m, n, bits, _p(packed), _s(stream)))
+
+
+def kronq_unpack(packed, n: int, bits: int, codes, stream=None):
+    _dev(codes, torch.uint8, "codes", 2)
+    _dev(packed, (torch.int32, torch.uint32), "packed", 2)
+    _contig(codes, "codes"); _contig(packed, "packed")
+    m = codes.shape[0]
+    _check("kronq_unpack", lib().kronq_unpack(_p(packed), m, n, bits, _p(codes), _s(stream)))
+
+
+def kronq_layer_loss(W_ref, W_hat, HX, HG, out, ws, stream=None):
+    for t, nm in ((W_ref, "W_ref"), (W_hat, "W_hat"), (HX, "H_X"), (HG, "H_G")):
+        _dev(t, torch.float32, nm, 2)
+        _contig(t, nm)
+    _dev(out, torch.float64, "loss_out")
+    m, n = W_ref.shape
+    _check("kronq_layer_loss", lib().kronq_layer_loss(
+        _p(W_ref), _p(W_hat), m, n, _p(HX), _p(HG), _p(out), _p(ws),
+        ws.numel() * ws.element_size(), _s(stream)))
+
+
+def kronq_selftest_wait(info, limit_ns: int, stream=None):
+    _dev(info, torch.int32, "info")
+    _check("kronq_selftest_wait", lib().kronq_selftest_wait(_p(info), int(limit_ns), _s(stream)))
+
+
+def packed_words(n: int, bits: int) -> int:
+    return (n * bits + 31) // 32

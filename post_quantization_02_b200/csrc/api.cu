@@ -1,0 +1,158 @@
+// extern "C" entry points of libkronq (declared in include/kronq.h).
+// Host-side argument checks live next to each launcher; this file only maps
+// the ABI onto them and provides the shared host helpers.
+#include <atomic>
+
+#include "common.cuh"
+
+size_t kq_cholesky_ws(int64_t n);
+size_t kq_biip_ws(int64_t m, int64_t n);
+size_t kq_quantize_ws(int64_t m);
+size_t kq_loss_ws(int64_t m, int64_t n);
+int kq_covariance(const uint16_t* A, int64_t N, int64_t d, int64_t lda, float* H, int64_t ldh,
+                  float alpha, float beta, int32_t* info, cudaStream_t st);
+int kq_sensitivity(const float* HX, int64_t n, const float* HG, int64_t m, double* out,
+                   cudaStream_t st);
+int kq_biip_rotate(float* W, int64_t m, int64_t n, float* HX, float* HG, const int8_t* su,
+                   const int8_t* sv, float alpha, int mode, int inverse, float* SX, float* SG,
+                   void* ws, size_t ws_bytes, cudaStream_t st);
+int kq_cholesky_inv(const float* H, int64_t n, float damp_rel, float* U, int32_t* info, void* ws,
+                    size_t ws_bytes, cudaStream_t st);
+int kq_quantize_layer(float* W, int64_t m, int64_t n, const float* U, int bits, int group,
+                      int block, uint8_t* codes, float* scales, uint8_t* zeros, float* W_hat,
+                      int32_t* info, void* ws, size_t ws_bytes, cudaStream_t st);
+int kq_pack(const uint8_t* codes, int64_t m, int64_t n, int bits, uint32_t* packed,
+            cudaStream_t st);
+int kq_unpack(const uint32_t* packed, int64_t m, int64_t n, int bits, uint8_t* codes,
+              cudaStream_t st);
+int kq_layer_loss(const float* Wr, const float* Wh, int64_t m, int64_t n, const float* HX,
+                  const float* HG, double* out, void* ws, size_t ws_bytes, cudaStream_t st);
+
+namespace kqh {
+
+int num_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!cache[dev]) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+      v = 148;
+    cache[dev] = v;
+  }
+  return cache[dev];
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+static std::atomic<unsigned long long> g_launches{0};
+
+int launch_status() {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return cudaGetLastError() == cudaSuccess ? KRONQ_OK : KRONQ_ERR_CUDA;
+}
+
+unsigned long long launches() { return g_launches.load(std::memory_order_relaxed); }
+
+}  // namespace kqh
+
+static cudaStream_t S(void* s) { return static_cast<cudaStream_t>(s); }
+
+// Waits on an mbarrier that nothing ever arrives on, with the given limit:
+// the bounded-wait path of the pipelined kernels, made to run out on purpose.
+__global__ void selftest_wait_kernel(int32_t* info, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort;
+  if (threadIdx.x == 0) {
+    kq::mbar_init(&bar, 1);
+    abort = 0;
+    kq::fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) kq::mbar_wait(&bar, 0, &abort, info, limit_ns);
+  __syncthreads();
+}
+
+extern "C" {
+
+const char* kronq_status_string(int st) {
+  switch (st) {
+    case KRONQ_OK: return "ok";
+    case KRONQ_ERR_INVALID_ARG: return "invalid argument";
+    case KRONQ_ERR_UNSUPPORTED: return "unsupported";
+    case KRONQ_ERR_NOT_PD: return "matrix not positive definite";
+    case KRONQ_ERR_CUDA: return "CUDA error";
+    case KRONQ_ERR_TIMEOUT: return "device wait timed out";
+    case KRONQ_ERR_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+int kronq_abi_version(void) { return 100; }
+
+uint64_t kronq_launch_count(void) { return kqh::launches(); }
+
+int kronq_selftest_wait(int32_t* info, int64_t limit_ns, void* stream) {
+  if (!info || limit_ns <= 0 || limit_ns > 2000000000ll) return KRONQ_ERR_INVALID_ARG;
+  selftest_wait_kernel<<<1, 32, 0, S(stream)>>>(info, (unsigned long long)limit_ns);
+  return kqh::launch_status();
+}
+
+size_t kronq_workspace_size(int64_t m, int64_t n, int bits, int group, int block) {
+  (void)bits; (void)group; (void)block;
+  if (m <= 0 || n <= 0) return 0;
+  size_t s = kq_biip_ws(m, n);
+  const size_t c = kq_cholesky_ws(n), q = kq_quantize_ws(m), l = kq_loss_ws(m, n);
+  if (c > s) s = c;
+  if (q > s) s = q;
+  if (l > s) s = l;
+  return s;
+}
+
+int kronq_covariance(const uint16_t* A, int64_t N, int64_t d, int64_t lda, float* H, int64_t ldh,
+                     float alpha, float beta, int32_t* info, void* stream) {
+  return kq_covariance(A, N, d, lda, H, ldh, alpha, beta, info, S(stream));
+}
+
+int kronq_sensitivity(const float* H_X, int64_t n, const float* H_G, int64_t m, double* out,
+                      void* stream) {
+  return kq_sensitivity(H_X, n, H_G, m, out, S(stream));
+}
+
+int kronq_biip_rotate(float* W, int64_t m, int64_t n, float* H_X, float* H_G,
+                      const int8_t* sign_u, const int8_t* sign_v, float alpha, int mode,
+                      int inverse, float* S_X, float* S_G, void* ws, size_t ws_bytes,
+                      void* stream) {
+  return kq_biip_rotate(W, m, n, H_X, H_G, sign_u, sign_v, alpha, mode, inverse, S_X, S_G, ws,
+                        ws_bytes, S(stream));
+}
+
+int kronq_cholesky_inv(const float* H, int64_t n, float damp_rel, float* U_c, int32_t* info,
+                       void* ws, size_t ws_bytes, void* stream) {
+  return kq_cholesky_inv(H, n, damp_rel, U_c, info, ws, ws_bytes, S(stream));
+}
+
+int kronq_quantize_layer(float* W, int64_t m, int64_t n, const float* U_c, int bits, int group,
+                         int block, uint8_t* codes, float* scales, uint8_t* zeros, float* W_hat,
+                         int32_t* info, void* ws, size_t ws_bytes, void* stream) {
+  return kq_quantize_layer(W, m, n, U_c, bits, group, block, codes, scales, zeros, W_hat, info, ws,
+                           ws_bytes, S(stream));
+}
+
+int kronq_pack(const uint8_t* codes, int64_t m, int64_t n, int bits, uint32_t* packed,
+               void* stream) {
+  return kq_pack(codes, m, n, bits, packed, S(stream));
+}
+
+int kronq_unpack(const uint32_t* packed, int64_t m, int64_t n, int bits, uint8_t* codes,
+                 void* stream) {
+  return kq_unpack(packed, m, n, bits, codes, S(stream));
+}
+
+int kronq_layer_loss(const float* W_ref, const float* W_hat, int64_t m, int64_t n,
+                     const float* H_X, const float* H_G, double* loss_out, void* ws,
+                     size_t ws_bytes, void* stream) {
+  return kq_layer_loss(W_ref, W_hat, m, n, H_X, H_G, loss_out, ws, ws_bytes, S(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,420 @@
+// Bidirectional incoherence processing and the sensitivity score.
+//
+// KronQ summary (hyper.ai), "Method", Eqs. 11-12: diagonal rescale of both
+// dimensions of W (S_X on columns, S_G on rows; S_G is KronQ's addition),
+// then W' = U W V^T, H_X' = V H_X V^T, H_G' = U H_G U^T with randomized
+// Hadamard transforms; Eq. 14: s = tr(H_G') tr(H_X').
+//
+// Transform of a length-d vector, d = Q * L2 with L2 = 2^k2 <= 4096:
+//   x -> (M_Q (x) H_L2 / sqrt(L2)) D x,   M_Q = C_q (x) H_{2^k1} / sqrt(2^k1)
+// (C_q the orthonormal DCT-II, q the odd part of d).  This is the same matrix
+// as C_q (x) H_{2^k} / sqrt(2^k): a Sylvester Hadamard of size 2^k1 L2 splits
+// into H_{2^k1} on the high index bits and H_L2 on the low ones.  Within a
+// segment of L2 consecutive entries: Walsh-Hadamard butterflies; across the
+// Q segments: a dense Q x Q mix.
+//
+// Passes over HBM: a row pass (one CTA per row, the row staged in shared
+// memory, scaling and signs fused into the load) and a column pass (64-row..
+// 4096-row segments of 8-column panels in shared memory, then the Q-mix).
+#include "common.cuh"
+
+namespace {
+
+constexpr int RT_THREADS = 256;
+constexpr int CP_COLS = 8;  // columns per panel in the column pass
+
+struct Split {
+  int L2, Q, q, k1;
+};
+
+bool split_width(int64_t d, Split& s) {
+  if (d < 16 || d % 16) return false;
+  int64_t q = d;
+  int k = 0;
+  while (q % 2 == 0) { q /= 2; ++k; }
+  if (q > 63) return false;
+  const int k2 = k < 12 ? k : 12;
+  s.L2 = 1 << k2;
+  s.k1 = k - k2;
+  s.q = (int)q;
+  s.Q = (int)q << s.k1;
+  return s.Q <= 64;
+}
+
+// M = C_q (x) H_{2^k1} / sqrt(2^k1), Q x Q, row-major.
+__global__ void make_mix_kernel(float* __restrict__ M, int q, int k1) {
+  const int Q = q << k1;
+  const double PI = 3.14159265358979323846;
+  for (int e = threadIdx.x; e < Q * Q; e += blockDim.x) {
+    const int s = e / Q, t = e % Q;
+    const int p = s >> k1, a = s & ((1 << k1) - 1);
+    const int p2 = t >> k1, a2 = t & ((1 << k1) - 1);
+    double c = sqrt(2.0 / q) * cos(PI * (2 * p2 + 1) * p / (2.0 * q));
+    if (p == 0) c *= sqrt(0.5);
+    const double h = (__popc(a & a2) & 1) ? -1.0 : 1.0;
+    M[e] = (float)(c * h / sqrt((double)(1 << k1)));
+  }
+}
+
+__global__ void colnorm_kernel(const float* __restrict__ W, int m, int n, double* __restrict__ cn) {
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= n) return;
+  const int rows_per = (m + gridDim.y - 1) / gridDim.y;
+  const int r0 = blockIdx.y * rows_per, r1 = min(m, r0 + rows_per);
+  double s = 0.0;
+  for (int i = r0; i < r1; ++i) {
+    const double v = W[(int64_t)i * n + j];
+    s += v * v;
+  }
+  atomicAdd(&cn[j], s);
+}
+
+// S = (H_jj / norm2_j)^alpha (1 when either is not positive); also 1/S.
+__global__ void scale_from_diag_kernel(const float* __restrict__ H, int d,
+                                       const double* __restrict__ norm2, float alpha,
+                                       float* __restrict__ S, float* __restrict__ rS, int active) {
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= d) return;
+  float s = 1.f;
+  if (active) {
+    const double h = H[(int64_t)j * d + j], nn = norm2[j];
+    if (h > 0.0 && nn > 0.0) s = (float)pow(h / nn, (double)alpha);
+  }
+  S[j] = s;
+  rS[j] = 1.f / s;
+}
+
+// ||(W S_X)_i,:||^2, one warp per row.
+__global__ void rownorm_kernel(const float* __restrict__ W, int m, int n,
+                               const float* __restrict__ SX, double* __restrict__ rn) {
+  const int row = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  const int lane = threadIdx.x & 31;
+  if (row >= m) return;
+  double s = 0.0;
+  for (int j = lane; j < n; j += 32) {
+    const double v = (double)(W[(int64_t)row * n + j] * SX[j]);
+    s += v * v;
+  }
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane == 0) rn[row] = s;
+}
+
+__global__ void recip_kernel(const float* __restrict__ S, float* __restrict__ rS, int d) {
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j < d) rS[j] = 1.f / S[j];
+}
+
+// X[r][c] *= rs[r] cs[c]
+__global__ void scale_only_kernel(float* __restrict__ X, int R, int C, const float* __restrict__ rs,
+                                  const float* __restrict__ cs) {
+  const int64_t total = (int64_t)R * C;
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int r = (int)(e / C), c = (int)(e % C);
+    X[e] *= rs[r] * cs[c];
+  }
+}
+
+// In-shared-memory Walsh-Hadamard butterflies on Q segments of L2 entries.
+__device__ void fwht_segments(float* x, int L2, int Q) {
+  const int half = L2 >> 1;
+  const int pairs = half * Q;
+  for (int h = 1; h < L2; h <<= 1) {
+    for (int p = threadIdx.x; p < pairs; p += blockDim.x) {
+      const int s = p / half, qq = p - s * half;
+      const int i = s * L2 + (qq / h) * 2 * h + (qq % h);
+      const float a = x[i], b = x[i + h];
+      x[i] = a + b;
+      x[i + h] = a - b;
+    }
+    __syncthreads();
+  }
+}
+
+// y[s L2 + r] = sum_t M[s][t] x[t L2 + r]  (M^T when transpose), in place.
+__device__ void mix_segments(float* x, int L2, int Q, const float* __restrict__ M, bool transpose) {
+  float v[64];
+  for (int r = threadIdx.x; r < L2; r += blockDim.x) {
+    for (int t = 0; t < Q; ++t) v[t] = x[t * L2 + r];
+    for (int s = 0; s < Q; ++s) {
+      float acc = 0.f;
+      for (int t = 0; t < Q; ++t) acc = fmaf(transpose ? M[t * Q + s] : M[s * Q + t], v[t], acc);
+      x[s * L2 + r] = acc;
+    }
+  }
+  __syncthreads();
+}
+
+// One row per CTA.  forward: x <- T D (rs[r] cs[c] x);  inverse: x <- rs[r] cs[c] D T^T x.
+__global__ void __launch_bounds__(RT_THREADS)
+row_transform_kernel(float* __restrict__ X, int R, int C, const float* __restrict__ rs,
+                     const float* __restrict__ cs, const int8_t* __restrict__ sign, int L2, int Q,
+                     const float* __restrict__ M, int inverse) {
+  extern __shared__ float x[];
+  const int r = blockIdx.x;
+  if (r >= R) return;
+  float* row = X + (int64_t)r * C;
+  const float rsc = rs ? rs[r] : 1.f;
+  const float norm = rsqrtf((float)L2);
+  for (int c = threadIdx.x; c < C; c += blockDim.x) {
+    float v = row[c];
+    if (!inverse) v = v * (rsc * (cs ? cs[c] : 1.f)) * (float)sign[c];
+    x[c] = v;
+  }
+  __syncthreads();
+  if (inverse && Q > 1) mix_segments(x, L2, Q, M, true);
+  fwht_segments(x, L2, Q);
+  if (!inverse && Q > 1) mix_segments(x, L2, Q, M, false);
+  for (int c = threadIdx.x; c < C; c += blockDim.x) {
+    float v = x[c] * norm;
+    if (inverse) v = v * (float)sign[c] * (rsc * (cs ? cs[c] : 1.f));
+    row[c] = v;
+  }
+}
+
+// Column pass, step 1: Walsh-Hadamard along rows inside each L2-row segment,
+// on a panel of CP_COLS columns (signs of the rows first when forward, last
+// when inverse; normalized by 1/sqrt(L2)).
+__global__ void __launch_bounds__(256)
+col_fht_kernel(float* __restrict__ X, int R, int C, const int8_t* __restrict__ sign, int L2,
+               int inverse) {
+  extern __shared__ float p[];  // [L2][CP_COLS]
+  const int seg = blockIdx.y, c0 = blockIdx.x * CP_COLS;
+  const int r0 = seg * L2;
+  const float norm = rsqrtf((float)L2);
+  for (int e = threadIdx.x; e < L2 * CP_COLS; e += blockDim.x) {
+    const int rr = e / CP_COLS, cc = e % CP_COLS;
+    float v = 0.f;
+    if (c0 + cc < C) v = X[(int64_t)(r0 + rr) * C + c0 + cc];
+    if (!inverse) v *= (float)sign[r0 + rr];
+    p[e] = v;
+  }
+  __syncthreads();
+  const int half = L2 >> 1;
+  for (int h = 1; h < L2; h <<= 1) {
+    for (int e = threadIdx.x; e < half * CP_COLS; e += blockDim.x) {
+      const int pr = e / CP_COLS, cc = e % CP_COLS;
+      const int i = (pr / h) * 2 * h + (pr % h);
+      const float a = p[i * CP_COLS + cc], b = p[(i + h) * CP_COLS + cc];
+      p[i * CP_COLS + cc] = a + b;
+      p[(i + h) * CP_COLS + cc] = a - b;
+    }
+    __syncthreads();
+  }
+  for (int e = threadIdx.x; e < L2 * CP_COLS; e += blockDim.x) {
+    const int rr = e / CP_COLS, cc = e % CP_COLS;
+    if (c0 + cc >= C) continue;
+    float v = p[e] * norm;
+    if (inverse) v *= (float)sign[r0 + rr];
+    X[(int64_t)(r0 + rr) * C + c0 + cc] = v;
+  }
+}
+
+// Column pass, step 2: rows {s L2 + r : s < Q} mixed by M (or M^T), 64 columns per CTA.
+__global__ void __launch_bounds__(64)
+col_mix_kernel(float* __restrict__ X, int C, int L2, int Q, const float* __restrict__ M,
+               int transpose) {
+  __shared__ float v[64][65];
+  __shared__ float Ms[64 * 64];
+  const int r = blockIdx.y, c = blockIdx.x * 64 + threadIdx.x;
+  for (int e = threadIdx.x; e < Q * Q; e += blockDim.x) Ms[e] = M[e];
+  for (int t = 0; t < Q; ++t) v[t][threadIdx.x] = (c < C) ? X[(int64_t)(t * L2 + r) * C + c] : 0.f;
+  __syncthreads();
+  if (c >= C) return;
+  for (int s = 0; s < Q; ++s) {
+    float acc = 0.f;
+    for (int t = 0; t < Q; ++t) acc = fmaf(transpose ? Ms[t * Q + s] : Ms[s * Q + t], v[t][threadIdx.x], acc);
+    X[(int64_t)(s * L2 + r) * C + c] = acc;
+  }
+}
+
+__global__ void sensitivity_kernel(const float* __restrict__ HX, int n, const float* __restrict__ HG,
+                                   int m, double* __restrict__ out) {
+  __shared__ double sx[256], sg[256];
+  double a = 0.0, b = 0.0;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) a += (double)HX[(int64_t)i * n + i];
+  for (int i = threadIdx.x; i < m; i += blockDim.x) b += (double)HG[(int64_t)i * m + i];
+  sx[threadIdx.x] = a;
+  sg[threadIdx.x] = b;
+  __syncthreads();
+  for (int w = 128; w > 0; w >>= 1) {
+    if (threadIdx.x < w) {
+      sx[threadIdx.x] += sx[threadIdx.x + w];
+      sg[threadIdx.x] += sg[threadIdx.x + w];
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    out[0] = sx[0] * sg[0];
+    out[1] = sx[0];
+    out[2] = sg[0];
+  }
+}
+
+size_t a256(size_t b) { return (b + 255) & ~(size_t)255; }
+
+bool g_row_attr = false, g_col_attr = false;
+
+int set_attrs() {
+  if (!g_row_attr) {
+    if (cudaFuncSetAttribute(row_transform_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             200 * 1024) != cudaSuccess)
+      return KRONQ_ERR_CUDA;
+    g_row_attr = true;
+  }
+  if (!g_col_attr) {
+    if (cudaFuncSetAttribute(col_fht_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             4096 * CP_COLS * 4) != cudaSuccess)
+      return KRONQ_ERR_CUDA;
+    g_col_attr = true;
+  }
+  return KRONQ_OK;
+}
+
+// Apply T D along rows (row pass, with scaling) of an R x C matrix.
+int row_pass(float* X, int R, int C, const float* rs, const float* cs, const int8_t* sign,
+             const Split& sp, const float* M, int inverse, cudaStream_t st) {
+  const size_t smem = (size_t)C * sizeof(float);
+  if (smem > 200 * 1024) return KRONQ_ERR_UNSUPPORTED;
+  row_transform_kernel<<<R, RT_THREADS, smem, st>>>(X, R, C, rs, cs, sign, sp.L2, sp.Q, M, inverse);
+  KQ_CHECK_LAUNCH();
+  return KRONQ_OK;
+}
+
+// Apply T D along columns of an R x C matrix (R = Q * L2).
+int col_pass(float* X, int R, int C, const int8_t* sign, const Split& sp, const float* M,
+             int inverse, cudaStream_t st) {
+  const dim3 g1((C + CP_COLS - 1) / CP_COLS, sp.Q);
+  const size_t smem = (size_t)sp.L2 * CP_COLS * sizeof(float);
+  if (inverse && sp.Q > 1) {
+    col_mix_kernel<<<dim3((C + 63) / 64, sp.L2), 64, 0, st>>>(X, C, sp.L2, sp.Q, M, 1);
+    KQ_CHECK_LAUNCH();
+  }
+  col_fht_kernel<<<g1, 256, smem, st>>>(X, R, C, sign, sp.L2, inverse);
+  KQ_CHECK_LAUNCH();
+  if (!inverse && sp.Q > 1) {
+    col_mix_kernel<<<dim3((C + 63) / 64, sp.L2), 64, 0, st>>>(X, C, sp.L2, sp.Q, M, 0);
+    KQ_CHECK_LAUNCH();
+  }
+  (void)R;
+  return KRONQ_OK;
+}
+
+}  // namespace
+
+size_t kq_biip_ws(int64_t m, int64_t n) {
+  return a256((size_t)(m + n) * sizeof(double)) + 2 * a256((size_t)(m + n) * sizeof(float)) +
+         2 * a256(64 * 64 * sizeof(float));
+}
+
+int kq_sensitivity(const float* HX, int64_t n, const float* HG, int64_t m, double* out,
+                   cudaStream_t st) {
+  if (!HX || !HG || !out || n <= 0 || m <= 0 || n > INT32_MAX || m > INT32_MAX)
+    return KRONQ_ERR_INVALID_ARG;
+  sensitivity_kernel<<<1, 256, 0, st>>>(HX, (int)n, HG, (int)m, out);
+  KQ_CHECK_LAUNCH();
+  return KRONQ_OK;
+}
+
+int kq_biip_rotate(float* W, int64_t m64, int64_t n64, float* HX, float* HG, const int8_t* su,
+                   const int8_t* sv, float alpha, int mode, int inverse, float* SX, float* SG,
+                   void* ws, size_t ws_bytes, cudaStream_t st) {
+  if (mode < 0 || mode > 3 || (inverse != 0 && inverse != 1)) return KRONQ_ERR_INVALID_ARG;
+  if (!W || !su || !sv || !SX || !SG || m64 <= 0 || n64 <= 0) return KRONQ_ERR_INVALID_ARG;
+  if (!inverse && (!HX || !HG)) return KRONQ_ERR_INVALID_ARG;
+  if (!(alpha >= 0.f)) return KRONQ_ERR_INVALID_ARG;
+  if (m64 % 16 || n64 % 16) return KRONQ_ERR_INVALID_ARG;
+  if (m64 > 65536 || n64 > 65536) return KRONQ_ERR_UNSUPPORTED;
+  Split spm, spn;
+  if (!split_width(m64, spm) || !split_width(n64, spn)) return KRONQ_ERR_UNSUPPORTED;
+  if (!ws || ws_bytes < kq_biip_ws(m64, n64) || !kqh::aligned(ws, 256)) return KRONQ_ERR_WORKSPACE;
+  int st0 = set_attrs();
+  if (st0 != KRONQ_OK) return st0;
+  const int m = (int)m64, n = (int)n64;
+  const bool in_s = mode == 0 || mode == 3, out_s = mode == 0 || mode == 2;
+  const bool in_r = mode != 2, out_r = mode != 3;
+
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  double* cn = reinterpret_cast<double*>(w);
+  double* rn = cn + n;
+  w += a256((size_t)(m + n) * sizeof(double));
+  float* rSX = reinterpret_cast<float*>(w);
+  float* rSG = rSX + n;
+  w += a256((size_t)(m + n) * sizeof(float));
+  w += a256((size_t)(m + n) * sizeof(float));  // spare slot
+  float* Mn = reinterpret_cast<float*>(w);
+  w += a256(64 * 64 * sizeof(float));
+  float* Mm = reinterpret_cast<float*>(w);
+
+  if (spn.Q > 1) { make_mix_kernel<<<1, 256, 0, st>>>(Mn, spn.q, spn.k1); KQ_CHECK_LAUNCH(); }
+  if (spm.Q > 1) { make_mix_kernel<<<1, 256, 0, st>>>(Mm, spm.q, spm.k1); KQ_CHECK_LAUNCH(); }
+  const int sms = kqh::num_sms();
+
+  if (inverse) {
+    recip_kernel<<<(n + 255) / 256, 256, 0, st>>>(SX, rSX, n);
+    KQ_CHECK_LAUNCH();
+    recip_kernel<<<(m + 255) / 256, 256, 0, st>>>(SG, rSG, m);
+    KQ_CHECK_LAUNCH();
+    if (out_r) {
+      int s = col_pass(W, m, n, su, spm, Mm, 1, st);
+      if (s) return s;
+    }
+    if (in_r) {
+      int s = row_pass(W, m, n, rSG, rSX, sv, spn, Mn, 1, st);
+      if (s) return s;
+    } else {
+      scale_only_kernel<<<4 * sms, 256, 0, st>>>(W, m, n, rSG, rSX);
+      KQ_CHECK_LAUNCH();
+    }
+    return KRONQ_OK;
+  }
+
+  // ---- rescale factors
+  if (cudaMemsetAsync(cn, 0, (size_t)n * sizeof(double), st) != cudaSuccess) return KRONQ_ERR_CUDA;
+  if (in_s) {
+    colnorm_kernel<<<dim3((n + 255) / 256, 32), 256, 0, st>>>(W, m, n, cn);
+    KQ_CHECK_LAUNCH();
+  }
+  scale_from_diag_kernel<<<(n + 255) / 256, 256, 0, st>>>(HX, n, cn, alpha, SX, rSX, in_s);
+  KQ_CHECK_LAUNCH();
+  if (out_s) {
+    rownorm_kernel<<<(m + 7) / 8, 256, 0, st>>>(W, m, n, SX, rn);
+    KQ_CHECK_LAUNCH();
+  }
+  scale_from_diag_kernel<<<(m + 255) / 256, 256, 0, st>>>(HG, m, rn, alpha, SG, rSG, out_s);
+  KQ_CHECK_LAUNCH();
+
+  // ---- W' = U (S_G W S_X) V^T
+  if (in_r) {
+    int s = row_pass(W, m, n, SG, SX, sv, spn, Mn, 0, st);
+    if (s) return s;
+  } else {
+    scale_only_kernel<<<4 * sms, 256, 0, st>>>(W, m, n, SG, SX);
+    KQ_CHECK_LAUNCH();
+  }
+  if (out_r) {
+    int s = col_pass(W, m, n, su, spm, Mm, 0, st);
+    if (s) return s;
+  }
+  // ---- H_X' = V S_X^-1 H_X S_X^-1 V^T
+  if (in_r) {
+    int s = row_pass(HX, n, n, rSX, rSX, sv, spn, Mn, 0, st);
+    if (s) return s;
+    s = col_pass(HX, n, n, sv, spn, Mn, 0, st);
+    if (s) return s;
+  } else if (in_s) {
+    scale_only_kernel<<<4 * sms, 256, 0, st>>>(HX, n, n, rSX, rSX);
+    KQ_CHECK_LAUNCH();
+  }
+  // ---- H_G' = U S_G^-1 H_G S_G^-1 U^T
+  if (out_r) {
+    int s = row_pass(HG, m, m, rSG, rSG, su, spm, Mm, 0, st);
+    if (s) return s;
+    s = col_pass(HG, m, m, su, spm, Mm, 0, st);
+    if (s) return s;
+  } else if (out_s) {
+    scale_only_kernel<<<4 * sms, 256, 0, st>>>(HG, m, m, rSG, rSG);
+    KQ_CHECK_LAUNCH();
+  }
+  return KRONQ_OK;
+}

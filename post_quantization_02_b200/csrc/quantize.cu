@@ -1,0 +1,370 @@
+// Column-wise OBS quantization of the rotated weights (GPTQ-style), packing,
+// and the layer-loss helper.
+//
+// KronQ summary (hyper.ai), "Method", Prop. 1: H_G cancels in the column
+// update, so every row of W' is solved with the inverse Cholesky factor U_c
+// of H_X alone, and rows never interact.  KronQ review (pith.science),
+// appendix, Algorithm 2: columns in blocks of B = 128 with an error buffer E
+// and lazy updates of the trailing columns.
+//
+// Per block of 128 columns:
+//   obs_block_kernel  32 rows per CTA, 8 threads per row, 16 columns of the
+//                     block held in registers by each thread; the 128 x 128
+//                     diagonal block of U_c in shared memory.  For each column
+//                     j: the owning thread quantizes, the scaled error
+//                     e = (w - w_hat) / U_c[j,j] is broadcast to the row's 8
+//                     threads with one shuffle, each thread applies
+//                     w_k -= e U_c[j,k] to its columns k > j.  No block-wide
+//                     synchronisation inside the column loop.
+//   lazy_update       W[:, i+128:] -= E U_c[i:i+128, i+128:]
+#include "common.cuh"
+#include "gemm_simt.cuh"
+
+namespace {
+
+constexpr int QB = 128;          // column block
+constexpr int ROWS_PER_CTA = 32;
+constexpr int US_LD = QB + 4;    // padded row of the U_c block in shared memory
+
+struct Grid {
+  float scale;
+  float zero;
+};
+
+// Asymmetric grid of [lo, hi] in fp32: lo = min(0, min w), hi = max(0, max w).
+__device__ __forceinline__ Grid make_grid(float mn, float mx, float maxq) {
+  const float lo = fminf(mn, 0.f), hi = fmaxf(mx, 0.f);
+  Grid g;
+  if (lo == 0.f && hi == 0.f) {
+    g.scale = 1.f;
+    g.zero = 0.f;
+  } else {
+    g.scale = __fdiv_rn(hi - lo, maxq);
+    g.zero = fminf(fmaxf(rintf(__fdiv_rn(-lo, g.scale)), 0.f), maxq);
+  }
+  return g;
+}
+
+// Per-channel grid from the whole row, one warp per row.
+__global__ void row_params_kernel(const float* __restrict__ W, int m, int n, int bits,
+                                  float* __restrict__ scales, uint8_t* __restrict__ zeros) {
+  const int row = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  const int lane = threadIdx.x & 31;
+  if (row >= m) return;
+  float mn = INFINITY, mx = -INFINITY;
+  const float* w = W + (int64_t)row * n;
+  for (int j = lane; j < n; j += 32) {
+    const float v = w[j];
+    mn = fminf(mn, v);
+    mx = fmaxf(mx, v);
+  }
+  for (int o = 16; o > 0; o >>= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  if (lane == 0) {
+    const Grid g = make_grid(mn, mx, (float)((1 << bits) - 1));
+    scales[row] = g.scale;
+    zeros[row] = (uint8_t)g.zero;
+  }
+}
+
+template <int GROUP>  // 0: per-channel grid; else 32, 64 or 128
+__global__ void __launch_bounds__(256)
+obs_block_kernel(const float* __restrict__ W, int m, int n, const float* __restrict__ U, int i1,
+                 int bits, uint8_t* __restrict__ codes, float* __restrict__ scales,
+                 uint8_t* __restrict__ zeros, float* __restrict__ W_hat, float* __restrict__ E) {
+  extern __shared__ float smem[];
+  float* Us = smem;                    // [QB][US_LD]
+  float* rdiag = smem + QB * US_LD;    // [QB]
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int chunk = tid & 7;           // which 16 columns of the block
+  const int row = blockIdx.x * ROWS_PER_CTA + (tid >> 3);
+  const bool live = row < m;
+  const float maxq = (float)((1 << bits) - 1);
+  const int G = GROUP ? n / GROUP : 1;
+
+  for (int e = tid; e < QB * QB / 4; e += blockDim.x) {
+    const int r = e / (QB / 4), c4 = e % (QB / 4);
+    const float4 u = *reinterpret_cast<const float4*>(U + (int64_t)(i1 + r) * n + i1 + c4 * 4);
+    *reinterpret_cast<float4*>(Us + r * US_LD + c4 * 4) = u;
+  }
+  for (int j = tid; j < QB; j += blockDim.x) rdiag[j] = 1.f / U[(int64_t)(i1 + j) * n + i1 + j];
+
+  float w[16];
+  {
+    const float* src = W + (int64_t)(live ? row : 0) * n + i1 + chunk * 16;
+#pragma unroll
+    for (int k = 0; k < 16; k += 4) {
+      float4 v = live ? *reinterpret_cast<const float4*>(src + k) : make_float4(0.f, 0.f, 0.f, 0.f);
+      w[k] = v.x; w[k + 1] = v.y; w[k + 2] = v.z; w[k + 3] = v.w;
+    }
+  }
+  float scale = 1.f, zero = 0.f;
+  if (GROUP == 0 && live) {
+    scale = scales[row];
+    zero = (float)zeros[row];
+  }
+  __syncthreads();
+
+  float qv[16], ev[16], hv[16];
+#pragma unroll
+  for (int j = 0; j < QB; ++j) {
+    const int c = j >> 4, jj = j & 15;
+    if (GROUP > 0 && (j % (GROUP > 0 ? GROUP : 1)) == 0) {
+      // grid of columns j .. j+GROUP-1 from the current (updated) weights
+      const int c_lo = j >> 4, c_hi = (j + GROUP) >> 4;  // chunks [c_lo, c_hi)
+      const bool in = chunk >= c_lo && chunk < c_hi;
+      float mn = INFINITY, mx = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        mn = fminf(mn, in ? w[k] : INFINITY);
+        mx = fmaxf(mx, in ? w[k] : -INFINITY);
+      }
+#pragma unroll
+      for (int o = 1; o < 8; o <<= 1) {
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      }
+      const Grid g = make_grid(mn, mx, maxq);
+      scale = g.scale;
+      zero = g.zero;
+      if (live && chunk == c) {
+        const int gi = (i1 + j) / (GROUP > 0 ? GROUP : 1);
+        scales[(int64_t)row * G + gi] = scale;
+        zeros[(int64_t)row * G + gi] = (uint8_t)zero;
+      }
+    }
+    // quantize this thread's copy of column j (meaningful on the owner only)
+    const float x = w[jj];
+    const float q = fminf(fmaxf(rintf(__fdiv_rn(x, scale)) + zero, 0.f), maxq);
+    const float wh = scale * (q - zero);
+    float e = (x - wh) * rdiag[j];
+    e = __shfl_sync(0xffffffffu, e, (lane & ~7) | c);
+    const bool own = chunk == c;
+    qv[jj] = own ? q : qv[jj];
+    hv[jj] = own ? wh : hv[jj];
+    ev[jj] = own ? e : ev[jj];
+    // w_k -= e U[j][k] for this thread's columns k > j
+    const float* ur = Us + j * US_LD + chunk * 16;
+#pragma unroll
+    for (int k = 0; k < 16; k += 4) {
+      const float4 u = *reinterpret_cast<const float4*>(ur + k);
+      const float uu[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const int col = chunk * 16 + k + t;
+        w[k + t] = fmaf(-e, (col > j) ? uu[t] : 0.f, w[k + t]);
+      }
+    }
+  }
+  if (!live) return;
+  const int64_t off = (int64_t)row * n + i1 + chunk * 16;
+  {
+    uint32_t pk[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      pk[k] = (uint32_t)qv[4 * k] | ((uint32_t)qv[4 * k + 1] << 8) | ((uint32_t)qv[4 * k + 2] << 16) |
+              ((uint32_t)qv[4 * k + 3] << 24);
+    *reinterpret_cast<uint4*>(codes + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  }
+  float* e_dst = E + (int64_t)row * QB + chunk * 16;
+#pragma unroll
+  for (int k = 0; k < 16; k += 4)
+    *reinterpret_cast<float4*>(e_dst + k) = make_float4(ev[k], ev[k + 1], ev[k + 2], ev[k + 3]);
+  if (W_hat) {
+#pragma unroll
+    for (int k = 0; k < 16; k += 4)
+      *reinterpret_cast<float4*>(W_hat + off + k) = make_float4(hv[k], hv[k + 1], hv[k + 2], hv[k + 3]);
+  }
+}
+
+// W[:, i2:] -= E U[i1:i2, i2:]
+__global__ void __launch_bounds__(256) lazy_update_kernel(float* W, int m, int n,
+                                                          const float* __restrict__ E,
+                                                          const float* __restrict__ U, int i1) {
+  const int i2 = i1 + QB;
+  kq::gemm_tile64<false, false>(E, QB, U + (int64_t)i1 * n + i2, n, W + i2, n, m, n - i2, QB, -1.f,
+                                1.f, blockIdx.y, blockIdx.x);
+}
+
+template <bool TA, bool TB>
+__global__ void __launch_bounds__(256) gemm_kernel(const float* A, int64_t lda, const float* B,
+                                                   int64_t ldb, float* C, int64_t ldc, int M, int N,
+                                                   int K, float alpha, float beta) {
+  kq::gemm_tile64<TA, TB>(A, lda, B, ldb, C, ldc, M, N, K, alpha, beta, blockIdx.y, blockIdx.x);
+}
+
+__global__ void sub_kernel(const float* __restrict__ a, const float* __restrict__ b,
+                           float* __restrict__ c, int64_t total) {
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
+       e += (int64_t)gridDim.x * blockDim.x)
+    c[e] = a[e] - b[e];
+}
+
+__global__ void dot_kernel(const float* __restrict__ a, const float* __restrict__ b, int64_t total,
+                           double* out) {
+  __shared__ double red[256];
+  double s = 0.0;
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
+       e += (int64_t)gridDim.x * blockDim.x)
+    s += (double)a[e] * (double)b[e];
+  red[threadIdx.x] = s;
+  __syncthreads();
+  for (int w = 128; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) atomicAdd(out, red[0]);
+}
+
+// ------------------------------------------------------------------ packing
+__global__ void pack_kernel(const uint8_t* __restrict__ codes, int64_t m, int64_t n, int bits,
+                            int64_t wpr, uint32_t* __restrict__ packed, int32_t* bad) {
+  const int per = 32 / bits;
+  const uint32_t mask = (1u << bits) - 1u;
+  const int64_t total = m * wpr;
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = e / wpr, wi = e % wpr;
+    const int64_t j0 = wi * per;
+    uint32_t word = 0;
+    for (int t = 0; t < per; ++t) {
+      const int64_t j = j0 + t;
+      if (j >= n) break;
+      const uint32_t c = codes[r * n + j];
+      if (c > mask && bad) atomicCAS(bad, 0, KRONQ_ERR_INVALID_ARG);
+      word |= (c & mask) << (t * bits);
+    }
+    packed[e] = word;
+  }
+}
+
+__global__ void unpack_kernel(const uint32_t* __restrict__ packed, int64_t m, int64_t n, int bits,
+                              int64_t wpr, uint8_t* __restrict__ codes) {
+  const int per = 32 / bits;
+  const uint32_t mask = (1u << bits) - 1u;
+  const int64_t total = m * n;
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = e / n, j = e % n;
+    codes[e] = (uint8_t)((packed[r * wpr + j / per] >> ((j % per) * bits)) & mask);
+  }
+}
+
+size_t a256(size_t b) { return (b + 255) & ~(size_t)255; }
+
+template <int GROUP>
+int launch_block(const float* W, int m, int n, const float* U, int i1, int bits, uint8_t* codes,
+                 float* scales, uint8_t* zeros, float* W_hat, float* E, cudaStream_t st) {
+  static bool attr = false;
+  const size_t smem = (size_t)(QB * US_LD + QB) * sizeof(float);
+  if (!attr) {
+    if (cudaFuncSetAttribute(obs_block_kernel<GROUP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+      return KRONQ_ERR_CUDA;
+    attr = true;
+  }
+  const int grid = (m + ROWS_PER_CTA - 1) / ROWS_PER_CTA;
+  obs_block_kernel<GROUP><<<grid, 256, smem, st>>>(W, m, n, U, i1, bits, codes, scales, zeros,
+                                                   W_hat, E);
+  KQ_CHECK_LAUNCH();
+  return KRONQ_OK;
+}
+
+}  // namespace
+
+size_t kq_quantize_ws(int64_t m) { return a256((size_t)m * QB * sizeof(float)); }
+
+size_t kq_loss_ws(int64_t m, int64_t n) { return 3 * a256((size_t)m * n * sizeof(float)); }
+
+int kq_quantize_layer(float* W, int64_t m64, int64_t n64, const float* U, int bits, int group,
+                      int block, uint8_t* codes, float* scales, uint8_t* zeros, float* W_hat,
+                      int32_t* info, void* ws, size_t ws_bytes, cudaStream_t st) {
+  (void)info;
+  if (!W || !U || !codes || !scales || !zeros || m64 <= 0 || n64 <= 0) return KRONQ_ERR_INVALID_ARG;
+  if (bits != 2 && bits != 3 && bits != 4 && bits != 8) return KRONQ_ERR_INVALID_ARG;
+  if (group != -1 && (group <= 0 || n64 % group)) return KRONQ_ERR_INVALID_ARG;
+  if (block != QB) return KRONQ_ERR_UNSUPPORTED;
+  if (group != -1 && group != 32 && group != 64 && group != 128) return KRONQ_ERR_UNSUPPORTED;
+  if (n64 % QB) return KRONQ_ERR_UNSUPPORTED;
+  if (m64 > INT32_MAX || n64 > 65536) return KRONQ_ERR_UNSUPPORTED;
+  if (!kqh::aligned(W, 16) || !kqh::aligned(U, 16) || !kqh::aligned(codes, 16) ||
+      (W_hat && !kqh::aligned(W_hat, 16)))
+    return KRONQ_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < kq_quantize_ws(m64) || !kqh::aligned(ws, 256)) return KRONQ_ERR_WORKSPACE;
+  const int m = (int)m64, n = (int)n64;
+  float* E = static_cast<float*>(ws);
+
+  if (group == -1) {
+    row_params_kernel<<<(m + 7) / 8, 256, 0, st>>>(W, m, n, bits, scales, zeros);
+    KQ_CHECK_LAUNCH();
+  }
+  for (int i1 = 0; i1 < n; i1 += QB) {
+    int s;
+    switch (group) {
+      case -1: s = launch_block<0>(W, m, n, U, i1, bits, codes, scales, zeros, W_hat, E, st); break;
+      case 32: s = launch_block<32>(W, m, n, U, i1, bits, codes, scales, zeros, W_hat, E, st); break;
+      case 64: s = launch_block<64>(W, m, n, U, i1, bits, codes, scales, zeros, W_hat, E, st); break;
+      default: s = launch_block<128>(W, m, n, U, i1, bits, codes, scales, zeros, W_hat, E, st); break;
+    }
+    if (s != KRONQ_OK) return s;
+    const int i2 = i1 + QB;
+    if (i2 < n) {
+      const dim3 grid((n - i2 + kq::GT - 1) / kq::GT, (m + kq::GT - 1) / kq::GT);
+      lazy_update_kernel<<<grid, 256, 0, st>>>(W, m, n, E, U, i1);
+      KQ_CHECK_LAUNCH();
+    }
+  }
+  return KRONQ_OK;
+}
+
+int kq_pack(const uint8_t* codes, int64_t m, int64_t n, int bits, uint32_t* packed,
+            cudaStream_t st) {
+  if (bits == 3) return KRONQ_ERR_UNSUPPORTED;
+  if (bits != 2 && bits != 4) return KRONQ_ERR_INVALID_ARG;
+  if (m < 0 || n < 0) return KRONQ_ERR_INVALID_ARG;
+  if (m == 0 || n == 0) return KRONQ_OK;
+  if (!codes || !packed || !kqh::aligned(packed, 4)) return KRONQ_ERR_INVALID_ARG;
+  const int64_t wpr = (n * bits + 31) / 32;
+  pack_kernel<<<4 * kqh::num_sms(), 256, 0, st>>>(codes, m, n, bits, wpr, packed, nullptr);
+  KQ_CHECK_LAUNCH();
+  return KRONQ_OK;
+}
+
+int kq_unpack(const uint32_t* packed, int64_t m, int64_t n, int bits, uint8_t* codes,
+              cudaStream_t st) {
+  if (bits == 3) return KRONQ_ERR_UNSUPPORTED;
+  if (bits != 2 && bits != 4) return KRONQ_ERR_INVALID_ARG;
+  if (m < 0 || n < 0) return KRONQ_ERR_INVALID_ARG;
+  if (m == 0 || n == 0) return KRONQ_OK;
+  if (!codes || !packed || !kqh::aligned(packed, 4)) return KRONQ_ERR_INVALID_ARG;
+  const int64_t wpr = (n * bits + 31) / 32;
+  unpack_kernel<<<4 * kqh::num_sms(), 256, 0, st>>>(packed, m, n, bits, wpr, codes);
+  KQ_CHECK_LAUNCH();
+  return KRONQ_OK;
+}
+
+int kq_layer_loss(const float* Wr, const float* Wh, int64_t m64, int64_t n64, const float* HX,
+                  const float* HG, double* out, void* ws, size_t ws_bytes, cudaStream_t st) {
+  if (!Wr || !Wh || !HX || !HG || !out || m64 <= 0 || n64 <= 0) return KRONQ_ERR_INVALID_ARG;
+  if (m64 > INT32_MAX || n64 > INT32_MAX) return KRONQ_ERR_UNSUPPORTED;
+  if (!ws || ws_bytes < kq_loss_ws(m64, n64) || !kqh::aligned(ws, 256)) return KRONQ_ERR_WORKSPACE;
+  const int m = (int)m64, n = (int)n64;
+  const size_t slab = a256((size_t)m * n * sizeof(float));
+  float* dW = static_cast<float*>(ws);
+  float* T1 = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + slab);
+  float* T2 = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + 2 * slab);
+  const int sms = kqh::num_sms();
+  sub_kernel<<<4 * sms, 256, 0, st>>>(Wr, Wh, dW, (int64_t)m * n);
+  KQ_CHECK_LAUNCH();
+  const dim3 g((n + 63) / 64, (m + 63) / 64);
+  gemm_kernel<false, false><<<g, 256, 0, st>>>(dW, n, HX, n, T1, n, m, n, n, 1.f, 0.f);
+  KQ_CHECK_LAUNCH();
+  gemm_kernel<false, false><<<g, 256, 0, st>>>(HG, m, dW, n, T2, n, m, n, m, 1.f, 0.f);
+  KQ_CHECK_LAUNCH();
+  if (cudaMemsetAsync(out, 0, sizeof(double), st) != cudaSuccess) return KRONQ_ERR_CUDA;
+  dot_kernel<<<2 * sms, 256, 0, st>>>(T1, T2, (int64_t)m * n, out);
+  KQ_CHECK_LAUNCH();
+  return KRONQ_OK;
+}

@@ -1,0 +1,115 @@
+"""The per-layer KronQ path as a sequence of libkronq calls on one stream.
+
+Order (KronQ review (pith.science), appendix: Algorithm 1 then Algorithm 2;
+KronQ summary (hyper.ai), "Method"):
+  covariances -> BiIP -> sensitivity -> damped inverse Cholesky ->
+  column-wise OBS quantization -> packing.
+
+PyTorch only allocates device memory and provides streams here; every step
+of the computation is a libkronq kernel.
+"""
+
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import torch
+
+from . import abi
+from .alloc import allocate_bits  # noqa: F401  (re-exported host logic)
+
+
+@dataclass
+class LayerResult:
+    codes: torch.Tensor          # m x n uint8
+    scales: torch.Tensor         # m x G fp32
+    zeros: torch.Tensor          # m x G uint8
+    packed: torch.Tensor | None  # m x words int32 (2- and 4-bit)
+    sens: torch.Tensor           # 3 fp64 on device: s, tr(H_X'), tr(H_G')
+    S_X: torch.Tensor
+    S_G: torch.Tensor
+    W_rot: torch.Tensor | None   # W' (kept when asked for)
+    W_hat: torch.Tensor | None
+    H_X: torch.Tensor            # rotated H_X'
+    H_G: torch.Tensor            # rotated H_G'
+    U_c: torch.Tensor
+    info: torch.Tensor           # device int32 status word
+
+
+def covariance(A: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """H = A^T A / N for a token-major bf16 matrix A (N x d) on the device."""
+    N, d = A.shape
+    H = out if out is not None else torch.empty((d, d), dtype=torch.float32, device=A.device)
+    abi.kronq_covariance(A, H, 1.0 / max(N, 1), 0.0, stream=stream)
+    return H
+
+
+def quantize_sublayer(W: torch.Tensor, HX: torch.Tensor, HG: torch.Tensor,
+                      sign_u: torch.Tensor, sign_v: torch.Tensor, bits: int, group: int = -1,
+                      alpha: float = 0.25, mode: str = "full", damp: float = 0.01,
+                      block: int = 128, keep: bool = False, ws: torch.Tensor | None = None,
+                      in_place: bool = False, stream=None) -> LayerResult:
+    """BiIP -> sensitivity -> inverse Cholesky -> OBS -> pack for one sublayer.
+
+    W (m x n fp32), HX (n x n fp32), HG (m x m fp32) are device tensors.  They
+    are cloned unless in_place is set (then W, HX, HG are overwritten)."""
+    m, n = W.shape
+    dev = W.device
+    if not in_place:
+        W, HX, HG = W.clone(), HX.clone(), HG.clone()
+    if ws is None:
+        ws = abi.workspace(m, n, bits, group, block, dev)
+    info = torch.zeros(1, dtype=torch.int32, device=dev)
+    SX = torch.empty(n, dtype=torch.float32, device=dev)
+    SG = torch.empty(m, dtype=torch.float32, device=dev)
+    abi.kronq_biip_rotate(W, HX, HG, sign_u, sign_v, alpha, mode, 0, SX, SG, ws, stream=stream)
+    sens = torch.empty(3, dtype=torch.float64, device=dev)
+    abi.kronq_sensitivity(HX, HG, sens, stream=stream)
+    U = torch.empty((n, n), dtype=torch.float32, device=dev)
+    abi.kronq_cholesky_inv(HX, damp, U, info, ws, stream=stream)
+    W_rot = W.clone() if keep else None
+    G = 1 if group == -1 else n // group
+    codes = torch.empty((m, n), dtype=torch.uint8, device=dev)
+    scales = torch.empty((m, G), dtype=torch.float32, device=dev)
+    zeros = torch.empty((m, G), dtype=torch.uint8, device=dev)
+    W_hat = torch.empty((m, n), dtype=torch.float32, device=dev) if keep else None
+    abi.kronq_quantize_layer(W, U, bits, group, block, codes, scales, zeros, W_hat, info, ws,
+                             stream=stream)
+    packed = None
+    if bits in (2, 4):
+        packed = torch.empty((m, abi.packed_words(n, bits)), dtype=torch.int32, device=dev)
+        abi.kronq_pack(codes, bits, packed, stream=stream)
+    return LayerResult(codes, scales, zeros, packed, sens, SX, SG, W_rot, W_hat, HX, HG, U, info)
+
+
+def covariance_from_host(A_host: torch.Tensor, H: torch.Tensor, chunk_rows: int = 16384,
+                         copy_stream=None, stream=None, staging=None) -> int:
+    """Stream a pinned host bf16 matrix through two device staging buffers:
+    the copy of chunk c+1 overlaps the covariance of chunk c.  Returns the
+    bytes copied host -> device."""
+    N, d = A_host.shape
+    dev = H.device
+    stream = stream or torch.cuda.current_stream(dev)
+    copy_stream = copy_stream or torch.cuda.Stream(dev)
+    if staging is None:
+        staging = [torch.empty((chunk_rows, d), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    done = [torch.cuda.Event(), torch.cuda.Event()]
+    used = [torch.cuda.Event(), torch.cuda.Event()]
+    nchunks = (N + chunk_rows - 1) // chunk_rows
+    if nchunks == 0:
+        abi.kronq_covariance(A_host[:0].to(dev), H, 0.0, 0.0, stream=stream)
+        return 0
+    copied = 0
+    for c in range(nchunks):
+        b = c & 1
+        r0, r1 = c * chunk_rows, min(N, (c + 1) * chunk_rows)
+        with torch.cuda.stream(copy_stream):
+            if c >= 2:
+                copy_stream.wait_event(used[b])
+            staging[b][: r1 - r0].copy_(A_host[r0:r1], non_blocking=True)
+            done[b].record(copy_stream)
+        copied += (r1 - r0) * d * 2
+        stream.wait_event(done[b])
+        abi.kronq_covariance(staging[b][: r1 - r0], H, 1.0 / N, 0.0 if c == 0 else 1.0, stream=stream)
+        used[b].record(stream)
+    return copied

@@ -1,0 +1,108 @@
+"""The C ABI: libkronq.so loads, exports every symbol include/kronq.h
+declares, and rejects bad arguments on the host (no kernel is launched by any
+call here; these run without a GPU)."""
+
+import ctypes
+import re
+
+import pytest
+
+from conftest import ROOT
+
+HEADER = ROOT / "include" / "kronq.h"
+
+
+def _declared():
+    text = re.sub(r"/\*.*?\*/", "", HEADER.read_text(), flags=re.S)
+    return sorted(set(re.findall(r"\b(kronq_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from post_quantization_02_b200 import build, abi
+    build.build()
+    return abi.lib()
+
+
+def test_header_declares_the_path():
+    names = _declared()
+    for required in ("kronq_covariance", "kronq_sensitivity", "kronq_biip_rotate",
+                     "kronq_cholesky_inv", "kronq_quantize_layer", "kronq_pack", "kronq_unpack",
+                     "kronq_layer_loss", "kronq_workspace_size", "kronq_status_string"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    for name in _declared():
+        assert hasattr(L, name), name
+        assert ctypes.cast(getattr(L, name), ctypes.c_void_p).value
+
+
+def test_status_strings_and_version(L):
+    assert L.kronq_status_string(0) == b"ok"
+    assert L.kronq_status_string(-3) == b"matrix not positive definite"
+    assert L.kronq_status_string(12345) == b"unknown status"
+    assert L.kronq_abi_version() == 100
+
+
+def test_workspace_size(L):
+    ws = L.kronq_workspace_size(4096, 4096, 4, -1, 128)
+    # the inverse Cholesky needs two n x n fp32 scratch matrices
+    assert ws >= 2 * 4096 * 4096 * 4
+    assert L.kronq_workspace_size(0, 4096, 4, -1, 128) == 0
+
+
+def test_host_side_argument_errors(L):
+    null = None
+    # pack: 3-bit is not packable; bad widths invalid
+    assert L.kronq_pack(null, 4, 16, 3, null, null) == -2
+    assert L.kronq_pack(null, 4, 16, 5, null, null) == -1
+    assert L.kronq_unpack(null, 4, 16, 3, null, null) == -2
+    # empty inputs are a no-op
+    assert L.kronq_pack(null, 0, 16, 4, null, null) == 0
+    # quantize: group must divide n, block must be 128
+    assert L.kronq_quantize_layer(null, 4, 256, null, 4, -1, 128, null, null, null, null, null,
+                                  null, 0, null) == -1
+    ptr = ctypes.c_void_p(16)  # never dereferenced: rejected before any launch
+    assert L.kronq_quantize_layer(ptr, 4, 256, ptr, 4, 96, 128, ptr, ptr, ptr, null, null,
+                                  null, 0, null) == -1
+    assert L.kronq_quantize_layer(ptr, 4, 256, ptr, 4, -1, 64, ptr, ptr, ptr, null, null,
+                                  null, 0, null) == -2
+    assert L.kronq_quantize_layer(ptr, 4, 256, ptr, 5, -1, 128, ptr, ptr, ptr, null, null,
+                                  null, 0, null) == -1
+    # workspace too small
+    assert L.kronq_quantize_layer(ptr, 4, 256, ptr, 4, -1, 128, ptr, ptr, ptr, null, null,
+                                  null, 0, null) == -6
+    # cholesky: aliasing and workspace
+    assert L.kronq_cholesky_inv(ptr, 64, ctypes.c_float(0.01), ptr, null, null, 0, null) == -1
+    assert L.kronq_cholesky_inv(ptr, 64, ctypes.c_float(0.01), ctypes.c_void_p(32), null, null,
+                                0, null) == -6
+    # biip: widths must be multiples of 16; an odd part above 63 is unsupported
+    assert L.kronq_biip_rotate(ptr, 24, 64, ptr, ptr, ptr, ptr, ctypes.c_float(0.25), 0, 0, ptr,
+                               ptr, null, 0, null) == -1
+    assert L.kronq_biip_rotate(ptr, 16 * 65, 64, ptr, ptr, ptr, ptr, ctypes.c_float(0.25), 0, 0,
+                               ptr, ptr, null, 0, null) == -2
+    assert L.kronq_biip_rotate(ptr, 64, 64, ptr, ptr, ptr, ptr, ctypes.c_float(0.25), 7, 0, ptr,
+                               ptr, null, 0, null) == -1
+    # covariance: misaligned leading dimension, tiny width
+    assert L.kronq_covariance(ptr, 10, 100, 100 + 3, ptr, 100, ctypes.c_float(1.0),
+                              ctypes.c_float(0.0), null, null) == -1
+    assert L.kronq_covariance(ptr, 10, 40, 40, ptr, 40, ctypes.c_float(1.0),
+                              ctypes.c_float(0.0), null, null) == -2
+    assert L.kronq_covariance(null, 10, 0, 0, null, 0, ctypes.c_float(1.0),
+                              ctypes.c_float(0.0), null, null) == 0
+
+
+def test_binding_refuses_host_tensors():
+    import torch
+    from post_quantization_02_b200 import abi
+    with pytest.raises(ValueError):
+        abi.kronq_covariance(torch.zeros(4, 64, dtype=torch.bfloat16),
+                             torch.zeros(64, 64), 1.0)
+
+
+def test_product_never_imports_the_oracle():
+    pkg = ROOT / "post_quantization_02_b200"
+    for f in list(pkg.glob("*.py")) + list((pkg / "csrc").glob("*")):
+        text = f.read_text(errors="ignore")
+        assert "oracle" not in re.findall(r"\b(?:import|from)\s+(\w+)", text), f

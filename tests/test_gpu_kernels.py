@@ -1,0 +1,224 @@
+"""Parity of every libkronq entry point with the fp64 oracle, through the C
+ABI, on seeded inputs sized to span several tiles with ragged tails.
+
+Tolerances (spec bar): covariances <= 1e-4 relative Frobenius
+(bf16 inputs, fp32 accumulation); packing bit-exact; codes >= 99.9 %
+identical with the row loss within 1 %.  Rotation and inverse Cholesky are
+intermediate fp32 stages: their bound (1e-5 and 1e-4 relative Frobenius)
+comes from fp32 rounding over log2(d) butterfly stages and from the
+conditioning of the damped matrix.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from gpu_helpers import bf16_dev, bf16_host, rel_fro, signs, spd, t, widen
+from oracle import biip as obiip
+from oracle import cholesky as ochol
+from oracle import covariance as ocov
+from oracle import pack as opack
+from oracle import quantizer as oq
+from post_quantization_02_b200 import abi
+
+pytestmark = pytest.mark.gpu
+
+
+def _x(r, N, d, kind="t4"):
+    if kind == "t4":
+        z = r.standard_normal((N, d)) / np.sqrt(r.gamma(2.0, size=(N, d)) / 2.0)
+        z[:, r.permutation(d)[: max(1, d // 200)]] *= 20.0
+    else:
+        z = r.standard_normal((N, d)) * np.exp(r.uniform(-3, 0, d))[None, :]
+    return bf16_host(z.astype(np.float32))
+
+
+# -------------------------------------------------------------- covariance
+@pytest.mark.parametrize("N,d,kind", [(2048, 256, "t4"), (1000, 200, "g"), (4097, 520, "t4"),
+                                      (130, 72, "g"), (64, 64, "t4"), (777, 1000, "g"),
+                                      (20000, 384, "t4"), (33, 129, "g")])
+def test_covariance_matches_oracle(cuda, N, d, kind):
+    r = np.random.default_rng(N * 7 + d)
+    bits = _x(r, N, d, kind)
+    H = torch.full((d, d), float("nan"), device=cuda)
+    abi.kronq_covariance(bf16_dev(bits, cuda), H, 1.0 / N, 0.0)
+    Hg = H.cpu().numpy()
+    ref = ocov.covariance(widen(bits))
+    assert rel_fro(Hg, ref) <= 1e-4
+    assert np.array_equal(Hg, Hg.T)
+    np.testing.assert_allclose(np.diag(Hg), np.diag(ref), rtol=1e-4)
+
+
+def test_covariance_padded_rows_beta_and_streaming(cuda):
+    r = np.random.default_rng(5)
+    N, d, pad = 3000, 264, 16
+    bits = _x(r, N, d + pad, "t4")
+    A = bf16_dev(bits, cuda)[:, :d]                 # lda = d + pad
+    ref = ocov.covariance(widen(bits)[:, :d])
+    # streamed over ragged chunks with alpha = 1/N, beta = 0 then 1
+    H = torch.full((d, d), float("nan"), device=cuda)
+    cuts = [0, 1000, 1001, 2500, N]
+    for i in range(len(cuts) - 1):
+        abi.kronq_covariance(A[cuts[i]:cuts[i + 1]], H, 1.0 / N, 0.0 if i == 0 else 1.0)
+    assert rel_fro(H.cpu().numpy(), ref) <= 1e-4
+    # beta != 0 with a symmetric start
+    H0 = spd(r, d)
+    H = t(H0, cuda)
+    abi.kronq_covariance(A, H, 0.5 / N, 0.25)
+    assert rel_fro(H.cpu().numpy(), 0.5 * ref + 0.25 * H0.astype(np.float64)) <= 1e-4
+    # N = 0: H <- beta H
+    H = t(H0, cuda)
+    abi.kronq_covariance(A[:0], H, 1.0, 2.0)
+    np.testing.assert_array_equal(H.cpu().numpy(), 2.0 * H0)
+
+
+# ------------------------------------------------------------- sensitivity
+def test_sensitivity_is_trace_product(cuda):
+    r = np.random.default_rng(1)
+    HX, HG = spd(r, 96), spd(r, 48)
+    out = torch.zeros(3, dtype=torch.float64, device=cuda)
+    abi.kronq_sensitivity(t(HX, cuda), t(HG, cuda), out)
+    s, tx, tg = out.cpu().tolist()
+    np.testing.assert_allclose(tx, np.trace(HX.astype(np.float64)), rtol=1e-12)
+    np.testing.assert_allclose(tg, np.trace(HG.astype(np.float64)), rtol=1e-12)
+    np.testing.assert_allclose(s, tx * tg, rtol=1e-14)
+
+
+# -------------------------------------------------------------------- BiIP
+def _biip_case(r, m, n):
+    W = (r.standard_normal((m, n)) * 0.02 * np.exp(r.uniform(-1, 1, n))[None, :]).astype(np.float32)
+    return W, spd(r, n), spd(r, m), signs(r, m), signs(r, n)
+
+
+@pytest.mark.parametrize("m,n", [(256, 256), (64, 112), (688, 96), (128, 448), (32, 8192),
+                                 (4096, 64), (112, 11008 // 8)])
+@pytest.mark.parametrize("mode", ["full", "no_rescale", "su_only", "sv_only"])
+def test_biip_matches_oracle(cuda, m, n, mode):
+    r = np.random.default_rng(m + 3 * n)
+    W, HX, HG, su, sv = _biip_case(r, m, n)
+    Wd, HXd, HGd = t(W, cuda), t(HX, cuda), t(HG, cuda)
+    SX = torch.empty(n, device=cuda)
+    SG = torch.empty(m, device=cuda)
+    ws = abi.workspace(m, n, device=cuda)
+    abi.kronq_biip_rotate(Wd, HXd, HGd, t(su, cuda), t(sv, cuda), 0.25, mode, 0, SX, SG, ws)
+    Wr, HXr, HGr, SXr, SGr = obiip.biip(W, HX, HG, su, sv, 0.25, mode)
+    np.testing.assert_allclose(SX.cpu().numpy(), SXr, rtol=2e-6)
+    np.testing.assert_allclose(SG.cpu().numpy(), SGr, rtol=2e-6)
+    assert rel_fro(Wd.cpu().numpy(), Wr) <= 1e-5
+    assert rel_fro(HXd.cpu().numpy(), HXr) <= 1e-5
+    assert rel_fro(HGd.cpu().numpy(), HGr) <= 1e-5
+    # exact inverse on W
+    abi.kronq_biip_rotate(Wd, None, None, t(su, cuda), t(sv, cuda), 0.25, mode, 1, SX, SG, ws)
+    assert rel_fro(Wd.cpu().numpy(), W) <= 1e-5
+
+
+# ---------------------------------------------------------- inverse Cholesky
+@pytest.mark.parametrize("n", [64, 72, 200, 256, 1000])
+def test_cholesky_inv_matches_oracle(cuda, n):
+    r = np.random.default_rng(n)
+    H = spd(r, n, spread=1.5)
+    U = torch.full((n, n), float("nan"), device=cuda)
+    info = torch.zeros(1, dtype=torch.int32, device=cuda)
+    ws = abi.workspace(n, n, device=cuda)
+    abi.kronq_cholesky_inv(t(H, cuda), 0.01, U, info, ws)
+    Ug = U.cpu().numpy().astype(np.float64)
+    Uref = ochol.inverse_cholesky(ochol.damp(H, 0.01))
+    assert info.item() == 0
+    assert rel_fro(Ug, Uref) <= 1e-4
+    assert np.all(np.tril(Ug, -1) == 0)
+    Hd = ochol.damp(H, 0.01)
+    assert rel_fro(Ug.T @ Ug @ Hd, np.eye(n)) <= 1e-4
+
+
+def test_cholesky_flags_not_positive_definite(cuda):
+    n = 96
+    H = -np.eye(n, dtype=np.float32)
+    U = torch.empty((n, n), device=cuda)
+    info = torch.zeros(1, dtype=torch.int32, device=cuda)
+    abi.kronq_cholesky_inv(t(H, cuda), 0.0, U, info, abi.workspace(n, n, device=cuda))
+    torch.cuda.synchronize()
+    assert info.item() == -3
+
+
+# --------------------------------------------------------------- quantizer
+@pytest.mark.parametrize("m,n,bits,group", [(256, 256, 4, -1), (100, 384, 2, 128),
+                                            (37, 128, 3, -1), (64, 512, 2, 32), (300, 256, 4, 64),
+                                            (128, 640, 8, -1), (130, 1024, 2, -1)])
+def test_quantize_layer_matches_oracle(cuda, m, n, bits, group):
+    r = np.random.default_rng(m * n + bits)
+    W = (r.standard_normal((m, n)) * 0.02).astype(np.float32)
+    U = ochol.inverse_cholesky(ochol.damp(spd(r, n, spread=1.0), 0.01)).astype(np.float32)
+    G = 1 if group == -1 else n // group
+    codes = torch.empty((m, n), dtype=torch.uint8, device=cuda)
+    scales = torch.empty((m, G), device=cuda)
+    zeros = torch.empty((m, G), dtype=torch.uint8, device=cuda)
+    What = torch.empty((m, n), device=cuda)
+    ws = abi.workspace(m, n, bits, group, device=cuda)
+    abi.kronq_quantize_layer(t(W, cuda), t(U, cuda), bits, group, 128, codes, scales, zeros, What,
+                             None, ws)
+    ref = oq.obs_quantize(W, U, bits, group)
+    cg = codes.cpu().numpy()
+    same = (cg == ref["codes"]).mean()
+    assert same >= 0.999, same
+    if group == -1:
+        np.testing.assert_array_equal(scales.cpu().numpy(), ref["scale"])
+        np.testing.assert_array_equal(zeros.cpu().numpy(), ref["zero"])
+    else:
+        assert (zeros.cpu().numpy() == ref["zero"]).mean() >= 0.999
+    Hd = np.linalg.inv(U.astype(np.float64).T @ U.astype(np.float64))
+    lg = oq.row_losses(W - What.cpu().numpy(), Hd).sum()
+    lr = oq.row_losses(W - ref["W_hat"], Hd).sum()
+    assert abs(lg / lr - 1) <= 0.01
+    # codes lie on the grid of their row / group
+    assert cg.max() <= 2 ** bits - 1
+
+
+# ------------------------------------------------------------------ packing
+@pytest.mark.parametrize("m,n,bits", [(5, 96, 4), (7, 100, 4), (3, 17, 2), (64, 4096, 2), (1, 8, 4)])
+def test_pack_unpack_bit_exact(cuda, m, n, bits):
+    r = np.random.default_rng(m * n)
+    codes = r.integers(0, 2 ** bits, (m, n), dtype=np.uint8)
+    codes[0, : min(n, 2 ** bits)] = np.arange(min(n, 2 ** bits))
+    packed = torch.full((m, abi.packed_words(n, bits)), -1, dtype=torch.int32, device=cuda)
+    abi.kronq_pack(t(codes, cuda), bits, packed)
+    ref = opack.pack(codes, bits)
+    np.testing.assert_array_equal(packed.cpu().numpy().view(np.uint32), ref)
+    back = torch.zeros((m, n), dtype=torch.uint8, device=cuda)
+    abi.kronq_unpack(packed, n, bits, back)
+    np.testing.assert_array_equal(back.cpu().numpy(), codes)
+
+
+def test_pack_three_bit_unsupported(cuda):
+    codes = torch.zeros((2, 32), dtype=torch.uint8, device=cuda)
+    packed = torch.zeros((2, 3), dtype=torch.int32, device=cuda)
+    with pytest.raises(abi.KronqError) as e:
+        abi.kronq_pack(codes, 3, packed)
+    assert e.value.code == -2
+
+
+# ---------------------------------------------------------------- layer loss
+def test_layer_loss_helper(cuda):
+    r = np.random.default_rng(9)
+    m, n = 96, 160
+    Wr = r.standard_normal((m, n)).astype(np.float32)
+    Wh = (Wr + 0.01 * r.standard_normal((m, n))).astype(np.float32)
+    HX, HG = spd(r, n), spd(r, m)
+    out = torch.zeros(1, dtype=torch.float64, device=cuda)
+    abi.kronq_layer_loss(t(Wr, cuda), t(Wh, cuda), t(HX, cuda), t(HG, cuda), out,
+                         abi.workspace(m, n, device=cuda))
+    ref = oq.layer_loss(Wr.astype(np.float64) - Wh, HX, HG)
+    np.testing.assert_allclose(out.item(), ref, rtol=1e-4)
+
+
+# ------------------------------------------------------- failure detection
+def test_bounded_wait_times_out_and_context_survives(cuda):
+    info = torch.zeros(1, dtype=torch.int32, device=cuda)
+    abi.kronq_selftest_wait(info, 20_000_000)      # 20 ms on a barrier nothing arrives on
+    torch.cuda.synchronize()
+    assert info.item() == -5
+    # the context is still usable
+    codes = torch.ones((2, 16), dtype=torch.uint8, device=cuda)
+    packed = torch.zeros((2, 2), dtype=torch.int32, device=cuda)
+    abi.kronq_pack(codes, 2, packed)
+    torch.cuda.synchronize()
+    assert packed[0, 0].item() == 0x55555555
