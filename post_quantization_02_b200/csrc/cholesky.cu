@@ -3,19 +3,29 @@
 // KronQ review (pith.science), appendix, Algorithm 2, steps 1-2:
 // H_X <- H_X + lambda mean(diag H_X) I, then the inverse Cholesky factor.
 //
-// Route (fp32): with J the index reversal, R = J H_d J = L L^T (lower
-// Cholesky), and U_c = J L^-1 J: then U_c^T U_c = J L^-T L^-1 J = (J R J)^-1
-// = H_d^-1 and U_c is upper triangular.  So: reverse-copy and damp, blocked
-// right-looking Cholesky (64-wide panels: one CTA factors and inverts the
-// diagonal block in shared memory, the panel below is multiplied by that
-// inverse, the trailing lower triangle gets a rank-64 update), blocked
-// forward substitution for L^-1 (block row by block row), reverse-copy out.
+// Route (fp32 throughout): with J the index reversal, R = J H_d J = L L^T
+// (lower Cholesky) and U_c = J L^-1 J; then U_c^T U_c = J (L L^T)^-1 J =
+// H_d^-1 and U_c is upper triangular.
+//
+// One right-looking sweep over 128-wide panels computes L and Y = L^-1
+// together (block forward substitution of L Y = I carried along with the
+// factorisation).  Step p (rows k = 128 p ...):
+//   panel kernel   every CTA factors the 128 x 128 diagonal block
+//                  R_pp = L_pp L_pp^T and inverts L_pp in shared memory, then
+//                  either turns 128 rows of the panel into L_ip = R_ip L_pp^-T,
+//                  or finishes 128 columns of block row p of Y:
+//                  Y_pj = L_pp^-1 A_pj  (A_pj = -sum_{q<p} L_pq Y_qj), Y_pp = L_pp^-1.
+//   update kernel  for every block row i > p: the trailing lower triangle
+//                  R_ij -= L_ip L_jp^T and the accumulators A_ij -= L_ip Y_pj
+//                  (j <= p), as 128 x 128 fp32 GEMM tiles with K = 128.
+// Then U_c[a][b] = Y[n-1-a][n-1-b] (a <= b).
 #include "common.cuh"
 #include "gemm_simt.cuh"
 
 namespace {
 
-constexpr int NB = 64;
+constexpr int NB = 128;
+constexpr int LDD = NB + 1;   // padded leading dimension of the diagonal block in smem
 
 __global__ void diag_sum_kernel(const float* __restrict__ H, int n, double* out) {
   __shared__ double red[256];
@@ -30,9 +40,10 @@ __global__ void diag_sum_kernel(const float* __restrict__ H, int n, double* out)
   if (threadIdx.x == 0) *out = red[0];
 }
 
-// R[a][b] = H[n-1-a][n-1-b] + delta [a == b], delta = damp_rel * mean(diag H)
+// R[a][b] = H[n-1-a][n-1-b] + delta [a == b], delta = damp_rel * mean(diag H); Y = 0.
 __global__ void reverse_damp_kernel(const float* __restrict__ H, int n, float* __restrict__ R,
-                                    float damp_rel, const double* __restrict__ diag_sum) {
+                                    float* __restrict__ Y, float damp_rel,
+                                    const double* __restrict__ diag_sum) {
   const float delta = (float)((double)damp_rel * (*diag_sum / (double)n));
   const int64_t total = (int64_t)n * n;
   for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
@@ -41,136 +52,201 @@ __global__ void reverse_damp_kernel(const float* __restrict__ H, int n, float* _
     float v = H[(int64_t)(n - 1 - a) * n + (n - 1 - b)];
     if (a == b) v += delta;
     R[e] = v;
+    Y[e] = 0.f;
   }
 }
 
-// Factor the diagonal block R[k:k+nb, k:k+nb] = L L^T in place (lower part,
-// upper part zeroed) and write L^-1 to Linv (nb x nb, leading dim NB).
-__global__ void __launch_bounds__(256) potrf_diag_kernel(float* __restrict__ R, int n, int k,
-                                                         float* __restrict__ Linv, int32_t* info) {
-  __shared__ float A[NB][NB + 1];
-  __shared__ float X[NB][NB + 1];
-  __shared__ int bad;
-  const int nb = min(NB, n - k);
+// Lower Cholesky of the kb x kb block in D (in place, fp32), then X = L^-1.
+// Rows/columns kb .. NB-1 are padded with the identity.
+//
+// Register-tiled: thread (ty, tx) = (tid / 16, tid % 16) keeps the 8 x 8 tile
+// D[8ty .. 8ty+7][8tx .. 8tx+7] in registers.  Column step j: every thread
+// reads the raw pivot column (published in shared memory) and applies
+// D[i][c] -= D[i][j] D[c][j] / D[j][j] to its whole tile.  Entries that are
+// already final (columns <= j) or never used (above the diagonal) absorb
+// harmless updates: each column is copied to D in shared memory when it is
+// published (right after its last update), and only those copies are used
+// afterwards.  Warps whose 16 rows all lie above the pivot skip the update.
+// One barrier per step.  The inverse runs the same way by rows: row p of X
+// is final once divided by L[p][p] and is published into X; rows below
+// subtract L[i][p] times it.
+__device__ void factor_and_invert(float* D, float* X, int kb, int* bad) {
+  __shared__ float colbuf[2][NB];
+  __shared__ float dall[NB];
   const int tid = threadIdx.x;
-  if (tid == 0) bad = 0;
-  for (int e = tid; e < NB * NB; e += blockDim.x) {
-    const int i = e / NB, j = e % NB;
-    A[i][j] = (i < nb && j <= i) ? R[(int64_t)(k + i) * n + (k + j)] : 0.f;
-  }
+  const int ty = tid >> 4, tx = tid & 15;
+  const int warp_last_row = 16 * (tid >> 5) + 15;
+  float a[8][8];
+#pragma unroll
+  for (int r = 0; r < 8; ++r)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) a[r][c] = D[(8 * ty + r) * LDD + 8 * tx + c];
+  if (tid < NB) colbuf[0][tid] = D[tid * LDD];   // column 0 (raw)
   __syncthreads();
-  for (int j = 0; j < nb; ++j) {
-    if (tid == 0) {
-      const float d = A[j][j];
+  for (int jb = 0; jb < NB / 8; ++jb) {
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) {
+      const int j = 8 * jb + jj;
+      const int b = jj & 1;               // j & 1 (8 * jb is even)
+      float d = colbuf[b][j];
       if (!(d > 0.f) || !isfinite(d)) {
-        bad = 1;
-        A[j][j] = 1.f;  // keep going with a placeholder; the result is flagged
-      } else {
-        A[j][j] = sqrtf(d);
+        if (tid == 0 && j < kb) *bad = 1;
+        d = 1.f;
       }
+      if (tid == 0) dall[j] = d;
+      if (warp_last_row > j) {
+        const float rd = __frcp_rn(d);
+        float ci[8], cc[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) ci[r] = colbuf[b][8 * ty + r];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) cc[c] = colbuf[b][8 * tx + c] * rd;
+#pragma unroll
+        for (int r = 0; r < 8; ++r)
+#pragma unroll
+          for (int c = 0; c < 8; ++c) a[r][c] = fmaf(-ci[r], cc[c], a[r][c]);
+      }
+      // publish column j + 1: its values received their last update just now
+      const int jn = j + 1;
+      if (jn < NB && tx == (jn >> 3)) {
+        const int cl = (jj + 1) & 7;  // compile-time after unrolling
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          const int i = 8 * ty + r;
+          const float v = (i >= jn) ? a[r][cl] : 0.f;
+          colbuf[b ^ 1][i] = v;
+          D[i * LDD + jn] = v;
+        }
+      }
+      __syncthreads();
     }
-    __syncthreads();
-    const float piv = A[j][j];
-    for (int i = j + 1 + tid; i < nb; i += blockDim.x) A[i][j] = A[i][j] / piv;
-    __syncthreads();
-    const int rem = nb - j - 1;
-    for (int e = tid; e < rem * rem; e += blockDim.x) {
-      const int i = j + 1 + e / rem, c = j + 1 + e % rem;
-      if (c <= i) A[i][c] = fmaf(-A[i][j], A[c][j], A[i][c]);
-    }
-    __syncthreads();
   }
-  // X = L^-1, one column per thread by forward substitution
-  if (tid < NB) {
-    const int c = tid;
-    for (int i = 0; i < NB; ++i) {
-      float v = 0.f;
-      if (i < nb && c < nb && i >= c) {
-        v = (i == c) ? 1.f : 0.f;
-        for (int p = c; p < i; ++p) v = fmaf(-A[i][p], X[p][c], v);
-        v = v / A[i][i];
+  // L[i][c] = raw[i][c] / sqrt(d_c) (i > c), L[c][c] = sqrt(d_c), upper part 0
+  for (int e = tid; e < NB * NB; e += blockDim.x) {
+    const int i = e >> 7, c = e & (NB - 1);
+    float v = 0.f;
+    if (c == i) v = sqrtf(dall[c]);
+    else if (c < i) v = D[i * LDD + c] * rsqrtf(dall[c]);
+    D[i * LDD + c] = v;
+  }
+  __syncthreads();
+  // X = L^-1 (x: accumulators of the rows of X, same tiling)
+  float x[8][8];
+#pragma unroll
+  for (int r = 0; r < 8; ++r)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) x[r][c] = (8 * ty + r == 8 * tx + c) ? 1.f : 0.f;
+  for (int pb = 0; pb < NB / 8; ++pb) {
+#pragma unroll
+    for (int pp = 0; pp < 8; ++pp) {
+      const int p = 8 * pb + pp;
+      const int b = pp & 1;
+      if (ty == pb) {
+        // finalise and publish row p (entries right of the diagonal are 0)
+        const float rl = __frcp_rn(D[p * LDD + p]);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const int col = 8 * tx + c;
+          const float v = (col <= p) ? x[pp][c] * rl : 0.f;
+          colbuf[b][col] = v;
+          X[p * LDD + col] = v;
+        }
       }
-      X[i][c] = v;
+      __syncthreads();
+      if (warp_last_row > p) {
+        float li[8], xr[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) li[r] = D[(8 * ty + r) * LDD + p];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) xr[c] = colbuf[b][8 * tx + c];
+#pragma unroll
+        for (int r = 0; r < 8; ++r)
+#pragma unroll
+          for (int c = 0; c < 8; ++c) x[r][c] = fmaf(-li[r], xr[c], x[r][c]);
+      }
     }
   }
   __syncthreads();
-  for (int e = tid; e < NB * NB; e += blockDim.x) {
+}
+
+__global__ void __launch_bounds__(256) panel_kernel(float* R, float* Y, int n, int k, int p,
+                                                    int tiles_L, int32_t* info) {
+  extern __shared__ float sm[];
+  float* D = sm;                       // [NB][LDD]
+  float* X = sm + NB * LDD;            // [NB][LDD]
+  kq::Gemm128Smem& gs = *reinterpret_cast<kq::Gemm128Smem*>(sm + 2 * NB * LDD);
+  __shared__ int bad;
+  const int kb = min(NB, n - k);
+  if (threadIdx.x == 0) bad = 0;
+  for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
     const int i = e / NB, j = e % NB;
-    if (i < nb && j < nb) {
-      R[(int64_t)(k + i) * n + (k + j)] = (j <= i) ? A[i][j] : 0.f;
-      Linv[i * NB + j] = X[i][j];
+    float v = 0.f;
+    if (i < kb && j <= i) v = R[(int64_t)(k + i) * n + (k + j)];
+    else if (i == j) v = 1.f;
+    D[i * LDD + j] = v;
+  }
+  __syncthreads();
+  factor_and_invert(D, X, kb, &bad);
+  if (blockIdx.x == 0 && threadIdx.x == 0 && bad) kq::record_error(info, KRONQ_ERR_NOT_PD);
+
+  if ((int)blockIdx.x < tiles_L) {
+    // 128 rows of the panel: L_ip = R_ip L_pp^-T (in place)
+    const int r0 = k + kb + NB * blockIdx.x;
+    float* P = R + (int64_t)r0 * n + k;
+    kq::gemm128<true>(gs, P, n, X, LDD, P, n, n - r0 < NB ? n - r0 : NB, kb, kb, 1.f, 0.f);
+  } else {
+    const int j = blockIdx.x - tiles_L;  // column block of Y's block row p
+    if (j < p) {
+      float* B = Y + (int64_t)k * n + NB * j;
+      kq::gemm128<false>(gs, X, LDD, B, n, B, n, kb, NB, kb, 1.f, 0.f);
+    } else {
+      for (int e = threadIdx.x; e < kb * kb; e += blockDim.x) {
+        const int a = e / kb, b = e % kb;
+        Y[(int64_t)(k + a) * n + k + b] = X[a * LDD + b];
+      }
     }
   }
-  if (tid == 0 && bad) kq::record_error(info, KRONQ_ERR_NOT_PD);
 }
 
-// Panel below the diagonal block: P <- P L_kk^-T (in place, one 64-column tile).
-__global__ void __launch_bounds__(256) trsm_panel_kernel(float* R, int n, int k,
-                                                         const float* __restrict__ Linv) {
-  const int nb = min(NB, n - k);
-  const int r0 = k + nb;
-  float* P = R + (int64_t)r0 * n + k;
-  kq::gemm_tile64<false, true>(P, n, Linv, NB, P, n, n - r0, nb, nb, 1.f, 0.f, blockIdx.x, 0);
-}
-
-// Trailing lower triangle: T <- T - P P^T.
-__global__ void __launch_bounds__(256) syrk_lower_kernel(float* R, int n, int k) {
-  const int tm = blockIdx.y, tn = blockIdx.x;
-  if (tn > tm) return;
-  const int nb = min(NB, n - k);
-  const int r0 = k + nb;
-  const float* P = R + (int64_t)r0 * n + k;
-  float* T = R + (int64_t)r0 * n + r0;
-  kq::gemm_tile64<false, true>(P, n, P, n, T, n, n - r0, n - r0, nb, -1.f, 1.f, tm, tn);
-}
-
-// Block row i of X = L^-1, step 1: S_j = L[i, j:i] X[j:i, j] for every block j < i.
-__global__ void __launch_bounds__(256) trtri_gemm_kernel(const float* __restrict__ L,
-                                                         const float* __restrict__ X, int n, int i,
-                                                         float* __restrict__ S) {
-  const int j = blockIdx.x;
-  const int r0 = i * NB, c0 = j * NB;
-  const int rows = min(NB, n - r0);
-  const int K = r0 - c0;
-  kq::gemm_tile64<false, false>(L + (int64_t)r0 * n + c0, n, X + (int64_t)c0 * n + c0, n,
-                                S + c0, n, rows, NB, K, 1.f, 0.f, 0, 0);
-}
-
-// Step 2: X[i, j] = -L_ii^-1 S_j for j < i (one GEMM over all of them), X_ii = L_ii^-1.
-__global__ void __launch_bounds__(256) trtri_scale_kernel(float* __restrict__ X, int n, int i,
-                                                          const float* __restrict__ S,
-                                                          const float* __restrict__ Linv_ii) {
-  const int r0 = i * NB;
-  const int rows = min(NB, n - r0);
-  if ((int)blockIdx.x == i) {
-    for (int e = threadIdx.x; e < rows * rows; e += blockDim.x) {
-      const int a = e / rows, b = e % rows;
-      X[(int64_t)(r0 + a) * n + r0 + b] = Linv_ii[a * NB + b];
-    }
-    return;
+// Trailing updates after panel p.  blockIdx.y: block row below the panel;
+// blockIdx.x < p+1: Y accumulator column block; else: trailing R column block.
+__global__ void __launch_bounds__(256) update_kernel(float* R, float* Y, int n, int k, int p) {
+  __shared__ kq::Gemm128Smem gs;
+  const int kb = min(NB, n - k);
+  const int ti = blockIdx.y, tj = blockIdx.x;
+  const int r0 = k + kb + NB * ti;
+  const int M = min(NB, n - r0);
+  const float* L = R + (int64_t)r0 * n + k;
+  if (tj <= p) {
+    float* C = Y + (int64_t)r0 * n + NB * tj;
+    kq::gemm128<false>(gs, L, n, Y + (int64_t)k * n + NB * tj, n, C, n, M, NB, kb, -1.f, 1.f);
+  } else {
+    const int sj = tj - (p + 1);
+    if (sj > ti) return;
+    const int c0 = k + kb + NB * sj;
+    float* C = R + (int64_t)r0 * n + c0;
+    kq::gemm128<true>(gs, L, n, R + (int64_t)c0 * n + k, n, C, n, M, min(NB, n - c0), kb, -1.f, 1.f);
   }
-  kq::gemm_tile64<false, false>(Linv_ii, NB, S, n, X + (int64_t)r0 * n, n, rows, r0, rows, -1.f,
-                                0.f, 0, blockIdx.x);
 }
 
-// U[a][b] = X[n-1-a][n-1-b] for a <= b, 0 below the diagonal.
-__global__ void reverse_out_kernel(const float* __restrict__ X, int n, float* __restrict__ U) {
+// U[a][b] = Y[n-1-a][n-1-b] for a <= b, 0 below the diagonal.
+__global__ void reverse_out_kernel(const float* __restrict__ Y, int n, float* __restrict__ U) {
   const int64_t total = (int64_t)n * n;
   for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
        e += (int64_t)gridDim.x * blockDim.x) {
     const int a = (int)(e / n), b = (int)(e % n);
-    U[e] = (a <= b) ? X[(int64_t)(n - 1 - a) * n + (n - 1 - b)] : 0.f;
+    U[e] = (a <= b) ? Y[(int64_t)(n - 1 - a) * n + (n - 1 - b)] : 0.f;
   }
 }
 
 size_t align256(size_t b) { return (b + 255) & ~(size_t)255; }
 
+constexpr size_t kPanelSmem = (size_t)2 * NB * LDD * sizeof(float) + sizeof(kq::Gemm128Smem);
+
 }  // namespace
 
 size_t kq_cholesky_ws(int64_t n) {
-  const int64_t nblk = (n + NB - 1) / NB;
-  return align256(sizeof(double)) + 2 * align256((size_t)n * n * sizeof(float)) +
-         align256((size_t)nblk * NB * NB * sizeof(float)) + align256((size_t)NB * n * sizeof(float));
+  return align256(sizeof(double)) + 2 * align256((size_t)n * n * sizeof(float));
 }
 
 int kq_cholesky_inv(const float* H, int64_t n64, float damp_rel, float* U, int32_t* info, void* ws,
@@ -180,46 +256,40 @@ int kq_cholesky_inv(const float* H, int64_t n64, float damp_rel, float* U, int32
   if (!H || !U || H == U) return KRONQ_ERR_INVALID_ARG;
   if (n64 > 65536) return KRONQ_ERR_UNSUPPORTED;
   if (!ws || ws_bytes < kq_cholesky_ws(n64) || !kqh::aligned(ws, 256)) return KRONQ_ERR_WORKSPACE;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(panel_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kPanelSmem) != cudaSuccess)
+      return KRONQ_ERR_CUDA;
+    attr = true;
+  }
   const int n = (int)n64;
   uint8_t* w = static_cast<uint8_t*>(ws);
   double* dsum = reinterpret_cast<double*>(w);
   w += align256(sizeof(double));
   float* R = reinterpret_cast<float*>(w);
   w += align256((size_t)n * n * sizeof(float));
-  float* X = reinterpret_cast<float*>(w);
-  w += align256((size_t)n * n * sizeof(float));
-  float* Ld = reinterpret_cast<float*>(w);
-  w += align256((size_t)((n + NB - 1) / NB) * NB * NB * sizeof(float));
-  float* S = reinterpret_cast<float*>(w);
+  float* Y = reinterpret_cast<float*>(w);
 
   const int sms = kqh::num_sms();
   diag_sum_kernel<<<1, 256, 0, st>>>(H, n, dsum);
   KQ_CHECK_LAUNCH();
-  reverse_damp_kernel<<<4 * sms, 256, 0, st>>>(H, n, R, damp_rel, dsum);
+  reverse_damp_kernel<<<4 * sms, 256, 0, st>>>(H, n, R, Y, damp_rel, dsum);
   KQ_CHECK_LAUNCH();
   const int nblk = (n + NB - 1) / NB;
-  for (int b = 0; b < nblk; ++b) {
-    const int k = b * NB;
-    potrf_diag_kernel<<<1, 256, 0, st>>>(R, n, k, Ld + (size_t)b * NB * NB, info);
+  for (int p = 0; p < nblk; ++p) {
+    const int k = p * NB;
+    const int kb = n - k < NB ? n - k : NB;
+    const int rest = n - k - kb;
+    const int tiles_L = (rest + NB - 1) / NB;
+    panel_kernel<<<tiles_L + p + 1, 256, kPanelSmem, st>>>(R, Y, n, k, p, tiles_L, info);
     KQ_CHECK_LAUNCH();
-    const int rest = n - k - NB;
     if (rest > 0) {
-      const int tiles = (rest + kq::GT - 1) / kq::GT;
-      trsm_panel_kernel<<<tiles, 256, 0, st>>>(R, n, k, Ld + (size_t)b * NB * NB);
-      KQ_CHECK_LAUNCH();
-      syrk_lower_kernel<<<dim3(tiles, tiles), 256, 0, st>>>(R, n, k);
+      update_kernel<<<dim3(p + 1 + tiles_L, tiles_L), 256, 0, st>>>(R, Y, n, k, p);
       KQ_CHECK_LAUNCH();
     }
   }
-  for (int i = 0; i < nblk; ++i) {
-    if (i > 0) {
-      trtri_gemm_kernel<<<i, 256, 0, st>>>(R, X, n, i, S);
-      KQ_CHECK_LAUNCH();
-    }
-    trtri_scale_kernel<<<i + 1, 256, 0, st>>>(X, n, i, S, Ld + (size_t)i * NB * NB);
-    KQ_CHECK_LAUNCH();
-  }
-  reverse_out_kernel<<<4 * sms, 256, 0, st>>>(X, n, U);
+  reverse_out_kernel<<<4 * sms, 256, 0, st>>>(Y, n, U);
   KQ_CHECK_LAUNCH();
   return KRONQ_OK;
 }

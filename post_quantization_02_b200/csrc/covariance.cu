@@ -13,10 +13,11 @@
 //   warp 1      one thread issues tcgen05.mma (M=128, N=256, K=16, bf16 in,
 //               fp32 accumulate in TMEM) and commits each stage back to the
 //               producer, and each finished tile to the epilogue.
-//   warp 2      allocates / frees the 512 TMEM columns (two accumulators, so
-//               the epilogue of tile t overlaps the MMAs of tile t+1).
-//   warps 4-7   epilogue: tcgen05.ld 32 lanes x 32 columns at a time,
-//               H = alpha acc + beta H for the elements on or above the
+//   warp 2      allocates / frees the 512 TMEM columns: the accumulator
+//               (256) and an fp32 master (256) that the epilogue folds each
+//               4096-token partial sum into.
+//   warps 4-7   epilogue: folds (tcgen05.ld / add / tcgen05.st), then per tile
+//               H = alpha master + beta H for the elements on or above the
 //               diagonal, stored twice: in place (row-contiguous vector
 //               stores) and mirrored (for a fixed column the 32 lanes of a
 //               warp write 32 consecutive floats of the transposed row).
@@ -32,11 +33,15 @@
 namespace {
 
 constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+// K-slabs per accumulation chunk: the tensor core's fp32 accumulation rounds
+// towards zero (measured: ~ -6e-8 relative per K=16 step), so partial sums
+// over 4096 tokens are folded into H with round-to-nearest fp32 adds.
+constexpr int KC_ITERS = 64;
 constexpr int BOX_BYTES = 64 * BK * 2;              // 64 features x 64 tokens of bf16
 constexpr int A_BYTES = BM * BK * 2;                // 16 KB
 constexpr int B_BYTES = BN * BK * 2;                // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;      // 48 KB
-constexpr int TMEM_COLS = 2 * BN;
+constexpr int TMEM_COLS = 2 * BN;  // accumulator + master
 constexpr int THREADS = 256;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
 constexpr uint32_t IDESC = kq::idesc_f16(BM, BN, /*bf16*/ 1, /*A MN-major*/ 1, /*B MN-major*/ 1);
@@ -44,8 +49,8 @@ constexpr uint32_t IDESC = kq::idesc_f16(BM, BN, /*bf16*/ 1, /*A MN-major*/ 1, /
 struct Bars {
   uint64_t full[STAGES];
   uint64_t empty[STAGES];
-  uint64_t tfull[2];
-  uint64_t tempty[2];
+  uint64_t tfull;
+  uint64_t tempty;
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -92,10 +97,8 @@ cov_tc_kernel(const __grid_constant__ CUtensorMap tmap, float* __restrict__ H, i
       kq::mbar_init(&bars->full[s], 1);
       kq::mbar_init(&bars->empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      kq::mbar_init(&bars->tfull[b], 1);
-      kq::mbar_init(&bars->tempty[b], 4);
-    }
+    kq::mbar_init(&bars->tfull, 1);
+    kq::mbar_init(&bars->tempty, 4);
     kq::mbar_init(&bars->drain, 1);
     bars->abort = 0;
     kq::fence_barrier_init();
@@ -141,32 +144,34 @@ cov_tc_kernel(const __grid_constant__ CUtensorMap tmap, float* __restrict__ H, i
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------ MMA issuer
-      int it = 0, tl = 0;
+      // One accumulator (TMEM columns [0, BN)); it is handed to the epilogue
+      // after every chunk of KC_ITERS K-slabs and reused once folded.
+      int it = 0, cc = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++tl) {
-        const int buf = tl & 1;
-        const uint32_t aph = (uint32_t)(tl >> 1) & 1u;
-        if (!kq::mbar_wait(&bars->tempty[buf], aph ^ 1u, abort, info)) break;
-        kq::tc_fence_after();
-        const uint32_t d_tmem = tmem + (uint32_t)(buf * BN);
-        for (int kb = 0; kb < k_iters; ++kb, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-          if (!kq::mbar_wait(&bars->full[s], ph, abort, info)) { ok = false; break; }
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        for (int k0 = 0; k0 < k_iters && ok; k0 += KC_ITERS, ++cc) {
+          const int k1 = min(k_iters, k0 + KC_ITERS);
+          if (!kq::mbar_wait(&bars->tempty, ((uint32_t)cc & 1u) ^ 1u, abort, info)) { ok = false; break; }
           kq::tc_fence_after();
-          const uint32_t a_addr = kq::smem_u32(tiles + s * STAGE_BYTES);
-          const uint32_t b_addr = a_addr + A_BYTES;
+          for (int kb = k0; kb < k1; ++kb, ++it) {
+            const int s = it % STAGES;
+            const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+            if (!kq::mbar_wait(&bars->full[s], ph, abort, info)) { ok = false; break; }
+            kq::tc_fence_after();
+            const uint32_t a_addr = kq::smem_u32(tiles + s * STAGE_BYTES);
+            const uint32_t b_addr = a_addr + A_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            // MN-major, 128B swizzle: 8-row K atoms 1024 B apart (SBO), 64-wide
-            // feature atoms one TMA box apart (LBO); K step of 16 rows = 2048 B.
-            const uint64_t ad = kq::smem_desc(a_addr + kk * 2048, BOX_BYTES, 1024, kq::kLayoutSwizzle128B);
-            const uint64_t bd = kq::smem_desc(b_addr + kk * 2048, BOX_BYTES, 1024, kq::kLayoutSwizzle128B);
-            kq::mma_f16(d_tmem, ad, bd, IDESC, (kb | kk) != 0);
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              // MN-major, 128B swizzle: 8-row K atoms 1024 B apart (SBO), 64-wide
+              // feature atoms one TMA box apart (LBO); K step of 16 rows = 2048 B.
+              const uint64_t ad = kq::smem_desc(a_addr + kk * 2048, BOX_BYTES, 1024, kq::kLayoutSwizzle128B);
+              const uint64_t bd = kq::smem_desc(b_addr + kk * 2048, BOX_BYTES, 1024, kq::kLayoutSwizzle128B);
+              kq::mma_f16(tmem, ad, bd, IDESC, (kb != k0) || (kk != 0));
+            }
+            kq::mma_commit(&bars->empty[s]);
           }
-          kq::mma_commit(&bars->empty[s]);
+          if (ok) kq::mma_commit(&bars->tfull);
         }
-        if (ok) kq::mma_commit(&bars->tfull[buf]);
       }
       // wind down: all MMAs issued by this thread complete before TMEM is freed
       kq::mma_commit(&bars->drain);
@@ -174,55 +179,88 @@ cov_tc_kernel(const __grid_constant__ CUtensorMap tmap, float* __restrict__ H, i
     }
   } else if (warp >= 4) {
     // -------------------------------------------------- epilogue
+    // Each chunk's partial sum is folded into the fp32 master (TMEM columns
+    // [BN, 2 BN)) with ordinary round-to-nearest adds, so the tensor core's
+    // own accumulation only ever spans KC_ITERS * BK tokens.  The accumulator
+    // is released as soon as the fold is done; after the last chunk of a tile
+    // the master is written out (H = alpha master + beta H_old) together with
+    // its mirror image.
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
-    int tl = 0;
-    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++tl) {
-      const int buf = tl & 1;
-      const uint32_t aph = (uint32_t)(tl >> 1) & 1u;
-      if (!kq::mbar_wait(&bars->tfull[buf], aph, abort, info)) break;
-      kq::tc_fence_after();
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    int cc = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
       int rb, cb;
       tile_coords(t, ncb, rb, cb);
       const int i0 = rb * BM, j0 = cb * BN;
       const int row0 = i0 + q * 32;             // first row of this warp's 32 lanes
       const int row = row0 + lane;
+      for (int k0 = 0; k0 < k_iters; k0 += KC_ITERS, ++cc) {
+        const bool first = k0 == 0, last = k0 + KC_ITERS >= k_iters;
+        if (!kq::mbar_wait(&bars->tfull, (uint32_t)cc & 1u, abort, info)) { ok = false; break; }
+        kq::tc_fence_after();
 #pragma unroll 1
-      for (int c = 0; c < BN; c += 32) {
-        const int jc = j0 + c;
-        if (jc >= d) break;                       // columns past the matrix (uniform)
-        if (jc + 31 < row0) continue;             // strictly below the diagonal: another tile's mirror
-        float v[32];
-        kq::tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN + c), v);
-        kq::tmem_wait_ld();
-        if (row < d) {
-          float* dst = H + (int64_t)row * ldh + jc;
-          if (beta != 0.f) {
+        for (int c = 0; c < BN; c += 32) {
+          if (j0 + c >= d) break;                   // columns past the matrix (uniform)
+          if (j0 + c + 31 < row0) continue;         // strictly below the diagonal: never stored
+          float v[32], mst[32];
+          __syncwarp();
+          kq::tmem_ld32(tmem + lane_off + (uint32_t)c, v);
+          if (!first) kq::tmem_ld32(tmem + lane_off + (uint32_t)(BN + c), mst);
+          kq::tmem_wait_ld();
+          if (!first) {
+#pragma unroll
+            for (int k = 0; k < 32; ++k) v[k] += mst[k];
+          }
+          kq::tmem_st32(tmem + lane_off + (uint32_t)(BN + c), v);
+        }
+        kq::tmem_wait_st();
+        kq::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) kq::mbar_arrive(&bars->tempty);   // accumulator free again
+        if (!last) continue;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          const int jc = j0 + c;
+          if (jc >= d) break;
+          if (jc + 31 < row0) continue;
+          float v[32];
+          __syncwarp();
+          kq::tmem_ld32(tmem + lane_off + (uint32_t)(BN + c), v);
+          kq::tmem_wait_ld();
+          if (row < d) {
+            float* dst = H + (int64_t)row * ldh + jc;
+            if (jc >= row0 + 31 && jc + 32 <= d) {
+              // whole chunk on or above the diagonal for every lane: vector stores
+#pragma unroll
+              for (int k = 0; k < 32; k += 4) {
+                float4 o = make_float4(alpha * v[k], alpha * v[k + 1], alpha * v[k + 2], alpha * v[k + 3]);
+                if (beta != 0.f) {
+                  const float4 h = *reinterpret_cast<const float4*>(dst + k);
+                  o.x = fmaf(beta, h.x, o.x); o.y = fmaf(beta, h.y, o.y);
+                  o.z = fmaf(beta, h.z, o.z); o.w = fmaf(beta, h.w, o.w);
+                }
+                v[k] = o.x; v[k + 1] = o.y; v[k + 2] = o.z; v[k + 3] = o.w;
+                *reinterpret_cast<float4*>(dst + k) = o;
+              }
+            } else {
+#pragma unroll
+              for (int k = 0; k < 32; ++k) {
+                if (jc + k < d && jc + k >= row) {
+                  float o = alpha * v[k];
+                  if (beta != 0.f) o = fmaf(beta, dst[k], o);
+                  v[k] = o;
+                  dst[k] = o;
+                }
+              }
+            }
+            // mirror: H[j][row] for j > row; for each j the warp writes 32 consecutive floats
 #pragma unroll
             for (int k = 0; k < 32; ++k)
-              if (jc + k < d && jc + k >= row) v[k] = alpha * v[k] + beta * dst[k];
-          } else {
-#pragma unroll
-            for (int k = 0; k < 32; ++k) v[k] *= alpha;
+              if (jc + k < d && jc + k > row) H[(int64_t)(jc + k) * ldh + row] = v[k];
           }
-          if (jc >= row0 + 31 && jc + 32 <= d) {
-            // whole chunk on or above the diagonal for every lane: vector stores
-#pragma unroll
-            for (int k = 0; k < 32; k += 4)
-              *reinterpret_cast<float4*>(dst + k) = make_float4(v[k], v[k + 1], v[k + 2], v[k + 3]);
-          } else {
-#pragma unroll
-            for (int k = 0; k < 32; ++k)
-              if (jc + k < d && jc + k >= row) dst[k] = v[k];
-          }
-          // mirror: H[j][row] for j > row; for each j the warp writes 32 consecutive floats
-#pragma unroll
-          for (int k = 0; k < 32; ++k)
-            if (jc + k < d && jc + k > row) H[(int64_t)(jc + k) * ldh + row] = v[k];
         }
       }
-      kq::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) kq::mbar_arrive(&bars->tempty[buf]);
     }
   }
 

@@ -31,6 +31,19 @@ struct Grid {
   float zero;
 };
 
+// round(x / scale) with x / scale rounded to fp32 first (round half to even),
+// i.e. exactly rintf(__fdiv_rn(x, scale)).  Fast path: qa = x * RN(1/scale)
+// is within |q| * 1.8e-7 of the correctly rounded quotient q (two roundings
+// of 2^-24 each, plus q's own), i.e. within 4.6e-5 for |q| < 256; so both
+// round to the same integer unless qa lies within 1e-4 of a half-integer.
+// Only then (or for |qa| >= 256) is the division carried out.
+__device__ __forceinline__ float round_quotient(float x, float scale, float rscale) {
+  const float qa = x * rscale;
+  const float fr = qa - floorf(qa);
+  if (fabsf(fr - 0.5f) > 1e-4f && fabsf(qa) < 256.f) return rintf(qa);
+  return rintf(__fdiv_rn(x, scale));
+}
+
 // Asymmetric grid of [lo, hi] in fp32: lo = min(0, min w), hi = max(0, max w).
 __device__ __forceinline__ Grid make_grid(float mn, float mx, float maxq) {
   const float lo = fminf(mn, 0.f), hi = fmaxf(mx, 0.f);
@@ -105,6 +118,7 @@ obs_block_kernel(const float* __restrict__ W, int m, int n, const float* __restr
     scale = scales[row];
     zero = (float)zeros[row];
   }
+  float rscale = __frcp_rn(scale);
   __syncthreads();
 
   float qv[16], ev[16], hv[16];
@@ -129,6 +143,7 @@ obs_block_kernel(const float* __restrict__ W, int m, int n, const float* __restr
       const Grid g = make_grid(mn, mx, maxq);
       scale = g.scale;
       zero = g.zero;
+      rscale = __frcp_rn(scale);
       if (live && chunk == c) {
         const int gi = (i1 + j) / (GROUP > 0 ? GROUP : 1);
         scales[(int64_t)row * G + gi] = scale;
@@ -137,7 +152,7 @@ obs_block_kernel(const float* __restrict__ W, int m, int n, const float* __restr
     }
     // quantize this thread's copy of column j (meaningful on the owner only)
     const float x = w[jj];
-    const float q = fminf(fmaxf(rintf(__fdiv_rn(x, scale)) + zero, 0.f), maxq);
+    const float q = fminf(fmaxf(round_quotient(x, scale, rscale) + zero, 0.f), maxq);
     const float wh = scale * (q - zero);
     float e = (x - wh) * rdiag[j];
     e = __shfl_sync(0xffffffffu, e, (lane & ~7) | c);
@@ -179,13 +194,16 @@ obs_block_kernel(const float* __restrict__ W, int m, int n, const float* __restr
   }
 }
 
-// W[:, i2:] -= E U[i1:i2, i2:]
+// W[:, i2:] -= E U[i1:i2, i2:]  (128 x 128 output tiles, K = 128)
 __global__ void __launch_bounds__(256) lazy_update_kernel(float* W, int m, int n,
                                                           const float* __restrict__ E,
                                                           const float* __restrict__ U, int i1) {
+  __shared__ kq::Gemm128Smem gs;
   const int i2 = i1 + QB;
-  kq::gemm_tile64<false, false>(E, QB, U + (int64_t)i1 * n + i2, n, W + i2, n, m, n - i2, QB, -1.f,
-                                1.f, blockIdx.y, blockIdx.x);
+  const int r0 = blockIdx.y * kq::G2, c0 = i2 + blockIdx.x * kq::G2;
+  kq::gemm128<false>(gs, E + (int64_t)r0 * QB, QB, U + (int64_t)i1 * n + c0, n,
+                     W + (int64_t)r0 * n + c0, n, min(kq::G2, m - r0), min(kq::G2, n - c0), QB,
+                     -1.f, 1.f);
 }
 
 template <bool TA, bool TB>
@@ -311,7 +329,7 @@ int kq_quantize_layer(float* W, int64_t m64, int64_t n64, const float* U, int bi
     if (s != KRONQ_OK) return s;
     const int i2 = i1 + QB;
     if (i2 < n) {
-      const dim3 grid((n - i2 + kq::GT - 1) / kq::GT, (m + kq::GT - 1) / kq::GT);
+      const dim3 grid((n - i2 + kq::G2 - 1) / kq::G2, (m + kq::G2 - 1) / kq::G2);
       lazy_update_kernel<<<grid, 256, 0, st>>>(W, m, n, E, U, i1);
       KQ_CHECK_LAUNCH();
     }

@@ -49,6 +49,7 @@ def test_workspace_size(L):
     ws = L.kronq_workspace_size(4096, 4096, 4, -1, 128)
     # the inverse Cholesky needs two n x n fp32 scratch matrices
     assert ws >= 2 * 4096 * 4096 * 4
+    assert L.kronq_launch_count() >= 0
     assert L.kronq_workspace_size(0, 4096, 4, -1, 128) == 0
 
 

@@ -36,14 +36,17 @@ def _x(r, N, d, kind="t4"):
 # -------------------------------------------------------------- covariance
 @pytest.mark.parametrize("N,d,kind", [(2048, 256, "t4"), (1000, 200, "g"), (4097, 520, "t4"),
                                       (130, 72, "g"), (64, 64, "t4"), (777, 1000, "g"),
-                                      (20000, 384, "t4"), (33, 129, "g")])
+                                      (20000, 384, "t4"), (33, 129, "g"), (70000, 256, "t4"),
+                                      (8193, 136, "g")])
 def test_covariance_matches_oracle(cuda, N, d, kind):
     r = np.random.default_rng(N * 7 + d)
-    bits = _x(r, N, d, kind)
-    H = torch.full((d, d), float("nan"), device=cuda)
-    abi.kronq_covariance(bf16_dev(bits, cuda), H, 1.0 / N, 0.0)
+    lda = (d + 7) // 8 * 8                       # the ABI wants lda % 8 == 0
+    bits = _x(r, N, lda, kind)
+    ldh = (d + 3) // 4 * 4                       # and ldh % 4 == 0
+    H = torch.full((d, ldh), float("nan"), device=cuda)[:, :d]
+    abi.kronq_covariance(bf16_dev(bits, cuda)[:, :d], H, 1.0 / N, 0.0)
     Hg = H.cpu().numpy()
-    ref = ocov.covariance(widen(bits))
+    ref = ocov.covariance(widen(bits)[:, :d])
     assert rel_fro(Hg, ref) <= 1e-4
     assert np.array_equal(Hg, Hg.T)
     np.testing.assert_allclose(np.diag(Hg), np.diag(ref), rtol=1e-4)
@@ -222,3 +225,24 @@ def test_bounded_wait_times_out_and_context_survives(cuda):
     abi.kronq_pack(codes, 2, packed)
     torch.cuda.synchronize()
     assert packed[0, 0].item() == 0x55555555
+
+
+def test_quantize_exact_ties_round_half_to_even(cuda):
+    """Weights exactly on half-steps: the code decision (round half to even of
+    the fp32 quotient) must match the oracle's bit for bit."""
+    m, n = 4, 128
+    W = np.zeros((m, n), dtype=np.float32)
+    W[:, 0] = 0.0
+    W[:, 1] = 15.0                                   # grid: lo 0, hi 15 -> scale 1, zero 0
+    W[:, 2:32] = np.arange(30, dtype=np.float32)[None, :] * 0.5   # 0, 0.5, 1, ..., 14.5
+    W[1] *= 0.25                                      # scale 0.25: exact multiples again
+    W[2] *= -1.0                                      # lo -15: zero 15
+    U = np.eye(n, dtype=np.float32)                   # no propagation: OBS == rounding
+    codes = torch.empty((m, n), dtype=torch.uint8, device=cuda)
+    scales = torch.empty((m, 1), device=cuda)
+    zeros = torch.empty((m, 1), dtype=torch.uint8, device=cuda)
+    abi.kronq_quantize_layer(t(W, cuda), t(U, cuda), 4, -1, 128, codes, scales, zeros, None, None,
+                             abi.workspace(m, n, 4, -1, device=cuda))
+    ref = oq.obs_quantize(W, U, 4, -1)
+    np.testing.assert_array_equal(codes.cpu().numpy(), ref["codes"])
+    assert list(ref["codes"][0, 2:8]) == [0, 0, 1, 2, 2, 2]
