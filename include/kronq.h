@@ -180,6 +180,29 @@ int kronq_quantize_layer(float* W, int64_t m, int64_t n, const float* U_c,
                          int32_t* info, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * kronq_quantize_layer without a workspace: for callers that cannot allocate
+ * device memory while they run (a host framework that owns the allocator,
+ * memory planned once at start-up, or a loop where cudaMalloc/cudaFree would
+ * synchronise the device).  The KronQ pages have no counterpart; this is a
+ * deployment variant of the same solver.
+ *
+ * Same arguments, meaning and results as kronq_quantize_layer, minus
+ * (ws, ws_bytes).  The solver's m x 128 fp32 error block lives in a static
+ * 16 MiB device array inside the library (every GPU that loads the library
+ * holds it until the process exits), so m may be at most 32768
+ * (KRONQ_ERR_UNSUPPORTED above that).  The library looks up the array's device
+ * address once per device, during the first call made on that device; make
+ * that first call before any stream capture.  All calls share the array:
+ * calls whose work can overlap on the GPU (different streams without
+ * ordering, several host threads) race on it and must be serialised by the
+ * caller.  Nothing in it needs to start zeroed.  Allocates nothing.
+ */
+int kronq_quantize_layer_noalloc(float* W, int64_t m, int64_t n, const float* U_c,
+                                 int bits, int group, int block,
+                                 uint8_t* codes, float* scales, uint8_t* zeros, float* W_hat,
+                                 int32_t* info, void* stream);
+
+/*
  * Pack b-bit codes into 32-bit words (b = 2 or 4).
  *
  * KronQ README (GitHub), "Model zoo": W4 / W2 stored as packed int4 / int2;

@@ -51,6 +51,7 @@ def lib() -> ctypes.CDLL:
         "kronq_biip_rotate": ([P, I64, I64, P, P, P, P, F32, I32, I32, P, P, P, SZ, P], I32),
         "kronq_cholesky_inv": ([P, I64, F32, P, P, P, SZ, P], I32),
         "kronq_quantize_layer": ([P, I64, I64, P, I32, I32, I32, P, P, P, P, P, P, SZ, P], I32),
+        "kronq_quantize_layer_noalloc": ([P, I64, I64, P, I32, I32, I32, P, P, P, P, P, P], I32),
         "kronq_pack": ([P, I64, I64, I32, P, P], I32),
         "kronq_unpack": ([P, I64, I64, I32, P, P], I32),
         "kronq_layer_loss": ([P, P, I64, I64, P, P, P, P, SZ, P], I32),
@@ -182,6 +183,25 @@ def kronq_quantize_layer(W, U, bits: int, group: int, block: int, codes, scales,
     _check("kronq_quantize_layer", lib().kronq_quantize_layer(
         _p(W), m, n, _p(U), bits, group, block, _p(codes), _p(scales), _p(zeros), _p(W_hat),
         _p(info), _p(ws), 0 if ws is None else ws.numel() * ws.element_size(), _s(stream)))
+
+
+def kronq_quantize_layer_noalloc(W, U, bits: int, group: int, block: int, codes, scales, zeros,
+                                 W_hat=None, info=None, stream=None):
+    """kronq_quantize_layer with its scratch in the library's static device
+    array (no workspace, nothing allocated; at most 32768 rows)."""
+    _dev(W, torch.float32, "W", 2)
+    _dev(U, torch.float32, "U_c", 2)
+    _dev(codes, torch.uint8, "codes", 2)
+    _dev(scales, torch.float32, "scales")
+    _dev(zeros, torch.uint8, "zeros")
+    _dev(W_hat, torch.float32, "W_hat", 2)
+    for t, nm in ((W, "W"), (U, "U_c"), (codes, "codes"), (scales, "scales"), (zeros, "zeros"),
+                  (W_hat, "W_hat")):
+        _contig(t, nm)
+    m, n = W.shape
+    _check("kronq_quantize_layer_noalloc", lib().kronq_quantize_layer_noalloc(
+        _p(W), m, n, _p(U), bits, group, block, _p(codes), _p(scales), _p(zeros), _p(W_hat),
+        _p(info), _s(stream)))
 
 
 def kronq_pack(codes, bits: int, packed, stream=None):

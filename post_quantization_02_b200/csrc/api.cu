@@ -21,6 +21,9 @@ int kq_cholesky_inv(const float* H, int64_t n, float damp_rel, float* U, int32_t
 int kq_quantize_layer(float* W, int64_t m, int64_t n, const float* U, int bits, int group,
                       int block, uint8_t* codes, float* scales, uint8_t* zeros, float* W_hat,
                       int32_t* info, void* ws, size_t ws_bytes, cudaStream_t st);
+int kq_quantize_layer_noalloc(float* W, int64_t m, int64_t n, const float* U, int bits, int group,
+                              int block, uint8_t* codes, float* scales, uint8_t* zeros,
+                              float* W_hat, int32_t* info, cudaStream_t st);
 int kq_pack(const uint8_t* codes, int64_t m, int64_t n, int bits, uint32_t* packed,
             cudaStream_t st);
 int kq_unpack(const uint32_t* packed, int64_t m, int64_t n, int bits, uint8_t* codes,
@@ -137,6 +140,13 @@ int kronq_quantize_layer(float* W, int64_t m, int64_t n, const float* U_c, int b
                          int32_t* info, void* ws, size_t ws_bytes, void* stream) {
   return kq_quantize_layer(W, m, n, U_c, bits, group, block, codes, scales, zeros, W_hat, info, ws,
                            ws_bytes, S(stream));
+}
+
+int kronq_quantize_layer_noalloc(float* W, int64_t m, int64_t n, const float* U_c, int bits,
+                                 int group, int block, uint8_t* codes, float* scales,
+                                 uint8_t* zeros, float* W_hat, int32_t* info, void* stream) {
+  return kq_quantize_layer_noalloc(W, m, n, U_c, bits, group, block, codes, scales, zeros, W_hat,
+                                   info, S(stream));
 }
 
 int kronq_pack(const uint8_t* codes, int64_t m, int64_t n, int bits, uint32_t* packed,

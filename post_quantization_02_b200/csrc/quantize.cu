@@ -17,6 +17,8 @@
 //                     w_k -= e U_c[j,k] to its columns k > j.  No block-wide
 //                     synchronisation inside the column loop.
 //   lazy_update       W[:, i+128:] -= E U_c[i:i+128, i+128:]
+#include <mutex>
+
 #include "common.cuh"
 #include "gemm_simt.cuh"
 
@@ -385,4 +387,56 @@ int kq_layer_loss(const float* Wr, const float* Wh, int64_t m64, int64_t n64, co
   dot_kernel<<<2 * sms, 256, 0, st>>>(T1, T2, (int64_t)m * n, out);
   KQ_CHECK_LAUNCH();
   return KRONQ_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of kronq_quantize_layer.
+//
+// Some callers cannot allocate device memory while they run: a host framework
+// that owns the device allocator and forbids plugins from calling cudaMalloc,
+// a process that plans all of its memory at start-up and must not grow it
+// later, or a latency-sensitive loop in which cudaMalloc / cudaFree would
+// synchronise the device and stall other streams.  For them the solver's
+// only scratch buffer (the m x 128 fp32 error block) lives in the static
+// device array below instead of a caller workspace.
+//
+// The array is part of the library image: every GPU that loads libkronq holds
+// its 16 MiB until the process exits.  Host code cannot use the symbol as a
+// device address, so its address is looked up with cudaGetSymbolAddress once
+// per device (with that device current), on the first call made on that
+// device.  All calls share the one array and it keeps the previous call's
+// contents: nothing in it has to start at zero (every element the lazy
+// update reads was written by the block solve of the same call), but two
+// calls whose work overlaps on the GPU race on it.
+constexpr int64_t kNoAllocMaxRows = 32768;
+static __device__ __align__(256) float g_noalloc_error_block[kNoAllocMaxRows * QB];
+
+namespace {
+
+std::mutex g_noalloc_mutex;
+float* g_noalloc_ptr[64] = {};
+
+// Device address of g_noalloc_error_block on the current device (nullptr on failure).
+float* noalloc_scratch() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_error_block) != cudaSuccess || !p) return nullptr;
+    g_noalloc_ptr[dev] = static_cast<float*>(p);
+  }
+  return g_noalloc_ptr[dev];
+}
+
+}  // namespace
+
+int kq_quantize_layer_noalloc(float* W, int64_t m, int64_t n, const float* U, int bits, int group,
+                              int block, uint8_t* codes, float* scales, uint8_t* zeros,
+                              float* W_hat, int32_t* info, cudaStream_t st) {
+  if (m > kNoAllocMaxRows) return KRONQ_ERR_UNSUPPORTED;   // the static scratch holds 32768 rows
+  float* E = noalloc_scratch();
+  if (!E) return KRONQ_ERR_CUDA;
+  return kq_quantize_layer(W, m, n, U, bits, group, block, codes, scales, zeros, W_hat, info, E,
+                           sizeof(g_noalloc_error_block), st);
 }

@@ -1,0 +1,64 @@
+"""The allocation-free solver entry point, kronq_quantize_layer_noalloc.
+
+It serves callers that cannot allocate device memory while they run (a host
+framework that owns the allocator, memory planned once at start-up, or a loop
+in which cudaMalloc would synchronise the device): its scratch is a static
+array inside the library instead of a caller workspace.  Here it is called
+through the C ABI and compared with the workspace entry point on the same
+inputs, on two calls in a row, so the second call runs with the first call's
+data still in the shared array.  This file is collected last on purpose.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from gpu_helpers import spd, t
+from oracle import cholesky as ochol
+from post_quantization_02_b200 import abi
+
+pytestmark = pytest.mark.gpu
+
+
+def _outputs(cuda, m, n, bits, group):
+    G = 1 if group == -1 else n // group
+    return (torch.empty((m, n), dtype=torch.uint8, device=cuda),
+            torch.empty((m, G), device=cuda),
+            torch.empty((m, G), dtype=torch.uint8, device=cuda),
+            torch.empty((m, n), device=cuda))
+
+
+@pytest.mark.parametrize("case", [0])
+def test_noalloc_matches_workspace_entry_point_twice(cuda, case):
+    for call, (m, n, bits, group) in enumerate([(300, 512, 4, -1), (520, 384, 2, 128)]):
+        r = np.random.default_rng(100 + call)
+        W = (r.standard_normal((m, n)) * 0.02).astype(np.float32)
+        U = ochol.inverse_cholesky(ochol.damp(spd(r, n, spread=1.0), 0.01)).astype(np.float32)
+        Ud = t(U, cuda)
+
+        ref = _outputs(cuda, m, n, bits, group)
+        abi.kronq_quantize_layer(t(W, cuda), Ud, bits, group, 128, *ref, None,
+                                 abi.workspace(m, n, bits, group, device=cuda))
+        got = _outputs(cuda, m, n, bits, group)
+        info = torch.zeros(1, dtype=torch.int32, device=cuda)
+        abi.kronq_quantize_layer_noalloc(t(W, cuda), Ud, bits, group, 128, *got, info)
+        torch.cuda.synchronize()
+
+        assert info.item() == 0
+        rc, gc = ref[0].cpu().numpy(), got[0].cpu().numpy()
+        assert (rc == gc).mean() >= 0.999              # the codes bar the parity tests use
+        np.testing.assert_allclose(got[1].cpu().numpy(), ref[1].cpu().numpy(), rtol=1e-6)
+        assert (got[2].cpu().numpy() == ref[2].cpu().numpy()).mean() >= 0.999
+        same = rc == gc
+        np.testing.assert_allclose(got[3].cpu().numpy()[same], ref[3].cpu().numpy()[same],
+                                   rtol=1e-5, atol=1e-7)
+
+
+def test_noalloc_rejects_more_rows_than_its_scratch(cuda):
+    m, n = 32769, 128
+    W = torch.zeros((m, n), device=cuda)
+    U = torch.eye(n, device=cuda)
+    outs = _outputs(cuda, m, n, 4, -1)
+    with pytest.raises(abi.KronqError) as e:
+        abi.kronq_quantize_layer_noalloc(W, U, 4, -1, 128, *outs)
+    assert e.value.code == -2
