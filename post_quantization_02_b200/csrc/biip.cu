@@ -21,7 +21,7 @@
 namespace {
 
 constexpr int RT_THREADS = 256;
-constexpr int CP_COLS = 8;  // columns per panel in the column pass
+constexpr int CP_COLS = 8;  // columns per panel in the column pass (shifts below assume 8)
 
 struct Split {
   int L2, Q, q, k1;
@@ -115,14 +115,15 @@ __global__ void scale_only_kernel(float* __restrict__ X, int R, int C, const flo
   }
 }
 
-// In-shared-memory Walsh-Hadamard butterflies on Q segments of L2 entries.
-__device__ void fwht_segments(float* x, int L2, int Q) {
-  const int half = L2 >> 1;
+// In-shared-memory Walsh-Hadamard butterflies on Q segments of L2 = 2^lg2
+// entries (pair p of stage h = 2^lh: i = (p >> lh) << (lh+1) | (p & (h-1))).
+__device__ void fwht_segments(float* x, int lg2, int Q) {
+  const int half = 1 << (lg2 - 1);
   const int pairs = half * Q;
-  for (int h = 1; h < L2; h <<= 1) {
+  for (int lh = 0; lh < lg2; ++lh) {
+    const int h = 1 << lh;
     for (int p = threadIdx.x; p < pairs; p += blockDim.x) {
-      const int s = p / half, qq = p - s * half;
-      const int i = s * L2 + (qq / h) * 2 * h + (qq % h);
+      const int i = ((p >> lh) << (lh + 1)) | (p & (h - 1));
       const float a = x[i], b = x[i + h];
       x[i] = a + b;
       x[i + h] = a - b;
@@ -163,7 +164,7 @@ row_transform_kernel(float* __restrict__ X, int R, int C, const float* __restric
   }
   __syncthreads();
   if (inverse && Q > 1) mix_segments(x, L2, Q, M, true);
-  fwht_segments(x, L2, Q);
+  fwht_segments(x, 31 - __clz(L2), Q);
   if (!inverse && Q > 1) mix_segments(x, L2, Q, M, false);
   for (int c = threadIdx.x; c < C; c += blockDim.x) {
     float v = x[c] * norm;
@@ -183,7 +184,7 @@ col_fht_kernel(float* __restrict__ X, int R, int C, const int8_t* __restrict__ s
   const int r0 = seg * L2;
   const float norm = rsqrtf((float)L2);
   for (int e = threadIdx.x; e < L2 * CP_COLS; e += blockDim.x) {
-    const int rr = e / CP_COLS, cc = e % CP_COLS;
+    const int rr = e >> 3, cc = e & (CP_COLS - 1);
     float v = 0.f;
     if (c0 + cc < C) v = X[(int64_t)(r0 + rr) * C + c0 + cc];
     if (!inverse) v *= (float)sign[r0 + rr];
@@ -191,10 +192,11 @@ col_fht_kernel(float* __restrict__ X, int R, int C, const int8_t* __restrict__ s
   }
   __syncthreads();
   const int half = L2 >> 1;
-  for (int h = 1; h < L2; h <<= 1) {
+  for (int lh = 0; (1 << lh) < L2; ++lh) {
+    const int h = 1 << lh;
     for (int e = threadIdx.x; e < half * CP_COLS; e += blockDim.x) {
-      const int pr = e / CP_COLS, cc = e % CP_COLS;
-      const int i = (pr / h) * 2 * h + (pr % h);
+      const int pr = e >> 3, cc = e & (CP_COLS - 1);   // CP_COLS == 8
+      const int i = ((pr >> lh) << (lh + 1)) | (pr & (h - 1));
       const float a = p[i * CP_COLS + cc], b = p[(i + h) * CP_COLS + cc];
       p[i * CP_COLS + cc] = a + b;
       p[(i + h) * CP_COLS + cc] = a - b;
@@ -202,7 +204,7 @@ col_fht_kernel(float* __restrict__ X, int R, int C, const int8_t* __restrict__ s
     __syncthreads();
   }
   for (int e = threadIdx.x; e < L2 * CP_COLS; e += blockDim.x) {
-    const int rr = e / CP_COLS, cc = e % CP_COLS;
+    const int rr = e >> 3, cc = e & (CP_COLS - 1);
     if (c0 + cc >= C) continue;
     float v = p[e] * norm;
     if (inverse) v *= (float)sign[r0 + rr];

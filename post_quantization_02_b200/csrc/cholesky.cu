@@ -56,120 +56,113 @@ __global__ void reverse_damp_kernel(const float* __restrict__ H, int n, float* _
   }
 }
 
-// Lower Cholesky of the kb x kb block in D (in place, fp32), then X = L^-1.
-// Rows/columns kb .. NB-1 are padded with the identity.
+// X = L^-1 for the lower Cholesky factor L of the 128 x 128 block in D
+// (fp32; rows/columns kb .. NB-1 are padded with the identity by the caller;
+// D is overwritten with scratch).
 //
-// Register-tiled: thread (ty, tx) = (tid / 16, tid % 16) keeps the 8 x 8 tile
-// D[8ty .. 8ty+7][8tx .. 8tx+7] in registers.  Column step j: every thread
-// reads the raw pivot column (published in shared memory) and applies
-// D[i][c] -= D[i][j] D[c][j] / D[j][j] to its whole tile.  Entries that are
-// already final (columns <= j) or never used (above the diagonal) absorb
-// harmless updates: each column is copied to D in shared memory when it is
-// published (right after its last update), and only those copies are used
-// afterwards.  Warps whose 16 rows all lie above the pivot skip the update.
-// One barrier per step.  The inverse runs the same way by rows: row p of X
-// is final once divided by L[p][p] and is published into X; rows below
-// subtract L[i][p] times it.
+// One sweep of 128 column steps does the factorisation and the inverse
+// together: at step j the pivot column of the Schur complement and the
+// accumulated row j of L^-1 are both final, so with r = 1/sqrt(d_j):
+//   L[i][j] = S[i][j] r,   Y[j][:] = A[j][:] r,
+//   S[i][c] -= L[i][j] L[c][j]      (the trailing Schur complement)
+//   A[i][:] -= L[i][j] Y[j][:]      (i > j, the rows of L^-1 still open).
+// Thread (ty, tx) keeps the 8 x 8 tiles of S and A at rows 8ty.., columns
+// 8tx.. in registers; warp w owns the column tiles tx = 2w, 2w+1 (ty = lane
+// mod 16), so at step j a warp's choice is uniform: tiles with columns > j
+// need the S update, tiles with columns <= j the A update (only the tile
+// holding column j needs both).  Entries that are already final or never
+// used absorb harmless updates.  After its last update, column j+1 of S and
+// row j+1 of A are published to shared memory; one barrier per step.
 __device__ void factor_and_invert(float* D, float* X, int kb, int* bad) {
-  __shared__ float colbuf[2][NB];
-  __shared__ float dall[NB];
+  __shared__ __align__(16) float colbuf[2][NB];
+  __shared__ __align__(16) float rowbuf[2][NB];
   const int tid = threadIdx.x;
-  const int ty = tid >> 4, tx = tid & 15;
-  const int warp_last_row = 16 * (tid >> 5) + 15;
-  float a[8][8];
+  const int ty = tid & 15, tx = ((tid >> 5) << 1) | ((tid >> 4) & 1);
+  float a[8][8], y[8][8];
 #pragma unroll
   for (int r = 0; r < 8; ++r)
 #pragma unroll
-    for (int c = 0; c < 8; ++c) a[r][c] = D[(8 * ty + r) * LDD + 8 * tx + c];
-  if (tid < NB) colbuf[0][tid] = D[tid * LDD];   // column 0 (raw)
+    for (int c = 0; c < 8; ++c) {
+      a[r][c] = D[(8 * ty + r) * LDD + 8 * tx + c];
+      y[r][c] = (8 * ty + r == 8 * tx + c) ? 1.f : 0.f;
+    }
+  if (tid < NB) {
+    colbuf[0][tid] = D[tid * LDD];          // column 0 of S
+    rowbuf[0][tid] = (tid == 0) ? 1.f : 0.f;  // row 0 of A (identity)
+  }
   __syncthreads();
   for (int jb = 0; jb < NB / 8; ++jb) {
 #pragma unroll
     for (int jj = 0; jj < 8; ++jj) {
       const int j = 8 * jb + jj;
-      const int b = jj & 1;               // j & 1 (8 * jb is even)
+      const int b = jj & 1;                 // j & 1 (8 * jb is even)
       float d = colbuf[b][j];
       if (!(d > 0.f) || !isfinite(d)) {
         if (tid == 0 && j < kb) *bad = 1;
         d = 1.f;
       }
-      if (tid == 0) dall[j] = d;
-      if (warp_last_row > j) {
-        const float rd = __frcp_rn(d);
-        float ci[8], cc[8];
-#pragma unroll
-        for (int r = 0; r < 8; ++r) ci[r] = colbuf[b][8 * ty + r];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) cc[c] = colbuf[b][8 * tx + c] * rd;
-#pragma unroll
-        for (int r = 0; r < 8; ++r)
-#pragma unroll
-          for (int c = 0; c < 8; ++c) a[r][c] = fmaf(-ci[r], cc[c], a[r][c]);
-      }
-      // publish column j + 1: its values received their last update just now
-      const int jn = j + 1;
-      if (jn < NB && tx == (jn >> 3)) {
-        const int cl = (jj + 1) & 7;  // compile-time after unrolling
-#pragma unroll
-        for (int r = 0; r < 8; ++r) {
-          const int i = 8 * ty + r;
-          const float v = (i >= jn) ? a[r][cl] : 0.f;
-          colbuf[b ^ 1][i] = v;
-          D[i * LDD + jn] = v;
+      const float rs = rsqrtf(d);
+      if (tid < NB) X[j * LDD + tid] = rowbuf[b][tid] * rs;   // row j of L^-1, final
+      const bool do_s = 8 * tx + 7 > j, do_a = 8 * tx <= j;
+      {
+        float li[8], lc[8], yj[8];
+        {
+          const float4 p0 = *reinterpret_cast<const float4*>(&colbuf[b][8 * ty]);
+          const float4 p1 = *reinterpret_cast<const float4*>(&colbuf[b][8 * ty + 4]);
+          const float4 q0 = *reinterpret_cast<const float4*>(&colbuf[b][8 * tx]);
+          const float4 q1 = *reinterpret_cast<const float4*>(&colbuf[b][8 * tx + 4]);
+          const float4 y0 = *reinterpret_cast<const float4*>(&rowbuf[b][8 * tx]);
+          const float4 y1 = *reinterpret_cast<const float4*>(&rowbuf[b][8 * tx + 4]);
+          li[0] = p0.x; li[1] = p0.y; li[2] = p0.z; li[3] = p0.w;
+          li[4] = p1.x; li[5] = p1.y; li[6] = p1.z; li[7] = p1.w;
+          lc[0] = q0.x; lc[1] = q0.y; lc[2] = q0.z; lc[3] = q0.w;
+          lc[4] = q1.x; lc[5] = q1.y; lc[6] = q1.z; lc[7] = q1.w;
+          yj[0] = y0.x; yj[1] = y0.y; yj[2] = y0.z; yj[3] = y0.w;
+          yj[4] = y1.x; yj[5] = y1.y; yj[6] = y1.z; yj[7] = y1.w;
         }
-      }
-      __syncthreads();
-    }
-  }
-  // L[i][c] = raw[i][c] / sqrt(d_c) (i > c), L[c][c] = sqrt(d_c), upper part 0
-  for (int e = tid; e < NB * NB; e += blockDim.x) {
-    const int i = e >> 7, c = e & (NB - 1);
-    float v = 0.f;
-    if (c == i) v = sqrtf(dall[c]);
-    else if (c < i) v = D[i * LDD + c] * rsqrtf(dall[c]);
-    D[i * LDD + c] = v;
-  }
-  __syncthreads();
-  // X = L^-1 (x: accumulators of the rows of X, same tiling)
-  float x[8][8];
+        // published values are raw: scale L[.][j] by r, and Y[j][.] by r
 #pragma unroll
-  for (int r = 0; r < 8; ++r)
-#pragma unroll
-    for (int c = 0; c < 8; ++c) x[r][c] = (8 * ty + r == 8 * tx + c) ? 1.f : 0.f;
-  for (int pb = 0; pb < NB / 8; ++pb) {
-#pragma unroll
-    for (int pp = 0; pp < 8; ++pp) {
-      const int p = 8 * pb + pp;
-      const int b = pp & 1;
-      if (ty == pb) {
-        // finalise and publish row p (entries right of the diagonal are 0)
-        const float rl = __frcp_rn(D[p * LDD + p]);
+        for (int r = 0; r < 8; ++r) li[r] *= rs;
+        const float rs2 = rs * rs;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-          const int col = 8 * tx + c;
-          const float v = (col <= p) ? x[pp][c] * rl : 0.f;
-          colbuf[b][col] = v;
-          X[p * LDD + col] = v;
+          lc[c] *= rs;
+          yj[c] *= rs;
+        }
+        (void)rs2;
+        if (do_s) {
+#pragma unroll
+          for (int r = 0; r < 8; ++r)
+#pragma unroll
+            for (int c = 0; c < 8; ++c) a[r][c] = fmaf(-li[r], lc[c], a[r][c]);
+        }
+        if (do_a) {
+#pragma unroll
+          for (int r = 0; r < 8; ++r)
+#pragma unroll
+            for (int c = 0; c < 8; ++c) y[r][c] = fmaf(-li[r], yj[c], y[r][c]);
+        }
+      }
+      // publish column j+1 of S and row j+1 of A (their last update was just now)
+      const int jn = j + 1;
+      if (jn < NB) {
+        if (tx == (jn >> 3)) {
+          const int cl = (jj + 1) & 7;        // compile-time after unrolling
+#pragma unroll
+          for (int r = 0; r < 8; ++r) colbuf[b ^ 1][8 * ty + r] = (8 * ty + r >= jn) ? a[r][cl] : 0.f;
+        }
+        if (ty == (jn >> 3)) {
+          const int rl = (jj + 1) & 7;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) rowbuf[b ^ 1][8 * tx + c] = (8 * tx + c <= jn) ? y[rl][c] : 0.f;
         }
       }
       __syncthreads();
-      if (warp_last_row > p) {
-        float li[8], xr[8];
-#pragma unroll
-        for (int r = 0; r < 8; ++r) li[r] = D[(8 * ty + r) * LDD + p];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) xr[c] = colbuf[b][8 * tx + c];
-#pragma unroll
-        for (int r = 0; r < 8; ++r)
-#pragma unroll
-          for (int c = 0; c < 8; ++c) x[r][c] = fmaf(-li[r], xr[c], x[r][c]);
-      }
     }
   }
-  __syncthreads();
 }
 
-__global__ void __launch_bounds__(256) panel_kernel(float* R, float* Y, int n, int k, int p,
+__global__ void __launch_bounds__(256, 1) panel_kernel(float* R, float* Y, int n, int k, int p,
                                                     int tiles_L, int32_t* info) {
   extern __shared__ float sm[];
   float* D = sm;                       // [NB][LDD]

@@ -89,11 +89,15 @@ __global__ void __launch_bounds__(256)
 obs_block_kernel(const float* __restrict__ W, int m, int n, const float* __restrict__ U, int i1,
                  int bits, uint8_t* __restrict__ codes, float* __restrict__ scales,
                  uint8_t* __restrict__ zeros, float* __restrict__ W_hat, float* __restrict__ E) {
+  // Thread `chunk` (0..7) of a row owns the 16 columns 32 s + 4 chunk + t
+  // (s, t in 0..3), held in w[4 s + t]: for a fixed s the 8 threads of a row
+  // read 8 consecutive float4 of a U row, so the shared-memory reads are
+  // free of bank conflicts.  Column j = 32 s + 4 c + t belongs to thread c.
   extern __shared__ float smem[];
   float* Us = smem;                    // [QB][US_LD]
   float* rdiag = smem + QB * US_LD;    // [QB]
   const int tid = threadIdx.x, lane = tid & 31;
-  const int chunk = tid & 7;           // which 16 columns of the block
+  const int chunk = tid & 7;
   const int row = blockIdx.x * ROWS_PER_CTA + (tid >> 3);
   const bool live = row < m;
   const float maxq = (float)((1 << bits) - 1);
@@ -108,11 +112,11 @@ obs_block_kernel(const float* __restrict__ W, int m, int n, const float* __restr
 
   float w[16];
   {
-    const float* src = W + (int64_t)(live ? row : 0) * n + i1 + chunk * 16;
+    const float* src = W + (int64_t)(live ? row : 0) * n + i1 + 4 * chunk;
 #pragma unroll
-    for (int k = 0; k < 16; k += 4) {
-      float4 v = live ? *reinterpret_cast<const float4*>(src + k) : make_float4(0.f, 0.f, 0.f, 0.f);
-      w[k] = v.x; w[k + 1] = v.y; w[k + 2] = v.z; w[k + 3] = v.w;
+    for (int sg = 0; sg < 4; ++sg) {
+      const float4 v = live ? *reinterpret_cast<const float4*>(src + 32 * sg) : make_float4(0.f, 0.f, 0.f, 0.f);
+      w[4 * sg] = v.x; w[4 * sg + 1] = v.y; w[4 * sg + 2] = v.z; w[4 * sg + 3] = v.w;
     }
   }
   float scale = 1.f, zero = 0.f;
@@ -125,74 +129,74 @@ obs_block_kernel(const float* __restrict__ W, int m, int n, const float* __restr
 
   float qv[16], ev[16], hv[16];
 #pragma unroll
-  for (int j = 0; j < QB; ++j) {
-    const int c = j >> 4, jj = j & 15;
-    if (GROUP > 0 && (j % (GROUP > 0 ? GROUP : 1)) == 0) {
-      // grid of columns j .. j+GROUP-1 from the current (updated) weights
-      const int c_lo = j >> 4, c_hi = (j + GROUP) >> 4;  // chunks [c_lo, c_hi)
-      const bool in = chunk >= c_lo && chunk < c_hi;
-      float mn = INFINITY, mx = -INFINITY;
-#pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        mn = fminf(mn, in ? w[k] : INFINITY);
-        mx = fmaxf(mx, in ? w[k] : -INFINITY);
-      }
-#pragma unroll
-      for (int o = 1; o < 8; o <<= 1) {
-        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      }
-      const Grid g = make_grid(mn, mx, maxq);
-      scale = g.scale;
-      zero = g.zero;
-      rscale = __frcp_rn(scale);
-      if (live && chunk == c) {
-        const int gi = (i1 + j) / (GROUP > 0 ? GROUP : 1);
-        scales[(int64_t)row * G + gi] = scale;
-        zeros[(int64_t)row * G + gi] = (uint8_t)zero;
-      }
-    }
-    // quantize this thread's copy of column j (meaningful on the owner only)
-    const float x = w[jj];
-    const float q = fminf(fmaxf(round_quotient(x, scale, rscale) + zero, 0.f), maxq);
-    const float wh = scale * (q - zero);
-    float e = (x - wh) * rdiag[j];
-    e = __shfl_sync(0xffffffffu, e, (lane & ~7) | c);
-    const bool own = chunk == c;
-    qv[jj] = own ? q : qv[jj];
-    hv[jj] = own ? wh : hv[jj];
-    ev[jj] = own ? e : ev[jj];
-    // w_k -= e U[j][k] for this thread's columns k > j
-    const float* ur = Us + j * US_LD + chunk * 16;
-#pragma unroll
-    for (int k = 0; k < 16; k += 4) {
-      const float4 u = *reinterpret_cast<const float4*>(ur + k);
-      const float uu[4] = {u.x, u.y, u.z, u.w};
+  for (int sg = 0; sg < 4; ++sg) {
+#pragma unroll 1
+    for (int c = 0; c < 8; ++c) {
+      const bool own = chunk == c;
+      const int src = (lane & ~7) | c;
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
-        const int col = chunk * 16 + k + t;
-        w[k + t] = fmaf(-e, (col > j) ? uu[t] : 0.f, w[k + t]);
+        const int j = 32 * sg + 4 * c + t;
+        if (GROUP > 0 && t == 0 && (j % (GROUP > 0 ? GROUP : 1)) == 0) {
+          // grid of columns j .. j+GROUP-1 (groups sg .. sg + GROUP/32 - 1 of every thread)
+          float mn = INFINITY, mx = -INFINITY;
+#pragma unroll
+          for (int k = 4 * sg; k < 4 * sg + (GROUP >= 32 ? GROUP / 8 : 4) && k < 16; ++k) {
+            mn = fminf(mn, w[k]);
+            mx = fmaxf(mx, w[k]);
+          }
+#pragma unroll
+          for (int o = 1; o < 8; o <<= 1) {
+            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          }
+          const Grid g = make_grid(mn, mx, maxq);
+          scale = g.scale;
+          zero = g.zero;
+          rscale = __frcp_rn(scale);
+          if (live && own) {
+            const int gi = (i1 + j) / (GROUP > 0 ? GROUP : 1);
+            scales[(int64_t)row * G + gi] = scale;
+            zeros[(int64_t)row * G + gi] = (uint8_t)zero;
+          }
+        }
+        // quantize this thread's copy of column j (meaningful on the owner only)
+        const float x = w[4 * sg + t];
+        const float q = fminf(fmaxf(round_quotient(x, scale, rscale) + zero, 0.f), maxq);
+        const float wh = scale * (q - zero);
+        const float e_own = (x - wh) * rdiag[j];
+        const float e_bc = __shfl_sync(0xffffffffu, e_own, src);
+        const float e = own ? e_own : e_bc;          // the owner skips the shuffle latency
+        qv[4 * sg + t] = own ? q : qv[4 * sg + t];
+        hv[4 * sg + t] = own ? wh : hv[4 * sg + t];
+        ev[4 * sg + t] = own ? e_own : ev[4 * sg + t];
+        // w_k -= e U[j][k] for this thread's columns k > j (groups left of sg are done)
+        const float* ur = Us + j * US_LD + 4 * chunk;
+#pragma unroll
+        for (int s2 = sg; s2 < 4; ++s2) {
+          const float4 u = *reinterpret_cast<const float4*>(ur + 32 * s2);
+          const float uu[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int t2 = 0; t2 < 4; ++t2) {
+            const float coef = (s2 > sg || 4 * chunk + t2 > 4 * c + t) ? uu[t2] : 0.f;
+            w[4 * s2 + t2] = fmaf(-e, coef, w[4 * s2 + t2]);
+          }
+        }
       }
     }
   }
   if (!live) return;
-  const int64_t off = (int64_t)row * n + i1 + chunk * 16;
-  {
-    uint32_t pk[4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k)
-      pk[k] = (uint32_t)qv[4 * k] | ((uint32_t)qv[4 * k + 1] << 8) | ((uint32_t)qv[4 * k + 2] << 16) |
-              ((uint32_t)qv[4 * k + 3] << 24);
-    *reinterpret_cast<uint4*>(codes + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-  }
-  float* e_dst = E + (int64_t)row * QB + chunk * 16;
-#pragma unroll
-  for (int k = 0; k < 16; k += 4)
-    *reinterpret_cast<float4*>(e_dst + k) = make_float4(ev[k], ev[k + 1], ev[k + 2], ev[k + 3]);
-  if (W_hat) {
-#pragma unroll
-    for (int k = 0; k < 16; k += 4)
-      *reinterpret_cast<float4*>(W_hat + off + k) = make_float4(hv[k], hv[k + 1], hv[k + 2], hv[k + 3]);
+  for (int sg = 0; sg < 4; ++sg) {
+    const int64_t off = (int64_t)row * n + i1 + 32 * sg + 4 * chunk;
+    const uint32_t pk = (uint32_t)qv[4 * sg] | ((uint32_t)qv[4 * sg + 1] << 8) |
+                        ((uint32_t)qv[4 * sg + 2] << 16) | ((uint32_t)qv[4 * sg + 3] << 24);
+    *reinterpret_cast<uint32_t*>(codes + off) = pk;
+    *reinterpret_cast<float4*>(E + (int64_t)row * QB + 32 * sg + 4 * chunk) =
+        make_float4(ev[4 * sg], ev[4 * sg + 1], ev[4 * sg + 2], ev[4 * sg + 3]);
+    if (W_hat)
+      *reinterpret_cast<float4*>(W_hat + off) =
+          make_float4(hv[4 * sg], hv[4 * sg + 1], hv[4 * sg + 2], hv[4 * sg + 3]);
   }
 }
 
