@@ -46,6 +46,9 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="calibration tokens per X/G (default: the workload's; smaller only for "
+                         "profiler captures)")
     return ap.parse_args()
 
 
@@ -56,6 +59,14 @@ def workload_desc(cfg) -> str:
     return (f"{cfg.name}: {subs}; X/G {cfg.tokens} tokens bf16 ({cfg.x_dist} X with outlier "
             f"channels x{cfg.x_outlier_scale:g}, G scales over {cfg.g_decades:g} decades); "
             f"{bits} asymmetric {g}; BiIP alpha {cfg.alpha}, damp {cfg.damp}")
+
+
+def l2_note(cfg) -> str:
+    sizes = [cfg.tokens * s.width * 2 for s in cfg.sites] + [cfg.tokens * s.m * 2 for s in cfg.sublayers]
+    small = min(sizes)
+    verdict = "larger than" if small > 126 * 2 ** 20 else "NOT larger than"
+    return (f"inputs {verdict} L2, no flush: each X/G is {small / 2 ** 30:.2f} GiB or more "
+            f"({cfg.tokens} tokens, bf16)")
 
 
 # ------------------------------------------------------------- clocks
@@ -366,8 +377,10 @@ def main():
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     abi.lib()
-    cfg0 = synth.get_config(args.config)
     import dataclasses
+    cfg0 = synth.get_config(args.config)
+    if args.tokens:
+        cfg0 = dataclasses.replace(cfg0, tokens=args.tokens)
     cfg = dataclasses.replace(cfg0, seed=cfg0.seed + rank)   # each rank: its own layer (weak scaling)
 
     # ---- seeded inputs on the host (pinned for the end-to-end leg), then HBM
@@ -528,7 +541,7 @@ def main():
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded generator; stands in for WikiText-2 activations and LLaMA weights)",
             "config": {"workload": workload, "parallelism": f"replicas x{world} (one layer per GPU)",
-                       "l2": "inputs larger than L2 (X and G are 2 GiB each at 262144 x 4096 bf16)",
+                       "l2": l2_note(cfg0),
                        "solver_dtype": "fp32", "input_gen_s": round(t_gen, 1)},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
             "clocks": clocks,

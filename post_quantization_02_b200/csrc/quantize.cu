@@ -16,11 +16,15 @@
 //                     threads with one shuffle, each thread applies
 //                     w_k -= e U_c[j,k] to its columns k > j.  No block-wide
 //                     synchronisation inside the column loop.
-//   lazy_update       W[:, i+128:] -= E U_c[i:i+128, i+128:]
+//   lazy update       W[:, i+128:] -= E U_c[i:i+128, i+128:] on the tensor cores
+//                     (kq_lazy_update_tc, tf32 with a three-term split)
 #include <mutex>
 
 #include "common.cuh"
 #include "gemm_simt.cuh"
+
+int kq_lazy_update_tc(float* W, int64_t m, int64_t n, const float* E, const float* U, int i1,
+                      int32_t* info, cudaStream_t st);
 
 namespace {
 
@@ -200,18 +204,6 @@ obs_block_kernel(const float* __restrict__ W, int m, int n, const float* __restr
   }
 }
 
-// W[:, i2:] -= E U[i1:i2, i2:]  (128 x 128 output tiles, K = 128)
-__global__ void __launch_bounds__(256) lazy_update_kernel(float* W, int m, int n,
-                                                          const float* __restrict__ E,
-                                                          const float* __restrict__ U, int i1) {
-  __shared__ kq::Gemm128Smem gs;
-  const int i2 = i1 + QB;
-  const int r0 = blockIdx.y * kq::G2, c0 = i2 + blockIdx.x * kq::G2;
-  kq::gemm128<false>(gs, E + (int64_t)r0 * QB, QB, U + (int64_t)i1 * n + c0, n,
-                     W + (int64_t)r0 * n + c0, n, min(kq::G2, m - r0), min(kq::G2, n - c0), QB,
-                     -1.f, 1.f);
-}
-
 template <bool TA, bool TB>
 __global__ void __launch_bounds__(256) gemm_kernel(const float* A, int64_t lda, const float* B,
                                                    int64_t ldb, float* C, int64_t ldc, int M, int N,
@@ -305,7 +297,6 @@ size_t kq_loss_ws(int64_t m, int64_t n) { return 3 * a256((size_t)m * n * sizeof
 int kq_quantize_layer(float* W, int64_t m64, int64_t n64, const float* U, int bits, int group,
                       int block, uint8_t* codes, float* scales, uint8_t* zeros, float* W_hat,
                       int32_t* info, void* ws, size_t ws_bytes, cudaStream_t st) {
-  (void)info;
   if (!W || !U || !codes || !scales || !zeros || m64 <= 0 || n64 <= 0) return KRONQ_ERR_INVALID_ARG;
   if (bits != 2 && bits != 3 && bits != 4 && bits != 8) return KRONQ_ERR_INVALID_ARG;
   if (group != -1 && (group <= 0 || n64 % group)) return KRONQ_ERR_INVALID_ARG;
@@ -335,9 +326,8 @@ int kq_quantize_layer(float* W, int64_t m64, int64_t n64, const float* U, int bi
     if (s != KRONQ_OK) return s;
     const int i2 = i1 + QB;
     if (i2 < n) {
-      const dim3 grid((n - i2 + kq::G2 - 1) / kq::G2, (m + kq::G2 - 1) / kq::G2);
-      lazy_update_kernel<<<grid, 256, 0, st>>>(W, m, n, E, U, i1);
-      KQ_CHECK_LAUNCH();
+      s = kq_lazy_update_tc(W, m, n, E, U, i1, info, st);
+      if (s != KRONQ_OK) return s;
     }
   }
   return KRONQ_OK;
