@@ -53,23 +53,31 @@ def _scale(h_diag: np.ndarray, norm2: np.ndarray, alpha: float) -> np.ndarray:
     return s
 
 
-def rescale(W, HX, HG, alpha: float, mode: str = "full"):
-    """Eq. 11 (reading above).  Returns W, H_X, H_G rescaled and S_X, S_G."""
-    W = np.array(W, dtype=np.float64)
-    HX = np.array(HX, dtype=np.float64)
-    HG = np.array(HG, dtype=np.float64)
+def scales(W, hx_diag, hg_diag, alpha: float, mode: str = "full"):
+    """S_X and S_G of Eq. 11 (reading above) from W and the two diagonals:
+    S_X from the column norms of W, S_G from the row norms of W diag(S_X)."""
+    W = np.asarray(W, dtype=np.float64)
     m, n = W.shape
     in_s, out_s, _, _ = sides(mode)
     SX = np.ones(n)
     SG = np.ones(m)
     if in_s:
-        SX = _scale(np.diag(HX).copy(), (W * W).sum(axis=0), alpha)
-        W = W * SX[None, :]
-        HX = HX / np.outer(SX, SX)
+        SX = _scale(np.array(hx_diag, dtype=np.float64), (W * W).sum(axis=0), alpha)
     if out_s:
-        SG = _scale(np.diag(HG).copy(), (W * W).sum(axis=1), alpha)
-        W = W * SG[:, None]
-        HG = HG / np.outer(SG, SG)
+        WS = W * SX[None, :]
+        SG = _scale(np.array(hg_diag, dtype=np.float64), (WS * WS).sum(axis=1), alpha)
+    return SX, SG
+
+
+def rescale(W, HX, HG, alpha: float, mode: str = "full"):
+    """Eq. 11 (reading above).  Returns W, H_X, H_G rescaled and S_X, S_G."""
+    W = np.array(W, dtype=np.float64)
+    HX = np.array(HX, dtype=np.float64)
+    HG = np.array(HG, dtype=np.float64)
+    SX, SG = scales(W, np.diag(HX), np.diag(HG), alpha, mode)
+    W = W * SX[None, :] * SG[:, None]
+    HX = HX / np.outer(SX, SX)
+    HG = HG / np.outer(SG, SG)
     return W, HX, HG, SX, SG
 
 
@@ -104,3 +112,49 @@ def unbiip_w(Wp, SX, SG, sign_u, sign_v, mode: str = "full"):
     if in_r:
         W = transform.apply_t(W, sign_v)
     return W / np.asarray(SG)[:, None] / np.asarray(SX)[None, :]
+
+
+def biip_entries(W, HX, HG, sign_u, sign_v, alpha: float, mode: str, w_rows, w_cols,
+                 hx_idx, hg_idx):
+    """Selected entries of the BiIP outputs at any size, without forming the
+    whole transforms:
+      W'[w_rows][:, w_cols]   = (U_r S_G) W (S_X V_c^T),
+      H_X'[hx_idx][:, hx_idx] = V_a S_X^-1 H_X S_X^-1 V_a^T,
+      H_G'[hg_idx][:, hg_idx] = U_a S_G^-1 H_G S_G^-1 U_a^T,
+    where U_r, V_c, V_a, U_a are the selected rows of U = T_m D_u and
+    V = T_n D_v (identity rows on a side the mode does not rotate).  The
+    same products as rescale + rotate, associated so only the selected rows
+    and columns are formed.  Returns (W' block, H_X' block, H_G' block,
+    S_X, S_G); H_X / H_G may be None."""
+    m, n = W.shape
+    _, _, in_r, out_r = sides(mode)
+    hxd = np.diag(HX) if HX is not None else np.ones(n)
+    hgd = np.diag(HG) if HG is not None else np.ones(m)
+    SX, SG = scales(W, hxd, hgd, alpha, mode)
+
+    def sel(d, idx, signs, rot):
+        if rot:
+            return transform.rows(d, idx, signs)
+        E = np.zeros((len(idx), d))
+        E[np.arange(len(idx)), np.asarray(idx)] = 1.0
+        return E
+
+    def left(A, M, panel=2048):
+        # A @ M with M widened to fp64 one row panel at a time (M may be a
+        # wide fp32 matrix that would not fit in memory as fp64 at once)
+        out = np.zeros((A.shape[0], M.shape[1]))
+        for p in range(0, M.shape[0], panel):
+            out += A[:, p:p + panel] @ np.asarray(M[p:p + panel], dtype=np.float64)
+        return out
+
+    Ur = sel(m, w_rows, sign_u, out_r) * SG[None, :]
+    Vc = sel(n, w_cols, sign_v, in_r) * SX[None, :]
+    Wb = left(Ur, W) @ Vc.T
+    HXb = HGb = None
+    if HX is not None:
+        Va = sel(n, hx_idx, sign_v, in_r) / SX[None, :]
+        HXb = left(Va, HX) @ Va.T
+    if HG is not None:
+        Ua = sel(m, hg_idx, sign_u, out_r) / SG[None, :]
+        HGb = left(Ua, HG) @ Ua.T
+    return Wb, HXb, HGb, SX, SG

@@ -49,3 +49,21 @@ def inverse_cholesky(H: np.ndarray) -> np.ndarray:
     except np.linalg.LinAlgError as e:
         raise NotPositiveDefinite(str(e)) from None
     return Lh.T
+
+
+def inverse_cholesky_trailing(H: np.ndarray, k: int, lam: float = 0.0) -> np.ndarray:
+    """U[k:, k:] of U = inverse_cholesky(damp(H, lam)), from H[k:, k:] and the
+    mean of diag(H) alone.
+
+    With R = U^-1 (upper), H_d = R R^T, and since R is upper the trailing
+    block obeys H_d[k:, k:] = R[k:, k:] R[k:, k:]^T; the inverse of an upper
+    triangular matrix has the inverse of its trailing block as its own
+    trailing block, so U[k:, k:] = inverse_cholesky(H_d[k:, k:]).  The
+    damping adds lam * mean(diag(H)) of the WHOLE matrix.  Lets a test check
+    a wide factor on its last columns without the n^3 inverse."""
+    H = np.asarray(H)
+    n = H.shape[0]
+    mu = float(np.mean(np.diag(H).astype(np.float64))) if n else 0.0
+    B = np.array(H[k:, k:], dtype=np.float64)
+    B[np.arange(n - k), np.arange(n - k)] += lam * mu
+    return inverse_cholesky(B)

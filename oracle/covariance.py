@@ -39,6 +39,15 @@ def covariance_block(chunks, rows: np.ndarray, cols: np.ndarray, n_total: int) -
     return H / n_total
 
 
+def covariance_diag(chunks, d: int, n_total: int) -> np.ndarray:
+    """diag(H) = (1/N) sum_t a_t[j]^2 for every j, over row chunks of A."""
+    s = np.zeros(d)
+    for C in chunks:
+        C = np.asarray(C, dtype=np.float64)
+        s += np.einsum("tj,tj->j", C, C)
+    return s / n_total
+
+
 def vec(M: np.ndarray) -> np.ndarray:
     """Column-stacking vec: vec(g x^T) = x (x) g."""
     return np.asarray(M).reshape(-1, order="F")

@@ -156,7 +156,17 @@ def layer_loss(dW: np.ndarray, HX: np.ndarray, HG: np.ndarray) -> float:
     return float(np.sum(M * dW))
 
 
-def row_losses(dW: np.ndarray, HX: np.ndarray) -> np.ndarray:
-    """dW_i H_X dW_i^T for each row (the part of the loss the solver sees)."""
+def row_losses(dW: np.ndarray, HX: np.ndarray, lam: float = 0.0) -> np.ndarray:
+    """dW_i H dW_i^T for each row (the part of the loss the solver sees),
+    with H = H_X + lam * mean(diag(H_X)) I (lam = 0: H_X itself).  H_X may be
+    fp32; it is widened to fp64 one row panel at a time."""
     dW = np.asarray(dW, dtype=np.float64)
-    return np.einsum("ij,ij->i", dW @ np.asarray(HX, dtype=np.float64), dW)
+    n = dW.shape[1]
+    P = np.zeros_like(dW)
+    for p in range(0, n, 2048):
+        P += dW[:, p:p + 2048] @ np.asarray(HX[p:p + 2048], dtype=np.float64)
+    out = np.einsum("ij,ij->i", P, dW)
+    if lam:
+        mu = float(np.mean(np.diag(HX).astype(np.float64)))
+        out += lam * mu * np.einsum("ij,ij->i", dW, dW)
+    return out

@@ -45,3 +45,14 @@ def allocate_bits(scores, params, target_avg: float = 3.0, base: int = 2, top: i
                 used += up * params[i]
                 break
     return bits
+
+
+def sensitivity_from_diagonals(hx_diag, hg_diag, SX, SG) -> float:
+    """The same s after BiIP, from the diagonals before it: the rotation is
+    orthogonal, so tr(V H V^T) = tr(H), and the rescale divides entry j of
+    the diagonal by S_j^2; hence s = (sum_j H_X[j,j] / S_X[j]^2) *
+    (sum_i H_G[i,i] / S_G[i]^2), fp64.  Lets a test score a sublayer of any
+    width without forming the rotated matrices."""
+    tx = float(np.sum(np.asarray(hx_diag, dtype=np.float64) / np.asarray(SX, dtype=np.float64) ** 2))
+    tg = float(np.sum(np.asarray(hg_diag, dtype=np.float64) / np.asarray(SG, dtype=np.float64) ** 2))
+    return tg * tx

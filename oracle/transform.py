@@ -107,3 +107,12 @@ def apply_t(y: np.ndarray, signs: np.ndarray | None = None) -> np.ndarray:
     if signs is not None:
         x = x * np.asarray(signs, dtype=np.float64)
     return x
+
+
+def rows(d: int, idx, signs: np.ndarray | None = None) -> np.ndarray:
+    """Rows idx of the d x d matrix T_d D, without forming it: row i is
+    (T_d D)^T e_i, i.e. apply_t of the i-th unit vector."""
+    idx = np.asarray(idx, dtype=np.int64)
+    E = np.zeros((len(idx), d))
+    E[np.arange(len(idx)), idx] = 1.0
+    return apply_t(E, signs)

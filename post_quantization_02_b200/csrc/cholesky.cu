@@ -7,20 +7,24 @@
 // (lower Cholesky) and U_c = J L^-1 J; then U_c^T U_c = J (L L^T)^-1 J =
 // H_d^-1 and U_c is upper triangular.
 //
-// One right-looking sweep over 128-wide panels computes L and Y = L^-1
-// together (block forward substitution of L Y = I carried along with the
-// factorisation).  Step p (rows k = 128 p ...):
+// The matrix is padded with the identity to np = a multiple of 128 (which
+// leaves the leading blocks of L and L^-1 unchanged).  One right-looking
+// sweep over 128-wide panels computes L and Z = L^-T together (block
+// forward substitution of L Y = I carried along with the factorisation,
+// stored transposed so that every product has both operands K-major).
+// Step p (rows k = 128 p ...):
 //   panel kernel   every CTA factors the 128 x 128 diagonal block
 //                  R_pp = L_pp L_pp^T and inverts L_pp in shared memory, then
 //                  either turns 128 rows of the panel into L_ip = R_ip L_pp^-T,
-//                  or finishes 128 columns of block row p of Y:
-//                  Y_pj = L_pp^-1 A_pj  (A_pj = -sum_{q<p} L_pq Y_qj), Y_pp = L_pp^-1.
-//   update kernel  for every block row i > p: the trailing lower triangle
-//                  R_ij -= L_ip L_jp^T and the accumulators A_ij -= L_ip Y_pj
-//                  (j <= p), as 128 x 128 fp32 GEMM tiles with K = 128.
-// Then U_c[a][b] = Y[n-1-a][n-1-b] (a <= b).
+//                  or finishes 128 rows of block column p of Z:
+//                  Z_jp = B_jp L_pp^-T (B_jp = -sum_{q<p} Z_jq L_pq^T), Z_pp = L_pp^-T.
+//   update         one tensor-core launch (tf32, three-term split) for
+//                  R[k+128:, k+128:] -= L L^T (lower triangle) and
+//                  Z[:k+128, k+128:] -= Z[:k+128, k:k+128] L^T, L = the panel rows.
+// Then U_c[a][b] = Z[n-1-b][n-1-a] (a <= b).
 #include "common.cuh"
 #include "gemm_simt.cuh"
+#include "gemm_tc.cuh"
 
 namespace {
 
@@ -40,121 +44,176 @@ __global__ void diag_sum_kernel(const float* __restrict__ H, int n, double* out)
   if (threadIdx.x == 0) *out = red[0];
 }
 
-// R[a][b] = H[n-1-a][n-1-b] + delta [a == b], delta = damp_rel * mean(diag H); Y = 0.
-__global__ void reverse_damp_kernel(const float* __restrict__ H, int n, float* __restrict__ R,
-                                    float* __restrict__ Y, float damp_rel,
+// R[a][b] = H[n-1-a][n-1-b] + delta [a == b] for a, b < n, the identity on
+// the padding up to np (a multiple of 128), delta = damp_rel * mean(diag H);
+// Z = 0.  Padding with the identity leaves the leading n x n blocks of the
+// factor and of its inverse unchanged.
+__global__ void reverse_damp_kernel(const float* __restrict__ H, int n, int np,
+                                    float* __restrict__ R, float* __restrict__ Z, float damp_rel,
                                     const double* __restrict__ diag_sum) {
   const float delta = (float)((double)damp_rel * (*diag_sum / (double)n));
-  const int64_t total = (int64_t)n * n;
+  const int64_t total = (int64_t)np * np;
   for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
        e += (int64_t)gridDim.x * blockDim.x) {
-    const int a = (int)(e / n), b = (int)(e % n);
-    float v = H[(int64_t)(n - 1 - a) * n + (n - 1 - b)];
-    if (a == b) v += delta;
+    const int a = (int)(e / np), b = (int)(e % np);
+    float v;
+    if (a < n && b < n) {
+      v = H[(int64_t)(n - 1 - a) * n + (n - 1 - b)];
+      if (a == b) v += delta;
+    } else {
+      v = (a == b) ? 1.f : 0.f;
+    }
     R[e] = v;
-    Y[e] = 0.f;
+    Z[e] = 0.f;
+  }
+}
+
+// One warp factors the 32 x 32 diagonal block at offset o of D (lower part
+// valid, already updated) and inverts the factor: on return D holds L_oo
+// and X holds L_oo^-1 (both lower).  Lane i keeps row i of the block in
+// registers; pivot step j needs no barrier: the pivot comes from lane j,
+// the column L[:, j] and the row j of L^-1 travel by shuffles.
+//   L[i][j] = a_i[j] r,  r = 1 / sqrt(a_j[j])
+//   a_i[c] -= L[i][j] L[c][j]            (c > j, the Schur complement)
+//   Y[j][:] = y_j[:] r,  y_i[:] -= L[i][j] Y[j][:]   (i > j, rows of L^-1)
+__device__ __forceinline__ void warp_leaf32(float* D, float* X, int o, int kb, int* bad) {
+  const int i = threadIdx.x & 31;
+  constexpr unsigned FULL = 0xffffffffu;
+  float a[32], y[32];
+#pragma unroll
+  for (int c = 0; c < 32; ++c) {
+    a[c] = (c <= i) ? D[(o + i) * LDD + o + c] : 0.f;
+    y[c] = (c == i) ? 1.f : 0.f;
+  }
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    float d = __shfl_sync(FULL, a[j], j);
+    if (!(d > 0.f) || !isfinite(d)) {
+      if (i == 0 && o + j < kb) *bad = 1;
+      d = 1.f;
+    }
+    const float r = rsqrtf(d);
+    const float l = (i >= j) ? a[j] * r : 0.f;
+    a[j] = l;
+#pragma unroll
+    for (int c = j + 1; c < 32; ++c) a[c] = fmaf(-l, __shfl_sync(FULL, l, c), a[c]);
+#pragma unroll
+    for (int c = 0; c <= j; ++c) {
+      const float yj = __shfl_sync(FULL, y[c], j) * r;
+      y[c] = (i == j) ? yj : fmaf(-l, yj, y[c]);
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < 32; ++c) {
+    if (c <= i) {
+      D[(o + i) * LDD + o + c] = a[c];
+      X[(o + i) * LDD + o + c] = y[c];
+    }
   }
 }
 
 // X = L^-1 for the lower Cholesky factor L of the 128 x 128 block in D
-// (fp32; rows/columns kb .. NB-1 are padded with the identity by the caller;
-// D is overwritten with scratch).
+// (fp32; rows / columns kb .. NB-1 padded with the identity by the caller).
+// On return D's lower triangle holds L and X (zero above the diagonal)
+// holds L^-1.  256 threads.
 //
-// One sweep of 128 column steps does the factorisation and the inverse
-// together: at step j the pivot column of the Schur complement and the
-// accumulated row j of L^-1 are both final, so with r = 1/sqrt(d_j):
-//   L[i][j] = S[i][j] r,   Y[j][:] = A[j][:] r,
-//   S[i][c] -= L[i][j] L[c][j]      (the trailing Schur complement)
-//   A[i][:] -= L[i][j] Y[j][:]      (i > j, the rows of L^-1 still open).
-// Thread (ty, tx) keeps the 8 x 8 tiles of S and A at rows 8ty.., columns
-// 8tx.. in registers; warp w owns the column tiles tx = 2w, 2w+1 (ty = lane
-// mod 16), so at step j a warp's choice is uniform: tiles with columns > j
-// need the S update, tiles with columns <= j the A update (only the tile
-// holding column j needs both).  Entries that are already final or never
-// used absorb harmless updates.  After its last update, column j+1 of S and
-// row j+1 of A are published to shared memory; one barrier per step.
+// Right-looking over four 32-wide blocks b (o = 32 b), carrying L^-1 along
+// (block forward substitution of L Y = I, accumulators in X below the
+// diagonal blocks):
+//   1. warp 0: L_bb and Y_bb = L_bb^-1                          (warp_leaf32)
+//   2. L_cb = D_cb Y_bb^T (c > b);  Y_bj = Y_bb Acc_bj (j < b)
+//   3. D_cd -= L_cb L_db^T (b < d <= c);  Acc_cj -= L_cb Y_bj (c > b, j <= b)
+// Steps 2 and 3 are small GEMMs out of shared memory, register-tiled.
 __device__ void factor_and_invert(float* D, float* X, int kb, int* bad) {
-  __shared__ __align__(16) float colbuf[2][NB];
-  __shared__ __align__(16) float rowbuf[2][NB];
   const int tid = threadIdx.x;
-  const int ty = tid & 15, tx = ((tid >> 5) << 1) | ((tid >> 4) & 1);
-  float a[8][8], y[8][8];
-#pragma unroll
-  for (int r = 0; r < 8; ++r)
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      a[r][c] = D[(8 * ty + r) * LDD + 8 * tx + c];
-      y[r][c] = (8 * ty + r == 8 * tx + c) ? 1.f : 0.f;
-    }
-  if (tid < NB) {
-    colbuf[0][tid] = D[tid * LDD];          // column 0 of S
-    rowbuf[0][tid] = (tid == 0) ? 1.f : 0.f;  // row 0 of A (identity)
-  }
+  for (int e = tid; e < NB * LDD; e += blockDim.x) X[e] = 0.f;
   __syncthreads();
-  for (int jb = 0; jb < NB / 8; ++jb) {
+  for (int b = 0; b < NB / 32; ++b) {
+    const int o = 32 * b;
+    const int o2 = o + 32;
+    const int R1 = NB - o2;                 // rows below the diagonal block
+    if (tid < 32) warp_leaf32(D, X, o, kb, bad);
+    __syncthreads();
+    // ---- step 2: thread (tr, tc) = (tid / 8, tid % 8)
+    {
+      const int tr = tid >> 3, tc = tid & 7;
+      float acc1[3][4], acc2[12];
+      // L_cb rows o2 + tr + 32 s, columns o + 4 tc .. +3
 #pragma unroll
-    for (int jj = 0; jj < 8; ++jj) {
-      const int j = 8 * jb + jj;
-      const int b = jj & 1;                 // j & 1 (8 * jb is even)
-      float d = colbuf[b][j];
-      if (!(d > 0.f) || !isfinite(d)) {
-        if (tid == 0 && j < kb) *bad = 1;
-        d = 1.f;
+      for (int s = 0; s < 3; ++s)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc1[s][q] = 0.f;
+#pragma unroll
+      for (int q = 0; q < 12; ++q) acc2[q] = 0.f;
+      const int nj = o >> 3;                // Y_bj columns per thread: o / 8
+#pragma unroll 4
+      for (int t = 0; t < 32; ++t) {
+        float bv[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) bv[q] = X[(o + 4 * tc + q) * LDD + o + t];   // Y_bb[c][t]
+#pragma unroll
+        for (int s = 0; s < 3; ++s) {
+          if (32 * s < R1) {
+            const float av = D[(o2 + tr + 32 * s) * LDD + o + t];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) acc1[s][q] = fmaf(av, bv[q], acc1[s][q]);
+          }
+        }
+        const float yv = X[(o + tr) * LDD + o + t];                            // Y_bb[r][t]
+#pragma unroll
+        for (int q = 0; q < 12; ++q)
+          if (q < nj) acc2[q] = fmaf(yv, X[(o + t) * LDD + tc * nj + q], acc2[q]);   // Acc[t][c']
       }
-      const float rs = rsqrtf(d);
-      if (tid < NB) X[j * LDD + tid] = rowbuf[b][tid] * rs;   // row j of L^-1, final
-      const bool do_s = 8 * tx + 7 > j, do_a = 8 * tx <= j;
-      {
-        float li[8], lc[8], yj[8];
-        {
-          const float4 p0 = *reinterpret_cast<const float4*>(&colbuf[b][8 * ty]);
-          const float4 p1 = *reinterpret_cast<const float4*>(&colbuf[b][8 * ty + 4]);
-          const float4 q0 = *reinterpret_cast<const float4*>(&colbuf[b][8 * tx]);
-          const float4 q1 = *reinterpret_cast<const float4*>(&colbuf[b][8 * tx + 4]);
-          const float4 y0 = *reinterpret_cast<const float4*>(&rowbuf[b][8 * tx]);
-          const float4 y1 = *reinterpret_cast<const float4*>(&rowbuf[b][8 * tx + 4]);
-          li[0] = p0.x; li[1] = p0.y; li[2] = p0.z; li[3] = p0.w;
-          li[4] = p1.x; li[5] = p1.y; li[6] = p1.z; li[7] = p1.w;
-          lc[0] = q0.x; lc[1] = q0.y; lc[2] = q0.z; lc[3] = q0.w;
-          lc[4] = q1.x; lc[5] = q1.y; lc[6] = q1.z; lc[7] = q1.w;
-          yj[0] = y0.x; yj[1] = y0.y; yj[2] = y0.z; yj[3] = y0.w;
-          yj[4] = y1.x; yj[5] = y1.y; yj[6] = y1.z; yj[7] = y1.w;
+      __syncthreads();
+#pragma unroll
+      for (int s = 0; s < 3; ++s)
+        if (32 * s < R1)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) D[(o2 + tr + 32 * s) * LDD + o + 4 * tc + q] = acc1[s][q];
+#pragma unroll
+      for (int q = 0; q < 12; ++q)
+        if (q < nj) X[(o + tr) * LDD + tc * nj + q] = acc2[q];
+      __syncthreads();
+    }
+    if (R1 == 0) break;
+    // ---- step 3: rows o2 + tr + 16 s, columns 8 tc .. 8 tc + 7 (all 128)
+    {
+      const int tr = tid >> 4, tc = tid & 15;
+      const int ns = R1 >> 4;               // 6, 4 or 2 rows per thread
+      float acc[6][8];
+#pragma unroll
+      for (int s = 0; s < 6; ++s)
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[s][q] = 0.f;
+      const int c0 = 8 * tc;
+      const bool left = c0 < o2;            // Acc / Y columns (j <= b), else trailing D
+#pragma unroll 2
+      for (int t = 0; t < 32; ++t) {
+        float bv[8];
+        if (left) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) bv[q] = X[(o + t) * LDD + c0 + q];          // Y_b[t][c]
+        } else {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) bv[q] = D[(c0 + q) * LDD + o + t];          // L[c][o+t]
         }
-        // published values are raw: scale L[.][j] by r, and Y[j][.] by r
 #pragma unroll
-        for (int r = 0; r < 8; ++r) li[r] *= rs;
-        const float rs2 = rs * rs;
+        for (int s = 0; s < 6; ++s) {
+          if (s < ns) {
+            const float av = D[(o2 + tr + 16 * s) * LDD + o + t];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          lc[c] *= rs;
-          yj[c] *= rs;
-        }
-        (void)rs2;
-        if (do_s) {
-#pragma unroll
-          for (int r = 0; r < 8; ++r)
-#pragma unroll
-            for (int c = 0; c < 8; ++c) a[r][c] = fmaf(-li[r], lc[c], a[r][c]);
-        }
-        if (do_a) {
-#pragma unroll
-          for (int r = 0; r < 8; ++r)
-#pragma unroll
-            for (int c = 0; c < 8; ++c) y[r][c] = fmaf(-li[r], yj[c], y[r][c]);
+            for (int q = 0; q < 8; ++q) acc[s][q] = fmaf(av, bv[q], acc[s][q]);
+          }
         }
       }
-      // publish column j+1 of S and row j+1 of A (their last update was just now)
-      const int jn = j + 1;
-      if (jn < NB) {
-        if (tx == (jn >> 3)) {
-          const int cl = (jj + 1) & 7;        // compile-time after unrolling
 #pragma unroll
-          for (int r = 0; r < 8; ++r) colbuf[b ^ 1][8 * ty + r] = (8 * ty + r >= jn) ? a[r][cl] : 0.f;
-        }
-        if (ty == (jn >> 3)) {
-          const int rl = (jj + 1) & 7;
+      for (int s = 0; s < 6; ++s) {
+        if (s < ns) {
+          const int r = o2 + tr + 16 * s;
+          float* dst = left ? &X[r * LDD + c0] : &D[r * LDD + c0];
 #pragma unroll
-          for (int c = 0; c < 8; ++c) rowbuf[b ^ 1][8 * tx + c] = (8 * tx + c <= jn) ? y[rl][c] : 0.f;
+          for (int q = 0; q < 8; ++q)
+            if (left || c0 + q <= r) dst[q] -= acc[s][q];
         }
       }
       __syncthreads();
@@ -162,7 +221,7 @@ __device__ void factor_and_invert(float* D, float* X, int kb, int* bad) {
   }
 }
 
-__global__ void __launch_bounds__(256, 1) panel_kernel(float* R, float* Y, int n, int k, int p,
+__global__ void __launch_bounds__(256, 1) panel_kernel(float* R, float* Z, int n, int k, int p,
                                                     int tiles_L, int32_t* info) {
   extern __shared__ float sm[];
   float* D = sm;                       // [NB][LDD]
@@ -188,47 +247,39 @@ __global__ void __launch_bounds__(256, 1) panel_kernel(float* R, float* Y, int n
     float* P = R + (int64_t)r0 * n + k;
     kq::gemm128<true>(gs, P, n, X, LDD, P, n, n - r0 < NB ? n - r0 : NB, kb, kb, 1.f, 0.f);
   } else {
-    const int j = blockIdx.x - tiles_L;  // column block of Y's block row p
+    const int j = blockIdx.x - tiles_L;  // row block of Z's column block p
     if (j < p) {
-      float* B = Y + (int64_t)k * n + NB * j;
-      kq::gemm128<false>(gs, X, LDD, B, n, B, n, kb, NB, kb, 1.f, 0.f);
+      // Z_jp = Acc_jp L_pp^-T (in place)
+      float* B = Z + (int64_t)(NB * j) * n + k;
+      kq::gemm128<true>(gs, B, n, X, LDD, B, n, NB, kb, kb, 1.f, 0.f);
     } else {
+      // Z_pp = L_pp^-T (upper; X is zero above its diagonal)
       for (int e = threadIdx.x; e < kb * kb; e += blockDim.x) {
         const int a = e / kb, b = e % kb;
-        Y[(int64_t)(k + a) * n + k + b] = X[a * LDD + b];
+        Z[(int64_t)(k + a) * n + k + b] = X[b * LDD + a];
       }
     }
   }
 }
 
-// Trailing updates after panel p.  blockIdx.y: block row below the panel;
-// blockIdx.x < p+1: Y accumulator column block; else: trailing R column block.
-__global__ void __launch_bounds__(256) update_kernel(float* R, float* Y, int n, int k, int p) {
-  __shared__ kq::Gemm128Smem gs;
-  const int kb = min(NB, n - k);
-  const int ti = blockIdx.y, tj = blockIdx.x;
-  const int r0 = k + kb + NB * ti;
-  const int M = min(NB, n - r0);
-  const float* L = R + (int64_t)r0 * n + k;
-  if (tj <= p) {
-    float* C = Y + (int64_t)r0 * n + NB * tj;
-    kq::gemm128<false>(gs, L, n, Y + (int64_t)k * n + NB * tj, n, C, n, M, NB, kb, -1.f, 1.f);
-  } else {
-    const int sj = tj - (p + 1);
-    if (sj > ti) return;
-    const int c0 = k + kb + NB * sj;
-    float* C = R + (int64_t)r0 * n + c0;
-    kq::gemm128<true>(gs, L, n, R + (int64_t)c0 * n + k, n, C, n, M, min(NB, n - c0), kb, -1.f, 1.f);
+// U[a][b] = Z[n-1-b][n-1-a] for a <= b, 0 below the diagonal (Z has leading
+// dimension np): an anti-transpose through 32 x 32 shared-memory tiles,
+// coalesced on both sides.
+__global__ void __launch_bounds__(256) reverse_out_kernel(const float* __restrict__ Z, int n,
+                                                          int np, float* __restrict__ U) {
+  __shared__ float tile[32][33];
+  const int ta = blockIdx.y * 32, tb = blockIdx.x * 32;     // U tile origin (rows a, cols b)
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;   // 8 rows per pass
+  for (int r = ty; r < 32; r += 8) {
+    const int b = tb + r, a = ta + 31 - tx;                 // Z row n-1-b, column n-1-a
+    float v = 0.f;
+    if (b < n && a < n) v = Z[(int64_t)(n - 1 - b) * np + (n - 1 - a)];
+    tile[r][31 - tx] = v;                                   // tile[b - tb][a - ta]
   }
-}
-
-// U[a][b] = Y[n-1-a][n-1-b] for a <= b, 0 below the diagonal.
-__global__ void reverse_out_kernel(const float* __restrict__ Y, int n, float* __restrict__ U) {
-  const int64_t total = (int64_t)n * n;
-  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
-       e += (int64_t)gridDim.x * blockDim.x) {
-    const int a = (int)(e / n), b = (int)(e % n);
-    U[e] = (a <= b) ? Y[(int64_t)(n - 1 - a) * n + (n - 1 - b)] : 0.f;
+  __syncthreads();
+  for (int r = ty; r < 32; r += 8) {
+    const int a = ta + r, b = tb + tx;
+    if (a < n && b < n) U[(int64_t)a * n + b] = (a <= b) ? tile[tx][r] : 0.f;
   }
 }
 
@@ -236,10 +287,13 @@ size_t align256(size_t b) { return (b + 255) & ~(size_t)255; }
 
 constexpr size_t kPanelSmem = (size_t)2 * NB * LDD * sizeof(float) + sizeof(kq::Gemm128Smem);
 
+int64_t padded(int64_t n) { return (n + NB - 1) / NB * NB; }
+
 }  // namespace
 
 size_t kq_cholesky_ws(int64_t n) {
-  return align256(sizeof(double)) + 2 * align256((size_t)n * n * sizeof(float));
+  const int64_t np = padded(n);
+  return align256(sizeof(double)) + 2 * align256((size_t)np * np * sizeof(float));
 }
 
 int kq_cholesky_inv(const float* H, int64_t n64, float damp_rel, float* U, int32_t* info, void* ws,
@@ -257,32 +311,40 @@ int kq_cholesky_inv(const float* H, int64_t n64, float damp_rel, float* U, int32
     attr = true;
   }
   const int n = (int)n64;
+  const int np = (int)padded(n64);
   uint8_t* w = static_cast<uint8_t*>(ws);
   double* dsum = reinterpret_cast<double*>(w);
   w += align256(sizeof(double));
   float* R = reinterpret_cast<float*>(w);
-  w += align256((size_t)n * n * sizeof(float));
-  float* Y = reinterpret_cast<float*>(w);
+  w += align256((size_t)np * np * sizeof(float));
+  float* Z = reinterpret_cast<float*>(w);
 
   const int sms = kqh::num_sms();
   diag_sum_kernel<<<1, 256, 0, st>>>(H, n, dsum);
   KQ_CHECK_LAUNCH();
-  reverse_damp_kernel<<<4 * sms, 256, 0, st>>>(H, n, R, Y, damp_rel, dsum);
+  reverse_damp_kernel<<<4 * sms, 256, 0, st>>>(H, n, np, R, Z, damp_rel, dsum);
   KQ_CHECK_LAUNCH();
-  const int nblk = (n + NB - 1) / NB;
+  const int nblk = np / NB;
   for (int p = 0; p < nblk; ++p) {
     const int k = p * NB;
-    const int kb = n - k < NB ? n - k : NB;
-    const int rest = n - k - kb;
-    const int tiles_L = (rest + NB - 1) / NB;
-    panel_kernel<<<tiles_L + p + 1, 256, kPanelSmem, st>>>(R, Y, n, k, p, tiles_L, info);
+    const int rest = np - k - NB;
+    const int tiles_L = rest / NB;
+    panel_kernel<<<tiles_L + p + 1, 256, kPanelSmem, st>>>(R, Z, np, k, p, tiles_L, info);
     KQ_CHECK_LAUNCH();
     if (rest > 0) {
-      update_kernel<<<dim3(p + 1 + tiles_L, tiles_L), 256, 0, st>>>(R, Y, n, k, p);
-      KQ_CHECK_LAUNCH();
+      // trailing update on the tensor cores, the panel rows L_ip = L as B:
+      //   R[k+128:, k+128:] -= L L^T                 (lower triangle)
+      //   Z[:k+128, k+128:] -= Z[:k+128, k:k+128] L^T
+      const float* L = R + (int64_t)(k + NB) * np + k;
+      kq::GemmNT g[2];
+      g[0] = {L, np, L, np, R + (int64_t)(k + NB) * np + (k + NB), np, rest, rest, NB, -1.f, 1};
+      g[1] = {Z + k, np, L, np, Z + (k + NB), np, k + NB, rest, NB, -1.f, 0};
+      const int s = kq_gemm_nt_tc(g, 2, info, st);
+      if (s != KRONQ_OK) return s;
     }
   }
-  reverse_out_kernel<<<4 * sms, 256, 0, st>>>(Y, n, U);
+  const dim3 og((n + 31) / 32, (n + 31) / 32);
+  reverse_out_kernel<<<og, 256, 0, st>>>(Z, n, np, U);
   KQ_CHECK_LAUNCH();
   return KRONQ_OK;
 }

@@ -1,0 +1,309 @@
+// C += alpha * A B^T on the 5th-generation tensor cores with fp32-level
+// accuracy (tf32, three-term split: tf32x3.cuh), for up to two problems
+// per launch.  A is M x K and B is N x K, both row-major, so both reach the
+// tensor core K-major straight from TMA; C is M x N row-major, updated in
+// place.  A problem may ask for its lower triangle only (M = N, tiles with
+// tile column > tile row skipped, diagonal tiles written on and below the
+// diagonal): the symmetric rank-K update of a Cholesky factorisation.
+//
+// Persistent kernel, one CTA per SM, 384 threads, 128 x 128 output tiles,
+// K streamed in 32-wide chunks through a 3-stage ring:
+//   warp 0       TMA loads of the A and B chunk of a stage (16 KB each)
+//   warps 2-3    split each landed chunk into hi (in place) and lo
+//   warp 1       one thread issues 3 MMAs (M = N = 128, K = 8) per K step
+//                into one of two TMEM accumulators
+//   warps 4-11   read an accumulator back and update C (loads of C issued
+//                before the accumulator is waited for)
+// All waits are bounded; a wait that gives up records KRONQ_ERR_TIMEOUT in
+// `info` and the CTA winds down.
+#include "gemm_tc.cuh"
+
+#include "tf32x3.cuh"
+
+namespace {
+
+using kq::tf32x3::KC;
+
+constexpr int TM = 128, TN = 128;
+constexpr int STAGES = 3;
+constexpr int CHUNK = TM * KC * 4;             // 16 KB: 128 rows x 32 fp32
+constexpr int STAGE_BYTES = 4 * CHUNK;         // A (hi after split), A lo, B (hi), B lo
+constexpr int THREADS = 384;
+constexpr int SPLITTERS = 64;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+constexpr int TMEM_COLS = 2 * TN;
+
+struct Bars {
+  uint64_t full[STAGES];
+  uint64_t lo[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+struct Maps {
+  CUtensorMap a[2];
+  CUtensorMap b[2];
+};
+
+struct Problem {
+  float* C;
+  int64_t ldc;
+  int M, N, K;
+  float alpha;
+  int lower;
+  int ntn;     // tile columns (rectangular problems)
+  int tiles;
+};
+
+struct Problems {
+  Problem p[2];
+  int count;
+  int total_tiles;
+};
+
+struct Tile {
+  int prob, tm, tn, kchunks;
+};
+
+__device__ __forceinline__ Tile tile_of(const Problems& P, int t) {
+  Tile r;
+  r.prob = (P.count > 1 && t >= P.p[0].tiles) ? 1 : 0;
+  if (r.prob) t -= P.p[0].tiles;
+  const Problem& q = P.p[r.prob];
+  if (q.lower) {
+    int tm = (int)((sqrtf(8.f * (float)t + 1.f) - 1.f) * 0.5f);
+    while ((tm + 1) * (tm + 2) / 2 <= t) ++tm;
+    while (tm * (tm + 1) / 2 > t) --tm;
+    r.tm = tm;
+    r.tn = t - tm * (tm + 1) / 2;
+  } else {
+    r.tm = t / q.ntn;
+    r.tn = t % q.ntn;
+  }
+  r.kchunks = (q.K + KC - 1) / KC;
+  return r;
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+gemm_nt_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Problems P,
+                  int32_t* info) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* stages = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  Bars* bars = reinterpret_cast<Bars*>(stages + STAGES * STAGE_BYTES);
+  volatile int* abort = &bars->abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      kq::mbar_init(&bars->full[s], 1);
+      kq::mbar_init(&bars->lo[s], SPLITTERS);
+      kq::mbar_init(&bars->empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      kq::mbar_init(&bars->tfull[b], 1);
+      kq::mbar_init(&bars->tempty[b], 8);
+    }
+    kq::mbar_init(&bars->drain, 1);
+    bars->abort = 0;
+    kq::fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    for (int i = 0; i < P.count; ++i) {
+      kq::prefetch_tmap(&maps.a[i]);
+      kq::prefetch_tmap(&maps.b[i]);
+    }
+  }
+  if (warp == 2) kq::tmem_alloc(&bars->tmem_base, TMEM_COLS);
+  kq::tc_fence_before();
+  __syncthreads();
+  kq::tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------ TMA producer
+      int it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < P.total_tiles && ok; t += gridDim.x) {
+        const Tile tl = tile_of(P, t);
+        for (int kc = 0; kc < tl.kchunks; ++kc, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+          if (!kq::mbar_wait(&bars->empty[s], ph ^ 1u, abort, info)) { ok = false; break; }
+          uint8_t* st = stages + s * STAGE_BYTES;
+          kq::mbar_arrive_expect_tx(&bars->full[s], 2 * CHUNK);
+          kq::tma_load_2d(st, &maps.a[tl.prob], &bars->full[s], kc * KC, tl.tm * TM);
+          kq::tma_load_2d(st + 2 * CHUNK, &maps.b[tl.prob], &bars->full[s], kc * KC, tl.tn * TN);
+        }
+      }
+      // wait for the copies still in flight before the CTA can exit
+      for (int s = 0; s < STAGES; ++s) {
+        const int armed = (it > s) ? (it - s + STAGES - 1) / STAGES : 0;
+        if (armed > 0) kq::tf32x3::drain_wait(&bars->full[s], (uint32_t)(armed - 1) & 1u, info);
+      }
+    }
+  } else if (warp == 2 || warp == 3) {
+    // ------------------------------------------------------ hi / lo split
+    const int t0 = (warp - 2) * 32 + lane;
+    int it = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < P.total_tiles && ok; t += gridDim.x) {
+      const Tile tl = tile_of(P, t);
+      for (int kc = 0; kc < tl.kchunks; ++kc, ++it) {
+        const int s = it % STAGES;
+        const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+        if (!kq::mbar_wait(&bars->full[s], ph, abort, info)) { ok = false; break; }
+        uint8_t* st = stages + s * STAGE_BYTES;
+        kq::tf32x3::split_smem(st, st + CHUNK, CHUNK / 16, t0, SPLITTERS);
+        kq::tf32x3::split_smem(st + 2 * CHUNK, st + 3 * CHUNK, CHUNK / 16, t0, SPLITTERS);
+        kq::mbar_arrive(&bars->lo[s]);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------ MMA issuer
+      int it = 0, tcount = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < P.total_tiles && ok; t += gridDim.x, ++tcount) {
+        const Tile tl = tile_of(P, t);
+        const int buf = tcount & 1;
+        const uint32_t aph = (uint32_t)(tcount >> 1) & 1u;
+        if (!kq::mbar_wait(&bars->tempty[buf], aph ^ 1u, abort, info)) break;
+        kq::tc_fence_after();
+        const uint32_t d_tmem = tmem + (uint32_t)(buf * TN);
+        for (int kc = 0; kc < tl.kchunks; ++kc, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+          if (!kq::mbar_wait(&bars->lo[s], ph, abort, info)) { ok = false; break; }
+          kq::tc_fence_after();
+          const uint32_t a = kq::smem_u32(stages + s * STAGE_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < KC / 8; ++kk)
+            kq::tf32x3::mma3(d_tmem, a, a + CHUNK, a + 2 * CHUNK, a + 3 * CHUNK, kk,
+                             (kc == 0 && kk == 0) ? 0u : 1u);
+          kq::mma_commit(&bars->empty[s]);
+        }
+        if (ok) kq::mma_commit(&bars->tfull[buf]);
+      }
+      kq::mma_commit(&bars->drain);
+      kq::tf32x3::drain_wait(&bars->drain, 0, info);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------ epilogue: C += alpha acc
+    // warp w: TMEM lane quadrant w % 4 (tile rows), columns [64 h, 64 h + 64)
+    const int q = warp & 3, h = (warp - 4) >> 2;
+    int tcount = 0;
+    for (int t = blockIdx.x; t < P.total_tiles; t += gridDim.x, ++tcount) {
+      const Tile tl = tile_of(P, t);
+      const Problem& pr = P.p[tl.prob];
+      const int buf = tcount & 1;
+      const uint32_t aph = (uint32_t)(tcount >> 1) & 1u;
+      const int row = tl.tm * TM + q * 32 + lane;
+      const int cbase = tl.tn * TN + 64 * h;
+      // columns this thread may write: below M, below N, and on / below the
+      // diagonal in a lower-triangle problem's diagonal tile
+      int cend = min(pr.N, cbase + 64);
+      if (pr.lower && tl.tm == tl.tn) cend = min(cend, row + 1);
+      const bool full = row < pr.M && cend == cbase + 64;
+      float4 c[16];
+      float* crow = pr.C + (int64_t)row * pr.ldc + cbase;
+      if (full) {
+        const float4* src = reinterpret_cast<const float4*>(crow);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) c[k] = src[k];
+      }
+      if (!kq::mbar_wait(&bars->tfull[buf], aph, abort, info)) break;
+      kq::tc_fence_after();
+      float v[64];
+      {
+        float v0[32], v1[32];
+        __syncwarp();
+        const uint32_t ta = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * TN + 64 * h);
+        kq::tmem_ld32(ta, v0);
+        kq::tmem_ld32(ta + 32, v1);
+        kq::tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 32; ++k) { v[k] = v0[k]; v[32 + k] = v1[k]; }
+      }
+      kq::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) kq::mbar_arrive(&bars->tempty[buf]);
+      const float al = pr.alpha;
+      if (full) {
+        float4* dst = reinterpret_cast<float4*>(crow);
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+          dst[k] = make_float4(fmaf(al, v[4 * k], c[k].x), fmaf(al, v[4 * k + 1], c[k].y),
+                               fmaf(al, v[4 * k + 2], c[k].z), fmaf(al, v[4 * k + 3], c[k].w));
+      } else if (row < pr.M) {
+#pragma unroll
+        for (int k = 0; k < 64; ++k)
+          if (cbase + k < cend) crow[k] = fmaf(al, v[k], crow[k]);
+      }
+    }
+  }
+
+  kq::tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    kq::tc_fence_after();
+    kq::tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+}  // namespace
+
+int kq_gemm_nt_tc(const kq::GemmNT* probs, int count, int32_t* info, cudaStream_t st) {
+  if (count < 1 || count > 2) return KRONQ_ERR_INVALID_ARG;
+  Maps maps;
+  Problems P;
+  P.count = 0;
+  P.total_tiles = 0;
+  for (int i = 0; i < count; ++i) {
+    const kq::GemmNT& g = probs[i];
+    if (g.M <= 0 || g.N <= 0 || g.K <= 0) continue;
+    if (!g.A || !g.B || !g.C || g.lda % 4 || g.ldb % 4 || g.ldc % 4 ||
+        !kqh::aligned(g.A, 16) || !kqh::aligned(g.B, 16) || !kqh::aligned(g.C, 16))
+      return KRONQ_ERR_INVALID_ARG;
+    if (g.lower && g.M != g.N) return KRONQ_ERR_INVALID_ARG;
+    const int j = P.count;
+    if (!kqh::make_map_f32(&maps.a[j], g.A, g.K, g.M, g.lda, KC, TM) ||
+        !kqh::make_map_f32(&maps.b[j], g.B, g.K, g.N, g.ldb, KC, TN))
+      return KRONQ_ERR_CUDA;
+    Problem& q = P.p[j];
+    q.C = g.C;
+    q.ldc = g.ldc;
+    q.M = g.M;
+    q.N = g.N;
+    q.K = g.K;
+    q.alpha = g.alpha;
+    q.lower = g.lower;
+    const int ntm = (g.M + TM - 1) / TM;
+    q.ntn = (g.N + TN - 1) / TN;
+    q.tiles = g.lower ? ntm * (ntm + 1) / 2 : ntm * q.ntn;
+    P.total_tiles += q.tiles;
+    ++P.count;
+  }
+  if (P.count == 0) return KRONQ_OK;
+  if (P.count == 1) {
+    maps.a[1] = maps.a[0];
+    maps.b[1] = maps.b[0];
+    P.p[1] = P.p[0];
+  }
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(gemm_nt_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SMEM_BYTES) != cudaSuccess)
+      return KRONQ_ERR_CUDA;
+    attr = true;
+  }
+  const int grid = P.total_tiles < kqh::num_sms() ? P.total_tiles : kqh::num_sms();
+  gemm_nt_tc_kernel<<<grid, THREADS, SMEM_BYTES, st>>>(maps, P, info);
+  KQ_CHECK_LAUNCH();
+  return KRONQ_OK;
+}

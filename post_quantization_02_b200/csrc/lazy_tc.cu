@@ -20,12 +20,14 @@
 // warp 1 issues the MMAs (M = 128, N = 128, K = 8, three per K-step) into one
 // of two TMEM accumulators; warps 4-11 read the accumulator back and update
 // W in place, with the tile's W loads issued ahead of the MMAs.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
-#include "common.cuh"
+#include "tf32x3.cuh"
 
 namespace {
+
+using kq::tf32x3::drain_wait;
+using kq::tf32x3::fence_to_tensor_core;
+using kq::tf32x3::swz128;
+using kq::tf32x3::split_smem;
 
 constexpr int TM = 128, TN = 128, KB = 128;  // tile rows, tile columns, block width (K)
 constexpr int KC = 32;                        // K values per 128-byte swizzle row of fp32
@@ -39,9 +41,6 @@ constexpr int THREADS = 384;
 constexpr int SPLITTERS = 64;                 // warps 2 and 3
 constexpr int SMEM_BYTES = B_BYTES + STAGES * STAGE_BYTES + 1024 + 256;
 constexpr int TMEM_COLS = 2 * TN;
-// kind::tf32: formats 2 = TF32, A and B K-major
-constexpr uint32_t IDESC = (1u << 4) | (2u << 7) | (2u << 10) | (0u << 15) | (0u << 16) |
-                           ((uint32_t)(TN >> 3) << 17) | ((uint32_t)(TM >> 4) << 24);
 
 struct Bars {
   uint64_t ufull;            // U tile landed (MN-major, in the stage area)
@@ -55,47 +54,6 @@ struct Bars {
   uint32_t tmem_base;
   int abort;
 };
-
-__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                         uint32_t accumulate) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(IDESC), "r"(accumulate)
-      : "memory");
-}
-
-// Byte address inside a tile of 128-byte rows written with the 128-byte
-// swizzle (16-byte chunk index XOR row mod 8); tiles are 1024-byte aligned.
-__device__ __forceinline__ int swz128(int row, int byte) {
-  return row * 128 + ((((byte >> 4) ^ (row & 7)) << 4) | (byte & 15));
-}
-
-__device__ __forceinline__ float tf32_hi(float v) {
-  return __uint_as_float(__float_as_uint(v) & 0xFFFFE000u);
-}
-
-__device__ __forceinline__ void fence_to_tensor_core() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-// In place: hi = x with its low 13 mantissa bits cleared (exactly a tf32
-// value, so the tensor core uses it unchanged whatever its own conversion
-// does), and lo = x - hi (exact in fp32) into dst; n4 float4 by `nthreads`.
-__device__ __forceinline__ void split_lo_smem(uint8_t* src, uint8_t* dst, int n4, int t,
-                                              int nthreads) {
-  float4* s4 = reinterpret_cast<float4*>(src);
-  float4* d4 = reinterpret_cast<float4*>(dst);
-  for (int e = t; e < n4; e += nthreads) {
-    const float4 v = s4[e];
-    float4 h, o;
-    h.x = tf32_hi(v.x); h.y = tf32_hi(v.y); h.z = tf32_hi(v.z); h.w = tf32_hi(v.w);
-    o.x = v.x - h.x; o.y = v.y - h.y; o.z = v.z - h.z; o.w = v.w - h.w;
-    s4[e] = h;
-    d4[e] = o;
-  }
-  fence_to_tensor_core();
-}
 
 // The U tile (K = 128 rows of U, 128 columns) lands MN-major as 4 K-chunks x
 // 4 boxes of 32 K-rows x 32 columns; it is split into hi / lo and transposed
@@ -111,24 +69,13 @@ __device__ __forceinline__ void split_transpose_u(const uint8_t* land, uint8_t* 
     const float vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const float h = tf32_hi(vv[j]);
+      const float h = kq::tf32x3::hi(vv[j]);
       const int d = kc * KTILE + swz128(4 * nq + j, kk * 4);
       *reinterpret_cast<float*>(hi + d) = h;
       *reinterpret_cast<float*>(lo + d) = vv[j] - h;
     }
   }
   fence_to_tensor_core();
-}
-
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, int32_t* info) {
-  if (kq::mbar_try_wait(bar, parity)) return;
-  unsigned long long t0 = kq::globaltimer();
-  while (!kq::mbar_try_wait(bar, parity)) {
-    if (kq::globaltimer() - t0 > kq::kWaitLimitNs) {
-      kq::record_error(info, KRONQ_ERR_TIMEOUT);
-      return;
-    }
-  }
 }
 
 // CTA (tn, r): column tile tn of W[:, i2:], row blocks r, r + R, ...
@@ -215,7 +162,7 @@ lazy_tc_kernel(const __grid_constant__ CUtensorMap tm_e, const __grid_constant__
           const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
           if (!kq::mbar_wait(&bars->full[s], ph, abort, info)) { ok = false; break; }
           uint8_t* st = stages + s * STAGE_BYTES;
-          split_lo_smem(st, st + KTILE, KTILE / 16, t, SPLITTERS);
+          split_smem(st, st + KTILE, KTILE / 16, t, SPLITTERS);
           kq::mbar_arrive(&bars->lo[s]);
         }
       }
@@ -241,17 +188,9 @@ lazy_tc_kernel(const __grid_constant__ CUtensorMap tm_e, const __grid_constant__
           kq::tc_fence_after();
           const uint32_t ah = kq::smem_u32(stages + s * STAGE_BYTES), al = ah + KTILE;
 #pragma unroll
-          for (int kk = 0; kk < KC / 8; ++kk) {
-            // K-major, 128-byte swizzle, 8-row atoms 1024 B apart; K step of 8 = 32 B
-            const uint64_t a_h = kq::smem_desc(ah + kk * 32, 16, 1024, kq::kLayoutSwizzle128B);
-            const uint64_t a_l = kq::smem_desc(al + kk * 32, 16, 1024, kq::kLayoutSwizzle128B);
-            const uint64_t b_h = kq::smem_desc(bh + kc * KTILE + kk * 32, 16, 1024, kq::kLayoutSwizzle128B);
-            const uint64_t b_l = kq::smem_desc(bl + kc * KTILE + kk * 32, 16, 1024, kq::kLayoutSwizzle128B);
-            const uint32_t first = (kc == 0 && kk == 0) ? 0u : 1u;
-            mma_tf32(d_tmem, a_l, b_h, first);
-            mma_tf32(d_tmem, a_h, b_l, 1u);
-            mma_tf32(d_tmem, a_h, b_h, 1u);
-          }
+          for (int kk = 0; kk < KC / 8; ++kk)
+            kq::tf32x3::mma3(d_tmem, ah, al, bh + kc * KTILE, bl + kc * KTILE, kk,
+                             (kc == 0 && kk == 0) ? 0u : 1u);
           kq::mma_commit(&bars->empty[s]);
         }
         if (ok) kq::mma_commit(&bars->tfull[buf]);
@@ -316,32 +255,6 @@ lazy_tc_kernel(const __grid_constant__ CUtensorMap tm_e, const __grid_constant__
   }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return nullptr;
-    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
-bool make_map(CUtensorMap* map, const float* ptr, int64_t cols, int64_t rows, uint32_t box_cols,
-              uint32_t box_rows) {
-  auto enc = encode_fn();
-  if (!enc) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)cols * 4};
-  cuuint32_t box[2] = {box_cols, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(ptr), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 }  // namespace
 
 // W[:, i1+128:] -= E U[i1:i1+128, i1+128:] with E: m x 128, U: n x n (both fp32, row-major).
@@ -350,7 +263,8 @@ int kq_lazy_update_tc(float* W, int64_t m, int64_t n, const float* E, const floa
   const int64_t i2 = i1 + KB;
   if (i2 >= n) return KRONQ_OK;
   CUtensorMap me, mu;
-  if (!make_map(&me, E, KB, m, KC, TM) || !make_map(&mu, U, n, n, 32, KC)) return KRONQ_ERR_CUDA;
+  if (!kqh::make_map_f32(&me, E, KB, m, KB, KC, TM) || !kqh::make_map_f32(&mu, U, n, n, n, 32, KC))
+    return KRONQ_ERR_CUDA;
   static bool attr = false;
   if (!attr) {
     if (cudaFuncSetAttribute(lazy_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

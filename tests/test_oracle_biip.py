@@ -122,3 +122,23 @@ def test_rotation_spreads_a_spike():
     _, HXp, _ = biip.rotate(np.zeros((4, n)), HX, np.eye(4), _signs(r, 4), _signs(r, n))
     d = np.diag(HXp)
     np.testing.assert_allclose(d, np.full(n, np.trace(HX) / n), rtol=1e-12)
+
+
+@pytest.mark.parametrize("m,n", [(56, 64), (16, 344), (86, 28)])
+@pytest.mark.parametrize("mode", ["full", "no_rescale", "su_only", "sv_only"])
+def test_sampled_entries_equal_the_whole_transform(m, n, mode):
+    """The selected-entries form (used at widths where the whole fp64
+    transform is too slow) equals rescale + rotate, including odd factors."""
+    r = np.random.default_rng(m * n)
+    W = r.standard_normal((m, n)) * np.exp(r.uniform(-1, 1, n))[None, :]
+    HX, HG = _spd(r, n), _spd(r, m)
+    su, sv = _signs(r, m), _signs(r, n)
+    Wp, HXp, HGp, SX, SG = biip.biip(W, HX, HG, su, sv, 0.25, mode)
+    wr, wc = r.choice(m, 7, replace=False), r.choice(n, 9, replace=False)
+    hx, hg = r.choice(n, 11, replace=False), r.choice(m, 5, replace=False)
+    Wb, HXb, HGb, SXs, SGs = biip.biip_entries(W, HX, HG, su, sv, 0.25, mode, wr, wc, hx, hg)
+    np.testing.assert_allclose(SXs, SX, rtol=1e-14)
+    np.testing.assert_allclose(SGs, SG, rtol=1e-14)
+    np.testing.assert_allclose(Wb, Wp[np.ix_(wr, wc)], rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(HXb, HXp[np.ix_(hx, hx)], rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(HGb, HGp[np.ix_(hg, hg)], rtol=1e-10, atol=1e-12)

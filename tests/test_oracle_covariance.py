@@ -89,3 +89,11 @@ def test_vec_is_column_stacking(bad):
     assert list(cov.vec(M)) == [1, 4, 2, 5, 3, 6]
     g, x = np.array([1.0, 2.0]), np.array([3.0, 4.0, 5.0])
     np.testing.assert_array_equal(cov.vec(np.outer(g, x)), np.kron(x, g))
+
+
+def test_streamed_diagonal_matches_the_covariance():
+    r = np.random.default_rng(4)
+    A = r.standard_normal((301, 37))
+    chunks = [A[:100], A[100:101], A[101:]]
+    np.testing.assert_allclose(cov.covariance_diag(chunks, 37, 301), np.diag(cov.covariance(A)),
+                               rtol=1e-13)

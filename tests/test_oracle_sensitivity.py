@@ -67,3 +67,16 @@ def test_allocation_on_llama3_block_sizes_mixes_2_3_4():
     scores = [1, 2, 3, 4, 7, 6, 5]        # q k v o gate up down
     bits = S.allocate_bits(scores, params, 3.0)
     assert set(bits) == {2, 3, 4}
+
+
+def test_score_from_diagonals_equals_score_after_biip():
+    r = np.random.default_rng(3)
+    m, n = 24, 56
+    HX, HG = _spd(r, n), _spd(r, m, 2.0)
+    W = r.standard_normal((m, n)) * np.exp(r.uniform(-1, 1, n))[None, :]
+    su = (1 - 2 * r.integers(0, 2, m)).astype(np.int8)
+    sv = (1 - 2 * r.integers(0, 2, n)).astype(np.int8)
+    for mode in ("full", "sv_only", "su_only", "no_rescale"):
+        _, HXt, HGt, SX, SG = biip.biip(W, HX, HG, su, sv, 0.25, mode)
+        np.testing.assert_allclose(S.sensitivity_from_diagonals(np.diag(HX), np.diag(HG), SX, SG),
+                                   S.sensitivity(HXt, HGt), rtol=1e-12)

@@ -237,3 +237,24 @@ def test_layer_loss_matches_kronecker_quadratic_form():
     HX, HG = _spd(r, n), _spd(r, m)
     v = dW.reshape(-1, order="F")
     np.testing.assert_allclose(Q.layer_loss(dW, HX, HG), v @ np.kron(HX, HG) @ v, rtol=1e-12)
+
+
+@pytest.mark.parametrize("n,k", [(40, 0), (40, 17), (64, 63), (100, 36)])
+def test_inverse_cholesky_trailing_block(n, k):
+    """U[k:, k:] depends on H[k:, k:] only (upper factor of the inverse)."""
+    r = np.random.default_rng(n + k)
+    H = _spd(r, n)
+    np.testing.assert_allclose(C.inverse_cholesky_trailing(H, k, 0.01),
+                               C.inverse_cholesky(C.damp(H, 0.01))[k:, k:], rtol=1e-9, atol=1e-12)
+
+
+def test_row_losses_damping_argument_and_fp32_input():
+    r = np.random.default_rng(21)
+    n = 2100                                   # more than one 2048-row panel
+    H = _spd(r, n)
+    dW = r.standard_normal((3, n))
+    ref = np.einsum("ij,jk,ik->i", dW, C.damp(H, 0.01), dW)
+    np.testing.assert_allclose(Q.row_losses(dW, H, 0.01), ref, rtol=1e-11)
+    H32 = H.astype(np.float32)
+    np.testing.assert_allclose(Q.row_losses(dW, H32), np.einsum("ij,jk,ik->i", dW, H32.astype(np.float64), dW),
+                               rtol=1e-11)

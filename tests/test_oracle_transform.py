@@ -70,3 +70,11 @@ def test_power_of_two_is_normalized_hadamard():
     d = 16
     s = np.ones(d, dtype=np.int8)
     np.testing.assert_allclose(T.dense(d, s), T.sylvester(4) / 4.0, atol=1e-15)
+
+
+@pytest.mark.parametrize("d", [8, 56, 344, 112])
+def test_selected_rows_match_the_dense_matrix(d):
+    r = np.random.default_rng(d)
+    s = np.where(r.random(d) < 0.5, -1.0, 1.0)
+    idx = r.choice(d, min(d, 9), replace=False)
+    np.testing.assert_allclose(T.rows(d, idx, s), T.dense(d, s)[idx], atol=1e-13)
