@@ -23,13 +23,23 @@
 //                  Z[:k+128, k+128:] -= Z[:k+128, k:k+128] L^T, L = the panel rows.
 // Then U_c[a][b] = Z[n-1-b][n-1-a] (a <= b).
 #include "common.cuh"
-#include "gemm_simt.cuh"
 #include "gemm_tc.cuh"
+#include "tf32x3.cuh"
 
 namespace {
 
 constexpr int NB = 128;
-constexpr int LDD = NB + 1;   // padded leading dimension of the diagonal block in smem
+constexpr int LDD = NB + 1;   // D: odd row stride, column reads are conflict-free
+constexpr int LDX = NB + 4;   // X and the panel tile P: 16-byte rows for float4 reads
+constexpr int LDA = 100;      // As: K-major copy of the 32 columns just factored (<= 96 rows)
+constexpr int LDY = 36;       // YT: the 32 x 32 inverse block, transposed
+// shared memory of the panel kernel, in floats
+constexpr int SM_D = 0;
+constexpr int SM_X = SM_D + NB * LDD;
+constexpr int SM_P = SM_X + NB * LDX;
+constexpr int SM_AS = SM_P + 32 * LDX;
+constexpr int SM_YT = SM_AS + 32 * LDA;
+constexpr int SM_FLOATS = SM_YT + 32 * LDY;
 
 __global__ void diag_sum_kernel(const float* __restrict__ H, int n, double* out) {
   __shared__ double red[256];
@@ -69,14 +79,15 @@ __global__ void reverse_damp_kernel(const float* __restrict__ H, int n, int np,
 }
 
 // One warp factors the 32 x 32 diagonal block at offset o of D (lower part
-// valid, already updated) and inverts the factor: on return D holds L_oo
-// and X holds L_oo^-1 (both lower).  Lane i keeps row i of the block in
-// registers; pivot step j needs no barrier: the pivot comes from lane j,
-// the column L[:, j] and the row j of L^-1 travel by shuffles.
-//   L[i][j] = a_i[j] r,  r = 1 / sqrt(a_j[j])
-//   a_i[c] -= L[i][j] L[c][j]            (c > j, the Schur complement)
-//   Y[j][:] = y_j[:] r,  y_i[:] -= L[i][j] Y[j][:]   (i > j, rows of L^-1)
-__device__ __forceinline__ void warp_leaf32(float* D, float* X, int o, int kb, int* bad) {
+// valid, already updated) and inverts the factor: on return D holds L_oo,
+// X holds Y_oo = L_oo^-1 and YT its transpose.  Lane i keeps row i of the
+// block and row i of the accumulating inverse in registers; pivot step j
+// needs no barrier, the pivot, the column L[:, j] and the finished row j of
+// the inverse travel by shuffles:
+//   L[i][j] = a_i[j] r,  r = 1 / sqrt(a_j[j]),   a_i[c] -= L[i][j] L[c][j]  (c > j)
+//   Y[j][:] = y_j[:] r,  y_i[:] -= L[i][j] Y[j][:]                          (i > j)
+__device__ __forceinline__ void warp_leaf32(float* D, float* X, float* YT, int o, int kb,
+                                            int* bad) {
   const int i = threadIdx.x & 31;
   constexpr unsigned FULL = 0xffffffffu;
   float a[32], y[32];
@@ -95,6 +106,7 @@ __device__ __forceinline__ void warp_leaf32(float* D, float* X, int o, int kb, i
     const float r = rsqrtf(d);
     const float l = (i >= j) ? a[j] * r : 0.f;
     a[j] = l;
+    // the next pivot's column first: it is on the critical path
 #pragma unroll
     for (int c = j + 1; c < 32; ++c) a[c] = fmaf(-l, __shfl_sync(FULL, l, c), a[c]);
 #pragma unroll
@@ -107,8 +119,9 @@ __device__ __forceinline__ void warp_leaf32(float* D, float* X, int o, int kb, i
   for (int c = 0; c < 32; ++c) {
     if (c <= i) {
       D[(o + i) * LDD + o + c] = a[c];
-      X[(o + i) * LDD + o + c] = y[c];
+      X[(o + i) * LDX + o + c] = y[c];
     }
+    YT[c * LDY + i] = (c <= i) ? y[c] : 0.f;   // YT[c][i] = Y[i][c]
   }
 }
 
@@ -121,62 +134,65 @@ __device__ __forceinline__ void warp_leaf32(float* D, float* X, int o, int kb, i
 // (block forward substitution of L Y = I, accumulators in X below the
 // diagonal blocks):
 //   1. warp 0: L_bb and Y_bb = L_bb^-1                          (warp_leaf32)
-//   2. L_cb = D_cb Y_bb^T (c > b);  Y_bj = Y_bb Acc_bj (j < b)
+//   2. L_cb = D_cb Y_bb^T (c > b), also kept K-major in As;  Y_bj = Y_bb Acc_bj (j < b)
 //   3. D_cd -= L_cb L_db^T (b < d <= c);  Acc_cj -= L_cb Y_bj (c > b, j <= b)
-// Steps 2 and 3 are small GEMMs out of shared memory, register-tiled.
-__device__ void factor_and_invert(float* D, float* X, int kb, int* bad) {
+// Steps 2 and 3 are small register-tiled GEMMs out of shared memory whose
+// wide operands are read as contiguous float4 rows (YT, As, rows of X).
+__device__ void factor_and_invert(float* D, float* X, float* As, float* YT, int kb, int* bad) {
   const int tid = threadIdx.x;
-  for (int e = tid; e < NB * LDD; e += blockDim.x) X[e] = 0.f;
+  for (int e = tid; e < NB * LDX; e += blockDim.x) X[e] = 0.f;
   __syncthreads();
   for (int b = 0; b < NB / 32; ++b) {
     const int o = 32 * b;
     const int o2 = o + 32;
     const int R1 = NB - o2;                 // rows below the diagonal block
-    if (tid < 32) warp_leaf32(D, X, o, kb, bad);
+    if (tid < 32) warp_leaf32(D, X, YT, o, kb, bad);
     __syncthreads();
     // ---- step 2: thread (tr, tc) = (tid / 8, tid % 8)
     {
       const int tr = tid >> 3, tc = tid & 7;
+      const int nj = o >> 3;                // Y_bj columns per thread: o / 8
       float acc1[3][4], acc2[12];
-      // L_cb rows o2 + tr + 32 s, columns o + 4 tc .. +3
 #pragma unroll
       for (int s = 0; s < 3; ++s)
 #pragma unroll
         for (int q = 0; q < 4; ++q) acc1[s][q] = 0.f;
 #pragma unroll
       for (int q = 0; q < 12; ++q) acc2[q] = 0.f;
-      const int nj = o >> 3;                // Y_bj columns per thread: o / 8
 #pragma unroll 4
       for (int t = 0; t < 32; ++t) {
-        float bv[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) bv[q] = X[(o + 4 * tc + q) * LDD + o + t];   // Y_bb[c][t]
+        const float4 bv = *reinterpret_cast<const float4*>(&YT[t * LDY + 4 * tc]);   // Y_bb[4tc+q][t]
 #pragma unroll
         for (int s = 0; s < 3; ++s) {
           if (32 * s < R1) {
             const float av = D[(o2 + tr + 32 * s) * LDD + o + t];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) acc1[s][q] = fmaf(av, bv[q], acc1[s][q]);
+            acc1[s][0] = fmaf(av, bv.x, acc1[s][0]);
+            acc1[s][1] = fmaf(av, bv.y, acc1[s][1]);
+            acc1[s][2] = fmaf(av, bv.z, acc1[s][2]);
+            acc1[s][3] = fmaf(av, bv.w, acc1[s][3]);
           }
         }
-        const float yv = X[(o + tr) * LDD + o + t];                            // Y_bb[r][t]
+        const float yv = X[(o + tr) * LDX + o + t];                            // Y_bb[tr][t]
 #pragma unroll
         for (int q = 0; q < 12; ++q)
-          if (q < nj) acc2[q] = fmaf(yv, X[(o + t) * LDD + tc * nj + q], acc2[q]);   // Acc[t][c']
+          if (q < nj) acc2[q] = fmaf(yv, X[(o + t) * LDX + tc * nj + q], acc2[q]);   // Acc[t][c']
       }
       __syncthreads();
 #pragma unroll
       for (int s = 0; s < 3; ++s)
         if (32 * s < R1)
 #pragma unroll
-          for (int q = 0; q < 4; ++q) D[(o2 + tr + 32 * s) * LDD + o + 4 * tc + q] = acc1[s][q];
+          for (int q = 0; q < 4; ++q) {
+            D[(o2 + tr + 32 * s) * LDD + o + 4 * tc + q] = acc1[s][q];
+            As[(4 * tc + q) * LDA + tr + 32 * s] = acc1[s][q];
+          }
 #pragma unroll
       for (int q = 0; q < 12; ++q)
-        if (q < nj) X[(o + tr) * LDD + tc * nj + q] = acc2[q];
+        if (q < nj) X[(o + tr) * LDX + tc * nj + q] = acc2[q];
       __syncthreads();
     }
     if (R1 == 0) break;
-    // ---- step 3: rows o2 + tr + 16 s, columns 8 tc .. 8 tc + 7 (all 128)
+    // ---- step 3: rows o2 + tr * ns + s, columns 8 tc .. 8 tc + 7 (all 128)
     {
       const int tr = tid >> 4, tc = tid & 15;
       const int ns = R1 >> 4;               // 6, 4 or 2 rows per thread
@@ -187,20 +203,17 @@ __device__ void factor_and_invert(float* D, float* X, int kb, int* bad) {
         for (int q = 0; q < 8; ++q) acc[s][q] = 0.f;
       const int c0 = 8 * tc;
       const bool left = c0 < o2;            // Acc / Y columns (j <= b), else trailing D
+      const float* Bp = left ? &X[o * LDX + c0] : &As[c0 - o2];
+      const int ldb = left ? LDX : LDA;
 #pragma unroll 2
       for (int t = 0; t < 32; ++t) {
-        float bv[8];
-        if (left) {
-#pragma unroll
-          for (int q = 0; q < 8; ++q) bv[q] = X[(o + t) * LDD + c0 + q];          // Y_b[t][c]
-        } else {
-#pragma unroll
-          for (int q = 0; q < 8; ++q) bv[q] = D[(c0 + q) * LDD + o + t];          // L[c][o+t]
-        }
+        const float4 b0 = *reinterpret_cast<const float4*>(Bp + t * ldb);
+        const float4 b1 = *reinterpret_cast<const float4*>(Bp + t * ldb + 4);
+        const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
         for (int s = 0; s < 6; ++s) {
           if (s < ns) {
-            const float av = D[(o2 + tr + 16 * s) * LDD + o + t];
+            const float av = As[t * LDA + tr * ns + s];                          // L[o2+r][o+t]
 #pragma unroll
             for (int q = 0; q < 8; ++q) acc[s][q] = fmaf(av, bv[q], acc[s][q]);
           }
@@ -209,11 +222,15 @@ __device__ void factor_and_invert(float* D, float* X, int kb, int* bad) {
 #pragma unroll
       for (int s = 0; s < 6; ++s) {
         if (s < ns) {
-          const int r = o2 + tr + 16 * s;
-          float* dst = left ? &X[r * LDD + c0] : &D[r * LDD + c0];
+          const int r = o2 + tr * ns + s;
+          if (left) {
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
-            if (left || c0 + q <= r) dst[q] -= acc[s][q];
+            for (int q = 0; q < 8; ++q) X[r * LDX + c0 + q] -= acc[s][q];
+          } else {
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              if (c0 + q <= r) D[r * LDD + c0 + q] -= acc[s][q];
+          }
         }
       }
       __syncthreads();
@@ -221,44 +238,127 @@ __device__ void factor_and_invert(float* D, float* X, int kb, int* bad) {
   }
 }
 
-__global__ void __launch_bounds__(256, 1) panel_kernel(float* R, float* Z, int n, int k, int p,
-                                                    int tiles_L, int32_t* info) {
-  extern __shared__ float sm[];
-  float* D = sm;                       // [NB][LDD]
-  float* X = sm + NB * LDD;            // [NB][LDD]
-  kq::Gemm128Smem& gs = *reinterpret_cast<kq::Gemm128Smem*>(sm + 2 * NB * LDD);
+KQ_DEV void bulk_copy_row(float* dst, const float* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          kq::smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(kq::smem_u32(bar))
+      : "memory");
+}
+
+// Write v to a row of fp32 and to its tf32 hi / lo planes.
+KQ_DEV void put_split(float* hi_plane, float* lo_plane, int64_t idx, float v) {
+  const float h = kq::tf32x3::hi(v);
+  hi_plane[idx] = h;
+  lo_plane[idx] = v - h;
+}
+
+// Panel step p (rows / columns k = 128 p ...) of the padded np x np matrices,
+// in 32-row slices (PR rows per CTA):
+//   CTA b < tiles_L:        L_ip = R_ip L_pp^-T for rows k+128+32b ..
+//                           -> the hi / lo planes Lh, Ll (np x 128, row 0 = row k+128)
+//   CTA tiles_L + j, j < 4p: Z_jp = B_jp L_pp^-T for Z rows 32j .. -> Z and the
+//                           planes Zh, Zl (row = Z row)
+//   CTA tiles_L + 4p:       Z_pp = L_pp^-T      -> Z and the planes
+// Every CTA first factors and inverts the diagonal block in shared memory;
+// the 32 x 128 slice it multiplies is fetched by bulk copies meanwhile.
+constexpr int PR = 32;
+
+__global__ void __launch_bounds__(256, 1) panel_kernel(const float* R, float* Z, float* Lh,
+                                                    float* Ll, float* Zh, float* Zl, int np, int k,
+                                                    int p, int tiles_L, int32_t* info) {
+  extern __shared__ __align__(16) float sm[];
+  float* D = sm + SM_D;
+  float* X = sm + SM_X;
+  float* P = sm + SM_P;
+  float* As = sm + SM_AS;
+  float* YT = sm + SM_YT;
   __shared__ int bad;
-  const int kb = min(NB, n - k);
-  if (threadIdx.x == 0) bad = 0;
-  for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
-    const int i = e / NB, j = e % NB;
-    float v = 0.f;
-    if (i < kb && j <= i) v = R[(int64_t)(k + i) * n + (k + j)];
-    else if (i == j) v = 1.f;
-    D[i * LDD + j] = v;
+  __shared__ int abort_flag;
+  __shared__ __align__(8) uint64_t pbar;
+  const int tid = threadIdx.x;
+  const int role_L = (int)blockIdx.x < tiles_L;
+  const int j = (int)blockIdx.x - tiles_L;
+  const bool has_tile = role_L || j < 4 * p;
+  const float* src = role_L ? R + (int64_t)(k + NB + PR * blockIdx.x) * np + k
+                            : Z + (int64_t)(PR * (j < 4 * p ? j : 0)) * np + k;
+  if (tid == 0) {
+    bad = 0;
+    abort_flag = 0;
+    kq::mbar_init(&pbar, 1);
+    kq::fence_barrier_init();
   }
   __syncthreads();
-  factor_and_invert(D, X, kb, &bad);
-  if (blockIdx.x == 0 && threadIdx.x == 0 && bad) kq::record_error(info, KRONQ_ERR_NOT_PD);
+  if (tid == 0 && has_tile) {
+    kq::mbar_arrive_expect_tx(&pbar, PR * NB * 4);
+    for (int r = 0; r < PR; ++r) bulk_copy_row(P + r * LDX, src + (int64_t)r * np, NB * 4, &pbar);
+  }
+  for (int e = tid; e < NB * NB; e += blockDim.x) {
+    const int i = e / NB, c = e % NB;
+    D[i * LDD + c] = (c <= i) ? R[(int64_t)(k + i) * np + (k + c)] : 0.f;
+  }
+  __syncthreads();
+  factor_and_invert(D, X, As, YT, NB, &bad);
+  if (blockIdx.x == 0 && tid == 0 && bad) kq::record_error(info, KRONQ_ERR_NOT_PD);
 
-  if ((int)blockIdx.x < tiles_L) {
-    // 128 rows of the panel: L_ip = R_ip L_pp^-T (in place)
-    const int r0 = k + kb + NB * blockIdx.x;
-    float* P = R + (int64_t)r0 * n + k;
-    kq::gemm128<true>(gs, P, n, X, LDD, P, n, n - r0 < NB ? n - r0 : NB, kb, kb, 1.f, 0.f);
-  } else {
-    const int j = blockIdx.x - tiles_L;  // row block of Z's column block p
-    if (j < p) {
-      // Z_jp = Acc_jp L_pp^-T (in place)
-      float* B = Z + (int64_t)(NB * j) * n + k;
-      kq::gemm128<true>(gs, B, n, X, LDD, B, n, NB, kb, kb, 1.f, 0.f);
-    } else {
-      // Z_pp = L_pp^-T (upper; X is zero above its diagonal)
-      for (int e = threadIdx.x; e < kb * kb; e += blockDim.x) {
-        const int a = e / kb, b = e % kb;
-        Z[(int64_t)(k + a) * n + k + b] = X[b * LDD + a];
-      }
+  if (!has_tile) {
+    // Z_pp = X^T (upper; X is zero above its diagonal)
+    for (int e = tid; e < NB * NB; e += blockDim.x) {
+      const int a = e / NB, c = e % NB;
+      const float v = X[c * LDX + a];
+      Z[(int64_t)(k + a) * np + k + c] = v;
+      put_split(Zh, Zl, (int64_t)(k + a) * NB + c, v);
     }
+    return;
+  }
+  if (!kq::mbar_wait(&pbar, 0, &abort_flag, info)) {
+    // give the copies in flight a bounded time to land before the CTA exits
+    kq::tf32x3::drain_wait(&pbar, 0, info);
+    return;
+  }
+  // C = P X^T (32 x 128): thread (ty, tx) owns rows ty, ty + 16 and columns tx + 16 jj
+  const int ty = tid >> 4, tx = tid & 15;
+  float acc[2][8];
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) acc[i][jj] = 0.f;
+#pragma unroll 4
+  for (int kk = 0; kk < NB; kk += 4) {
+    float4 pa[2], xb[8];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) pa[i] = *reinterpret_cast<const float4*>(&P[(ty + 16 * i) * LDX + kk]);
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj)
+      xb[jj] = *reinterpret_cast<const float4*>(&X[(tx + 16 * jj) * LDX + kk]);
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) {
+        acc[i][jj] = fmaf(pa[i].x, xb[jj].x, acc[i][jj]);
+        acc[i][jj] = fmaf(pa[i].y, xb[jj].y, acc[i][jj]);
+        acc[i][jj] = fmaf(pa[i].z, xb[jj].z, acc[i][jj]);
+        acc[i][jj] = fmaf(pa[i].w, xb[jj].w, acc[i][jj]);
+      }
+  }
+  if (role_L) {
+    const int64_t r0 = (int64_t)PR * blockIdx.x;      // plane row of this slice's first row
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj)
+        put_split(Lh, Ll, (r0 + ty + 16 * i) * NB + tx + 16 * jj, acc[i][jj]);
+  } else {
+    const int64_t r0 = (int64_t)PR * j;
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) {
+        const int64_t r = r0 + ty + 16 * i;
+        const int c = tx + 16 * jj;
+        Z[r * np + k + c] = acc[i][jj];
+        put_split(Zh, Zl, r * NB + c, acc[i][jj]);
+      }
   }
 }
 
@@ -285,7 +385,7 @@ __global__ void __launch_bounds__(256) reverse_out_kernel(const float* __restric
 
 size_t align256(size_t b) { return (b + 255) & ~(size_t)255; }
 
-constexpr size_t kPanelSmem = (size_t)2 * NB * LDD * sizeof(float) + sizeof(kq::Gemm128Smem);
+constexpr size_t kPanelSmem = (size_t)SM_FLOATS * sizeof(float);
 
 int64_t padded(int64_t n) { return (n + NB - 1) / NB * NB; }
 
@@ -293,7 +393,8 @@ int64_t padded(int64_t n) { return (n + NB - 1) / NB * NB; }
 
 size_t kq_cholesky_ws(int64_t n) {
   const int64_t np = padded(n);
-  return align256(sizeof(double)) + 2 * align256((size_t)np * np * sizeof(float));
+  return align256(sizeof(double)) + 2 * align256((size_t)np * np * sizeof(float)) +
+         4 * align256((size_t)np * NB * sizeof(float));
 }
 
 int kq_cholesky_inv(const float* H, int64_t n64, float damp_rel, float* U, int32_t* info, void* ws,
@@ -318,6 +419,13 @@ int kq_cholesky_inv(const float* H, int64_t n64, float damp_rel, float* U, int32
   float* R = reinterpret_cast<float*>(w);
   w += align256((size_t)np * np * sizeof(float));
   float* Z = reinterpret_cast<float*>(w);
+  w += align256((size_t)np * np * sizeof(float));
+  float* planes[4];
+  for (int i = 0; i < 4; ++i) {
+    planes[i] = reinterpret_cast<float*>(w);
+    w += align256((size_t)np * NB * sizeof(float));
+  }
+  float *Lh = planes[0], *Ll = planes[1], *Zh = planes[2], *Zl = planes[3];
 
   const int sms = kqh::num_sms();
   diag_sum_kernel<<<1, 256, 0, st>>>(H, n, dsum);
@@ -328,17 +436,18 @@ int kq_cholesky_inv(const float* H, int64_t n64, float damp_rel, float* U, int32
   for (int p = 0; p < nblk; ++p) {
     const int k = p * NB;
     const int rest = np - k - NB;
-    const int tiles_L = rest / NB;
-    panel_kernel<<<tiles_L + p + 1, 256, kPanelSmem, st>>>(R, Z, np, k, p, tiles_L, info);
+    const int tiles_L = rest / PR;
+    panel_kernel<<<tiles_L + 4 * p + 1, 256, kPanelSmem, st>>>(R, Z, Lh, Ll, Zh, Zl, np, k, p,
+                                                               tiles_L, info);
     KQ_CHECK_LAUNCH();
     if (rest > 0) {
-      // trailing update on the tensor cores, the panel rows L_ip = L as B:
+      // trailing update on the tensor cores, B = the panel rows L_ip (planes):
       //   R[k+128:, k+128:] -= L L^T                 (lower triangle)
       //   Z[:k+128, k+128:] -= Z[:k+128, k:k+128] L^T
-      const float* L = R + (int64_t)(k + NB) * np + k;
       kq::GemmNT g[2];
-      g[0] = {L, np, L, np, R + (int64_t)(k + NB) * np + (k + NB), np, rest, rest, NB, -1.f, 1};
-      g[1] = {Z + k, np, L, np, Z + (k + NB), np, k + NB, rest, NB, -1.f, 0};
+      g[0] = {Lh, Ll, NB, Lh, Ll, NB, R + (int64_t)(k + NB) * np + (k + NB), np, rest, rest, NB,
+              -1.f, 1};
+      g[1] = {Zh, Zl, NB, Lh, Ll, NB, Z + (k + NB), np, k + NB, rest, NB, -1.f, 0};
       const int s = kq_gemm_nt_tc(g, 2, info, st);
       if (s != KRONQ_OK) return s;
     }

@@ -1,18 +1,19 @@
 // C += alpha * A B^T on the 5th-generation tensor cores with fp32-level
 // accuracy (tf32, three-term split: tf32x3.cuh), for up to two problems
-// per launch.  A is M x K and B is N x K, both row-major, so both reach the
-// tensor core K-major straight from TMA; C is M x N row-major, updated in
-// place.  A problem may ask for its lower triangle only (M = N, tiles with
-// tile column > tile row skipped, diagonal tiles written on and below the
-// diagonal): the symmetric rank-K update of a Cholesky factorisation.
+// per launch.  A (M x K) and B (N x K) come pre-split: each as a hi plane
+// (tf32-exact) and a lo plane (the fp32 remainder), all row-major, so all
+// four reach the tensor core K-major straight from TMA.  C is M x N
+// row-major, updated in place.  A problem may ask for its lower triangle
+// only (M = N, tiles with tile column > tile row skipped, diagonal tiles
+// written on and below the diagonal): the symmetric rank-K update of a
+// Cholesky factorisation.
 //
-// Persistent kernel, one CTA per SM, 384 threads, 128 x 128 output tiles,
+// Persistent kernel, one CTA per SM, 320 threads, 128 x 128 output tiles,
 // K streamed in 32-wide chunks through a 3-stage ring:
-//   warp 0       TMA loads of the A and B chunk of a stage (16 KB each)
-//   warps 2-3    split each landed chunk into hi (in place) and lo
+//   warp 0       TMA loads of A_hi, A_lo, B_hi, B_lo of a stage (16 KB each)
 //   warp 1       one thread issues 3 MMAs (M = N = 128, K = 8) per K step
 //                into one of two TMEM accumulators
-//   warps 4-11   read an accumulator back and update C (loads of C issued
+//   warps 2-9    read an accumulator back and update C (loads of C issued
 //                before the accumulator is waited for)
 // All waits are bounded; a wait that gives up records KRONQ_ERR_TIMEOUT in
 // `info` and the CTA winds down.
@@ -27,15 +28,14 @@ using kq::tf32x3::KC;
 constexpr int TM = 128, TN = 128;
 constexpr int STAGES = 3;
 constexpr int CHUNK = TM * KC * 4;             // 16 KB: 128 rows x 32 fp32
-constexpr int STAGE_BYTES = 4 * CHUNK;         // A (hi after split), A lo, B (hi), B lo
-constexpr int THREADS = 384;
-constexpr int SPLITTERS = 64;
+constexpr int STAGE_BYTES = 4 * CHUNK;         // A hi, A lo, B hi, B lo
+constexpr int THREADS = 320;
+constexpr int EPI_WARP0 = 2;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
 constexpr int TMEM_COLS = 2 * TN;
 
 struct Bars {
   uint64_t full[STAGES];
-  uint64_t lo[STAGES];
   uint64_t empty[STAGES];
   uint64_t tfull[2];
   uint64_t tempty[2];
@@ -45,8 +45,8 @@ struct Bars {
 };
 
 struct Maps {
-  CUtensorMap a[2];
-  CUtensorMap b[2];
+  CUtensorMap a_hi[2], a_lo[2];
+  CUtensorMap b_hi[2], b_lo[2];
 };
 
 struct Problem {
@@ -101,7 +101,6 @@ gemm_nt_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Pro
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       kq::mbar_init(&bars->full[s], 1);
-      kq::mbar_init(&bars->lo[s], SPLITTERS);
       kq::mbar_init(&bars->empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -114,11 +113,13 @@ gemm_nt_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Pro
   }
   if (warp == 0 && lane == 0) {
     for (int i = 0; i < P.count; ++i) {
-      kq::prefetch_tmap(&maps.a[i]);
-      kq::prefetch_tmap(&maps.b[i]);
+      kq::prefetch_tmap(&maps.a_hi[i]);
+      kq::prefetch_tmap(&maps.a_lo[i]);
+      kq::prefetch_tmap(&maps.b_hi[i]);
+      kq::prefetch_tmap(&maps.b_lo[i]);
     }
   }
-  if (warp == 2) kq::tmem_alloc(&bars->tmem_base, TMEM_COLS);
+  if (warp == EPI_WARP0) kq::tmem_alloc(&bars->tmem_base, TMEM_COLS);
   kq::tc_fence_before();
   __syncthreads();
   kq::tc_fence_after();
@@ -136,32 +137,18 @@ gemm_nt_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Pro
           const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
           if (!kq::mbar_wait(&bars->empty[s], ph ^ 1u, abort, info)) { ok = false; break; }
           uint8_t* st = stages + s * STAGE_BYTES;
-          kq::mbar_arrive_expect_tx(&bars->full[s], 2 * CHUNK);
-          kq::tma_load_2d(st, &maps.a[tl.prob], &bars->full[s], kc * KC, tl.tm * TM);
-          kq::tma_load_2d(st + 2 * CHUNK, &maps.b[tl.prob], &bars->full[s], kc * KC, tl.tn * TN);
+          kq::mbar_arrive_expect_tx(&bars->full[s], 4 * CHUNK);
+          const int x = kc * KC, ya = tl.tm * TM, yb = tl.tn * TN;
+          kq::tma_load_2d(st, &maps.a_hi[tl.prob], &bars->full[s], x, ya);
+          kq::tma_load_2d(st + CHUNK, &maps.a_lo[tl.prob], &bars->full[s], x, ya);
+          kq::tma_load_2d(st + 2 * CHUNK, &maps.b_hi[tl.prob], &bars->full[s], x, yb);
+          kq::tma_load_2d(st + 3 * CHUNK, &maps.b_lo[tl.prob], &bars->full[s], x, yb);
         }
       }
       // wait for the copies still in flight before the CTA can exit
       for (int s = 0; s < STAGES; ++s) {
         const int armed = (it > s) ? (it - s + STAGES - 1) / STAGES : 0;
         if (armed > 0) kq::tf32x3::drain_wait(&bars->full[s], (uint32_t)(armed - 1) & 1u, info);
-      }
-    }
-  } else if (warp == 2 || warp == 3) {
-    // ------------------------------------------------------ hi / lo split
-    const int t0 = (warp - 2) * 32 + lane;
-    int it = 0;
-    bool ok = true;
-    for (int t = blockIdx.x; t < P.total_tiles && ok; t += gridDim.x) {
-      const Tile tl = tile_of(P, t);
-      for (int kc = 0; kc < tl.kchunks; ++kc, ++it) {
-        const int s = it % STAGES;
-        const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-        if (!kq::mbar_wait(&bars->full[s], ph, abort, info)) { ok = false; break; }
-        uint8_t* st = stages + s * STAGE_BYTES;
-        kq::tf32x3::split_smem(st, st + CHUNK, CHUNK / 16, t0, SPLITTERS);
-        kq::tf32x3::split_smem(st + 2 * CHUNK, st + 3 * CHUNK, CHUNK / 16, t0, SPLITTERS);
-        kq::mbar_arrive(&bars->lo[s]);
       }
     }
   } else if (warp == 1) {
@@ -179,7 +166,7 @@ gemm_nt_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Pro
         for (int kc = 0; kc < tl.kchunks; ++kc, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-          if (!kq::mbar_wait(&bars->lo[s], ph, abort, info)) { ok = false; break; }
+          if (!kq::mbar_wait(&bars->full[s], ph, abort, info)) { ok = false; break; }
           kq::tc_fence_after();
           const uint32_t a = kq::smem_u32(stages + s * STAGE_BYTES);
 #pragma unroll
@@ -193,10 +180,11 @@ gemm_nt_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Pro
       kq::mma_commit(&bars->drain);
       kq::tf32x3::drain_wait(&bars->drain, 0, info);
     }
-  } else if (warp >= 4) {
+  } else {
     // ------------------------------------------------------ epilogue: C += alpha acc
-    // warp w: TMEM lane quadrant w % 4 (tile rows), columns [64 h, 64 h + 64)
-    const int q = warp & 3, h = (warp - 4) >> 2;
+    // warp w: TMEM lane quadrant w % 4 (tile rows; a warp may only read its
+    // own quadrant), columns [64 h, 64 h + 64)
+    const int q = warp & 3, h = (warp - EPI_WARP0) >> 2;
     int tcount = 0;
     for (int t = blockIdx.x; t < P.total_tiles; t += gridDim.x, ++tcount) {
       const Tile tl = tile_of(P, t);
@@ -250,7 +238,7 @@ gemm_nt_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Pro
 
   kq::tc_fence_before();
   __syncthreads();
-  if (warp == 2) {
+  if (warp == EPI_WARP0) {
     kq::tc_fence_after();
     kq::tmem_dealloc(tmem, TMEM_COLS);
   }
@@ -267,13 +255,16 @@ int kq_gemm_nt_tc(const kq::GemmNT* probs, int count, int32_t* info, cudaStream_
   for (int i = 0; i < count; ++i) {
     const kq::GemmNT& g = probs[i];
     if (g.M <= 0 || g.N <= 0 || g.K <= 0) continue;
-    if (!g.A || !g.B || !g.C || g.lda % 4 || g.ldb % 4 || g.ldc % 4 ||
-        !kqh::aligned(g.A, 16) || !kqh::aligned(g.B, 16) || !kqh::aligned(g.C, 16))
+    if (!g.A_hi || !g.A_lo || !g.B_hi || !g.B_lo || !g.C || g.lda % 4 || g.ldb % 4 || g.ldc % 4 ||
+        !kqh::aligned(g.A_hi, 16) || !kqh::aligned(g.A_lo, 16) || !kqh::aligned(g.B_hi, 16) ||
+        !kqh::aligned(g.B_lo, 16) || !kqh::aligned(g.C, 16))
       return KRONQ_ERR_INVALID_ARG;
     if (g.lower && g.M != g.N) return KRONQ_ERR_INVALID_ARG;
     const int j = P.count;
-    if (!kqh::make_map_f32(&maps.a[j], g.A, g.K, g.M, g.lda, KC, TM) ||
-        !kqh::make_map_f32(&maps.b[j], g.B, g.K, g.N, g.ldb, KC, TN))
+    if (!kqh::make_map_f32(&maps.a_hi[j], g.A_hi, g.K, g.M, g.lda, KC, TM) ||
+        !kqh::make_map_f32(&maps.a_lo[j], g.A_lo, g.K, g.M, g.lda, KC, TM) ||
+        !kqh::make_map_f32(&maps.b_hi[j], g.B_hi, g.K, g.N, g.ldb, KC, TN) ||
+        !kqh::make_map_f32(&maps.b_lo[j], g.B_lo, g.K, g.N, g.ldb, KC, TN))
       return KRONQ_ERR_CUDA;
     Problem& q = P.p[j];
     q.C = g.C;
@@ -290,11 +281,7 @@ int kq_gemm_nt_tc(const kq::GemmNT* probs, int count, int32_t* info, cudaStream_
     ++P.count;
   }
   if (P.count == 0) return KRONQ_OK;
-  if (P.count == 1) {
-    maps.a[1] = maps.a[0];
-    maps.b[1] = maps.b[0];
-    P.p[1] = P.p[0];
-  }
+  if (P.count == 1) P.p[1] = P.p[0];
   static bool attr = false;
   if (!attr) {
     if (cudaFuncSetAttribute(gemm_nt_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

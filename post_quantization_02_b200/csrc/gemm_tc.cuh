@@ -6,14 +6,19 @@
 
 namespace kq {
 
-// C (M x N, row-major, ldc) += alpha * A B^T with A M x K (lda) and B N x K
-// (ldb), both row-major.  lower = 1: M == N and only the lower triangle of C
-// (tile by tile, the diagonal tiles on and below the diagonal) is updated.
-// Pointers 16-byte aligned, leading dimensions multiples of 4.
+// C (M x N, row-major, ldc) += alpha * A B^T with A M x K and B N x K, both
+// row-major and given pre-split: A = A_hi + A_lo with A_hi exactly a tf32
+// value (the low 13 mantissa bits clear) and A_lo the fp32 remainder, the
+// two planes sharing the leading dimension lda (B likewise, ldb).
+// lower = 1: M == N and only the lower triangle of C (tile by tile, the
+// diagonal tiles on and below the diagonal) is updated.  Pointers 16-byte
+// aligned, leading dimensions multiples of 4.
 struct GemmNT {
-  const float* A;
+  const float* A_hi;
+  const float* A_lo;
   int64_t lda;
-  const float* B;
+  const float* B_hi;
+  const float* B_lo;
   int64_t ldb;
   float* C;
   int64_t ldc;
