@@ -13,15 +13,16 @@
 // segment of L2 consecutive entries: Walsh-Hadamard butterflies; across the
 // Q segments: a dense Q x Q mix.
 //
-// Passes over HBM: a row pass (one CTA per row, the row staged in shared
-// memory, scaling and signs fused into the load) and a column pass (64-row..
-// 4096-row segments of 8-column panels in shared memory, then the Q-mix).
+// Passes over HBM: a row pass (per row segment: butterflies in registers,
+// scaling and signs fused into the load; rows with an odd factor: the row
+// staged in shared memory with the Q-mix) and a column pass (each thread
+// one column of a group of rows in registers, two launches for segments
+// longer than 64 rows, then the Q-mix).
 #include "common.cuh"
 
 namespace {
 
 constexpr int RT_THREADS = 256;
-constexpr int CP_COLS = 8;  // columns per panel in the column pass (shifts below assume 8)
 
 struct Split {
   int L2, Q, q, k1;
@@ -173,45 +174,6 @@ row_transform_kernel(float* __restrict__ X, int R, int C, const float* __restric
   }
 }
 
-// Column pass, step 1: Walsh-Hadamard along rows inside each L2-row segment,
-// on a panel of CP_COLS columns (signs of the rows first when forward, last
-// when inverse; normalized by 1/sqrt(L2)).
-__global__ void __launch_bounds__(256)
-col_fht_kernel(float* __restrict__ X, int R, int C, const int8_t* __restrict__ sign, int L2,
-               int inverse) {
-  extern __shared__ float p[];  // [L2][CP_COLS]
-  const int seg = blockIdx.y, c0 = blockIdx.x * CP_COLS;
-  const int r0 = seg * L2;
-  const float norm = rsqrtf((float)L2);
-  for (int e = threadIdx.x; e < L2 * CP_COLS; e += blockDim.x) {
-    const int rr = e >> 3, cc = e & (CP_COLS - 1);
-    float v = 0.f;
-    if (c0 + cc < C) v = X[(int64_t)(r0 + rr) * C + c0 + cc];
-    if (!inverse) v *= (float)sign[r0 + rr];
-    p[e] = v;
-  }
-  __syncthreads();
-  const int half = L2 >> 1;
-  for (int lh = 0; (1 << lh) < L2; ++lh) {
-    const int h = 1 << lh;
-    for (int e = threadIdx.x; e < half * CP_COLS; e += blockDim.x) {
-      const int pr = e >> 3, cc = e & (CP_COLS - 1);   // CP_COLS == 8
-      const int i = ((pr >> lh) << (lh + 1)) | (pr & (h - 1));
-      const float a = p[i * CP_COLS + cc], b = p[(i + h) * CP_COLS + cc];
-      p[i * CP_COLS + cc] = a + b;
-      p[(i + h) * CP_COLS + cc] = a - b;
-    }
-    __syncthreads();
-  }
-  for (int e = threadIdx.x; e < L2 * CP_COLS; e += blockDim.x) {
-    const int rr = e >> 3, cc = e & (CP_COLS - 1);
-    if (c0 + cc >= C) continue;
-    float v = p[e] * norm;
-    if (inverse) v *= (float)sign[r0 + rr];
-    X[(int64_t)(r0 + rr) * C + c0 + cc] = v;
-  }
-}
-
 // Column pass, step 2: rows {s L2 + r : s < Q} mixed by M (or M^T), 64 columns per CTA.
 __global__ void __launch_bounds__(64)
 col_mix_kernel(float* __restrict__ X, int C, int L2, int Q, const float* __restrict__ M,
@@ -227,6 +189,139 @@ col_mix_kernel(float* __restrict__ X, int C, int L2, int Q, const float* __restr
     float acc = 0.f;
     for (int t = 0; t < Q; ++t) acc = fmaf(transpose ? Ms[t * Q + s] : Ms[s * Q + t], v[t][threadIdx.x], acc);
     X[(int64_t)(s * L2 + r) * C + c] = acc;
+  }
+}
+
+// Row pass, fast path (one segment of L2 = 128 E entries per CTA, no odd
+// factor): Walsh-Hadamard butterflies in registers.  Thread t first holds
+// entries t + 128 k (coalesced loads; scaling and signs fused), which makes
+// the stages with h >= 128 thread-local; one padded shared-memory transpose
+// gives it entries E t .. E t + E - 1 for the stages h < E; the stages
+// E <= h < 128 pair thread t with t ^ (h / E) by shuffles.
+template <int E>
+__global__ void __launch_bounds__(128)
+row_fht_kernel(float* __restrict__ X, int C, const float* __restrict__ rs,
+               const float* __restrict__ cs, const int8_t* __restrict__ sign, int inverse) {
+  constexpr int L2 = 128 * E;
+  __shared__ float sm[L2 + L2 / 32];
+  const int t = threadIdx.x;
+  const int64_t r = blockIdx.x;
+  const int c0 = blockIdx.y * L2;
+  float* base = X + r * C + c0;
+  const float rsc = rs ? rs[r] : 1.f;
+  float v[E];
+#pragma unroll
+  for (int k = 0; k < E; ++k) {
+    const int c = c0 + t + 128 * k;
+    float x = base[t + 128 * k];
+    if (!inverse) x = x * (rsc * (cs ? cs[c] : 1.f)) * (float)sign[c];
+    v[k] = x;
+  }
+#pragma unroll
+  for (int h = 1; h < E; h <<= 1)
+#pragma unroll
+    for (int k = 0; k < E; ++k)
+      if (!(k & h)) {
+        const float a = v[k], b = v[k + h];
+        v[k] = a + b;
+        v[k + h] = a - b;
+      }
+#pragma unroll
+  for (int k = 0; k < E; ++k) {
+    const int i = t + 128 * k;
+    sm[i + (i >> 5)] = v[k];
+  }
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < E; ++k) {
+    const int i = E * t + k;
+    v[k] = sm[i + (i >> 5)];
+  }
+#pragma unroll
+  for (int h = 1; h < E; h <<= 1)
+#pragma unroll
+    for (int k = 0; k < E; ++k)
+      if (!(k & h)) {
+        const float a = v[k], b = v[k + h];
+        v[k] = a + b;
+        v[k + h] = a - b;
+      }
+#pragma unroll
+  for (int m = 1; m < 128 / E; m <<= 1) {
+    const bool upper = (t & m) != 0;
+#pragma unroll
+    for (int k = 0; k < E; ++k) {
+      const float o = __shfl_xor_sync(0xffffffffu, v[k], m);
+      v[k] = upper ? (o - v[k]) : (v[k] + o);
+    }
+  }
+  const float norm = rsqrtf((float)L2);
+#pragma unroll
+  for (int k = 0; k < E; ++k) {
+    const int c = c0 + E * t + k;
+    float x = v[k] * norm;
+    if (inverse) x = x * (float)sign[c] * (rsc * (cs ? cs[c] : 1.f));
+    v[k] = x;
+  }
+#pragma unroll
+  for (int k = 0; k < E; k += 4)
+    *reinterpret_cast<float4*>(base + E * t + k) = make_float4(v[k], v[k + 1], v[k + 2], v[k + 3]);
+}
+
+// Column pass, one factor H_{NR} (NR = 2^LG <= 64) of the Walsh-Hadamard
+// transform along rows, in registers: each thread owns one column and the
+// NR rows row(s) = seg L2 + hi (st NR) + lo + s st, s < NR, of one group
+// (coalesced row segments, no shared memory).  With st = 1 the groups are
+// NR consecutive rows; with st = 2^a and NR = L2 / st the rows with stride
+// st, so the two launches (I (x) H_{2^a}) then (H_{L2/2^a} (x) I) make the
+// whole H_{L2}.  first: signs of the rows before (forward); last: the
+// 1/sqrt(L2) normalisation and, when inverse, the signs after.
+template <int LG>
+__global__ void __launch_bounds__(128)
+col_fht_reg_kernel(float* __restrict__ X, int C, int L2, int st, const int8_t* __restrict__ sign,
+                   int first, int last, int inverse) {
+  constexpr int NR = 1 << LG;
+  const int c = blockIdx.x * 128 + threadIdx.x;
+  if (c >= C) return;
+  const int groups_per_seg = L2 / NR;
+  const int seg = blockIdx.y / groups_per_seg, g = blockIdx.y % groups_per_seg;
+  const int hi = g / st, lo = g % st;
+  const int64_t r0 = (int64_t)seg * L2 + (int64_t)hi * st * NR + lo;
+  const int64_t step = (int64_t)st * C;
+  float v[NR];
+  {
+    const float* p = X + r0 * C + c;
+#pragma unroll
+    for (int s = 0; s < NR; ++s) {
+      v[s] = *p;
+      p += step;
+    }
+  }
+  if (first && !inverse) {
+    const int8_t* sg = sign + r0;
+#pragma unroll
+    for (int s = 0; s < NR; ++s) v[s] = (sg[(int64_t)s * st] < 0) ? -v[s] : v[s];
+  }
+#pragma unroll
+  for (int h = 1; h < NR; h <<= 1)
+#pragma unroll
+    for (int s = 0; s < NR; ++s)
+      if (!(s & h)) {
+        const float a = v[s], b = v[s + h];
+        v[s] = a + b;
+        v[s + h] = a - b;
+      }
+  const float norm = last ? rsqrtf((float)L2) : 1.f;
+  if (last && inverse) {
+    const int8_t* sg = sign + r0;
+#pragma unroll
+    for (int s = 0; s < NR; ++s) v[s] = (sg[(int64_t)s * st] < 0) ? -v[s] : v[s];
+  }
+  float* p = X + r0 * C + c;
+#pragma unroll
+  for (int s = 0; s < NR; ++s) {
+    *p = v[s] * norm;
+    p += step;
   }
 }
 
@@ -255,7 +350,7 @@ __global__ void sensitivity_kernel(const float* __restrict__ HX, int n, const fl
 
 size_t a256(size_t b) { return (b + 255) & ~(size_t)255; }
 
-bool g_row_attr = false, g_col_attr = false;
+bool g_row_attr = false;
 
 int set_attrs() {
   if (!g_row_attr) {
@@ -264,18 +359,23 @@ int set_attrs() {
       return KRONQ_ERR_CUDA;
     g_row_attr = true;
   }
-  if (!g_col_attr) {
-    if (cudaFuncSetAttribute(col_fht_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             4096 * CP_COLS * 4) != cudaSuccess)
-      return KRONQ_ERR_CUDA;
-    g_col_attr = true;
-  }
   return KRONQ_OK;
 }
 
 // Apply T D along rows (row pass, with scaling) of an R x C matrix.
 int row_pass(float* X, int R, int C, const float* rs, const float* cs, const int8_t* sign,
              const Split& sp, const float* M, int inverse, cudaStream_t st) {
+  if (sp.Q == 1 && sp.L2 >= 512) {
+    const dim3 g(R, C / sp.L2);
+    switch (sp.L2) {
+      case 512: row_fht_kernel<4><<<g, 128, 0, st>>>(X, C, rs, cs, sign, inverse); break;
+      case 1024: row_fht_kernel<8><<<g, 128, 0, st>>>(X, C, rs, cs, sign, inverse); break;
+      case 2048: row_fht_kernel<16><<<g, 128, 0, st>>>(X, C, rs, cs, sign, inverse); break;
+      default: row_fht_kernel<32><<<g, 128, 0, st>>>(X, C, rs, cs, sign, inverse); break;
+    }
+    KQ_CHECK_LAUNCH();
+    return KRONQ_OK;
+  }
   const size_t smem = (size_t)C * sizeof(float);
   if (smem > 200 * 1024) return KRONQ_ERR_UNSUPPORTED;
   row_transform_kernel<<<R, RT_THREADS, smem, st>>>(X, R, C, rs, cs, sign, sp.L2, sp.Q, M, inverse);
@@ -283,22 +383,44 @@ int row_pass(float* X, int R, int C, const float* rs, const float* cs, const int
   return KRONQ_OK;
 }
 
-// Apply T D along columns of an R x C matrix (R = Q * L2).
+// One launch of col_fht_reg_kernel<lg> over every segment of an R x C matrix.
+int col_fht_launch(float* X, int R, int C, int L2, int lg, int stride, const int8_t* sign,
+                   int first, int last, int inverse, cudaStream_t st) {
+  const dim3 g((C + 127) / 128, R >> lg);
+  switch (lg) {
+    case 1: col_fht_reg_kernel<1><<<g, 128, 0, st>>>(X, C, L2, stride, sign, first, last, inverse); break;
+    case 2: col_fht_reg_kernel<2><<<g, 128, 0, st>>>(X, C, L2, stride, sign, first, last, inverse); break;
+    case 3: col_fht_reg_kernel<3><<<g, 128, 0, st>>>(X, C, L2, stride, sign, first, last, inverse); break;
+    case 4: col_fht_reg_kernel<4><<<g, 128, 0, st>>>(X, C, L2, stride, sign, first, last, inverse); break;
+    case 5: col_fht_reg_kernel<5><<<g, 128, 0, st>>>(X, C, L2, stride, sign, first, last, inverse); break;
+    case 6: col_fht_reg_kernel<6><<<g, 128, 0, st>>>(X, C, L2, stride, sign, first, last, inverse); break;
+    default: return KRONQ_ERR_UNSUPPORTED;
+  }
+  KQ_CHECK_LAUNCH();
+  return KRONQ_OK;
+}
+
+// Apply T D along columns of an R x C matrix (R = Q * L2): the Hadamard part
+// as H_{2^a} within groups of 2^a consecutive rows, then (when L2 > 64)
+// H_{L2 / 2^a} across them; the odd factor as a Q x Q mix of the segments.
 int col_pass(float* X, int R, int C, const int8_t* sign, const Split& sp, const float* M,
              int inverse, cudaStream_t st) {
-  const dim3 g1((C + CP_COLS - 1) / CP_COLS, sp.Q);
-  const size_t smem = (size_t)sp.L2 * CP_COLS * sizeof(float);
   if (inverse && sp.Q > 1) {
     col_mix_kernel<<<dim3((C + 63) / 64, sp.L2), 64, 0, st>>>(X, C, sp.L2, sp.Q, M, 1);
     KQ_CHECK_LAUNCH();
   }
-  col_fht_kernel<<<g1, 256, smem, st>>>(X, R, C, sign, sp.L2, inverse);
-  KQ_CHECK_LAUNCH();
+  const int k2 = 31 - __builtin_clz((unsigned)sp.L2);
+  const int a = k2 < 6 ? k2 : 6, b = k2 - a;
+  int s = col_fht_launch(X, R, C, sp.L2, a, 1, sign, 1, b == 0, inverse, st);
+  if (s != KRONQ_OK) return s;
+  if (b > 0) {
+    s = col_fht_launch(X, R, C, sp.L2, b, 1 << a, sign, 0, 1, inverse, st);
+    if (s != KRONQ_OK) return s;
+  }
   if (!inverse && sp.Q > 1) {
     col_mix_kernel<<<dim3((C + 63) / 64, sp.L2), 64, 0, st>>>(X, C, sp.L2, sp.Q, M, 0);
     KQ_CHECK_LAUNCH();
   }
-  (void)R;
   return KRONQ_OK;
 }
 

@@ -93,9 +93,13 @@ def _biip_case(r, m, n):
     return W, spd(r, n), spd(r, m), signs(r, m), signs(r, n)
 
 
-@pytest.mark.parametrize("m,n", [(256, 256), (64, 112), (688, 96), (128, 448), (32, 8192),
-                                 (4096, 64), (112, 11008 // 8)])
-@pytest.mark.parametrize("mode", ["full", "no_rescale", "su_only", "sv_only"])
+_BIIP_SHAPES = [(256, 256), (64, 112), (688, 96), (128, 448), (4096, 64), (112, 11008 // 8),
+                (1024, 512), (2048, 128), (64, 2048)]
+
+
+@pytest.mark.parametrize("m,n,mode", [(m, n, mode) for m, n in _BIIP_SHAPES
+                                      for mode in ("full", "no_rescale", "su_only", "sv_only")]
+                         + [(32, 8192, "full")])
 def test_biip_matches_oracle(cuda, m, n, mode):
     r = np.random.default_rng(m + 3 * n)
     W, HX, HG, su, sv = _biip_case(r, m, n)
