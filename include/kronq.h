@@ -187,10 +187,11 @@ int kronq_quantize_layer(float* W, int64_t m, int64_t n, const float* U_c,
  * deployment variant of the same solver.
  *
  * Same arguments, meaning and results as kronq_quantize_layer, minus
- * (ws, ws_bytes).  The solver's m x 128 fp32 error block lives in a static
- * 16 MiB device array inside the library (every GPU that loads the library
- * holds it until the process exits), so m may be at most 32768
- * (KRONQ_ERR_UNSUPPORTED above that).  The library looks up the array's device
+ * (ws, ws_bytes).  The solver's scratch (its m x 128 error block and the
+ * current block's n x 128 slab of U_c, both as tf32 hi / lo planes) lives in
+ * a static 64 MiB device array inside the library (every GPU that loads the
+ * library holds it until the process exits), so m and n may each be at most
+ * 32768 (KRONQ_ERR_UNSUPPORTED above that).  The library looks up the array's device
  * address once per device, during the first call made on that device; make
  * that first call before any stream capture.  All calls share the array:
  * calls whose work can overlap on the GPU (different streams without

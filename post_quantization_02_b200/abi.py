@@ -188,7 +188,7 @@ def kronq_quantize_layer(W, U, bits: int, group: int, block: int, codes, scales,
 def kronq_quantize_layer_noalloc(W, U, bits: int, group: int, block: int, codes, scales, zeros,
                                  W_hat=None, info=None, stream=None):
     """kronq_quantize_layer with its scratch in the library's static device
-    array (no workspace, nothing allocated; at most 32768 rows)."""
+    array (no workspace, nothing allocated; at most 32768 rows and 32768 columns)."""
     _dev(W, torch.float32, "W", 2)
     _dev(U, torch.float32, "U_c", 2)
     _dev(codes, torch.uint8, "codes", 2)

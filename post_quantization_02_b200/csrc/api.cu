@@ -7,7 +7,7 @@
 
 size_t kq_cholesky_ws(int64_t n);
 size_t kq_biip_ws(int64_t m, int64_t n);
-size_t kq_quantize_ws(int64_t m);
+size_t kq_quantize_ws(int64_t m, int64_t n);
 size_t kq_loss_ws(int64_t m, int64_t n);
 int kq_covariance(const uint16_t* A, int64_t N, int64_t d, int64_t lda, float* H, int64_t ldh,
                   float alpha, float beta, int32_t* info, cudaStream_t st);
@@ -105,7 +105,7 @@ size_t kronq_workspace_size(int64_t m, int64_t n, int bits, int group, int block
   (void)bits; (void)group; (void)block;
   if (m <= 0 || n <= 0) return 0;
   size_t s = kq_biip_ws(m, n);
-  const size_t c = kq_cholesky_ws(n), q = kq_quantize_ws(m), l = kq_loss_ws(m, n);
+  const size_t c = kq_cholesky_ws(n), q = kq_quantize_ws(m, n), l = kq_loss_ws(m, n);
   if (c > s) s = c;
   if (q > s) s = q;
   if (l > s) s = l;

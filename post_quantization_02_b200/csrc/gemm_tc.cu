@@ -13,8 +13,8 @@
 //   warp 0       TMA loads of A_hi, A_lo, B_hi, B_lo of a stage (16 KB each)
 //   warp 1       one thread issues 3 MMAs (M = N = 128, K = 8) per K step
 //                into one of two TMEM accumulators
-//   warps 2-9    read an accumulator back and update C (loads of C issued
-//                before the accumulator is waited for)
+//   warps 2-9    read an accumulator back and add it to C with TMA reduces
+//                (32 x 32 boxes staged in shared memory)
 // All waits are bounded; a wait that gives up records KRONQ_ERR_TIMEOUT in
 // `info` and the CTA winds down.
 #include "gemm_tc.cuh"
@@ -31,7 +31,8 @@ constexpr int CHUNK = TM * KC * 4;             // 16 KB: 128 rows x 32 fp32
 constexpr int STAGE_BYTES = 4 * CHUNK;         // A hi, A lo, B hi, B lo
 constexpr int THREADS = 320;
 constexpr int EPI_WARP0 = 2;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+constexpr int STG_BYTES = 32 * 32 * 4;           // one 32 x 32 fp32 box per epilogue warp
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 8 * STG_BYTES + 1024 + 256;
 constexpr int TMEM_COLS = 2 * TN;
 
 struct Bars {
@@ -47,7 +48,20 @@ struct Bars {
 struct Maps {
   CUtensorMap a_hi[2], a_lo[2];
   CUtensorMap b_hi[2], b_lo[2];
+  CUtensorMap c[2];
 };
+
+// C box += the 32 x 32 fp32 box in shared memory (TMA, bulk-group completion).
+KQ_DEV void tma_reduce_add_2d(const void* tmap, const void* src, int x, int y) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(tmap)),
+      "r"(kq::smem_u32(src)), "r"(x), "r"(y)
+      : "memory");
+}
+KQ_DEV void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+KQ_DEV void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+KQ_DEV void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 struct Problem {
   float* C;
@@ -94,7 +108,8 @@ gemm_nt_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Pro
   extern __shared__ uint8_t smem_raw[];
   uint8_t* stages = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  Bars* bars = reinterpret_cast<Bars*>(stages + STAGES * STAGE_BYTES);
+  uint8_t* staging = stages + STAGES * STAGE_BYTES;   // 1024-byte aligned
+  Bars* bars = reinterpret_cast<Bars*>(staging + 8 * STG_BYTES);
   volatile int* abort = &bars->abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -117,6 +132,7 @@ gemm_nt_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Pro
       kq::prefetch_tmap(&maps.a_lo[i]);
       kq::prefetch_tmap(&maps.b_hi[i]);
       kq::prefetch_tmap(&maps.b_lo[i]);
+      kq::prefetch_tmap(&maps.c[i]);
     }
   }
   if (warp == EPI_WARP0) kq::tmem_alloc(&bars->tmem_base, TMEM_COLS);
@@ -183,57 +199,66 @@ gemm_nt_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Pro
   } else {
     // ------------------------------------------------------ epilogue: C += alpha acc
     // warp w: TMEM lane quadrant w % 4 (tile rows; a warp may only read its
-    // own quadrant), columns [64 h, 64 h + 64)
+    // own quadrant), columns [64 h, 64 h + 64) as two 32 x 32 boxes.  Each box
+    // is scaled, written to the warp's staging buffer in the 128-byte-swizzled
+    // layout and added to C by a TMA reduce (the L2 does the read-modify-write).
     const int q = warp & 3, h = (warp - EPI_WARP0) >> 2;
+    uint8_t* stg = staging + (warp - EPI_WARP0) * STG_BYTES;
     int tcount = 0;
+    bool pending = false;
     for (int t = blockIdx.x; t < P.total_tiles; t += gridDim.x, ++tcount) {
       const Tile tl = tile_of(P, t);
       const Problem& pr = P.p[tl.prob];
       const int buf = tcount & 1;
       const uint32_t aph = (uint32_t)(tcount >> 1) & 1u;
-      const int row = tl.tm * TM + q * 32 + lane;
-      const int cbase = tl.tn * TN + 64 * h;
-      // columns this thread may write: below M, below N, and on / below the
-      // diagonal in a lower-triangle problem's diagonal tile
-      int cend = min(pr.N, cbase + 64);
-      if (pr.lower && tl.tm == tl.tn) cend = min(cend, row + 1);
-      const bool full = row < pr.M && cend == cbase + 64;
-      float4 c[16];
-      float* crow = pr.C + (int64_t)row * pr.ldc + cbase;
-      if (full) {
-        const float4* src = reinterpret_cast<const float4*>(crow);
-#pragma unroll
-        for (int k = 0; k < 16; ++k) c[k] = src[k];
-      }
+      const int rt = q * 32 + lane;                   // row inside the tile
       if (!kq::mbar_wait(&bars->tfull[buf], aph, abort, info)) break;
       kq::tc_fence_after();
-      float v[64];
-      {
-        float v0[32], v1[32];
-        __syncwarp();
-        const uint32_t ta = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * TN + 64 * h);
-        kq::tmem_ld32(ta, v0);
-        kq::tmem_ld32(ta + 32, v1);
-        kq::tmem_wait_ld();
-#pragma unroll
-        for (int k = 0; k < 32; ++k) { v[k] = v0[k]; v[32 + k] = v1[k]; }
-      }
+      float v[2][32];
+      __syncwarp();
+      const uint32_t ta = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * TN + 64 * h);
+      kq::tmem_ld32(ta, v[0]);
+      kq::tmem_ld32(ta + 32, v[1]);
+      kq::tmem_wait_ld();
       kq::tc_fence_before();
       __syncwarp();
       if (lane == 0) kq::mbar_arrive(&bars->tempty[buf]);
       const float al = pr.alpha;
-      if (full) {
-        float4* dst = reinterpret_cast<float4*>(crow);
+      const bool diag = pr.lower && tl.tm == tl.tn;
 #pragma unroll
-        for (int k = 0; k < 16; ++k)
-          dst[k] = make_float4(fmaf(al, v[4 * k], c[k].x), fmaf(al, v[4 * k + 1], c[k].y),
-                               fmaf(al, v[4 * k + 2], c[k].z), fmaf(al, v[4 * k + 3], c[k].w));
-      } else if (row < pr.M) {
+      for (int c2 = 0; c2 < 2; ++c2) {
+        const int ct = 64 * h + 32 * c2;              // first column inside the tile
+        if (pending) {
+          if (lane == 0) bulk_wait_read();            // staging free again
+          __syncwarp();
+        }
 #pragma unroll
-        for (int k = 0; k < 64; ++k)
-          if (cbase + k < cend) crow[k] = fmaf(al, v[k], crow[k]);
+        for (int ch = 0; ch < 8; ++ch) {
+          float4 o;
+          o.x = al * v[c2][4 * ch];
+          o.y = al * v[c2][4 * ch + 1];
+          o.z = al * v[c2][4 * ch + 2];
+          o.w = al * v[c2][4 * ch + 3];
+          if (diag) {                                 // keep the strict upper triangle untouched
+            const int c = ct + 4 * ch;
+            if (c > rt) o.x = 0.f;
+            if (c + 1 > rt) o.y = 0.f;
+            if (c + 2 > rt) o.z = 0.f;
+            if (c + 3 > rt) o.w = 0.f;
+          }
+          *reinterpret_cast<float4*>(stg + lane * 128 + ((ch ^ (lane & 7)) << 4)) = o;
+        }
+        kq::tf32x3::fence_to_tensor_core();
+        __syncwarp();
+        if (lane == 0) {
+          tma_reduce_add_2d(&maps.c[tl.prob], stg, tl.tn * TN + ct, tl.tm * TM + q * 32);
+          bulk_commit();
+        }
+        pending = true;
       }
     }
+    if (lane == 0) bulk_wait_all();                   // the reduces have landed in C
+    __syncwarp();
   }
 
   kq::tc_fence_before();
@@ -264,7 +289,8 @@ int kq_gemm_nt_tc(const kq::GemmNT* probs, int count, int32_t* info, cudaStream_
     if (!kqh::make_map_f32(&maps.a_hi[j], g.A_hi, g.K, g.M, g.lda, KC, TM) ||
         !kqh::make_map_f32(&maps.a_lo[j], g.A_lo, g.K, g.M, g.lda, KC, TM) ||
         !kqh::make_map_f32(&maps.b_hi[j], g.B_hi, g.K, g.N, g.ldb, KC, TN) ||
-        !kqh::make_map_f32(&maps.b_lo[j], g.B_lo, g.K, g.N, g.ldb, KC, TN))
+        !kqh::make_map_f32(&maps.b_lo[j], g.B_lo, g.K, g.N, g.ldb, KC, TN) ||
+        !kqh::make_map_f32(&maps.c[j], g.C, g.N, g.M, g.ldc, 32, 32))
       return KRONQ_ERR_CUDA;
     Problem& q = P.p[j];
     q.C = g.C;

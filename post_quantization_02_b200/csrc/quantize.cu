@@ -16,21 +16,23 @@
 //                     threads with one shuffle, each thread applies
 //                     w_k -= e U_c[j,k] to its columns k > j.  No block-wide
 //                     synchronisation inside the column loop.
+//                     The kernel also writes E and the slab U_c[i:i+128, i+128:]^T
+//                     as tf32 hi / lo planes (tf32x3.cuh) for the lazy update.
 //   lazy update       W[:, i+128:] -= E U_c[i:i+128, i+128:] on the tensor cores
-//                     (kq_lazy_update_tc, tf32 with a three-term split)
+//                     (kq_gemm_nt_tc: tf32, three-term split, TMA reduce into W)
 #include <mutex>
 
 #include "common.cuh"
 #include "gemm_simt.cuh"
-
-int kq_lazy_update_tc(float* W, int64_t m, int64_t n, const float* E, const float* U, int i1,
-                      int32_t* info, cudaStream_t st);
+#include "gemm_tc.cuh"
+#include "tf32x3.cuh"
 
 namespace {
 
 constexpr int QB = 128;          // column block
 constexpr int ROWS_PER_CTA = 32;
 constexpr int US_LD = QB + 4;    // padded row of the U_c block in shared memory
+constexpr int TT_LD = 33;        // transposition tile of the U_c slab (QB x 32)
 
 struct Grid {
   float scale;
@@ -92,7 +94,8 @@ template <int GROUP>  // 0: per-channel grid; else 32, 64 or 128
 __global__ void __launch_bounds__(256)
 obs_block_kernel(const float* __restrict__ W, int m, int n, const float* __restrict__ U, int i1,
                  int bits, uint8_t* __restrict__ codes, float* __restrict__ scales,
-                 uint8_t* __restrict__ zeros, float* __restrict__ W_hat, float* __restrict__ E) {
+                 uint8_t* __restrict__ zeros, float* __restrict__ W_hat, float* __restrict__ Eh,
+                 float* __restrict__ El, float* __restrict__ Uth, float* __restrict__ Utl) {
   // Thread `chunk` (0..7) of a row owns the 16 columns 32 s + 4 chunk + t
   // (s, t in 0..3), held in w[4 s + t]: for a fixed s the 8 threads of a row
   // read 8 consecutive float4 of a U row, so the shared-memory reads are
@@ -100,7 +103,32 @@ obs_block_kernel(const float* __restrict__ W, int m, int n, const float* __restr
   extern __shared__ float smem[];
   float* Us = smem;                    // [QB][US_LD]
   float* rdiag = smem + QB * US_LD;    // [QB]
+  float* Tt = rdiag + QB;              // [QB][TT_LD]
   const int tid = threadIdx.x, lane = tid & 31;
+
+  // The lazy update's B operand: Ut[c - i2][k] = U[i1 + k][c] for c >= i2,
+  // in 32-column slices spread over the CTAs, as tf32 hi / lo planes.
+  {
+    const int i2 = i1 + QB;
+    const int slices = (n - i2) / 32;
+    for (int sl = blockIdx.x; sl < slices; sl += gridDim.x) {
+      const int c0 = i2 + 32 * sl;
+      for (int e = tid; e < QB * 32; e += blockDim.x) {
+        const int k = e >> 5, cc = e & 31;
+        Tt[k * TT_LD + cc] = U[(int64_t)(i1 + k) * n + c0 + cc];
+      }
+      __syncthreads();
+      for (int e = tid; e < QB * 32; e += blockDim.x) {
+        const int cc = e >> 7, k = e & (QB - 1);
+        const float v = Tt[k * TT_LD + cc];
+        const float h = kq::tf32x3::hi(v);
+        const int64_t o = (int64_t)(c0 - i2 + cc) * QB + k;
+        Uth[o] = h;
+        Utl[o] = v - h;
+      }
+      __syncthreads();
+    }
+  }
   const int chunk = tid & 7;
   const int row = blockIdx.x * ROWS_PER_CTA + (tid >> 3);
   const bool live = row < m;
@@ -196,8 +224,20 @@ obs_block_kernel(const float* __restrict__ W, int m, int n, const float* __restr
     const uint32_t pk = (uint32_t)qv[4 * sg] | ((uint32_t)qv[4 * sg + 1] << 8) |
                         ((uint32_t)qv[4 * sg + 2] << 16) | ((uint32_t)qv[4 * sg + 3] << 24);
     *reinterpret_cast<uint32_t*>(codes + off) = pk;
-    *reinterpret_cast<float4*>(E + (int64_t)row * QB + 32 * sg + 4 * chunk) =
-        make_float4(ev[4 * sg], ev[4 * sg + 1], ev[4 * sg + 2], ev[4 * sg + 3]);
+    {
+      float4 eh, el;
+      eh.x = kq::tf32x3::hi(ev[4 * sg]);
+      eh.y = kq::tf32x3::hi(ev[4 * sg + 1]);
+      eh.z = kq::tf32x3::hi(ev[4 * sg + 2]);
+      eh.w = kq::tf32x3::hi(ev[4 * sg + 3]);
+      el.x = ev[4 * sg] - eh.x;
+      el.y = ev[4 * sg + 1] - eh.y;
+      el.z = ev[4 * sg + 2] - eh.z;
+      el.w = ev[4 * sg + 3] - eh.w;
+      const int64_t eo = (int64_t)row * QB + 32 * sg + 4 * chunk;
+      *reinterpret_cast<float4*>(Eh + eo) = eh;
+      *reinterpret_cast<float4*>(El + eo) = el;
+    }
     if (W_hat)
       *reinterpret_cast<float4*>(W_hat + off) =
           make_float4(hv[4 * sg], hv[4 * sg + 1], hv[4 * sg + 2], hv[4 * sg + 3]);
@@ -270,11 +310,16 @@ __global__ void unpack_kernel(const uint32_t* __restrict__ packed, int64_t m, in
 
 size_t a256(size_t b) { return (b + 255) & ~(size_t)255; }
 
+struct SolverScratch {
+  float *Eh, *El, *Uth, *Utl;
+};
+
 template <int GROUP>
 int launch_block(const float* W, int m, int n, const float* U, int i1, int bits, uint8_t* codes,
-                 float* scales, uint8_t* zeros, float* W_hat, float* E, cudaStream_t st) {
+                 float* scales, uint8_t* zeros, float* W_hat, const SolverScratch& sc,
+                 cudaStream_t st) {
   static bool attr = false;
-  const size_t smem = (size_t)(QB * US_LD + QB) * sizeof(float);
+  const size_t smem = (size_t)(QB * US_LD + QB + QB * TT_LD) * sizeof(float);
   if (!attr) {
     if (cudaFuncSetAttribute(obs_block_kernel<GROUP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)
@@ -283,14 +328,18 @@ int launch_block(const float* W, int m, int n, const float* U, int i1, int bits,
   }
   const int grid = (m + ROWS_PER_CTA - 1) / ROWS_PER_CTA;
   obs_block_kernel<GROUP><<<grid, 256, smem, st>>>(W, m, n, U, i1, bits, codes, scales, zeros,
-                                                   W_hat, E);
+                                                   W_hat, sc.Eh, sc.El, sc.Uth, sc.Utl);
   KQ_CHECK_LAUNCH();
   return KRONQ_OK;
 }
 
 }  // namespace
 
-size_t kq_quantize_ws(int64_t m) { return a256((size_t)m * QB * sizeof(float)); }
+// Scratch of the solver: E as hi / lo planes (m x 128 each) and the U_c slab
+// of the current block, transposed, as hi / lo planes (n x 128 each).
+size_t kq_quantize_ws(int64_t m, int64_t n) {
+  return 2 * a256((size_t)m * QB * sizeof(float)) + 2 * a256((size_t)n * QB * sizeof(float));
+}
 
 size_t kq_loss_ws(int64_t m, int64_t n) { return 3 * a256((size_t)m * n * sizeof(float)); }
 
@@ -307,9 +356,20 @@ int kq_quantize_layer(float* W, int64_t m64, int64_t n64, const float* U, int bi
   if (!kqh::aligned(W, 16) || !kqh::aligned(U, 16) || !kqh::aligned(codes, 16) ||
       (W_hat && !kqh::aligned(W_hat, 16)))
     return KRONQ_ERR_INVALID_ARG;
-  if (!ws || ws_bytes < kq_quantize_ws(m64) || !kqh::aligned(ws, 256)) return KRONQ_ERR_WORKSPACE;
+  if (!ws || ws_bytes < kq_quantize_ws(m64, n64) || !kqh::aligned(ws, 256))
+    return KRONQ_ERR_WORKSPACE;
   const int m = (int)m64, n = (int)n64;
-  float* E = static_cast<float*>(ws);
+  SolverScratch sc;
+  {
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    sc.Eh = reinterpret_cast<float*>(w);
+    w += a256((size_t)m * QB * sizeof(float));
+    sc.El = reinterpret_cast<float*>(w);
+    w += a256((size_t)m * QB * sizeof(float));
+    sc.Uth = reinterpret_cast<float*>(w);
+    w += a256((size_t)n * QB * sizeof(float));
+    sc.Utl = reinterpret_cast<float*>(w);
+  }
 
   if (group == -1) {
     row_params_kernel<<<(m + 7) / 8, 256, 0, st>>>(W, m, n, bits, scales, zeros);
@@ -318,15 +378,17 @@ int kq_quantize_layer(float* W, int64_t m64, int64_t n64, const float* U, int bi
   for (int i1 = 0; i1 < n; i1 += QB) {
     int s;
     switch (group) {
-      case -1: s = launch_block<0>(W, m, n, U, i1, bits, codes, scales, zeros, W_hat, E, st); break;
-      case 32: s = launch_block<32>(W, m, n, U, i1, bits, codes, scales, zeros, W_hat, E, st); break;
-      case 64: s = launch_block<64>(W, m, n, U, i1, bits, codes, scales, zeros, W_hat, E, st); break;
-      default: s = launch_block<128>(W, m, n, U, i1, bits, codes, scales, zeros, W_hat, E, st); break;
+      case -1: s = launch_block<0>(W, m, n, U, i1, bits, codes, scales, zeros, W_hat, sc, st); break;
+      case 32: s = launch_block<32>(W, m, n, U, i1, bits, codes, scales, zeros, W_hat, sc, st); break;
+      case 64: s = launch_block<64>(W, m, n, U, i1, bits, codes, scales, zeros, W_hat, sc, st); break;
+      default: s = launch_block<128>(W, m, n, U, i1, bits, codes, scales, zeros, W_hat, sc, st); break;
     }
     if (s != KRONQ_OK) return s;
     const int i2 = i1 + QB;
     if (i2 < n) {
-      s = kq_lazy_update_tc(W, m, n, E, U, i1, info, st);
+      // W[:, i2:] -= E U[i1:i2, i2:] = E (Ut)^T
+      const kq::GemmNT g = {sc.Eh, sc.El, QB, sc.Uth, sc.Utl, QB, W + i2, n, m, n - i2, QB, -1.f, 0};
+      s = kq_gemm_nt_tc(&g, 1, info, st);
       if (s != KRONQ_OK) return s;
     }
   }
@@ -391,33 +453,37 @@ int kq_layer_loss(const float* Wr, const float* Wh, int64_t m64, int64_t n64, co
 // a process that plans all of its memory at start-up and must not grow it
 // later, or a latency-sensitive loop in which cudaMalloc / cudaFree would
 // synchronise the device and stall other streams.  For them the solver's
-// only scratch buffer (the m x 128 fp32 error block) lives in the static
-// device array below instead of a caller workspace.
+// scratch (the error block and the transposed U_c slab, each as tf32 hi / lo
+// planes) lives in the static device array below instead of a caller
+// workspace.
 //
 // The array is part of the library image: every GPU that loads libkronq holds
-// its 16 MiB until the process exits.  Host code cannot use the symbol as a
-// device address, so its address is looked up with cudaGetSymbolAddress once
-// per device (with that device current), on the first call made on that
-// device.  All calls share the one array and it keeps the previous call's
-// contents: nothing in it has to start at zero (every element the lazy
-// update reads was written by the block solve of the same call), but two
-// calls whose work overlaps on the GPU race on it.
+// its 64 MiB until the process exits; it fits m <= 32768 rows and
+// n <= 32768 columns.  Host code cannot use the symbol as a device address,
+// so its address is looked up with cudaGetSymbolAddress once per device (with
+// that device current), on the first call made on that device.  All calls
+// share the one array and it keeps the previous call's contents: nothing in
+// it has to start at zero (every element the lazy update reads was written
+// by the block solve of the same call), but two calls whose work overlaps on
+// the GPU race on it.
 constexpr int64_t kNoAllocMaxRows = 32768;
-static __device__ __align__(256) float g_noalloc_error_block[kNoAllocMaxRows * QB];
+constexpr int64_t kNoAllocMaxCols = 32768;
+constexpr size_t kNoAllocBytes = (size_t)2 * (kNoAllocMaxRows + kNoAllocMaxCols) * QB * sizeof(float);
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocBytes / sizeof(float)];
 
 namespace {
 
 std::mutex g_noalloc_mutex;
 float* g_noalloc_ptr[64] = {};
 
-// Device address of g_noalloc_error_block on the current device (nullptr on failure).
+// Device address of g_noalloc_scratch on the current device (nullptr on failure).
 float* noalloc_scratch() {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
   std::lock_guard<std::mutex> lock(g_noalloc_mutex);
   if (!g_noalloc_ptr[dev]) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_error_block) != cudaSuccess || !p) return nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return nullptr;
     g_noalloc_ptr[dev] = static_cast<float*>(p);
   }
   return g_noalloc_ptr[dev];
@@ -428,9 +494,10 @@ float* noalloc_scratch() {
 int kq_quantize_layer_noalloc(float* W, int64_t m, int64_t n, const float* U, int bits, int group,
                               int block, uint8_t* codes, float* scales, uint8_t* zeros,
                               float* W_hat, int32_t* info, cudaStream_t st) {
-  if (m > kNoAllocMaxRows) return KRONQ_ERR_UNSUPPORTED;   // the static scratch holds 32768 rows
-  float* E = noalloc_scratch();
-  if (!E) return KRONQ_ERR_CUDA;
-  return kq_quantize_layer(W, m, n, U, bits, group, block, codes, scales, zeros, W_hat, info, E,
-                           sizeof(g_noalloc_error_block), st);
+  // the static scratch holds 32768 rows and 32768 columns
+  if (m > kNoAllocMaxRows || n > kNoAllocMaxCols) return KRONQ_ERR_UNSUPPORTED;
+  float* scratch = noalloc_scratch();
+  if (!scratch) return KRONQ_ERR_CUDA;
+  return kq_quantize_layer(W, m, n, U, bits, group, block, codes, scales, zeros, W_hat, info,
+                           scratch, sizeof(g_noalloc_scratch), st);
 }
