@@ -128,101 +128,141 @@ __device__ __forceinline__ void warp_leaf32(float* D, float* X, float* YT, int o
 // X = L^-1 for the lower Cholesky factor L of the 128 x 128 block in D
 // (fp32; rows / columns kb .. NB-1 padded with the identity by the caller).
 // On return D's lower triangle holds L and X (zero above the diagonal)
-// holds L^-1.  256 threads.
+// holds L^-1.  PANEL_THREADS (256) threads.
 //
 // Right-looking over four 32-wide blocks b (o = 32 b), carrying L^-1 along
 // (block forward substitution of L Y = I, accumulators in X below the
 // diagonal blocks):
 //   1. warp 0: L_bb and Y_bb = L_bb^-1                          (warp_leaf32)
 //   2. L_cb = D_cb Y_bb^T (c > b), also kept K-major in As;  Y_bj = Y_bb Acc_bj (j < b)
-//   3. D_cd -= L_cb L_db^T (b < d <= c);  Acc_cj -= L_cb Y_bj (c > b, j <= b)
-// Steps 2 and 3 are small register-tiled GEMMs out of shared memory whose
-// wide operands are read as contiguous float4 rows (YT, As, rows of X).
+//   3a. the next block column: D_{c,b+1} -= L_cb L_{b+1,b}^T
+//   3b. the rest: D_cd -= L_cb L_db^T (d > b+1);  Acc_cj -= L_cb Y_bj (j <= b)
+// with warp 0 factoring block b+1 (step 1 of the next round) while the other
+// warps do 3b.  Steps 2 and 3 are small register-tiled GEMMs out of shared
+// memory whose wide operands are read as contiguous rows (YT, As, rows of X).
+constexpr int PANEL_THREADS = 256;
+
 __device__ void factor_and_invert(float* D, float* X, float* As, float* YT, int kb, int* bad) {
   const int tid = threadIdx.x;
   for (int e = tid; e < NB * LDX; e += blockDim.x) X[e] = 0.f;
+  __syncthreads();
+  if (tid < 32) warp_leaf32(D, X, YT, 0, kb, bad);
   __syncthreads();
   for (int b = 0; b < NB / 32; ++b) {
     const int o = 32 * b;
     const int o2 = o + 32;
     const int R1 = NB - o2;                 // rows below the diagonal block
-    if (tid < 32) warp_leaf32(D, X, YT, o, kb, bad);
-    __syncthreads();
-    // ---- step 2: thread (tr, tc) = (tid / 8, tid % 8)
+    // ---- step 2: thread tid handles (tr, tc) = (tid / 16 + 16 u, tid % 16), u = 0, 1
     {
-      const int tr = tid >> 3, tc = tid & 7;
-      const int nj = o >> 3;                // Y_bj columns per thread: o / 8
-      float acc1[3][4], acc2[12];
+      const int tc = tid & 15;
+      const int nj = o >> 4;                // Y_bj columns per item: o / 16
+      float acc1[2][3][2], acc2[2][6];
 #pragma unroll
-      for (int s = 0; s < 3; ++s)
+      for (int u = 0; u < 2; ++u) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) acc1[s][q] = 0.f;
+        for (int s = 0; s < 3; ++s) acc1[u][s][0] = acc1[u][s][1] = 0.f;
 #pragma unroll
-      for (int q = 0; q < 12; ++q) acc2[q] = 0.f;
-#pragma unroll 4
+        for (int q = 0; q < 6; ++q) acc2[u][q] = 0.f;
+      }
+#pragma unroll 2
       for (int t = 0; t < 32; ++t) {
-        const float4 bv = *reinterpret_cast<const float4*>(&YT[t * LDY + 4 * tc]);   // Y_bb[4tc+q][t]
+        const float2 bv = *reinterpret_cast<const float2*>(&YT[t * LDY + 2 * tc]);   // Y_bb[2tc+q][t]
 #pragma unroll
-        for (int s = 0; s < 3; ++s) {
-          if (32 * s < R1) {
-            const float av = D[(o2 + tr + 32 * s) * LDD + o + t];
-            acc1[s][0] = fmaf(av, bv.x, acc1[s][0]);
-            acc1[s][1] = fmaf(av, bv.y, acc1[s][1]);
-            acc1[s][2] = fmaf(av, bv.z, acc1[s][2]);
-            acc1[s][3] = fmaf(av, bv.w, acc1[s][3]);
+        for (int u = 0; u < 2; ++u) {
+          const int tr = (tid >> 4) + 16 * u;
+#pragma unroll
+          for (int s = 0; s < 3; ++s) {
+            if (32 * s < R1) {
+              const float av = D[(o2 + tr + 32 * s) * LDD + o + t];
+              acc1[u][s][0] = fmaf(av, bv.x, acc1[u][s][0]);
+              acc1[u][s][1] = fmaf(av, bv.y, acc1[u][s][1]);
+            }
           }
-        }
-        const float yv = X[(o + tr) * LDX + o + t];                            // Y_bb[tr][t]
+          const float yv = X[(o + tr) * LDX + o + t];                          // Y_bb[tr][t]
 #pragma unroll
-        for (int q = 0; q < 12; ++q)
-          if (q < nj) acc2[q] = fmaf(yv, X[(o + t) * LDX + tc * nj + q], acc2[q]);   // Acc[t][c']
+          for (int q = 0; q < 6; ++q)
+            if (q < nj) acc2[u][q] = fmaf(yv, X[(o + t) * LDX + tc * nj + q], acc2[u][q]);  // Acc[t][c']
+        }
       }
       __syncthreads();
 #pragma unroll
-      for (int s = 0; s < 3; ++s)
-        if (32 * s < R1)
+      for (int u = 0; u < 2; ++u) {
+        const int tr = (tid >> 4) + 16 * u;
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            D[(o2 + tr + 32 * s) * LDD + o + 4 * tc + q] = acc1[s][q];
-            As[(4 * tc + q) * LDA + tr + 32 * s] = acc1[s][q];
-          }
+        for (int s = 0; s < 3; ++s)
+          if (32 * s < R1)
 #pragma unroll
-      for (int q = 0; q < 12; ++q)
-        if (q < nj) X[(o + tr) * LDX + tc * nj + q] = acc2[q];
+            for (int q = 0; q < 2; ++q) {
+              D[(o2 + tr + 32 * s) * LDD + o + 2 * tc + q] = acc1[u][s][q];
+              As[(2 * tc + q) * LDA + tr + 32 * s] = acc1[u][s][q];
+            }
+#pragma unroll
+        for (int q = 0; q < 6; ++q)
+          if (q < nj) X[(o + tr) * LDX + tc * nj + q] = acc2[u][q];
+      }
       __syncthreads();
     }
     if (R1 == 0) break;
-    // ---- step 3: rows o2 + tr * ns + s, columns 8 tc .. 8 tc + 7 (all 128)
-    {
-      const int tr = tid >> 4, tc = tid & 15;
-      const int ns = R1 >> 4;               // 6, 4 or 2 rows per thread
-      float acc[6][8];
+    // ---- step 3a: D[r][c] -= sum_t L[r][o+t] L[c][o+t], c in the next block column
+    for (int w = tid; w < 512; w += PANEL_THREADS) {
+      const int tr = w >> 4, tc = w & 15;          // rows tr + 32 s, columns 2 tc, 2 tc + 1
+      float acc[3][2];
 #pragma unroll
-      for (int s = 0; s < 6; ++s)
-#pragma unroll
-        for (int q = 0; q < 8; ++q) acc[s][q] = 0.f;
-      const int c0 = 8 * tc;
-      const bool left = c0 < o2;            // Acc / Y columns (j <= b), else trailing D
-      const float* Bp = left ? &X[o * LDX + c0] : &As[c0 - o2];
-      const int ldb = left ? LDX : LDA;
-#pragma unroll 2
+      for (int s = 0; s < 3; ++s) acc[s][0] = acc[s][1] = 0.f;
+#pragma unroll 4
       for (int t = 0; t < 32; ++t) {
-        const float4 b0 = *reinterpret_cast<const float4*>(Bp + t * ldb);
-        const float4 b1 = *reinterpret_cast<const float4*>(Bp + t * ldb + 4);
-        const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+        const float2 bv = *reinterpret_cast<const float2*>(&As[t * LDA + 2 * tc]);
 #pragma unroll
-        for (int s = 0; s < 6; ++s) {
-          if (s < ns) {
-            const float av = As[t * LDA + tr * ns + s];                          // L[o2+r][o+t]
-#pragma unroll
-            for (int q = 0; q < 8; ++q) acc[s][q] = fmaf(av, bv[q], acc[s][q]);
+        for (int s = 0; s < 3; ++s) {
+          if (32 * s < R1) {
+            const float av = As[t * LDA + tr + 32 * s];
+            acc[s][0] = fmaf(av, bv.x, acc[s][0]);
+            acc[s][1] = fmaf(av, bv.y, acc[s][1]);
           }
         }
       }
 #pragma unroll
-      for (int s = 0; s < 6; ++s) {
-        if (s < ns) {
-          const int r = o2 + tr * ns + s;
+      for (int s = 0; s < 3; ++s)
+        if (32 * s < R1) {
+          const int r = o2 + tr + 32 * s;
+#pragma unroll
+          for (int q = 0; q < 2; ++q)
+            if (o2 + 2 * tc + q <= r) D[r * LDD + o2 + 2 * tc + q] -= acc[s][q];
+        }
+    }
+    __syncthreads();
+    // ---- step 3b on warps 1.., the next diagonal block on warp 0
+    if (tid < 32) {
+      warp_leaf32(D, X, YT, o2, kb, bad);
+    } else {
+      // item = 4 rows x 8 columns; 12 column groups: 8 g < o2 (Acc), else past the next block
+      const int items = (R1 / 4) * 12;
+      for (int it = tid - 32; it < items; it += PANEL_THREADS - 32) {
+        const int rg = it / 12, g = it % 12;
+        const int c0 = (8 * g < o2) ? 8 * g : 8 * g + 32;
+        const bool left = c0 < o2;
+        const float* Bp = left ? &X[o * LDX + c0] : &As[c0 - o2];
+        const int ldb = left ? LDX : LDA;
+        float acc[4][8];
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+#pragma unroll
+          for (int q = 0; q < 8; ++q) acc[s][q] = 0.f;
+#pragma unroll 2
+        for (int t = 0; t < 32; ++t) {
+          const float4 b0 = *reinterpret_cast<const float4*>(Bp + t * ldb);
+          const float4 b1 = *reinterpret_cast<const float4*>(Bp + t * ldb + 4);
+          const float4 a4 = *reinterpret_cast<const float4*>(&As[t * LDA + 4 * rg]);
+          const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+          const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+          for (int s = 0; s < 4; ++s)
+#pragma unroll
+            for (int q = 0; q < 8; ++q) acc[s][q] = fmaf(av[s], bv[q], acc[s][q]);
+        }
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+          const int r = o2 + 4 * rg + s;
           if (left) {
 #pragma unroll
             for (int q = 0; q < 8; ++q) X[r * LDX + c0 + q] -= acc[s][q];
@@ -233,8 +273,8 @@ __device__ void factor_and_invert(float* D, float* X, float* As, float* YT, int 
           }
         }
       }
-      __syncthreads();
     }
+    __syncthreads();
   }
 }
 
@@ -264,7 +304,7 @@ KQ_DEV void put_split(float* hi_plane, float* lo_plane, int64_t idx, float v) {
 // the 32 x 128 slice it multiplies is fetched by bulk copies meanwhile.
 constexpr int PR = 32;
 
-__global__ void __launch_bounds__(256, 1) panel_kernel(const float* R, float* Z, float* Lh,
+__global__ void __launch_bounds__(PANEL_THREADS, 1) panel_kernel(const float* R, float* Z, float* Lh,
                                                     float* Ll, float* Zh, float* Zl, int np, int k,
                                                     int p, int tiles_L, int32_t* info) {
   extern __shared__ __align__(16) float sm[];
@@ -342,23 +382,23 @@ __global__ void __launch_bounds__(256, 1) panel_kernel(const float* R, float* Z,
       }
   }
   if (role_L) {
-    const int64_t r0 = (int64_t)PR * blockIdx.x;      // plane row of this slice's first row
 #pragma unroll
-    for (int i = 0; i < 2; ++i)
+    for (int i = 0; i < 2; ++i) {
+      const int64_t r = (int64_t)PR * blockIdx.x + ty + 16 * i;   // plane row
 #pragma unroll
-      for (int jj = 0; jj < 8; ++jj)
-        put_split(Lh, Ll, (r0 + ty + 16 * i) * NB + tx + 16 * jj, acc[i][jj]);
+      for (int jj = 0; jj < 8; ++jj) put_split(Lh, Ll, r * NB + tx + 16 * jj, acc[i][jj]);
+    }
   } else {
-    const int64_t r0 = (int64_t)PR * j;
 #pragma unroll
-    for (int i = 0; i < 2; ++i)
+    for (int i = 0; i < 2; ++i) {
+      const int64_t r = (int64_t)PR * j + ty + 16 * i;
 #pragma unroll
       for (int jj = 0; jj < 8; ++jj) {
-        const int64_t r = r0 + ty + 16 * i;
         const int c = tx + 16 * jj;
         Z[r * np + k + c] = acc[i][jj];
         put_split(Zh, Zl, r * NB + c, acc[i][jj]);
       }
+    }
   }
 }
 
@@ -437,7 +477,7 @@ int kq_cholesky_inv(const float* H, int64_t n64, float damp_rel, float* U, int32
     const int k = p * NB;
     const int rest = np - k - NB;
     const int tiles_L = rest / PR;
-    panel_kernel<<<tiles_L + 4 * p + 1, 256, kPanelSmem, st>>>(R, Z, Lh, Ll, Zh, Zl, np, k, p,
+    panel_kernel<<<tiles_L + 4 * p + 1, PANEL_THREADS, kPanelSmem, st>>>(R, Z, Lh, Ll, Zh, Zl, np, k, p,
                                                                tiles_L, info);
     KQ_CHECK_LAUNCH();
     if (rest > 0) {

@@ -70,6 +70,7 @@ struct Problem {
   float alpha;
   int lower;
   int ntn;     // tile columns (rectangular problems)
+  int t0;      // first tile of the problem's own tile order
   int tiles;
 };
 
@@ -88,6 +89,7 @@ __device__ __forceinline__ Tile tile_of(const Problems& P, int t) {
   r.prob = (P.count > 1 && t >= P.p[0].tiles) ? 1 : 0;
   if (r.prob) t -= P.p[0].tiles;
   const Problem& q = P.p[r.prob];
+  t += q.t0;
   if (q.lower) {
     int tm = (int)((sqrtf(8.f * (float)t + 1.f) - 1.f) * 0.5f);
     while ((tm + 1) * (tm + 2) / 2 <= t) ++tm;
@@ -271,7 +273,8 @@ gemm_nt_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Pro
 
 }  // namespace
 
-int kq_gemm_nt_tc(const kq::GemmNT* probs, int count, int32_t* info, cudaStream_t st) {
+int kq_gemm_nt_tc(const kq::GemmNT* probs, int count, int32_t* info, cudaStream_t st,
+                  int max_ctas) {
   if (count < 1 || count > 2) return KRONQ_ERR_INVALID_ARG;
   Maps maps;
   Problems P;
@@ -302,7 +305,12 @@ int kq_gemm_nt_tc(const kq::GemmNT* probs, int count, int32_t* info, cudaStream_
     q.lower = g.lower;
     const int ntm = (g.M + TM - 1) / TM;
     q.ntn = (g.N + TN - 1) / TN;
-    q.tiles = g.lower ? ntm * (ntm + 1) / 2 : ntm * q.ntn;
+    const int all = g.lower ? ntm * (ntm + 1) / 2 : ntm * q.ntn;
+    const int tb = g.tile_begin < 0 ? 0 : (g.tile_begin > all ? all : g.tile_begin);
+    const int te = (g.tile_end < 0 || g.tile_end > all) ? all : g.tile_end;
+    if (te <= tb) continue;
+    q.t0 = tb;
+    q.tiles = te - tb;
     P.total_tiles += q.tiles;
     ++P.count;
   }
@@ -315,7 +323,8 @@ int kq_gemm_nt_tc(const kq::GemmNT* probs, int count, int32_t* info, cudaStream_
       return KRONQ_ERR_CUDA;
     attr = true;
   }
-  const int grid = P.total_tiles < kqh::num_sms() ? P.total_tiles : kqh::num_sms();
+  int grid = P.total_tiles < kqh::num_sms() ? P.total_tiles : kqh::num_sms();
+  if (max_ctas > 0 && grid > max_ctas) grid = max_ctas;
   gemm_nt_tc_kernel<<<grid, THREADS, SMEM_BYTES, st>>>(maps, P, info);
   KQ_CHECK_LAUNCH();
   return KRONQ_OK;

@@ -25,6 +25,11 @@ struct GemmNT {
   int M, N, K;
   float alpha;
   int lower;
+  // only the problem's output tiles [tile_begin, tile_end) in its own tile
+  // order (row-major over 128 x 128 tiles; lower: row by row, columns up to
+  // the diagonal); tile_end < 0: to the last tile
+  int tile_begin = 0;
+  int tile_end = -1;
 };
 
 }  // namespace kq
@@ -32,4 +37,6 @@ struct GemmNT {
 // One launch for up to two independent problems (count 1 or 2); empty
 // problems are skipped.  Returns KRONQ_OK, KRONQ_ERR_INVALID_ARG or
 // KRONQ_ERR_CUDA.
-int kq_gemm_nt_tc(const kq::GemmNT* probs, int count, int32_t* info, cudaStream_t st);
+// max_ctas > 0 caps the persistent grid (to leave SMs to concurrent work).
+int kq_gemm_nt_tc(const kq::GemmNT* probs, int count, int32_t* info, cudaStream_t st,
+                  int max_ctas = 0);

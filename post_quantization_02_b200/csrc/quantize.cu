@@ -95,7 +95,8 @@ __global__ void __launch_bounds__(256)
 obs_block_kernel(const float* __restrict__ W, int m, int n, const float* __restrict__ U, int i1,
                  int bits, uint8_t* __restrict__ codes, float* __restrict__ scales,
                  uint8_t* __restrict__ zeros, float* __restrict__ W_hat, float* __restrict__ Eh,
-                 float* __restrict__ El, float* __restrict__ Uth, float* __restrict__ Utl) {
+                 float* __restrict__ El, int ld_e, float* __restrict__ Uth,
+                 float* __restrict__ Utl, int slab_end) {
   // Thread `chunk` (0..7) of a row owns the 16 columns 32 s + 4 chunk + t
   // (s, t in 0..3), held in w[4 s + t]: for a fixed s the 8 threads of a row
   // read 8 consecutive float4 of a U row, so the shared-memory reads are
@@ -106,11 +107,12 @@ obs_block_kernel(const float* __restrict__ W, int m, int n, const float* __restr
   float* Tt = rdiag + QB;              // [QB][TT_LD]
   const int tid = threadIdx.x, lane = tid & 31;
 
-  // The lazy update's B operand: Ut[c - i2][k] = U[i1 + k][c] for c >= i2,
-  // in 32-column slices spread over the CTAs, as tf32 hi / lo planes.
+  // The lazy update's B operand: Ut[c - i2][k] = U[i1 + k][c] for
+  // i2 <= c < slab_end (the rest of the super-block, or of the matrix with
+  // one level), in 32-column slices spread over the CTAs, as tf32 hi / lo planes.
   {
     const int i2 = i1 + QB;
-    const int slices = (n - i2) / 32;
+    const int slices = (slab_end - i2) / 32;
     for (int sl = blockIdx.x; sl < slices; sl += gridDim.x) {
       const int c0 = i2 + 32 * sl;
       for (int e = tid; e < QB * 32; e += blockDim.x) {
@@ -234,7 +236,7 @@ obs_block_kernel(const float* __restrict__ W, int m, int n, const float* __restr
       el.y = ev[4 * sg + 1] - eh.y;
       el.z = ev[4 * sg + 2] - eh.z;
       el.w = ev[4 * sg + 3] - eh.w;
-      const int64_t eo = (int64_t)row * QB + 32 * sg + 4 * chunk;
+      const int64_t eo = (int64_t)row * ld_e + 32 * sg + 4 * chunk;
       *reinterpret_cast<float4*>(Eh + eo) = eh;
       *reinterpret_cast<float4*>(El + eo) = el;
     }
@@ -311,13 +313,42 @@ __global__ void unpack_kernel(const uint32_t* __restrict__ packed, int64_t m, in
 size_t a256(size_t b) { return (b + 255) & ~(size_t)255; }
 
 struct SolverScratch {
-  float *Eh, *El, *Uth, *Utl;
+  int B2;                  // outer (super-)block width: 128 (one level) or 1024
+  float *Eh, *El;          // E of the super-block, m x B2 each
+  float *Uth, *Utl;        // inner slab U[i1:i1+128, i1+128:sb_end]^T, n x 128 each
+  float *Voh, *Vol;        // outer slab U[sb:sb_end, sb_end:]^T, n x B2 each (two levels only)
 };
+
+// Ut[c - col0][k] = U[row0 + k][c] for k < rows, col0 <= c < n, as tf32
+// hi / lo planes with leading dimension ld: one 32 x 32 tile per CTA.
+__global__ void __launch_bounds__(256) slab_transpose_kernel(const float* __restrict__ U, int n,
+                                                             int row0, int rows, int col0,
+                                                             float* __restrict__ Th,
+                                                             float* __restrict__ Tl, int ld) {
+  __shared__ float t[32][33];
+  const int kb = blockIdx.y * 32, cb = col0 + blockIdx.x * 32;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  for (int r = ty; r < 32; r += 8) {
+    const int k = kb + r, c = cb + tx;
+    t[r][tx] = (k < rows && c < n) ? U[(int64_t)(row0 + k) * n + c] : 0.f;
+  }
+  __syncthreads();
+  for (int r = ty; r < 32; r += 8) {
+    const int c = cb + r, k = kb + tx;
+    if (c < n && k < rows) {
+      const float v = t[tx][r];
+      const float h = kq::tf32x3::hi(v);
+      const int64_t o = (int64_t)(c - col0) * ld + k;
+      Th[o] = h;
+      Tl[o] = v - h;
+    }
+  }
+}
 
 template <int GROUP>
 int launch_block(const float* W, int m, int n, const float* U, int i1, int bits, uint8_t* codes,
-                 float* scales, uint8_t* zeros, float* W_hat, const SolverScratch& sc,
-                 cudaStream_t st) {
+                 float* scales, uint8_t* zeros, float* W_hat, const SolverScratch& sc, int sb,
+                 int slab_end, cudaStream_t st) {
   static bool attr = false;
   const size_t smem = (size_t)(QB * US_LD + QB + QB * TT_LD) * sizeof(float);
   if (!attr) {
@@ -328,18 +359,28 @@ int launch_block(const float* W, int m, int n, const float* U, int i1, int bits,
   }
   const int grid = (m + ROWS_PER_CTA - 1) / ROWS_PER_CTA;
   obs_block_kernel<GROUP><<<grid, 256, smem, st>>>(W, m, n, U, i1, bits, codes, scales, zeros,
-                                                   W_hat, sc.Eh, sc.El, sc.Uth, sc.Utl);
+                                                   W_hat, sc.Eh + (i1 - sb), sc.El + (i1 - sb),
+                                                   sc.B2, sc.Uth, sc.Utl, slab_end);
   KQ_CHECK_LAUNCH();
   return KRONQ_OK;
 }
 
+constexpr int QB2 = 1024;        // outer super-block of the two-level lazy update
+
+// Scratch of the solver with outer block B2: E of a super-block as hi / lo
+// planes (m x B2 each), the inner U_c slab transposed (n x 128 each) and,
+// with two levels, the outer slab transposed (n x B2 each).
+size_t solver_ws(int64_t m, int64_t n, int B2) {
+  size_t b = 2 * a256((size_t)m * B2 * sizeof(float)) + 2 * a256((size_t)n * QB * sizeof(float));
+  if (B2 > QB) b += 2 * a256((size_t)n * B2 * sizeof(float));
+  return b;
+}
+
 }  // namespace
 
-// Scratch of the solver: E as hi / lo planes (m x 128 each) and the U_c slab
-// of the current block, transposed, as hi / lo planes (n x 128 each).
-size_t kq_quantize_ws(int64_t m, int64_t n) {
-  return 2 * a256((size_t)m * QB * sizeof(float)) + 2 * a256((size_t)n * QB * sizeof(float));
-}
+// The size that enables the two-level lazy update; a workspace of at least
+// solver_ws(m, n, 128) runs the one-level update.
+size_t kq_quantize_ws(int64_t m, int64_t n) { return solver_ws(m, n, QB2); }
 
 size_t kq_loss_ws(int64_t m, int64_t n) { return 3 * a256((size_t)m * n * sizeof(float)); }
 
@@ -356,39 +397,75 @@ int kq_quantize_layer(float* W, int64_t m64, int64_t n64, const float* U, int bi
   if (!kqh::aligned(W, 16) || !kqh::aligned(U, 16) || !kqh::aligned(codes, 16) ||
       (W_hat && !kqh::aligned(W_hat, 16)))
     return KRONQ_ERR_INVALID_ARG;
-  if (!ws || ws_bytes < kq_quantize_ws(m64, n64) || !kqh::aligned(ws, 256))
-    return KRONQ_ERR_WORKSPACE;
+  if (!ws || !kqh::aligned(ws, 256)) return KRONQ_ERR_WORKSPACE;
+  // two levels (B2 = 1024: the outer update is a K = 1024 tensor-core GEMM)
+  // when the workspace allows, else one level
+  const int B2 = (n64 > QB && ws_bytes >= solver_ws(m64, n64, QB2)) ? QB2 : QB;
+  if (ws_bytes < solver_ws(m64, n64, B2)) return KRONQ_ERR_WORKSPACE;
   const int m = (int)m64, n = (int)n64;
   SolverScratch sc;
   {
     uint8_t* w = static_cast<uint8_t*>(ws);
+    sc.B2 = B2;
     sc.Eh = reinterpret_cast<float*>(w);
-    w += a256((size_t)m * QB * sizeof(float));
+    w += a256((size_t)m * B2 * sizeof(float));
     sc.El = reinterpret_cast<float*>(w);
-    w += a256((size_t)m * QB * sizeof(float));
+    w += a256((size_t)m * B2 * sizeof(float));
     sc.Uth = reinterpret_cast<float*>(w);
     w += a256((size_t)n * QB * sizeof(float));
     sc.Utl = reinterpret_cast<float*>(w);
+    w += a256((size_t)n * QB * sizeof(float));
+    sc.Voh = sc.Vol = nullptr;
+    if (B2 > QB) {
+      sc.Voh = reinterpret_cast<float*>(w);
+      w += a256((size_t)n * B2 * sizeof(float));
+      sc.Vol = reinterpret_cast<float*>(w);
+    }
   }
 
   if (group == -1) {
     row_params_kernel<<<(m + 7) / 8, 256, 0, st>>>(W, m, n, bits, scales, zeros);
     KQ_CHECK_LAUNCH();
   }
-  for (int i1 = 0; i1 < n; i1 += QB) {
-    int s;
-    switch (group) {
-      case -1: s = launch_block<0>(W, m, n, U, i1, bits, codes, scales, zeros, W_hat, sc, st); break;
-      case 32: s = launch_block<32>(W, m, n, U, i1, bits, codes, scales, zeros, W_hat, sc, st); break;
-      case 64: s = launch_block<64>(W, m, n, U, i1, bits, codes, scales, zeros, W_hat, sc, st); break;
-      default: s = launch_block<128>(W, m, n, U, i1, bits, codes, scales, zeros, W_hat, sc, st); break;
+  for (int sb = 0; sb < n; sb += B2) {
+    const int sb_end = sb + B2 < n ? sb + B2 : n;
+    const int slab_end = B2 > QB ? sb_end : n;
+    for (int i1 = sb; i1 < sb_end; i1 += QB) {
+      int s;
+      switch (group) {
+        case -1: s = launch_block<0>(W, m, n, U, i1, bits, codes, scales, zeros, W_hat, sc, sb, slab_end, st); break;
+        case 32: s = launch_block<32>(W, m, n, U, i1, bits, codes, scales, zeros, W_hat, sc, sb, slab_end, st); break;
+        case 64: s = launch_block<64>(W, m, n, U, i1, bits, codes, scales, zeros, W_hat, sc, sb, slab_end, st); break;
+        default: s = launch_block<128>(W, m, n, U, i1, bits, codes, scales, zeros, W_hat, sc, sb, slab_end, st); break;
+      }
+      if (s != KRONQ_OK) return s;
+      const int i2 = i1 + QB;
+      if (i2 < sb_end) {
+        // inner: W[:, i2:sb_end] -= E_blk U[i1:i2, i2:sb_end]
+        const kq::GemmNT g = {sc.Eh + (i1 - sb), sc.El + (i1 - sb), B2, sc.Uth, sc.Utl, QB,
+                              W + i2, n, m, sb_end - i2, QB, -1.f, 0};
+        s = kq_gemm_nt_tc(&g, 1, info, st);
+        if (s != KRONQ_OK) return s;
+      }
     }
-    if (s != KRONQ_OK) return s;
-    const int i2 = i1 + QB;
-    if (i2 < n) {
-      // W[:, i2:] -= E U[i1:i2, i2:] = E (Ut)^T
-      const kq::GemmNT g = {sc.Eh, sc.El, QB, sc.Uth, sc.Utl, QB, W + i2, n, m, n - i2, QB, -1.f, 0};
-      s = kq_gemm_nt_tc(&g, 1, info, st);
+    if (sb_end < n) {
+      // outer: W[:, sb_end:] -= E_sb U[sb:sb_end, sb_end:]   (K = sb_end - sb)
+      const int K = sb_end - sb;
+      const float* Bh = sc.Uth;
+      const float* Bl = sc.Utl;
+      int ldb = QB;
+      if (B2 > QB) {
+        const dim3 g((n - sb_end + 31) / 32, (K + 31) / 32);
+        slab_transpose_kernel<<<g, 256, 0, st>>>(U, n, sb, K, sb_end, sc.Voh, sc.Vol, B2);
+        KQ_CHECK_LAUNCH();
+        Bh = sc.Voh;
+        Bl = sc.Vol;
+        ldb = B2;
+      }
+      // (one level: the block kernel already wrote U[sb:sb_end, sb_end:]^T into Ut)
+      const kq::GemmNT g = {sc.Eh, sc.El, B2, Bh, Bl, ldb, W + sb_end, n, m, n - sb_end, K,
+                            -1.f, 0};
+      const int s = kq_gemm_nt_tc(&g, 1, info, st);
       if (s != KRONQ_OK) return s;
     }
   }

@@ -250,3 +250,45 @@ def test_quantize_exact_ties_round_half_to_even(cuda):
     ref = oq.obs_quantize(W, U, 4, -1)
     np.testing.assert_array_equal(codes.cpu().numpy(), ref["codes"])
     assert list(ref["codes"][0, 2:8]) == [0, 0, 1, 2, 2, 2]
+
+
+def test_quantize_two_level_lazy_update_matches_one_level_and_oracle(cuda):
+    """n = 2304 spans two full 1024-column super-blocks and a ragged one: the
+    two-level lazy update (outer K = 1024 products) and the one-level update
+    (chosen when the workspace only fits it) are both exact reassociations of
+    the unblocked loop."""
+    m, n, bits = 160, 2304, 4
+    r = np.random.default_rng(77)
+    W = (r.standard_normal((m, n)) * 0.02).astype(np.float32)
+    U = ochol.inverse_cholesky(ochol.damp(spd(r, n, spread=1.0), 0.01)).astype(np.float32)
+    ref = oq.obs_quantize(W, U, bits, -1)
+
+    def a256(b):
+        return (b + 255) // 256 * 256
+
+    one_level = 2 * a256(m * 128 * 4) + 2 * a256(n * 128 * 4)
+    outs = []
+    for ws in (abi.workspace(m, n, bits, -1, device=cuda),
+               torch.empty(one_level, dtype=torch.uint8, device=cuda)):
+        codes = torch.empty((m, n), dtype=torch.uint8, device=cuda)
+        scales = torch.empty((m, 1), device=cuda)
+        zeros = torch.empty((m, 1), dtype=torch.uint8, device=cuda)
+        What = torch.empty((m, n), device=cuda)
+        abi.kronq_quantize_layer(t(W, cuda), t(U, cuda), bits, -1, 128, codes, scales, zeros, What,
+                                 None, ws)
+        cg = codes.cpu().numpy()
+        assert (cg == ref["codes"]).mean() >= 0.999
+        outs.append((cg, What.cpu().numpy()))
+    Hd = np.linalg.inv(U.astype(np.float64).T @ U.astype(np.float64))
+    lr = oq.row_losses(W - ref["W_hat"], Hd).sum()
+    for cg, wh in outs:
+        assert abs(oq.row_losses(W - wh, Hd).sum() / lr - 1) <= 0.01
+    assert (outs[0][0] == outs[1][0]).mean() >= 0.999
+    # a workspace below the one-level size is refused
+    with pytest.raises(abi.KronqError) as e:
+        abi.kronq_quantize_layer(t(W, cuda), t(U, cuda), bits, -1, 128,
+                                 torch.empty((m, n), dtype=torch.uint8, device=cuda),
+                                 torch.empty((m, 1), device=cuda),
+                                 torch.empty((m, 1), dtype=torch.uint8, device=cuda), None, None,
+                                 torch.empty(one_level - 256, dtype=torch.uint8, device=cuda))
+    assert e.value.code == -6
