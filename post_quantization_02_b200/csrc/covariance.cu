@@ -6,30 +6,25 @@
 // whose operands are both "MN-major": for a K-slab of tokens the features
 // (the M and N indices of the tile) are contiguous in memory.
 //
-// Kernel structure (one CTA per SM, persistent over work units).  A unit is
-// one output tile and one chunk of KC_ITERS K-slabs (4096 tokens); units are
-// handed out chunk-major, so all CTAs stream the same token range at about
-// the same time (L2 reuse of X) and every CTA gets the same number of units.
+// Kernel structure (one CTA per SM, persistent over output tiles):
 //   warp 0      TMA producer: per K-slab of 64 tokens, two 64x64 boxes of the
 //               row panel (A, 128 features) and four of the column panel (B,
 //               256 features), 128-byte swizzled, into a 4-stage ring.
 //   warp 1      one thread issues tcgen05.mma (M=128, N=256, K=16, bf16 in,
-//               fp32 accumulate in TMEM) into one of two accumulators (one
-//               per unit, alternating) and commits each stage back to the
-//               producer and each finished unit to the epilogue.
-//   warp 2      allocates / frees the 512 TMEM columns.
-//   warps 4-7   epilogue: a unit's partial sum, times alpha, goes to H by TMA
-//               reduce-adds of 32 x 32 boxes staged in shared memory (fp32
-//               round-to-nearest adds in L2), while the tensor core already
-//               fills the other accumulator.
-// Folding every 4096-token partial sum with round-to-nearest adds matters:
-// the tensor core's own fp32 accumulation rounds towards zero (measured ~
-// -6e-8 relative per K=16 step), so it only ever spans one chunk.
-// Before the kernel H <- beta H (or 0); only tiles that touch the upper
-// triangle are computed, and a last pass copies the upper triangle onto the
-// lower one, so the whole symmetric d x d result is written by every call.
-// When beta != 0 the old upper triangle is read, so the old H must be
-// symmetric.
+//               fp32 accumulate in TMEM) and commits each stage back to the
+//               producer, and each finished tile to the epilogue.
+//   warp 2      allocates / frees the 512 TMEM columns: the accumulator
+//               (256) and an fp32 master (256) that the epilogue folds each
+//               4096-token partial sum into.
+//   warps 4-7   epilogue: folds (tcgen05.ld / add / tcgen05.st), then per tile
+//               H = alpha master + beta H for the elements on or above the
+//               diagonal, stored twice: in place (row-contiguous vector
+//               stores) and mirrored (for a fixed column the 32 lanes of a
+//               warp write 32 consecutive floats of the transposed row).
+// Only tiles that touch the upper triangle are computed; with the mirrored
+// stores every element of the symmetric d x d result is written once per
+// call (the diagonal twice, with the same value).  When beta != 0 the old
+// upper triangle is read, so the old H must be symmetric.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -46,17 +41,16 @@ constexpr int BOX_BYTES = 64 * BK * 2;              // 64 features x 64 tokens o
 constexpr int A_BYTES = BM * BK * 2;                // 16 KB
 constexpr int B_BYTES = BN * BK * 2;                // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;      // 48 KB
-constexpr int TMEM_COLS = 2 * BN;  // two accumulators
+constexpr int TMEM_COLS = 2 * BN;  // accumulator + master
 constexpr int THREADS = 256;
-constexpr int STG_BYTES = 32 * 32 * 4;              // one 32 x 32 fp32 box
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 8 * STG_BYTES + 1024 + 256;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
 constexpr uint32_t IDESC = kq::idesc_f16(BM, BN, /*bf16*/ 1, /*A MN-major*/ 1, /*B MN-major*/ 1);
 
 struct Bars {
   uint64_t full[STAGES];
   uint64_t empty[STAGES];
-  uint64_t tfull[2];
-  uint64_t tempty[2];
+  uint64_t tfull;
+  uint64_t tempty;
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -87,23 +81,13 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, int32
   }
 }
 
-// C box += the 32 x 32 fp32 box in shared memory (TMA, bulk-group completion).
-KQ_DEV void tma_reduce_add_2d(const void* tmap, const void* src, int x, int y) {
-  asm volatile(
-      "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
-          reinterpret_cast<uint64_t>(tmap)),
-      "r"(kq::smem_u32(src)), "r"(x), "r"(y)
-      : "memory");
-}
-
 __global__ void __launch_bounds__(THREADS, 1)
-cov_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ CUtensorMap hmap,
-              int k_iters, int ncb, int num_tiles, int num_units, float alpha, int32_t* info) {
+cov_tc_kernel(const __grid_constant__ CUtensorMap tmap, float* __restrict__ H, int64_t ldh, int d,
+              int k_iters, int ncb, int num_tiles, float alpha, float beta, int32_t* info) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* tiles = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* staging = tiles + STAGES * STAGE_BYTES;      // 1024-byte aligned
-  Bars* bars = reinterpret_cast<Bars*>(staging + 8 * STG_BYTES);
+  Bars* bars = reinterpret_cast<Bars*>(tiles + STAGES * STAGE_BYTES);
   volatile int* abort = &bars->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -113,18 +97,13 @@ cov_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
       kq::mbar_init(&bars->full[s], 1);
       kq::mbar_init(&bars->empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      kq::mbar_init(&bars->tfull[b], 1);
-      kq::mbar_init(&bars->tempty[b], 4);
-    }
+    kq::mbar_init(&bars->tfull, 1);
+    kq::mbar_init(&bars->tempty, 4);
     kq::mbar_init(&bars->drain, 1);
     bars->abort = 0;
     kq::fence_barrier_init();
   }
-  if (warp == 0 && lane == 0) {
-    kq::prefetch_tmap(&tmap);
-    kq::prefetch_tmap(&hmap);
-  }
+  if (warp == 0 && lane == 0) kq::prefetch_tmap(&tmap);
   if (warp == 2) kq::tmem_alloc(&bars->tmem_base, TMEM_COLS);
   kq::tc_fence_before();
   __syncthreads();
@@ -135,13 +114,12 @@ cov_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
     if (lane == 0) {
       // ------------------------------------------------ TMA producer
       int it = 0;
-      bool ok = true;
-      for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+      for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
         int rb, cb;
-        tile_coords(u % num_tiles, ncb, rb, cb);
+        tile_coords(t, ncb, rb, cb);
         const int i0 = rb * BM, j0 = cb * BN;
-        const int k0 = (u / num_tiles) * KC_ITERS, k1 = min(k_iters, k0 + KC_ITERS);
-        for (int kb = k0; kb < k1; ++kb, ++it) {
+        bool ok = true;
+        for (int kb = 0; kb < k_iters; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
           if (!kq::mbar_wait(&bars->empty[s], ph ^ 1u, abort, info)) { ok = false; break; }
@@ -155,6 +133,7 @@ cov_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
           for (int q = 0; q < 4; ++q)
             kq::tma_load_2d(b + q * BOX_BYTES, &tmap, &bars->full[s], j0 + 64 * q, y);
         }
+        if (!ok) break;
       }
       // wind down: every stage's last armed phase must have landed
       for (int s = 0; s < STAGES; ++s) {
@@ -165,32 +144,34 @@ cov_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------ MMA issuer
-      int it = 0, uc = 0;
+      // One accumulator (TMEM columns [0, BN)); it is handed to the epilogue
+      // after every chunk of KC_ITERS K-slabs and reused once folded.
+      int it = 0, cc = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x, ++uc) {
-        const int k0 = (u / num_tiles) * KC_ITERS, k1 = min(k_iters, k0 + KC_ITERS);
-        const int buf = uc & 1;
-        if (!kq::mbar_wait(&bars->tempty[buf], ((uint32_t)(uc >> 1) & 1u) ^ 1u, abort, info)) break;
-        kq::tc_fence_after();
-        const uint32_t acc = tmem + (uint32_t)(buf * BN);
-        for (int kb = k0; kb < k1; ++kb, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-          if (!kq::mbar_wait(&bars->full[s], ph, abort, info)) { ok = false; break; }
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        for (int k0 = 0; k0 < k_iters && ok; k0 += KC_ITERS, ++cc) {
+          const int k1 = min(k_iters, k0 + KC_ITERS);
+          if (!kq::mbar_wait(&bars->tempty, ((uint32_t)cc & 1u) ^ 1u, abort, info)) { ok = false; break; }
           kq::tc_fence_after();
-          const uint32_t a_addr = kq::smem_u32(tiles + s * STAGE_BYTES);
-          const uint32_t b_addr = a_addr + A_BYTES;
+          for (int kb = k0; kb < k1; ++kb, ++it) {
+            const int s = it % STAGES;
+            const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+            if (!kq::mbar_wait(&bars->full[s], ph, abort, info)) { ok = false; break; }
+            kq::tc_fence_after();
+            const uint32_t a_addr = kq::smem_u32(tiles + s * STAGE_BYTES);
+            const uint32_t b_addr = a_addr + A_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            // MN-major, 128B swizzle: 8-row K atoms 1024 B apart (SBO), 64-wide
-            // feature atoms one TMA box apart (LBO); K step of 16 rows = 2048 B.
-            const uint64_t ad = kq::smem_desc(a_addr + kk * 2048, BOX_BYTES, 1024, kq::kLayoutSwizzle128B);
-            const uint64_t bd = kq::smem_desc(b_addr + kk * 2048, BOX_BYTES, 1024, kq::kLayoutSwizzle128B);
-            kq::mma_f16(acc, ad, bd, IDESC, (kb != k0) || (kk != 0));
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              // MN-major, 128B swizzle: 8-row K atoms 1024 B apart (SBO), 64-wide
+              // feature atoms one TMA box apart (LBO); K step of 16 rows = 2048 B.
+              const uint64_t ad = kq::smem_desc(a_addr + kk * 2048, BOX_BYTES, 1024, kq::kLayoutSwizzle128B);
+              const uint64_t bd = kq::smem_desc(b_addr + kk * 2048, BOX_BYTES, 1024, kq::kLayoutSwizzle128B);
+              kq::mma_f16(tmem, ad, bd, IDESC, (kb != k0) || (kk != 0));
+            }
+            kq::mma_commit(&bars->empty[s]);
           }
-          kq::mma_commit(&bars->empty[s]);
+          if (ok) kq::mma_commit(&bars->tfull);
         }
-        if (ok) kq::mma_commit(&bars->tfull[buf]);
       }
       // wind down: all MMAs issued by this thread complete before TMEM is freed
       kq::mma_commit(&bars->drain);
@@ -198,51 +179,89 @@ cov_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
     }
   } else if (warp >= 4) {
     // -------------------------------------------------- epilogue
-    // warp q = warp - 4 reads TMEM lanes 32 q .. 32 q + 31 (tile rows) and
-    // adds the unit's partial sum into H box by box (32 columns at a time),
-    // alternating between two staging buffers.
-    const int q = warp & 3;
+    // Each chunk's partial sum is folded into the fp32 master (TMEM columns
+    // [BN, 2 BN)) with ordinary round-to-nearest adds, so the tensor core's
+    // own accumulation only ever spans KC_ITERS * BK tokens.  The accumulator
+    // is released as soon as the fold is done; after the last chunk of a tile
+    // the master is written out (H = alpha master + beta H_old) together with
+    // its mirror image.
+    const int q = warp & 3;  // TMEM lane quadrant this warp may access
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-    uint8_t* stg = staging + (warp - 4) * 2 * STG_BYTES;
-    int uc = 0, nbox = 0;
-    for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++uc) {
+    int cc = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
       int rb, cb;
-      tile_coords(u % num_tiles, ncb, rb, cb);
+      tile_coords(t, ncb, rb, cb);
       const int i0 = rb * BM, j0 = cb * BN;
-      const int buf = uc & 1;
-      if (!kq::mbar_wait(&bars->tfull[buf], (uint32_t)(uc >> 1) & 1u, abort, info)) break;
-      kq::tc_fence_after();
+      const int row0 = i0 + q * 32;             // first row of this warp's 32 lanes
+      const int row = row0 + lane;
+      for (int k0 = 0; k0 < k_iters; k0 += KC_ITERS, ++cc) {
+        const bool first = k0 == 0, last = k0 + KC_ITERS >= k_iters;
+        if (!kq::mbar_wait(&bars->tfull, (uint32_t)cc & 1u, abort, info)) { ok = false; break; }
+        kq::tc_fence_after();
 #pragma unroll 1
-      for (int c = 0; c < BN; c += 32) {
-        if (j0 + c + 31 < i0 + q * 32) continue;     // box strictly below the diagonal: skipped
-        float v[32];
-        __syncwarp();
-        kq::tmem_ld32(tmem + lane_off + (uint32_t)(buf * BN + c), v);
-        kq::tmem_wait_ld();
-        uint8_t* box = stg + (nbox & 1) * STG_BYTES;
-        if (nbox >= 2) {
-          if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+        for (int c = 0; c < BN; c += 32) {
+          if (j0 + c >= d) break;                   // columns past the matrix (uniform)
+          if (j0 + c + 31 < row0) continue;         // strictly below the diagonal: never stored
+          float v[32], mst[32];
           __syncwarp();
-        }
+          kq::tmem_ld32(tmem + lane_off + (uint32_t)c, v);
+          if (!first) kq::tmem_ld32(tmem + lane_off + (uint32_t)(BN + c), mst);
+          kq::tmem_wait_ld();
+          if (!first) {
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch)
-          *reinterpret_cast<float4*>(box + lane * 128 + ((ch ^ (lane & 7)) << 4)) =
-              make_float4(alpha * v[4 * ch], alpha * v[4 * ch + 1], alpha * v[4 * ch + 2],
-                          alpha * v[4 * ch + 3]);
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        __syncwarp();
-        if (lane == 0) {
-          tma_reduce_add_2d(&hmap, box, j0 + c, i0 + q * 32);
-          asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+            for (int k = 0; k < 32; ++k) v[k] += mst[k];
+          }
+          kq::tmem_st32(tmem + lane_off + (uint32_t)(BN + c), v);
         }
-        ++nbox;
+        kq::tmem_wait_st();
+        kq::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) kq::mbar_arrive(&bars->tempty);   // accumulator free again
+        if (!last) continue;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          const int jc = j0 + c;
+          if (jc >= d) break;
+          if (jc + 31 < row0) continue;
+          float v[32];
+          __syncwarp();
+          kq::tmem_ld32(tmem + lane_off + (uint32_t)(BN + c), v);
+          kq::tmem_wait_ld();
+          if (row < d) {
+            float* dst = H + (int64_t)row * ldh + jc;
+            if (jc >= row0 + 31 && jc + 32 <= d) {
+              // whole chunk on or above the diagonal for every lane: vector stores
+#pragma unroll
+              for (int k = 0; k < 32; k += 4) {
+                float4 o = make_float4(alpha * v[k], alpha * v[k + 1], alpha * v[k + 2], alpha * v[k + 3]);
+                if (beta != 0.f) {
+                  const float4 h = *reinterpret_cast<const float4*>(dst + k);
+                  o.x = fmaf(beta, h.x, o.x); o.y = fmaf(beta, h.y, o.y);
+                  o.z = fmaf(beta, h.z, o.z); o.w = fmaf(beta, h.w, o.w);
+                }
+                v[k] = o.x; v[k + 1] = o.y; v[k + 2] = o.z; v[k + 3] = o.w;
+                *reinterpret_cast<float4*>(dst + k) = o;
+              }
+            } else {
+#pragma unroll
+              for (int k = 0; k < 32; ++k) {
+                if (jc + k < d && jc + k >= row) {
+                  float o = alpha * v[k];
+                  if (beta != 0.f) o = fmaf(beta, dst[k], o);
+                  v[k] = o;
+                  dst[k] = o;
+                }
+              }
+            }
+            // mirror: H[j][row] for j > row; for each j the warp writes 32 consecutive floats
+#pragma unroll
+            for (int k = 0; k < 32; ++k)
+              if (jc + k < d && jc + k > row) H[(int64_t)(jc + k) * ldh + row] = v[k];
+          }
+        }
       }
-      kq::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) kq::mbar_arrive(&bars->tempty[buf]);   // accumulator free again
     }
-    if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-    __syncwarp();
   }
 
   kq::tc_fence_before();
@@ -250,24 +269,6 @@ cov_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
   if (warp == 2) {
     kq::tc_fence_after();
     kq::tmem_dealloc(tmem, TMEM_COLS);
-  }
-}
-
-// H[j][i] = H[i][j] for j > i (the computed upper triangle onto the lower
-// one), through 32 x 32 shared-memory tiles: coalesced reads and writes.
-__global__ void __launch_bounds__(256) mirror_kernel(float* __restrict__ H, int64_t ldh, int d) {
-  __shared__ float tile[32][33];
-  const int bi = blockIdx.y, bj = blockIdx.x;       // source tile: rows 32 bi, columns 32 bj
-  if (bj < bi) return;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  for (int r = ty; r < 32; r += 8) {
-    const int i = 32 * bi + r, j = 32 * bj + tx;
-    tile[r][tx] = (i < d && j < d) ? H[(int64_t)i * ldh + j] : 0.f;
-  }
-  __syncthreads();
-  for (int r = ty; r < 32; r += 8) {
-    const int j = 32 * bj + r, i = 32 * bi + tx;     // destination H[j][i]
-    if (i < d && j < d && j > i) H[(int64_t)j * ldh + i] = tile[tx][r];
   }
 }
 
@@ -313,37 +314,21 @@ int kq_covariance(const uint16_t* A, int64_t N, int64_t d, int64_t lda, float* H
 
   auto encode = get_encode();
   if (!encode) return KRONQ_ERR_CUDA;
-  CUtensorMap tmap, hmap;
-  {
-    cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)N};
-    cuuint64_t strides[1] = {(cuuint64_t)lda * 2};
-    cuuint32_t box[2] = {64, (cuuint32_t)BK};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(A), dims,
-                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return KRONQ_ERR_UNSUPPORTED;
-  }
-  {
-    cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)d};
-    cuuint64_t strides[1] = {(cuuint64_t)ldh * 4};
-    cuuint32_t box[2] = {32, 32};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = encode(&hmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, H, dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return KRONQ_ERR_UNSUPPORTED;
-  }
+  CUtensorMap tmap;
+  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)N};
+  cuuint64_t strides[1] = {(cuuint64_t)lda * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)BK};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(A), dims,
+                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return KRONQ_ERR_UNSUPPORTED;
 
   const int nrb = (int)((d + BM - 1) / BM), ncb = (int)((d + BN - 1) / BN);
   int num_tiles = 0;
   for (int cb = 0; cb < ncb; ++cb) num_tiles += (2 * cb + 2 < nrb) ? 2 * cb + 2 : nrb;
   const int k_iters = (int)((N + BK - 1) / BK);
-  const int chunks = (k_iters + KC_ITERS - 1) / KC_ITERS;
-  const int64_t units64 = (int64_t)num_tiles * chunks;
-  if (units64 > INT32_MAX) return KRONQ_ERR_UNSUPPORTED;
-  const int num_units = (int)units64;
 
   static bool attr_set = false;
   if (!attr_set) {
@@ -352,17 +337,9 @@ int kq_covariance(const uint16_t* A, int64_t N, int64_t d, int64_t lda, float* H
       return KRONQ_ERR_CUDA;
     attr_set = true;
   }
-  // H <- beta H, then the units add alpha A^T A into its upper tiles
-  if (beta != 1.f) {
-    scale_kernel<<<4 * kqh::num_sms(), 256, 0, st>>>(H, ldh, (int)d, beta);
-    KQ_CHECK_LAUNCH();
-  }
-  const int grid = num_units < kqh::num_sms() ? num_units : kqh::num_sms();
-  cov_tc_kernel<<<grid, THREADS, SMEM_BYTES, st>>>(tmap, hmap, k_iters, ncb, num_tiles, num_units,
-                                                   alpha, info);
-  KQ_CHECK_LAUNCH();
-  const int nt = (int)((d + 31) / 32);
-  mirror_kernel<<<dim3(nt, nt), 256, 0, st>>>(H, ldh, (int)d);
+  const int grid = num_tiles < kqh::num_sms() ? num_tiles : kqh::num_sms();
+  cov_tc_kernel<<<grid, THREADS, SMEM_BYTES, st>>>(tmap, H, ldh, (int)d, k_iters, ncb, num_tiles,
+                                                   alpha, beta, info);
   KQ_CHECK_LAUNCH();
   return KRONQ_OK;
 }
