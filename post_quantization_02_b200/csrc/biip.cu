@@ -192,80 +192,111 @@ col_mix_kernel(float* __restrict__ X, int C, int L2, int Q, const float* __restr
   }
 }
 
-// Row pass, fast path (one segment of L2 = 128 E entries per CTA, no odd
-// factor): Walsh-Hadamard butterflies in registers.  Thread t first holds
-// entries t + 128 k (coalesced loads; scaling and signs fused), which makes
-// the stages with h >= 128 thread-local; one padded shared-memory transpose
-// gives it entries E t .. E t + E - 1 for the stages h < E; the stages
-// E <= h < 128 pair thread t with t ^ (h / E) by shuffles.
+// Row pass, fast path (no odd factor): one segment of L2 = 128 E entries of
+// two rows per CTA, Walsh-Hadamard butterflies in registers.  Thread t first
+// holds entries t + 128 k (coalesced loads; the row scale and the column
+// factor cf = column scale x sign fused, cf loaded once for both rows), which
+// makes the stages with h >= 128 thread-local; one padded shared-memory
+// transpose gives it entries E t .. E t + E - 1 for the stages h < E; the
+// stages E <= h < 128 pair thread t with t ^ (h / E) by shuffles.
 template <int E>
 __global__ void __launch_bounds__(128)
-row_fht_kernel(float* __restrict__ X, int C, const float* __restrict__ rs,
-               const float* __restrict__ cs, const int8_t* __restrict__ sign, int inverse) {
+row_fht_kernel(float* __restrict__ X, int R, int C, const float* __restrict__ rs,
+               const float* __restrict__ cf, int inverse) {
   constexpr int L2 = 128 * E;
-  __shared__ float sm[L2 + L2 / 32];
+  constexpr int RPC = 2;                      // rows per CTA
+  __shared__ float sm[RPC][L2 + L2 / 32];
   const int t = threadIdx.x;
-  const int64_t r = blockIdx.x;
   const int c0 = blockIdx.y * L2;
-  float* base = X + r * C + c0;
-  const float rsc = rs ? rs[r] : 1.f;
-  float v[E];
+  const int64_t r0 = (int64_t)blockIdx.x * RPC;
+  const int nr = (R - r0) < RPC ? (int)(R - r0) : RPC;
+  float v[RPC][E];
+  float f[E];
 #pragma unroll
-  for (int k = 0; k < E; ++k) {
-    const int c = c0 + t + 128 * k;
-    float x = base[t + 128 * k];
-    if (!inverse) x = x * (rsc * (cs ? cs[c] : 1.f)) * (float)sign[c];
-    v[k] = x;
+  for (int k = 0; k < E; ++k) f[k] = cf[c0 + t + 128 * k];
+#pragma unroll
+  for (int q = 0; q < RPC; ++q) {
+    if (q < nr) {
+      const float* base = X + (r0 + q) * C + c0;
+      const float rsc = rs ? rs[r0 + q] : 1.f;
+#pragma unroll
+      for (int k = 0; k < E; ++k) {
+        const float x = base[t + 128 * k];
+        v[q][k] = inverse ? x : x * (rsc * f[k]);
+      }
+    } else {
+#pragma unroll
+      for (int k = 0; k < E; ++k) v[q][k] = 0.f;
+    }
   }
 #pragma unroll
-  for (int h = 1; h < E; h <<= 1)
+  for (int q = 0; q < RPC; ++q) {
 #pragma unroll
-    for (int k = 0; k < E; ++k)
-      if (!(k & h)) {
-        const float a = v[k], b = v[k + h];
-        v[k] = a + b;
-        v[k + h] = a - b;
-      }
+    for (int h = 1; h < E; h <<= 1)
 #pragma unroll
-  for (int k = 0; k < E; ++k) {
-    const int i = t + 128 * k;
-    sm[i + (i >> 5)] = v[k];
+      for (int k = 0; k < E; ++k)
+        if (!(k & h)) {
+          const float a = v[q][k], b = v[q][k + h];
+          v[q][k] = a + b;
+          v[q][k + h] = a - b;
+        }
+#pragma unroll
+    for (int k = 0; k < E; ++k) {
+      const int i = t + 128 * k;
+      sm[q][i + (i >> 5)] = v[q][k];
+    }
   }
   __syncthreads();
 #pragma unroll
-  for (int k = 0; k < E; ++k) {
-    const int i = E * t + k;
-    v[k] = sm[i + (i >> 5)];
-  }
-#pragma unroll
-  for (int h = 1; h < E; h <<= 1)
-#pragma unroll
-    for (int k = 0; k < E; ++k)
-      if (!(k & h)) {
-        const float a = v[k], b = v[k + h];
-        v[k] = a + b;
-        v[k + h] = a - b;
-      }
-#pragma unroll
-  for (int m = 1; m < 128 / E; m <<= 1) {
-    const bool upper = (t & m) != 0;
+  for (int q = 0; q < RPC; ++q) {
 #pragma unroll
     for (int k = 0; k < E; ++k) {
-      const float o = __shfl_xor_sync(0xffffffffu, v[k], m);
-      v[k] = upper ? (o - v[k]) : (v[k] + o);
+      const int i = E * t + k;
+      v[q][k] = sm[q][i + (i >> 5)];
+    }
+#pragma unroll
+    for (int h = 1; h < E; h <<= 1)
+#pragma unroll
+      for (int k = 0; k < E; ++k)
+        if (!(k & h)) {
+          const float a = v[q][k], b = v[q][k + h];
+          v[q][k] = a + b;
+          v[q][k + h] = a - b;
+        }
+#pragma unroll
+    for (int m = 1; m < 128 / E; m <<= 1) {
+      const bool upper = (t & m) != 0;
+#pragma unroll
+      for (int k = 0; k < E; ++k) {
+        const float o = __shfl_xor_sync(0xffffffffu, v[q][k], m);
+        v[q][k] = upper ? (o - v[q][k]) : (v[q][k] + o);
+      }
     }
   }
   const float norm = rsqrtf((float)L2);
 #pragma unroll
-  for (int k = 0; k < E; ++k) {
-    const int c = c0 + E * t + k;
-    float x = v[k] * norm;
-    if (inverse) x = x * (float)sign[c] * (rsc * (cs ? cs[c] : 1.f));
-    v[k] = x;
-  }
+  for (int q = 0; q < RPC; ++q) {
+    if (q >= nr) break;
+    float* base = X + (r0 + q) * C + c0;
+    const float rsc = rs ? rs[r0 + q] : 1.f;
 #pragma unroll
-  for (int k = 0; k < E; k += 4)
-    *reinterpret_cast<float4*>(base + E * t + k) = make_float4(v[k], v[k + 1], v[k + 2], v[k + 3]);
+    for (int k = 0; k < E; k += 4) {
+      float o[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        o[u] = v[q][k + u] * norm;
+        if (inverse) o[u] *= rsc * cf[c0 + E * t + k + u];
+      }
+      *reinterpret_cast<float4*>(base + E * t + k) = make_float4(o[0], o[1], o[2], o[3]);
+    }
+  }
+}
+
+// cf[c] = cs[c] sign[c] (cs may be null: 1).
+__global__ void col_factor_kernel(const float* __restrict__ cs, const int8_t* __restrict__ sign,
+                                  int C, float* __restrict__ cf) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c < C) cf[c] = (cs ? cs[c] : 1.f) * (float)sign[c];
 }
 
 // Column pass, one factor H_{NR} (NR = 2^LG <= 64) of the Walsh-Hadamard
@@ -364,14 +395,16 @@ int set_attrs() {
 
 // Apply T D along rows (row pass, with scaling) of an R x C matrix.
 int row_pass(float* X, int R, int C, const float* rs, const float* cs, const int8_t* sign,
-             const Split& sp, const float* M, int inverse, cudaStream_t st) {
+             const Split& sp, const float* M, int inverse, float* cf, cudaStream_t st) {
   if (sp.Q == 1 && sp.L2 >= 512) {
-    const dim3 g(R, C / sp.L2);
+    col_factor_kernel<<<(C + 255) / 256, 256, 0, st>>>(cs, sign, C, cf);
+    KQ_CHECK_LAUNCH();
+    const dim3 g((R + 1) / 2, C / sp.L2);
     switch (sp.L2) {
-      case 512: row_fht_kernel<4><<<g, 128, 0, st>>>(X, C, rs, cs, sign, inverse); break;
-      case 1024: row_fht_kernel<8><<<g, 128, 0, st>>>(X, C, rs, cs, sign, inverse); break;
-      case 2048: row_fht_kernel<16><<<g, 128, 0, st>>>(X, C, rs, cs, sign, inverse); break;
-      default: row_fht_kernel<32><<<g, 128, 0, st>>>(X, C, rs, cs, sign, inverse); break;
+      case 512: row_fht_kernel<4><<<g, 128, 0, st>>>(X, R, C, rs, cf, inverse); break;
+      case 1024: row_fht_kernel<8><<<g, 128, 0, st>>>(X, R, C, rs, cf, inverse); break;
+      case 2048: row_fht_kernel<16><<<g, 128, 0, st>>>(X, R, C, rs, cf, inverse); break;
+      default: row_fht_kernel<32><<<g, 128, 0, st>>>(X, R, C, rs, cf, inverse); break;
     }
     KQ_CHECK_LAUNCH();
     return KRONQ_OK;
@@ -465,7 +498,8 @@ int kq_biip_rotate(float* W, int64_t m64, int64_t n64, float* HX, float* HG, con
   float* rSX = reinterpret_cast<float*>(w);
   float* rSG = rSX + n;
   w += a256((size_t)(m + n) * sizeof(float));
-  w += a256((size_t)(m + n) * sizeof(float));  // spare slot
+  float* cf = reinterpret_cast<float*>(w);      // column factors of a row pass
+  w += a256((size_t)(m + n) * sizeof(float));
   float* Mn = reinterpret_cast<float*>(w);
   w += a256(64 * 64 * sizeof(float));
   float* Mm = reinterpret_cast<float*>(w);
@@ -484,7 +518,7 @@ int kq_biip_rotate(float* W, int64_t m64, int64_t n64, float* HX, float* HG, con
       if (s) return s;
     }
     if (in_r) {
-      int s = row_pass(W, m, n, rSG, rSX, sv, spn, Mn, 1, st);
+      int s = row_pass(W, m, n, rSG, rSX, sv, spn, Mn, 1, cf, st);
       if (s) return s;
     } else {
       scale_only_kernel<<<4 * sms, 256, 0, st>>>(W, m, n, rSG, rSX);
@@ -510,7 +544,7 @@ int kq_biip_rotate(float* W, int64_t m64, int64_t n64, float* HX, float* HG, con
 
   // ---- W' = U (S_G W S_X) V^T
   if (in_r) {
-    int s = row_pass(W, m, n, SG, SX, sv, spn, Mn, 0, st);
+    int s = row_pass(W, m, n, SG, SX, sv, spn, Mn, 0, cf, st);
     if (s) return s;
   } else {
     scale_only_kernel<<<4 * sms, 256, 0, st>>>(W, m, n, SG, SX);
@@ -522,7 +556,7 @@ int kq_biip_rotate(float* W, int64_t m64, int64_t n64, float* HX, float* HG, con
   }
   // ---- H_X' = V S_X^-1 H_X S_X^-1 V^T
   if (in_r) {
-    int s = row_pass(HX, n, n, rSX, rSX, sv, spn, Mn, 0, st);
+    int s = row_pass(HX, n, n, rSX, rSX, sv, spn, Mn, 0, cf, st);
     if (s) return s;
     s = col_pass(HX, n, n, sv, spn, Mn, 0, st);
     if (s) return s;
@@ -532,7 +566,7 @@ int kq_biip_rotate(float* W, int64_t m64, int64_t n64, float* HX, float* HG, con
   }
   // ---- H_G' = U S_G^-1 H_G S_G^-1 U^T
   if (out_r) {
-    int s = row_pass(HG, m, m, rSG, rSG, su, spm, Mm, 0, st);
+    int s = row_pass(HG, m, m, rSG, rSG, su, spm, Mm, 0, cf, st);
     if (s) return s;
     s = col_pass(HG, m, m, su, spm, Mm, 0, st);
     if (s) return s;

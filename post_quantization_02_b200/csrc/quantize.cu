@@ -20,6 +20,7 @@
 //                     as tf32 hi / lo planes (tf32x3.cuh) for the lazy update.
 //   lazy update       W[:, i+128:] -= E U_c[i:i+128, i+128:] on the tensor cores
 //                     (kq_gemm_nt_tc: tf32, three-term split, TMA reduce into W)
+#include <algorithm>
 #include <mutex>
 
 #include "common.cuh"
@@ -31,8 +32,10 @@ namespace {
 
 constexpr int QB = 128;          // column block
 constexpr int ROWS_PER_CTA = 32;
+constexpr int OBS_THREADS = 8 * ROWS_PER_CTA;   // 8 threads per row
 constexpr int US_LD = QB + 4;    // padded row of the U_c block in shared memory
-constexpr int TT_LD = 33;        // transposition tile of the U_c slab (QB x 32)
+constexpr int TT_W = 8;          // columns per transposition slice of the U_c slab
+constexpr int TT_LD = TT_W + 1;  // its shared-memory tile (QB x TT_W), padded
 
 struct Grid {
   float scale;
@@ -91,7 +94,7 @@ __global__ void row_params_kernel(const float* __restrict__ W, int m, int n, int
 }
 
 template <int GROUP>  // 0: per-channel grid; else 32, 64 or 128
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(OBS_THREADS)
 obs_block_kernel(const float* __restrict__ W, int m, int n, const float* __restrict__ U, int i1,
                  int bits, uint8_t* __restrict__ codes, float* __restrict__ scales,
                  uint8_t* __restrict__ zeros, float* __restrict__ W_hat, float* __restrict__ Eh,
@@ -109,18 +112,19 @@ obs_block_kernel(const float* __restrict__ W, int m, int n, const float* __restr
 
   // The lazy update's B operand: Ut[c - i2][k] = U[i1 + k][c] for
   // i2 <= c < slab_end (the rest of the super-block, or of the matrix with
-  // one level), in 32-column slices spread over the CTAs, as tf32 hi / lo planes.
+  // one level), in 8-column slices spread over all the CTAs (so that no CTA
+  // starts its column loop much later than the others), as tf32 hi / lo planes.
   {
     const int i2 = i1 + QB;
-    const int slices = (slab_end - i2) / 32;
+    const int slices = (slab_end - i2) / TT_W;
     for (int sl = blockIdx.x; sl < slices; sl += gridDim.x) {
-      const int c0 = i2 + 32 * sl;
-      for (int e = tid; e < QB * 32; e += blockDim.x) {
-        const int k = e >> 5, cc = e & 31;
+      const int c0 = i2 + TT_W * sl;
+      for (int e = tid; e < QB * TT_W; e += blockDim.x) {
+        const int k = e / TT_W, cc = e % TT_W;
         Tt[k * TT_LD + cc] = U[(int64_t)(i1 + k) * n + c0 + cc];
       }
       __syncthreads();
-      for (int e = tid; e < QB * 32; e += blockDim.x) {
+      for (int e = tid; e < QB * TT_W; e += blockDim.x) {
         const int cc = e >> 7, k = e & (QB - 1);
         const float v = Tt[k * TT_LD + cc];
         const float h = kq::tf32x3::hi(v);
@@ -298,6 +302,39 @@ __global__ void pack_kernel(const uint8_t* __restrict__ codes, int64_t m, int64_
   }
 }
 
+// Fast path for n % 16 == 0: 16 codes (one 16-byte load) per item give two
+// 32-bit words (4-bit) or one (2-bit); the flattened code index maps to the
+// flattened word index because rows hold whole items.
+template <int BITS>
+__global__ void pack16_kernel(const uint4* __restrict__ codes, int64_t items,
+                              uint32_t* __restrict__ packed) {
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < items;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const uint4 v = codes[e];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    if (BITS == 4) {
+      uint32_t o[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t a = w[2 * h], b = w[2 * h + 1];   // bytes c0..c3, c4..c7
+        o[h] = (a & 0xFu) | ((a >> 4) & 0xF0u) | ((a >> 8) & 0xF00u) | ((a >> 12) & 0xF000u) |
+               ((b & 0xFu) << 16) | ((b << 12) & 0xF00000u) | ((b << 8) & 0xF000000u) |
+               ((b << 4) & 0xF0000000u);
+      }
+      reinterpret_cast<uint2*>(packed)[e] = make_uint2(o[0], o[1]);
+    } else {
+      uint32_t o = 0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t a = w[q];
+        const uint32_t c = (a & 0x3u) | ((a >> 6) & 0xCu) | ((a >> 12) & 0x30u) | ((a >> 18) & 0xC0u);
+        o |= c << (8 * q);
+      }
+      packed[e] = o;
+    }
+  }
+}
+
 __global__ void unpack_kernel(const uint32_t* __restrict__ packed, int64_t m, int64_t n, int bits,
                               int64_t wpr, uint8_t* __restrict__ codes) {
   const int per = 32 / bits;
@@ -358,7 +395,7 @@ int launch_block(const float* W, int m, int n, const float* U, int i1, int bits,
     attr = true;
   }
   const int grid = (m + ROWS_PER_CTA - 1) / ROWS_PER_CTA;
-  obs_block_kernel<GROUP><<<grid, 256, smem, st>>>(W, m, n, U, i1, bits, codes, scales, zeros,
+  obs_block_kernel<GROUP><<<grid, OBS_THREADS, smem, st>>>(W, m, n, U, i1, bits, codes, scales, zeros,
                                                    W_hat, sc.Eh + (i1 - sb), sc.El + (i1 - sb),
                                                    sc.B2, sc.Uth, sc.Utl, slab_end);
   KQ_CHECK_LAUNCH();
@@ -480,6 +517,16 @@ int kq_pack(const uint8_t* codes, int64_t m, int64_t n, int bits, uint32_t* pack
   if (m == 0 || n == 0) return KRONQ_OK;
   if (!codes || !packed || !kqh::aligned(packed, 4)) return KRONQ_ERR_INVALID_ARG;
   const int64_t wpr = (n * bits + 31) / 32;
+  if (n % 16 == 0 && kqh::aligned(codes, 16) && kqh::aligned(packed, bits == 4 ? 8 : 4)) {
+    const int64_t items = m * n / 16;
+    const int grid = (int)std::min<int64_t>((items + 255) / 256, 8 * (int64_t)kqh::num_sms());
+    if (bits == 4)
+      pack16_kernel<4><<<grid, 256, 0, st>>>(reinterpret_cast<const uint4*>(codes), items, packed);
+    else
+      pack16_kernel<2><<<grid, 256, 0, st>>>(reinterpret_cast<const uint4*>(codes), items, packed);
+    KQ_CHECK_LAUNCH();
+    return KRONQ_OK;
+  }
   pack_kernel<<<4 * kqh::num_sms(), 256, 0, st>>>(codes, m, n, bits, wpr, packed, nullptr);
   KQ_CHECK_LAUNCH();
   return KRONQ_OK;
