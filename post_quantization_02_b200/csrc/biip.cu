@@ -273,6 +273,17 @@ row_fht_kernel(float* __restrict__ X, int R, int C, const float* __restrict__ rs
       }
     }
   }
+  // back to entries t + 128 k through shared memory, so that every store
+  // instruction writes 128 contiguous bytes per warp
+  __syncthreads();
+#pragma unroll
+  for (int q = 0; q < RPC; ++q)
+#pragma unroll
+    for (int k = 0; k < E; ++k) {
+      const int i = E * t + k;
+      sm[q][i + (i >> 5)] = v[q][k];
+    }
+  __syncthreads();
   const float norm = rsqrtf((float)L2);
 #pragma unroll
   for (int q = 0; q < RPC; ++q) {
@@ -280,14 +291,11 @@ row_fht_kernel(float* __restrict__ X, int R, int C, const float* __restrict__ rs
     float* base = X + (r0 + q) * C + c0;
     const float rsc = rs ? rs[r0 + q] : 1.f;
 #pragma unroll
-    for (int k = 0; k < E; k += 4) {
-      float o[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        o[u] = v[q][k + u] * norm;
-        if (inverse) o[u] *= rsc * cf[c0 + E * t + k + u];
-      }
-      *reinterpret_cast<float4*>(base + E * t + k) = make_float4(o[0], o[1], o[2], o[3]);
+    for (int k = 0; k < E; ++k) {
+      const int i = t + 128 * k;
+      float o = sm[q][i + (i >> 5)] * norm;
+      if (inverse) o *= rsc * f[k];
+      base[i] = o;
     }
   }
 }
