@@ -81,6 +81,70 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, int32
   }
 }
 
+// Row `row` of H, columns jc .. jc+31 (v = the fp32 sums): H = alpha v + beta H
+// for the elements on or above the diagonal, and their mirror images below
+// it.  row0 is the first row of the calling warp (rows row0 .. row0+31).
+__device__ __forceinline__ void store_row_chunk(float* __restrict__ H, int64_t ldh, int d, int row,
+                                                int row0, int jc, float (&v)[32], float alpha,
+                                                float beta) {
+  float* dst = H + (int64_t)row * ldh + jc;
+  if (jc >= row0 + 31 && jc + 32 <= d) {
+    // whole chunk on or above the diagonal for every lane: vector stores
+#pragma unroll
+    for (int k = 0; k < 32; k += 4) {
+      float4 o = make_float4(alpha * v[k], alpha * v[k + 1], alpha * v[k + 2], alpha * v[k + 3]);
+      if (beta != 0.f) {
+        const float4 h = *reinterpret_cast<const float4*>(dst + k);
+        o.x = fmaf(beta, h.x, o.x); o.y = fmaf(beta, h.y, o.y);
+        o.z = fmaf(beta, h.z, o.z); o.w = fmaf(beta, h.w, o.w);
+      }
+      v[k] = o.x; v[k + 1] = o.y; v[k + 2] = o.z; v[k + 3] = o.w;
+      *reinterpret_cast<float4*>(dst + k) = o;
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+      if (jc + k < d && jc + k >= row) {
+        float o = alpha * v[k];
+        if (beta != 0.f) o = fmaf(beta, dst[k], o);
+        v[k] = o;
+        dst[k] = o;
+      }
+    }
+  }
+  // mirror: H[j][row] for j > row; for each j the warp writes 32 consecutive floats
+#pragma unroll
+  for (int k = 0; k < 32; ++k)
+    if (jc + k < d && jc + k > row) H[(int64_t)(jc + k) * ldh + row] = v[k];
+}
+
+KQ_DEV void red_add_v4(float* p, float a, float b, float c, float e) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(e)
+               : "memory");
+}
+
+KQ_DEV void red_add(float* p, float a) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(a) : "memory");
+}
+
+// As store_row_chunk, for a tile that several CTA pairs share: adds alpha v
+// into H on and above the diagonal with reductions.  The mirror images are
+// copied once all parts are in (mirror_tiles_kernel), so that H stays exactly
+// symmetric whatever order the parts arrive in.
+__device__ __forceinline__ void add_row_chunk(float* __restrict__ H, int64_t ldh, int d, int row,
+                                              int row0, int jc, const float (&v)[32], float alpha) {
+  float* dst = H + (int64_t)row * ldh + jc;
+  if (jc >= row0 + 31 && jc + 32 <= d) {
+#pragma unroll
+    for (int k = 0; k < 32; k += 4)
+      red_add_v4(dst + k, alpha * v[k], alpha * v[k + 1], alpha * v[k + 2], alpha * v[k + 3]);
+  } else {
+#pragma unroll
+    for (int k = 0; k < 32; ++k)
+      if (jc + k < d && jc + k >= row) red_add(dst + k, alpha * v[k]);
+  }
+}
+
 __global__ void __launch_bounds__(THREADS, 1)
 cov_tc_kernel(const __grid_constant__ CUtensorMap tmap, float* __restrict__ H, int64_t ldh, int d,
               int k_iters, int ncb, int num_tiles, float alpha, float beta, int32_t* info) {
@@ -228,37 +292,7 @@ cov_tc_kernel(const __grid_constant__ CUtensorMap tmap, float* __restrict__ H, i
           __syncwarp();
           kq::tmem_ld32(tmem + lane_off + (uint32_t)(BN + c), v);
           kq::tmem_wait_ld();
-          if (row < d) {
-            float* dst = H + (int64_t)row * ldh + jc;
-            if (jc >= row0 + 31 && jc + 32 <= d) {
-              // whole chunk on or above the diagonal for every lane: vector stores
-#pragma unroll
-              for (int k = 0; k < 32; k += 4) {
-                float4 o = make_float4(alpha * v[k], alpha * v[k + 1], alpha * v[k + 2], alpha * v[k + 3]);
-                if (beta != 0.f) {
-                  const float4 h = *reinterpret_cast<const float4*>(dst + k);
-                  o.x = fmaf(beta, h.x, o.x); o.y = fmaf(beta, h.y, o.y);
-                  o.z = fmaf(beta, h.z, o.z); o.w = fmaf(beta, h.w, o.w);
-                }
-                v[k] = o.x; v[k + 1] = o.y; v[k + 2] = o.z; v[k + 3] = o.w;
-                *reinterpret_cast<float4*>(dst + k) = o;
-              }
-            } else {
-#pragma unroll
-              for (int k = 0; k < 32; ++k) {
-                if (jc + k < d && jc + k >= row) {
-                  float o = alpha * v[k];
-                  if (beta != 0.f) o = fmaf(beta, dst[k], o);
-                  v[k] = o;
-                  dst[k] = o;
-                }
-              }
-            }
-            // mirror: H[j][row] for j > row; for each j the warp writes 32 consecutive floats
-#pragma unroll
-            for (int k = 0; k < 32; ++k)
-              if (jc + k < d && jc + k > row) H[(int64_t)(jc + k) * ldh + row] = v[k];
-          }
+          if (row < d) store_row_chunk(H, ldh, d, row, row0, jc, v, alpha, beta);
         }
       }
     }
@@ -272,13 +306,314 @@ cov_tc_kernel(const __grid_constant__ CUtensorMap tmap, float* __restrict__ H, i
   }
 }
 
+// ------------------------------------------------------------------------
+// The same product on CTA pairs (cta_group::2): a cluster of two CTAs owns a
+// 256 x 256 tile of H.  Per K-slab of 64 tokens each CTA loads its 128 rows
+// of the tile's row panel and its 128 of the column panel (32 KB, against
+// 48 KB per 128 x 256 tile for one CTA alone), and the even CTA issues
+// tcgen05.mma.cta_group::2 with M = N = 256: the pair's two tensor cores
+// each compute their 128 x 256 half from 128 + 256 features staged across
+// both shared memories.  Per unit of tensor-core work the shared-memory
+// traffic drops by a third, and the same 192 KB ring covers 50 % more
+// K-slabs of load latency.  Each CTA folds and stores its own 128 rows
+// exactly as the single-CTA kernel does.
+//
+// Work is dealt out so that every pair streams the same tokens at the same
+// time (one 64-token slab of A then serves all pairs from L2, the reason the
+// covariance reads A from DRAM about once): with P pairs and T tiles, the
+// first W = T / P waves give each pair whole tiles.  Of the R = T mod P tiles
+// left, each goes to one pair for its first k* token chunks (chunks of
+// KC_ITERS K-slabs, the fold granularity) while the P - R pairs that would
+// otherwise sit idle take the last C - k* chunks of g = ceil(R / (P - R))
+// tiles each, k* balancing the two: k* = ceil(g C / (g + 1)).  Only two token
+// offsets are then in flight.  A tile split that way is added into H by its
+// two pairs with fp32 reductions, onto an H the host has zeroed (or scaled by
+// beta) first; with beta = 0 the sum 0 + a + b does not depend on the order.
+//
+// Barriers: full[s] of the even CTA counts the bytes of both CTAs' loads
+// (its producer arms it for 2 x 32 KB; the odd CTA's loads complete on it
+// through the cta_group::2 form of the TMA load); empty[s] and tfull exist
+// in both CTAs and receive one multicast tcgen05.commit each; tempty of the
+// even CTA collects the 8 epilogue warps of the pair.
+constexpr int P_BM = 128;                            // rows of the tile per CTA
+constexpr int P_TILE = 256;                          // the pair's square tile
+constexpr int P_STAGES = 7;
+constexpr int P_A_BYTES = P_BM * BK * 2;             // 16 KB
+constexpr int P_B_BYTES = (P_TILE / 2) * BK * 2;     // 16 KB
+constexpr int P_STAGE_BYTES = P_A_BYTES + P_B_BYTES; // 32 KB
+constexpr int P_SMEM_BYTES = P_STAGES * P_STAGE_BYTES + 1024 + 256;
+constexpr uint32_t P_IDESC = kq::idesc_f16(2 * P_BM, P_TILE, /*bf16*/ 1, /*A MN-major*/ 1, /*B MN-major*/ 1);
+static_assert(P_SMEM_BYTES <= 227 * 1024, "pair ring exceeds the shared-memory limit");
+
+struct PairBars {
+  uint64_t full[P_STAGES];
+  uint64_t empty[P_STAGES];
+  uint64_t tfull;
+  uint64_t tempty;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+// Square tiles in the upper triangle, ordered by column block: column block
+// cb holds the row blocks 0 .. cb, i.e. cb (cb + 1) / 2 tiles precede it.
+__device__ __forceinline__ void pair_tile_coords(int t, int& rb, int& cb) {
+  int c = (int)((sqrt(8.0 * (double)t + 1.0) - 1.0) * 0.5);
+  while ((long long)(c + 1) * (c + 2) / 2 <= t) ++c;
+  while ((long long)c * (c + 1) / 2 > t) --c;
+  cb = c;
+  rb = t - c * (c + 1) / 2;
+}
+
+struct PairSchedule {
+  int tiles, chunks;   // T, C
+  int waves, rest;     // W = T / P, R = T mod P
+  int per_helper;      // g
+  int kstar;           // k*
+};
+
+// The idx-th segment (tile t, chunks [c0, c1)) of pair p; false when p has
+// no more.
+__device__ __forceinline__ bool pair_segment(const PairSchedule& S, int p, int np, int idx, int& t,
+                                             int& c0, int& c1) {
+  if (idx < S.waves) {
+    t = p + idx * np;
+    c0 = 0;
+    c1 = S.chunks;
+    return true;
+  }
+  idx -= S.waves;
+  if (S.rest == 0) return false;
+  const int t0 = S.waves * np;
+  if (p < S.rest) {
+    if (idx > 0) return false;
+    t = t0 + p;
+    c0 = 0;
+    c1 = S.kstar;
+    return true;
+  }
+  if (S.kstar >= S.chunks || idx >= S.per_helper) return false;
+  const int i = (p - S.rest) * S.per_helper + idx;
+  if (i >= S.rest) return false;
+  t = t0 + i;
+  c0 = S.kstar;
+  c1 = S.chunks;
+  return true;
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+cov_pair_kernel(const __grid_constant__ CUtensorMap tmap, float* __restrict__ H, int64_t ldh, int d,
+                int k_iters, const PairSchedule sched, float alpha, float beta, int32_t* info) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* tiles = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  PairBars* bars = reinterpret_cast<PairBars*>(tiles + P_STAGES * P_STAGE_BYTES);
+  volatile int* abort = &bars->abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = kq::cluster_rank();
+  const int cid = (int)kq::cluster_id_x(), ncl = (int)kq::num_clusters_x();
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < P_STAGES; ++s) {
+      kq::mbar_init(&bars->full[s], 1);
+      kq::mbar_init(&bars->empty[s], 1);
+    }
+    kq::mbar_init(&bars->tfull, 1);
+    kq::mbar_init(&bars->tempty, 8);
+    kq::mbar_init(&bars->drain, 1);
+    bars->abort = 0;
+    kq::fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) kq::prefetch_tmap(&tmap);
+  if (warp == 2) kq::tmem_alloc_pair(&bars->tmem_base, TMEM_COLS);
+  kq::tc_fence_before();
+  kq::cluster_sync();          // the peer's barriers are initialised before any remote signal
+  kq::tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer (both CTAs)
+      int it = 0;
+      int t, c0, c1;
+      for (int sg = 0; pair_segment(sched, cid, ncl, sg, t, c0, c1); ++sg) {
+        int rb, cb;
+        pair_tile_coords(t, rb, cb);
+        const int i0 = rb * P_TILE + P_BM * (int)rank;          // this CTA's rows of the tile
+        const int j0 = cb * P_TILE + (P_TILE / 2) * (int)rank;  // this CTA's half of the columns
+        bool ok = true;
+        const int kb_end = min(k_iters, c1 * KC_ITERS);
+        for (int kb = c0 * KC_ITERS; kb < kb_end; ++kb, ++it) {
+          const int s = it % P_STAGES;
+          const uint32_t ph = (uint32_t)(it / P_STAGES) & 1u;
+          if (!kq::mbar_wait(&bars->empty[s], ph ^ 1u, abort, info)) { ok = false; break; }
+          uint8_t* a = tiles + s * P_STAGE_BYTES;
+          uint8_t* b = a + P_A_BYTES;
+          if (rank == 0) kq::mbar_arrive_expect_tx(&bars->full[s], 2 * P_STAGE_BYTES);
+          const uint32_t fb = kq::map_to_rank(kq::smem_u32(&bars->full[s]), 0);
+          const int y = kb * BK;
+          kq::tma_load_2d_pair(a, &tmap, fb, i0, y);
+          kq::tma_load_2d_pair(a + BOX_BYTES, &tmap, fb, i0 + 64, y);
+          kq::tma_load_2d_pair(b, &tmap, fb, j0, y);
+          kq::tma_load_2d_pair(b + BOX_BYTES, &tmap, fb, j0 + 64, y);
+        }
+        if (!ok) break;
+      }
+      // wind down (even CTA): every armed phase has landed, the odd CTA's
+      // bytes included, before the pair may exit
+      if (rank == 0) {
+        for (int s = 0; s < P_STAGES; ++s) {
+          const int armed = (it > s) ? (it - s + P_STAGES - 1) / P_STAGES : 0;
+          if (armed > 0) drain_wait(&bars->full[s], (uint32_t)(armed - 1) & 1u, info);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      // ------------------------------------------------ MMA issuer (even CTA)
+      int it = 0, cc = 0;
+      bool ok = true;
+      int t, c0, c1;
+      for (int sg = 0; ok && pair_segment(sched, cid, ncl, sg, t, c0, c1); ++sg) {
+        for (int ch = c0; ch < c1 && ok; ++ch, ++cc) {
+          const int k0 = ch * KC_ITERS, k1 = min(k_iters, k0 + KC_ITERS);
+          if (!kq::mbar_wait(&bars->tempty, ((uint32_t)cc & 1u) ^ 1u, abort, info)) { ok = false; break; }
+          kq::tc_fence_after();
+          for (int kb = k0; kb < k1; ++kb, ++it) {
+            const int s = it % P_STAGES;
+            const uint32_t ph = (uint32_t)(it / P_STAGES) & 1u;
+            if (!kq::mbar_wait(&bars->full[s], ph, abort, info)) { ok = false; break; }
+            kq::tc_fence_after();
+            const uint32_t a_addr = kq::smem_u32(tiles + s * P_STAGE_BYTES);
+            const uint32_t b_addr = a_addr + P_A_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              const uint64_t ad = kq::smem_desc(a_addr + kk * 2048, BOX_BYTES, 1024, kq::kLayoutSwizzle128B);
+              const uint64_t bd = kq::smem_desc(b_addr + kk * 2048, BOX_BYTES, 1024, kq::kLayoutSwizzle128B);
+              kq::mma_f16_pair(tmem, ad, bd, P_IDESC, (kb != k0) || (kk != 0));
+            }
+            kq::mma_commit_pair(&bars->empty[s], 0x3);
+          }
+          if (ok) kq::mma_commit_pair(&bars->tfull, 0x3);
+        }
+      }
+      kq::mma_commit_pair(&bars->drain, 0x1);
+      drain_wait(&bars->drain, 0, info);
+    }
+  } else if (warp >= 4) {
+    // -------------------------------------------------- epilogue (both CTAs)
+    const int q = warp & 3;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const uint32_t tempty_leader = kq::map_to_rank(kq::smem_u32(&bars->tempty), 0);
+    int cc = 0;
+    bool ok = true;
+    int t, c0, c1;
+    for (int sg = 0; ok && pair_segment(sched, cid, ncl, sg, t, c0, c1); ++sg) {
+      const bool shared_tile = c0 > 0 || c1 < sched.chunks;   // another pair adds the rest
+      int rb, cb;
+      pair_tile_coords(t, rb, cb);
+      const int i0 = rb * P_TILE + P_BM * (int)rank, j0 = cb * P_TILE;
+      const int row0 = i0 + q * 32;
+      const int row = row0 + lane;
+      for (int ch = c0; ch < c1; ++ch, ++cc) {
+        const bool first = ch == c0, last = ch == c1 - 1;
+        if (!kq::mbar_wait(&bars->tfull, (uint32_t)cc & 1u, abort, info)) { ok = false; break; }
+        kq::tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < P_TILE; c += 32) {
+          if (j0 + c >= d) break;
+          if (j0 + c + 31 < row0) continue;
+          float v[32], mst[32];
+          __syncwarp();
+          kq::tmem_ld32(tmem + lane_off + (uint32_t)c, v);
+          if (!first) kq::tmem_ld32(tmem + lane_off + (uint32_t)(P_TILE + c), mst);
+          kq::tmem_wait_ld();
+          if (!first) {
+#pragma unroll
+            for (int k = 0; k < 32; ++k) v[k] += mst[k];
+          }
+          kq::tmem_st32(tmem + lane_off + (uint32_t)(P_TILE + c), v);
+        }
+        kq::tmem_wait_st();
+        kq::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) kq::mbar_arrive_cluster(tempty_leader);
+        if (!last) continue;
+#pragma unroll 1
+        for (int c = 0; c < P_TILE; c += 32) {
+          const int jc = j0 + c;
+          if (jc >= d) break;
+          if (jc + 31 < row0) continue;
+          float v[32];
+          __syncwarp();
+          kq::tmem_ld32(tmem + lane_off + (uint32_t)(P_TILE + c), v);
+          kq::tmem_wait_ld();
+          if (row < d) {
+            if (shared_tile) add_row_chunk(H, ldh, d, row, row0, jc, v, alpha);
+            else store_row_chunk(H, ldh, d, row, row0, jc, v, alpha, beta);
+          }
+        }
+      }
+    }
+  }
+
+  kq::tc_fence_before();
+  kq::cluster_sync();          // no CTA leaves while the pair's MMAs or loads may touch it
+  if (warp == 2) {
+    kq::tc_fence_after();
+    kq::tmem_dealloc_pair(tmem, TMEM_COLS);
+  }
+}
+
+// The square tiles several pairs shared (at most one per pair boundary).
+constexpr int kMaxSharedTiles = 256;
+struct SharedTiles {
+  int count;
+  int tile[kMaxSharedTiles];
+};
+
+// For each listed 256 x 256 tile (rb <= cb): H[j][i] = H[i][j] for the tile's
+// elements above the diagonal, through 32 x 32 shared-memory transposes
+// (coalesced on both sides).  blockIdx.x = listed tile * 64 + 32 x 32 block.
+__global__ void __launch_bounds__(256) mirror_tiles_kernel(float* __restrict__ H, int64_t ldh, int d,
+                                                           const __grid_constant__ SharedTiles st) {
+  __shared__ float tile[32][33];
+  const int li = blockIdx.x >> 6, sb = blockIdx.x & 63;
+  int rb, cb;
+  pair_tile_coords(st.tile[li], rb, cb);
+  const int i0 = rb * P_TILE + (sb >> 3) * 32, j0 = cb * P_TILE + (sb & 7) * 32;   // source block
+  if (i0 >= d || j0 >= d || j0 + 31 < i0) return;                                  // nothing above the diagonal
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  for (int r = ty; r < 32; r += 8) {
+    const int i = i0 + r, j = j0 + tx;
+    tile[r][tx] = (i < d && j < d) ? H[(int64_t)i * ldh + j] : 0.f;
+  }
+  __syncthreads();
+  for (int r = ty; r < 32; r += 8) {
+    const int j = j0 + r, i = i0 + tx;                 // destination H[j][i] = H[i][j]
+    if (i < d && j < d && j > i) H[(int64_t)j * ldh + i] = tile[tx][r];
+  }
+}
+
+// H = beta H over d x d (ldh), zeros when beta = 0 (no read).
 __global__ void scale_kernel(float* __restrict__ H, int64_t ldh, int d, float beta) {
-  const int64_t total = (int64_t)d * d;
-  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
-       e += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t r = e / d, c = e % d;
-    float* p = H + r * ldh + c;
-    *p = (beta == 0.f) ? 0.f : beta * *p;
+  const bool vec = (d % 4) == 0 && (ldh % 4) == 0;
+  for (int r = blockIdx.x; r < d; r += gridDim.x) {
+    float* row = H + (int64_t)r * ldh;
+    if (vec) {
+      float4* row4 = reinterpret_cast<float4*>(row);
+      for (int c = threadIdx.x; c < d / 4; c += blockDim.x) {
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (beta != 0.f) {
+          v = row4[c];
+          v.x *= beta; v.y *= beta; v.z *= beta; v.w *= beta;
+        }
+        row4[c] = v;
+      }
+    } else {
+      for (int c = threadIdx.x; c < d; c += blockDim.x) row[c] = (beta == 0.f) ? 0.f : beta * row[c];
+    }
   }
 }
 
@@ -325,10 +660,66 @@ int kq_covariance(const uint16_t* A, int64_t N, int64_t d, int64_t lda, float* H
                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return KRONQ_ERR_UNSUPPORTED;
 
+  const int k_iters = (int)((N + BK - 1) / BK);
+  if (d > P_TILE) {
+    // CTA pairs on 256 x 256 tiles
+    const int ncb2 = (int)((d + P_TILE - 1) / P_TILE);
+    const int tiles2 = ncb2 * (ncb2 + 1) / 2;
+    static int max_pairs = 0;
+    if (max_pairs == 0) {
+      if (cudaFuncSetAttribute(cov_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               P_SMEM_BYTES) != cudaSuccess)
+        return KRONQ_ERR_CUDA;
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(2 * (kqh::num_sms() / 2), 1, 1);
+      cfg.blockDim = dim3(THREADS, 1, 1);
+      cfg.dynamicSmemBytes = P_SMEM_BYTES;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, cov_pair_kernel, &cfg) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        n = kqh::num_sms() / 2;
+      }
+      max_pairs = n < kMaxSharedTiles ? n : kMaxSharedTiles;
+    }
+    const int P = max_pairs;
+    PairSchedule sc;
+    sc.tiles = tiles2;
+    sc.chunks = (k_iters + KC_ITERS - 1) / KC_ITERS;
+    sc.waves = tiles2 / P;
+    sc.rest = tiles2 % P;
+    sc.per_helper = sc.rest > 0 ? (sc.rest + (P - sc.rest) - 1) / (P - sc.rest) : 0;
+    sc.kstar = sc.rest > 0 ? (sc.per_helper * sc.chunks + sc.per_helper) / (sc.per_helper + 1) : sc.chunks;
+    if (sc.kstar < 1) sc.kstar = 1;
+    if (sc.kstar > sc.chunks) sc.kstar = sc.chunks;
+    // the split tiles: the R tiles of the last, partial wave when helpers take their tail
+    SharedTiles list;
+    list.count = 0;
+    if (sc.rest > 0 && sc.kstar < sc.chunks) {
+      if (sc.rest > kMaxSharedTiles) return KRONQ_ERR_UNSUPPORTED;
+      for (int i = 0; i < sc.rest; ++i) list.tile[list.count++] = sc.waves * P + i;
+    }
+    const bool shared = list.count > 0;
+    const int pairs = (sc.waves == 0 && !shared) ? sc.rest : P;
+    if (shared && beta != 1.f) {
+      // shared tiles add into H: start from beta H (zeros when beta = 0); the
+      // tiles a single pair owns then store alpha sum + 1 * (beta H)
+      scale_kernel<<<2 * kqh::num_sms(), 256, 0, st>>>(H, ldh, (int)d, beta);
+      KQ_CHECK_LAUNCH();
+    }
+    const float beta_owned = shared ? (beta == 0.f ? 0.f : 1.f) : beta;
+    cov_pair_kernel<<<2 * pairs, THREADS, P_SMEM_BYTES, st>>>(tmap, H, ldh, (int)d, k_iters, sc,
+                                                             alpha, beta_owned, info);
+    KQ_CHECK_LAUNCH();
+    if (shared) {
+      mirror_tiles_kernel<<<list.count * 64, 256, 0, st>>>(H, ldh, (int)d, list);
+      KQ_CHECK_LAUNCH();
+    }
+    return KRONQ_OK;
+  }
+
   const int nrb = (int)((d + BM - 1) / BM), ncb = (int)((d + BN - 1) / BN);
   int num_tiles = 0;
   for (int cb = 0; cb < ncb; ++cb) num_tiles += (2 * cb + 2 < nrb) ? 2 * cb + 2 : nrb;
-  const int k_iters = (int)((N + BK - 1) / BK);
 
   static bool attr_set = false;
   if (!attr_set) {

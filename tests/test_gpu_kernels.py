@@ -37,7 +37,7 @@ def _x(r, N, d, kind="t4"):
 @pytest.mark.parametrize("N,d,kind", [(2048, 256, "t4"), (1000, 200, "g"), (4097, 520, "t4"),
                                       (130, 72, "g"), (64, 64, "t4"), (777, 1000, "g"),
                                       (20000, 384, "t4"), (33, 129, "g"), (70000, 256, "t4"),
-                                      (8193, 136, "g")])
+                                      (8193, 136, "g"), (300, 257, "g"), (5000, 3104, "t4")])
 def test_covariance_matches_oracle(cuda, N, d, kind):
     r = np.random.default_rng(N * 7 + d)
     lda = (d + 7) // 8 * 8                       # the ABI wants lda % 8 == 0
@@ -73,6 +73,24 @@ def test_covariance_padded_rows_beta_and_streaming(cuda):
     H = t(H0, cuda)
     abi.kronq_covariance(A[:0], H, 1.0, 2.0)
     np.testing.assert_array_equal(H.cpu().numpy(), 2.0 * H0)
+
+
+def test_covariance_shared_tiles_with_beta(cuda):
+    """Enough tokens that CTA pairs split a tile's K range between them and
+    add their parts into H (after the host-side scaling of H by beta)."""
+    r = np.random.default_rng(11)
+    N, d = 9000, 600
+    bits = _x(r, N, d, "t4")
+    A = bf16_dev(bits, cuda)
+    ref = ocov.covariance(widen(bits))
+    H0 = spd(r, d)
+    for beta in (0.0, 0.25, 1.0):
+        H = t(H0, cuda)
+        abi.kronq_covariance(A, H, 1.0 / N, beta)
+        want = ref + beta * H0.astype(np.float64)
+        Hg = H.cpu().numpy()
+        assert rel_fro(Hg, want) <= 1e-4, beta
+        assert np.array_equal(Hg, Hg.T)
 
 
 # ------------------------------------------------------------- sensitivity
