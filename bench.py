@@ -157,7 +157,7 @@ def kernel_source_sha() -> str:
 def load_traffic(workload: str):
     """DRAM bytes per launch of the covariance kernel from a committed ncu
     summary, only while the kernel source is the one that was profiled."""
-    p = ROOT / "profiles" / "cov_tc_kernel.traffic.json"
+    p = ROOT / "profiles" / "cov_pair_kernel.traffic.json"
     if not p.exists():
         return None
     d = json.loads(p.read_text())
@@ -521,7 +521,7 @@ def main():
     avg_ms = statistics.mean(cov_ms)
     achieved = statistics.mean(cov_flops) / (avg_ms / 1e3) / 1e12
     workload = workload_desc(cfg0)
-    roofline = {"bound": "tensor", "kernel": "cov_tc_kernel (kronq_covariance)",
+    roofline = {"bound": "tensor", "kernel": "cov_pair_kernel (kronq_covariance)",
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                 "traffic": load_traffic(workload),
                 "peak_source": f"{peak_src} {peak_kind}",
