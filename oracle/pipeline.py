@@ -53,21 +53,29 @@ def g_covariance(cfg, sub, tokens=None, threads=None) -> np.ndarray:
                        sub.m, tokens, threads)
 
 
-def quantize_sublayer(cfg, sub, HX, HG, bits, rows=None, W=None):
+def quantize_sublayer(cfg, sub, HX, HG, bits, rows=None, W=None, act_order=False, clip=False):
     """Steps 2-6 for one sublayer given its two covariances.
 
     rows: the rows of W' to run the column loop on (all when None); the loop
-    treats rows independently, so a subset gives those rows' exact results."""
+    treats rows independently, so a subset gives those rows' exact results.
+    act_order / clip: the README's --act_order and --w_clip (readings in
+    oracle/quantizer.py)."""
     if W is None:
         W = synth.make_w(cfg, sub)
     su, sv = synth.make_signs(cfg, sub)
     Wp, HXt, HGt, SX, SG = _biip.biip(W, HX, HG, su, sv, cfg.alpha, cfg.mode)
     s = sensitivity.sensitivity(HXt, HGt)
     Hd = cholesky.damp(HXt, cfg.damp)
-    Uc = cholesky.inverse_cholesky(Hd)
-    res = quantizer.obs_quantize_rows(Wp, Uc, bits, sub.group, rows=rows)
+    if act_order:
+        perm = quantizer.act_order_perm(HXt)
+        res = quantizer.obs_quantize_act_order(Wp, Hd, perm, bits, sub.group, clip=clip, rows=rows)
+        Uc = res.pop("U_perm")
+    else:
+        perm = None
+        Uc = cholesky.inverse_cholesky(Hd)
+        res = quantizer.obs_quantize_rows(Wp, Uc, bits, sub.group, rows=rows, clip=clip)
     out = {"W_rot": Wp, "HX_rot": HXt, "HG_rot": HGt, "S_X": SX, "S_G": SG, "s": s,
-           "U_c": Uc, "rows": np.arange(sub.m) if rows is None else np.asarray(rows)}
+           "U_c": Uc, "perm": perm, "rows": np.arange(sub.m) if rows is None else np.asarray(rows)}
     out.update(res)
     if bits in (2, 4):
         out["packed"] = pack.pack(res["codes"], bits)

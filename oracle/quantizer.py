@@ -11,8 +11,9 @@ Sources:
     plain unblocked loop: after column j, every later column k is updated at
     once.
   * KronQ README (GitHub), "Reproduce from scratch": --w_asym, --w_groupsize
-    -1 (per-channel) or 128, 2/3/4 bits; --w_clip and --act_order are left
-    off (the pages do not define them).
+    -1 (per-channel) or 128, 2/3/4 bits, and the flags --w_clip and
+    --act_order, which the pages name but do not define (readings below;
+    both are off unless asked for).
 
 Readings:
   * grid: lo = min(0, min w), hi = max(0, max w), scale = (hi - lo)/(2^b - 1),
@@ -27,6 +28,15 @@ Readings:
     group parameters at column j = 0 mod g from the current (already
     error-updated) columns j .. j+g-1.
   * column update: e = (w_j - w_hat_j) / U[j, j]; W[:, k] -= e U[j, k], k > j.
+  * --w_clip (reading): for each row (per-channel) or group, the grid is
+    chosen among the shrunk ranges [p lo, p hi], p = 1 - i/100 for
+    i = 0 .. 79, as the first one with the smallest squared quantization
+    error sum_k (w_k - w_hat_k)^2 over the row or group.  The grid of each
+    candidate and the differences w_k - w_hat_k are fp32 operations (the
+    decision precision above); the squares of those fp32 differences are
+    exact in fp64 and are summed in fp64, so that the choice does not hinge
+    on the order of the sum.
+  * --act_order (reading): act_order_perm below.
 """
 
 from __future__ import annotations
@@ -58,6 +68,62 @@ def grid_params(w: np.ndarray, bits: int):
     return scale, zero.astype(np.int64)
 
 
+CLIP_GRID = 100      # candidate shrink ratios p = 1 - i / CLIP_GRID ...
+CLIP_STEPS = 80      # ... for i = 0 .. CLIP_STEPS - 1
+
+
+def clip_ratio(i: int) -> np.float32:
+    """p_i = 1 - i/100, evaluated in fp64 and rounded once to fp32."""
+    return F32(1.0 - i * (1.0 / CLIP_GRID))
+
+
+def _grid_from_range(lo: np.ndarray, hi: np.ndarray, bits: int):
+    """(scale, zero) of the asymmetric grid of [lo, hi] (fp32, lo <= 0 <= hi)."""
+    maxq = F32(2 ** bits - 1)
+    zero_row = (lo == 0) & (hi == 0)
+    span = (hi - lo).astype(F32)
+    span[zero_row] = maxq
+    scale = (span / maxq).astype(F32)
+    zero = np.rint((-lo).astype(F32) / scale).astype(F32)
+    zero = np.clip(zero, F32(0), maxq)
+    scale[zero_row] = F32(1)
+    zero[zero_row] = F32(0)
+    return scale, zero.astype(np.int64)
+
+
+def sq_error(w32: np.ndarray, scale, zero, bits: int) -> np.ndarray:
+    """Per-row sum of (w - w_hat)^2: w_hat = scale (q - zero) and the
+    difference in fp32, the squares (exact) and their sum in fp64."""
+    scale = np.asarray(scale, dtype=F32).reshape(-1, 1)
+    zero = np.asarray(zero, dtype=np.int64).reshape(-1, 1)
+    q = quantize(w32, scale, zero, bits)
+    wh = (scale * (q - zero).astype(F32)).astype(F32)
+    d = (w32 - wh).astype(F32).astype(np.float64)
+    return np.sum(d * d, axis=1)
+
+
+def clip_grid_params(w: np.ndarray, bits: int):
+    """Per-row (scale, zero) of the --w_clip search (reading in the module
+    docstring): the first of the shrunk grids with the least squared error."""
+    w32 = np.asarray(w, dtype=np.float64).astype(F32)
+    if w32.ndim == 1:
+        w32 = w32[None, :]
+    lo = np.minimum(w32.min(axis=1), F32(0))
+    hi = np.maximum(w32.max(axis=1), F32(0))
+    best = np.full(w32.shape[0], np.inf)
+    scale = np.ones(w32.shape[0], dtype=F32)
+    zero = np.zeros(w32.shape[0], dtype=np.int64)
+    for i in range(CLIP_STEPS):
+        p = clip_ratio(i)
+        s1, z1 = _grid_from_range((lo * p).astype(F32), (hi * p).astype(F32), bits)
+        err = sq_error(w32, s1, z1, bits)
+        better = err < best
+        best[better] = err[better]
+        scale[better] = s1[better]
+        zero[better] = z1[better]
+    return scale, zero
+
+
 def quantize(w: np.ndarray, scale: np.ndarray, zero: np.ndarray, bits: int) -> np.ndarray:
     """Integer codes, decided in fp32 (reading in the module docstring)."""
     maxq = 2 ** bits - 1
@@ -78,12 +144,14 @@ def _check(n: int, group: int, bits: int):
         raise ValueError("group must be -1 or divide n")
 
 
-def obs_quantize(W: np.ndarray, U: np.ndarray, bits: int, group: int = -1):
+def obs_quantize(W: np.ndarray, U: np.ndarray, bits: int, group: int = -1, clip: bool = False):
     """Unblocked column-wise OBS loop on the rows of W (rows are independent).
 
     W: m x n (the rotated weights, widened to fp64).  U: n x n upper inverse
-    Cholesky factor of the damped H_X.  Returns a dict with codes (m x n),
-    scale and zero (m x n_groups), W_hat (m x n) and the scaled errors E."""
+    Cholesky factor of the damped H_X.  clip: the --w_clip grid search.
+    Returns a dict with codes (m x n), scale and zero (m x n_groups), W_hat
+    (m x n) and the scaled errors E."""
+    params = clip_grid_params if clip else grid_params
     W = np.array(W, dtype=np.float64)
     U = np.asarray(U, dtype=np.float64)
     m, n = W.shape
@@ -95,11 +163,11 @@ def obs_quantize(W: np.ndarray, U: np.ndarray, bits: int, group: int = -1):
     What = np.zeros((m, n))
     E = np.zeros((m, n))
     if group == -1:
-        scale, zero = grid_params(W, bits)
+        scale, zero = params(W, bits)
         scales[:, 0], zeros[:, 0] = scale, zero
     for j in range(n):
         if group != -1 and j % group == 0:
-            scale, zero = grid_params(W[:, j:j + group], bits)
+            scale, zero = params(W[:, j:j + group], bits)
             scales[:, j // group], zeros[:, j // group] = scale, zero
         w = W[:, j]
         q = quantize(w, scale, zero, bits)
@@ -113,7 +181,7 @@ def obs_quantize(W: np.ndarray, U: np.ndarray, bits: int, group: int = -1):
 
 
 def obs_quantize_rows(W: np.ndarray, U: np.ndarray, bits: int, group: int = -1,
-                      rows=None, chunk: int = 64, threads: int | None = None):
+                      rows=None, chunk: int = 64, threads: int | None = None, clip: bool = False):
     """obs_quantize on a subset of rows, in row chunks on a thread pool.
 
     Each row's arithmetic is exactly that of obs_quantize: the rows of the
@@ -123,10 +191,42 @@ def obs_quantize_rows(W: np.ndarray, U: np.ndarray, bits: int, group: int = -1,
     parts = [rows[i:i + chunk] for i in range(0, len(rows), chunk)]
     threads = threads or min(32, os.cpu_count() or 1)
     with ThreadPoolExecutor(threads) as ex:
-        res = list(ex.map(lambda r: obs_quantize(W[r], U, bits, group), parts))
+        res = list(ex.map(lambda r: obs_quantize(W[r], U, bits, group, clip), parts))
     if not res:
-        return obs_quantize(W[:0], U, bits, group)
+        return obs_quantize(W[:0], U, bits, group, clip)
     return {k: np.concatenate([r[k] for r in res], axis=0) for k in res[0]}
+
+
+def act_order_perm(H: np.ndarray) -> np.ndarray:
+    """--act_order (reading): the columns are quantized in descending order
+    of the diagonal of the (rotated, undamped) H_X handed to the solver, equal
+    diagonals in increasing column order.  perm[k] = the column quantized
+    k-th.  The solver then runs on W[:, perm] with H[perm][:, perm] (damping
+    and inverse Cholesky of the permuted matrix), and its codes and W_hat go
+    back to the original column order; with groups, a group is g consecutive
+    columns of the permuted order."""
+    d = np.asarray(np.diag(np.asarray(H)), dtype=np.float64)
+    return np.array(sorted(range(len(d)), key=lambda j: (-d[j], j)), dtype=np.int64)
+
+
+def obs_quantize_act_order(W: np.ndarray, H_damped: np.ndarray, perm: np.ndarray, bits: int,
+                           group: int = -1, clip: bool = False, rows=None):
+    """The column loop in the order perm (act_order_perm), results in the
+    original column order.  H_damped: the damped H_X (unpermuted); its
+    permuted copy gets its own inverse Cholesky factor.  scale / zero are
+    indexed by groups of the permuted order."""
+    from . import cholesky
+    perm = np.asarray(perm)
+    Up = cholesky.inverse_cholesky(np.asarray(H_damped, dtype=np.float64)[np.ix_(perm, perm)])
+    Wp = np.asarray(W, dtype=np.float64)[:, perm]
+    res = obs_quantize_rows(Wp, Up, bits, group, rows=rows, clip=clip)
+    out = dict(res)
+    for k in ("codes", "W_hat", "E"):
+        back = np.empty_like(res[k])
+        back[:, perm] = res[k]
+        out[k] = back
+    out["U_perm"] = Up
+    return out
 
 
 def rtn_quantize(W: np.ndarray, bits: int, group: int = -1):
