@@ -46,6 +46,10 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--act-order", action="store_true",
+                    help="quantize columns in descending H_X' diagonal order (README --act_order)")
+    ap.add_argument("--w-clip", action="store_true",
+                    help="clip-ratio search for every grid (README --w_clip)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="calibration tokens per X/G (default: the workload's; smaller only for "
                          "profiler captures)")
@@ -280,7 +284,7 @@ def run_reference(args, rank, world):
 class Layer:
     """Device buffers of one sublayer for the timed steps (allocated once)."""
 
-    def __init__(self, cfg, sub, dev, seed_offset, host):
+    def __init__(self, cfg, sub, dev, seed_offset, host, act_order=False):
         import numpy as np
         import torch
         import synth
@@ -307,9 +311,35 @@ class Layer:
         self.zeros = torch.empty((m, G), dtype=torch.uint8, device=dev)
         self.packed = torch.empty((m, abi.packed_words(n, 4)), dtype=torch.int32, device=dev)
         self.bits = sub.bits
+        self.perm = self.Hp = self.Wp = self.codes_p = None
+        if act_order:
+            self.perm = torch.empty(n, dtype=torch.int32, device=dev)
+            self.Hp = torch.empty((n, n), dtype=torch.float32, device=dev)
+            self.Wp = torch.empty((m, n), dtype=torch.float32, device=dev)
+            self.codes_p = torch.empty((m, n), dtype=torch.uint8, device=dev)
 
 
-def gpu_step(cfg, layers, X, ws, stream, cov_events=None):
+def solve_layer(cfg, L, ws, stream, act_order=False, clip=False):
+    """Damped inverse Cholesky and the column loop of one sublayer, with the
+    README's --act_order (column order by the H_X' diagonal, results back in
+    the original order) and --w_clip (clip-ratio search) when asked for."""
+    from post_quantization_02_b200 import abi
+    opts = abi.QUANT_CLIP if clip else 0
+    if not act_order:
+        abi.kronq_cholesky_inv(L.HX, cfg.damp, L.U, L.info, ws, stream=stream)
+        abi.kronq_quantize_layer_opt(L.W, L.U, L.bits, L.sub.group, cfg.block, opts, L.codes,
+                                     L.scales, L.zeros, None, L.info, ws, stream=stream)
+        return
+    abi.kronq_act_order(L.HX, L.perm, stream=stream)
+    abi.kronq_permute(L.HX, L.Hp, L.perm, abi.PERM_SYM, L.info, stream=stream)
+    abi.kronq_permute(L.W, L.Wp, L.perm, abi.PERM_COLS, L.info, stream=stream)
+    abi.kronq_cholesky_inv(L.Hp, cfg.damp, L.U, L.info, ws, stream=stream)
+    abi.kronq_quantize_layer_opt(L.Wp, L.U, L.bits, L.sub.group, cfg.block, opts, L.codes_p,
+                                 L.scales, L.zeros, None, L.info, ws, stream=stream)
+    abi.kronq_permute(L.codes_p, L.codes, L.perm, abi.UNPERM_COLS, L.info, stream=stream)
+
+
+def gpu_step(cfg, layers, X, ws, stream, cov_events=None, act_order=False, clip=False):
     """One pass of the whole path over every sublayer of the config."""
     import torch
     from post_quantization_02_b200 import abi, alloc
@@ -346,9 +376,7 @@ def gpu_step(cfg, layers, X, ws, stream, cov_events=None):
         for L, b in zip(layers, bits):
             L.bits = b
     for L in layers:
-        abi.kronq_cholesky_inv(L.HX, cfg.damp, L.U, L.info, ws, stream=stream)
-        abi.kronq_quantize_layer(L.W, L.U, L.bits, L.sub.group, cfg.block, L.codes, L.scales,
-                                 L.zeros, None, L.info, ws, stream=stream)
+        solve_layer(cfg, L, ws, stream, act_order, clip)
         if L.bits in (2, 4):
             pk = L.packed[:, : abi.packed_words(L.sub.n, L.bits)]
             abi.kronq_pack(L.codes, L.bits, pk.contiguous() if not pk.is_contiguous() else pk,
@@ -392,7 +420,7 @@ def main():
         host["G"][sub.name] = synth.make_g(cfg, sub)
     t_gen = time.perf_counter() - t_gen
     X = {s: torch.from_numpy(v.view(np.int16)).to(dev).view(torch.bfloat16) for s, v in host["X"].items()}
-    layers = [Layer(cfg, sub, dev, rank, host) for sub in cfg.sublayers]
+    layers = [Layer(cfg, sub, dev, rank, host, args.act_order) for sub in cfg.sublayers]
     mmax = max(s.m for s in cfg.sublayers)
     nmax = max(s.n for s in cfg.sublayers)
     ws = abi.workspace(mmax, nmax, device=dev)
@@ -401,7 +429,7 @@ def main():
 
     ncov = len(cfg.sites) + len(cfg.sublayers)
     for _ in range(args.warmup):
-        gpu_step(cfg, layers, X, ws, stream)
+        gpu_step(cfg, layers, X, ws, stream, None, args.act_order, args.w_clip)
     torch.cuda.synchronize()
     for L in layers:
         if L.info.item() != 0:
@@ -418,7 +446,7 @@ def main():
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record(stream)
     for k in range(args.steps):
-        gpu_step(cfg, layers, X, ws, stream, cov_events[k])
+        gpu_step(cfg, layers, X, ws, stream, cov_events[k], args.act_order, args.w_clip)
     end.record(stream)
     torch.cuda.synchronize()
     if world > 1:
@@ -471,9 +499,7 @@ def main():
                                       ws, stream=stream)
                 abi.kronq_sensitivity(L.HX, L.HG, L.sens, stream=stream)
             for L in layers:
-                abi.kronq_cholesky_inv(L.HX, cfg.damp, L.U, L.info, ws, stream=stream)
-                abi.kronq_quantize_layer(L.W, L.U, L.bits, L.sub.group, cfg.block, L.codes, L.scales,
-                                         L.zeros, None, L.info, ws, stream=stream)
+                solve_layer(cfg, L, ws, stream, args.act_order, args.w_clip)
                 pk, sc, zr = outs[L.sub.name]
                 if L.bits in (2, 4):
                     words = abi.packed_words(L.sub.n, L.bits)
@@ -542,7 +568,8 @@ def main():
             "data": "synthetic (seeded generator; stands in for WikiText-2 activations and LLaMA weights)",
             "config": {"workload": workload, "parallelism": f"replicas x{world} (one layer per GPU)",
                        "l2": l2_note(cfg0),
-                       "solver_dtype": "fp32", "input_gen_s": round(t_gen, 1)},
+                       "solver_dtype": "fp32", "input_gen_s": round(t_gen, 1),
+                       "act_order": args.act_order, "w_clip": args.w_clip},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
             "clocks": clocks,
         }

@@ -179,6 +179,60 @@ int kronq_quantize_layer(float* W, int64_t m, int64_t n, const float* U_c,
                          uint8_t* codes, float* scales, uint8_t* zeros, float* W_hat,
                          int32_t* info, void* ws, size_t ws_bytes, void* stream);
 
+/* Options of kronq_quantize_layer_opt (bit flags). */
+enum kronq_quant_option {
+  KRONQ_QUANT_CLIP = 1   /* --w_clip: clip-ratio search for every grid */
+};
+
+/*
+ * kronq_quantize_layer with options.  options = 0 is kronq_quantize_layer.
+ *
+ * KRONQ_QUANT_CLIP: the README's --w_clip (KronQ README (GitHub),
+ * "Reproduce from scratch"; the pages name the flag without defining it).
+ * Reading taken: each grid (per row before the loop, or per group at its
+ * first column) is the first of the shrunk ranges [p lo, p hi],
+ * p = 1 - i/100 for i = 0 .. 79, with the least squared error
+ * sum (w - w_hat)^2 over the row or group; the candidate grids and the
+ * differences are fp32 operations, the squares are summed in fp64.
+ * Other bits set: KRONQ_ERR_INVALID_ARG.  Everything else as
+ * kronq_quantize_layer.
+ */
+int kronq_quantize_layer_opt(float* W, int64_t m, int64_t n, const float* U_c,
+                             int bits, int group, int block, int options,
+                             uint8_t* codes, float* scales, uint8_t* zeros, float* W_hat,
+                             int32_t* info, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * The --act_order column order (KronQ README (GitHub), "Reproduce from
+ * scratch"; undefined on the pages).  Reading taken: columns in descending
+ * order of diag(H), equal values in increasing column order (NaN last).
+ * perm[k] = the column quantized k-th.  To quantize in that order: permute
+ * the columns of W and both sides of H_X with kronq_permute, factor the
+ * permuted H_X with kronq_cholesky_inv, run the solver, and scatter the
+ * codes (and W_hat) back with KRONQ_UNPERM_COLS; with groups, a group is g
+ * consecutive columns of the permuted order (scales / zeros are indexed by
+ * those groups).
+ * H: n x n fp32 device (only the diagonal is read).  perm: n int32 device.
+ */
+int kronq_act_order(const float* H, int64_t n, int32_t* perm, void* stream);
+
+/* kronq_permute modes. */
+enum kronq_perm_mode {
+  KRONQ_PERM_COLS = 0,    /* dst[r][k] = src[r][perm[k]]          */
+  KRONQ_UNPERM_COLS = 1,  /* dst[r][perm[k]] = src[r][k]          */
+  KRONQ_PERM_SYM = 2      /* dst[a][b] = src[perm[a]][perm[b]], m == n, fp32 */
+};
+
+/*
+ * Column (or symmetric) permutation of an m x n row-major matrix of 1-byte
+ * (codes) or 4-byte (fp32) elements; src and dst are distinct device
+ * buffers.  perm: n int32 device, a permutation of 0 .. n-1; entries out of
+ * range are skipped and reported as KRONQ_ERR_INVALID_ARG in the optional
+ * device word info.  Not in the pages: the plumbing of --act_order.
+ */
+int kronq_permute(const void* src, void* dst, int64_t m, int64_t n, int elem_bytes,
+                  const int32_t* perm, int mode, int32_t* info, void* stream);
+
 /*
  * kronq_quantize_layer without a workspace: for callers that cannot allocate
  * device memory while they run (a host framework that owns the allocator,

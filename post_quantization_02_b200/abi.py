@@ -22,6 +22,8 @@ STATUS = {
     -4: "CUDA error", -5: "device wait timed out", -6: "workspace missing or too small",
 }
 MODES = {"full": 0, "no_rescale": 1, "su_only": 2, "sv_only": 3}
+QUANT_CLIP = 1                      # kronq_quantize_layer_opt options
+PERM_COLS, UNPERM_COLS, PERM_SYM = 0, 1, 2   # kronq_permute modes
 
 _lib = None
 
@@ -52,6 +54,9 @@ def lib() -> ctypes.CDLL:
         "kronq_cholesky_inv": ([P, I64, F32, P, P, P, SZ, P], I32),
         "kronq_quantize_layer": ([P, I64, I64, P, I32, I32, I32, P, P, P, P, P, P, SZ, P], I32),
         "kronq_quantize_layer_noalloc": ([P, I64, I64, P, I32, I32, I32, P, P, P, P, P, P], I32),
+        "kronq_quantize_layer_opt": ([P, I64, I64, P, I32, I32, I32, I32, P, P, P, P, P, P, SZ, P], I32),
+        "kronq_act_order": ([P, I64, P, P], I32),
+        "kronq_permute": ([P, P, I64, I64, I32, P, I32, P, P], I32),
         "kronq_pack": ([P, I64, I64, I32, P, P], I32),
         "kronq_unpack": ([P, I64, I64, I32, P, P], I32),
         "kronq_layer_loss": ([P, P, I64, I64, P, P, P, P, SZ, P], I32),
@@ -183,6 +188,46 @@ def kronq_quantize_layer(W, U, bits: int, group: int, block: int, codes, scales,
     _check("kronq_quantize_layer", lib().kronq_quantize_layer(
         _p(W), m, n, _p(U), bits, group, block, _p(codes), _p(scales), _p(zeros), _p(W_hat),
         _p(info), _p(ws), 0 if ws is None else ws.numel() * ws.element_size(), _s(stream)))
+
+
+def kronq_quantize_layer_opt(W, U, bits: int, group: int, block: int, options: int, codes, scales,
+                             zeros, W_hat=None, info=None, ws=None, stream=None):
+    """kronq_quantize_layer with option flags (QUANT_CLIP: the --w_clip search)."""
+    _dev(W, torch.float32, "W", 2)
+    _dev(U, torch.float32, "U_c", 2)
+    _dev(codes, torch.uint8, "codes", 2)
+    _dev(scales, torch.float32, "scales")
+    _dev(zeros, torch.uint8, "zeros")
+    _dev(W_hat, torch.float32, "W_hat", 2)
+    for t, nm in ((W, "W"), (U, "U_c"), (codes, "codes"), (scales, "scales"), (zeros, "zeros"),
+                  (W_hat, "W_hat")):
+        _contig(t, nm)
+    m, n = W.shape
+    _check("kronq_quantize_layer_opt", lib().kronq_quantize_layer_opt(
+        _p(W), m, n, _p(U), bits, group, block, options, _p(codes), _p(scales), _p(zeros),
+        _p(W_hat), _p(info), _p(ws), 0 if ws is None else ws.numel() * ws.element_size(),
+        _s(stream)))
+
+
+def kronq_act_order(H, perm, stream=None):
+    """perm (int32, n) = the --act_order column order from diag(H)."""
+    _dev(H, torch.float32, "H", 2)
+    _dev(perm, torch.int32, "perm", 1)
+    _contig(H, "H")
+    _check("kronq_act_order", lib().kronq_act_order(_p(H), H.shape[0], _p(perm), _s(stream)))
+
+
+def kronq_permute(src, dst, perm, mode: int, info=None, stream=None):
+    """Column / symmetric permutation of a 2-D uint8 or fp32 tensor (see kronq.h)."""
+    _dev(src, (torch.float32, torch.uint8), "src", 2)
+    _dev(dst, src.dtype, "dst", 2)
+    _dev(perm, torch.int32, "perm", 1)
+    _contig(src, "src"); _contig(dst, "dst")
+    if dst.shape != src.shape or perm.numel() != src.shape[1]:
+        raise ValueError("kronq_permute: shapes do not match")
+    m, n = src.shape
+    _check("kronq_permute", lib().kronq_permute(_p(src), _p(dst), m, n, src.element_size(),
+                                                _p(perm), mode, _p(info), _s(stream)))
 
 
 def kronq_quantize_layer_noalloc(W, U, bits: int, group: int, block: int, codes, scales, zeros,

@@ -19,8 +19,11 @@ int kq_biip_rotate(float* W, int64_t m, int64_t n, float* HX, float* HG, const i
 int kq_cholesky_inv(const float* H, int64_t n, float damp_rel, float* U, int32_t* info, void* ws,
                     size_t ws_bytes, cudaStream_t st);
 int kq_quantize_layer(float* W, int64_t m, int64_t n, const float* U, int bits, int group,
-                      int block, uint8_t* codes, float* scales, uint8_t* zeros, float* W_hat,
-                      int32_t* info, void* ws, size_t ws_bytes, cudaStream_t st);
+                      int block, int options, uint8_t* codes, float* scales, uint8_t* zeros,
+                      float* W_hat, int32_t* info, void* ws, size_t ws_bytes, cudaStream_t st);
+int kq_act_order(const float* H, int64_t n, int32_t* perm, cudaStream_t st);
+int kq_permute(const void* src, void* dst, int64_t m, int64_t n, int elem_bytes,
+               const int32_t* perm, int mode, int32_t* info, cudaStream_t st);
 int kq_quantize_layer_noalloc(float* W, int64_t m, int64_t n, const float* U, int bits, int group,
                               int block, uint8_t* codes, float* scales, uint8_t* zeros,
                               float* W_hat, int32_t* info, cudaStream_t st);
@@ -138,8 +141,25 @@ int kronq_cholesky_inv(const float* H, int64_t n, float damp_rel, float* U_c, in
 int kronq_quantize_layer(float* W, int64_t m, int64_t n, const float* U_c, int bits, int group,
                          int block, uint8_t* codes, float* scales, uint8_t* zeros, float* W_hat,
                          int32_t* info, void* ws, size_t ws_bytes, void* stream) {
-  return kq_quantize_layer(W, m, n, U_c, bits, group, block, codes, scales, zeros, W_hat, info, ws,
-                           ws_bytes, S(stream));
+  return kq_quantize_layer(W, m, n, U_c, bits, group, block, 0, codes, scales, zeros, W_hat, info,
+                           ws, ws_bytes, S(stream));
+}
+
+int kronq_quantize_layer_opt(float* W, int64_t m, int64_t n, const float* U_c, int bits,
+                             int group, int block, int options, uint8_t* codes, float* scales,
+                             uint8_t* zeros, float* W_hat, int32_t* info, void* ws,
+                             size_t ws_bytes, void* stream) {
+  return kq_quantize_layer(W, m, n, U_c, bits, group, block, options, codes, scales, zeros, W_hat,
+                           info, ws, ws_bytes, S(stream));
+}
+
+int kronq_act_order(const float* H, int64_t n, int32_t* perm, void* stream) {
+  return kq_act_order(H, n, perm, S(stream));
+}
+
+int kronq_permute(const void* src, void* dst, int64_t m, int64_t n, int elem_bytes,
+                  const int32_t* perm, int mode, int32_t* info, void* stream) {
+  return kq_permute(src, dst, m, n, elem_bytes, perm, mode, info, S(stream));
 }
 
 int kronq_quantize_layer_noalloc(float* W, int64_t m, int64_t n, const float* U_c, int bits,

@@ -69,6 +69,88 @@ __device__ __forceinline__ Grid make_grid(float mn, float mx, float maxq) {
   return g;
 }
 
+// --w_clip (KronQ README (GitHub), "Reproduce from scratch"; the pages name
+// the flag without defining it).  Reading: among the shrunk ranges
+// [p lo, p hi], p = 1 - i/100 for i = 0 .. 79, take the first grid with the
+// least squared error sum (w - w_hat)^2 over the row or group.  The grid and
+// the differences are fp32 operations (no contraction), the squares of the
+// fp32 differences are exact in fp64 and summed in fp64, so the choice does
+// not depend on the order of the sum.
+constexpr int CLIP_STEPS = 80;
+
+__device__ __forceinline__ float clip_ratio(int i) {
+  return __double2float_rn(__dadd_rn(1.0, -__dmul_rn((double)i, 0.01)));
+}
+
+__device__ __forceinline__ Grid clip_grid(float lo, float hi, float p, float maxq) {
+  const float lo1 = __fmul_rn(lo, p), hi1 = __fmul_rn(hi, p);
+  Grid g;
+  if (lo1 == 0.f && hi1 == 0.f) {
+    g.scale = 1.f;
+    g.zero = 0.f;
+  } else {
+    g.scale = __fdiv_rn(__fsub_rn(hi1, lo1), maxq);
+    g.zero = fminf(fmaxf(rintf(__fdiv_rn(-lo1, g.scale)), 0.f), maxq);
+  }
+  return g;
+}
+
+// (w - w_hat)^2 for one weight on grid g, exact in fp64.
+__device__ __forceinline__ double clip_sq_err(float x, const Grid& g, float rscale, float maxq) {
+  const float q = fminf(fmaxf(round_quotient(x, g.scale, rscale) + g.zero, 0.f), maxq);
+  const float wh = __fmul_rn(g.scale, q - g.zero);
+  const double d = (double)__fsub_rn(x, wh);
+  return d * d;
+}
+
+// Per-channel grid with the clip search: one CTA of 256 threads per row.
+__global__ void __launch_bounds__(256) row_clip_params_kernel(const float* __restrict__ W, int m,
+                                                              int n, int bits,
+                                                              float* __restrict__ scales,
+                                                              uint8_t* __restrict__ zeros) {
+  __shared__ float rmn[8], rmx[8];
+  __shared__ double part[8][CLIP_STEPS];   // per-warp error sums of every candidate
+  const int row = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const float* w = W + (int64_t)row * n;
+  const float maxq = (float)((1 << bits) - 1);
+  float mn = INFINITY, mx = -INFINITY;
+  for (int j = tid; j < n; j += blockDim.x) {
+    const float v = w[j];
+    mn = fminf(mn, v);
+    mx = fmaxf(mx, v);
+  }
+  for (int o = 16; o > 0; o >>= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  if (lane == 0) { rmn[warp] = mn; rmx[warp] = mx; }
+  __syncthreads();
+  mn = rmn[0]; mx = rmx[0];
+  for (int k = 1; k < 8; ++k) { mn = fminf(mn, rmn[k]); mx = fmaxf(mx, rmx[k]); }
+  const float lo = fminf(mn, 0.f), hi = fmaxf(mx, 0.f);
+  for (int i = 0; i < CLIP_STEPS; ++i) {
+    const Grid g = clip_grid(lo, hi, clip_ratio(i), maxq);
+    const float rs = __frcp_rn(g.scale);
+    double acc = 0.0;
+    for (int j = tid; j < n; j += blockDim.x) acc += clip_sq_err(w[j], g, rs, maxq);
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) part[warp][i] = acc;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    double best = INFINITY;
+    int best_i = 0;
+    for (int i = 0; i < CLIP_STEPS; ++i) {
+      double tot = 0.0;
+      for (int k = 0; k < 8; ++k) tot += part[k][i];
+      if (tot < best) { best = tot; best_i = i; }
+    }
+    const Grid g = clip_grid(lo, hi, clip_ratio(best_i), maxq);
+    scales[row] = g.scale;
+    zeros[row] = (uint8_t)g.zero;
+  }
+}
+
 // Per-channel grid from the whole row, one warp per row.
 __global__ void row_params_kernel(const float* __restrict__ W, int m, int n, int bits,
                                   float* __restrict__ scales, uint8_t* __restrict__ zeros) {
@@ -93,7 +175,7 @@ __global__ void row_params_kernel(const float* __restrict__ W, int m, int n, int
   }
 }
 
-template <int GROUP>  // 0: per-channel grid; else 32, 64 or 128
+template <int GROUP, bool CLIP>  // GROUP 0: per-channel grid; else 32, 64 or 128.  CLIP: --w_clip
 __global__ void __launch_bounds__(OBS_THREADS)
 obs_block_kernel(const float* __restrict__ W, int m, int n, const float* __restrict__ U, int i1,
                  int bits, uint8_t* __restrict__ codes, float* __restrict__ scales,
@@ -188,7 +270,29 @@ obs_block_kernel(const float* __restrict__ W, int m, int n, const float* __restr
             mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
           }
-          const Grid g = make_grid(mn, mx, maxq);
+          Grid g = make_grid(mn, mx, maxq);
+          if (CLIP) {
+            // the clip search over this group: every candidate's error summed
+            // over the row's 8 threads, the total taken from the row's first
+            // thread so that all 8 make the same choice
+            const float lo = fminf(mn, 0.f), hi = fmaxf(mx, 0.f);
+            double best = INFINITY;
+            int best_i = 0;
+#pragma unroll 1
+            for (int ci = 0; ci < CLIP_STEPS; ++ci) {
+              const Grid gc = clip_grid(lo, hi, clip_ratio(ci), maxq);
+              const float rs = __frcp_rn(gc.scale);
+              double acc = 0.0;
+#pragma unroll
+              for (int k = 4 * sg; k < 4 * sg + (GROUP >= 32 ? GROUP / 8 : 4) && k < 16; ++k)
+                acc += clip_sq_err(w[k], gc, rs, maxq);
+#pragma unroll
+              for (int o = 1; o < 8; o <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+              acc = __shfl_sync(0xffffffffu, acc, lane & ~7);
+              if (acc < best) { best = acc; best_i = ci; }
+            }
+            g = clip_grid(lo, hi, clip_ratio(best_i), maxq);
+          }
           scale = g.scale;
           zero = g.zero;
           rscale = __frcp_rn(scale);
@@ -382,20 +486,20 @@ __global__ void __launch_bounds__(256) slab_transpose_kernel(const float* __rest
   }
 }
 
-template <int GROUP>
+template <int GROUP, bool CLIP>
 int launch_block(const float* W, int m, int n, const float* U, int i1, int bits, uint8_t* codes,
                  float* scales, uint8_t* zeros, float* W_hat, const SolverScratch& sc, int sb,
                  int slab_end, cudaStream_t st) {
   static bool attr = false;
   const size_t smem = (size_t)(QB * US_LD + QB + QB * TT_LD) * sizeof(float);
   if (!attr) {
-    if (cudaFuncSetAttribute(obs_block_kernel<GROUP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
+    if (cudaFuncSetAttribute(obs_block_kernel<GROUP, CLIP>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
       return KRONQ_ERR_CUDA;
     attr = true;
   }
   const int grid = (m + ROWS_PER_CTA - 1) / ROWS_PER_CTA;
-  obs_block_kernel<GROUP><<<grid, OBS_THREADS, smem, st>>>(W, m, n, U, i1, bits, codes, scales, zeros,
+  obs_block_kernel<GROUP, CLIP><<<grid, OBS_THREADS, smem, st>>>(W, m, n, U, i1, bits, codes, scales, zeros,
                                                    W_hat, sc.Eh + (i1 - sb), sc.El + (i1 - sb),
                                                    sc.B2, sc.Uth, sc.Utl, slab_end);
   KQ_CHECK_LAUNCH();
@@ -422,9 +526,11 @@ size_t kq_quantize_ws(int64_t m, int64_t n) { return solver_ws(m, n, QB2); }
 size_t kq_loss_ws(int64_t m, int64_t n) { return 3 * a256((size_t)m * n * sizeof(float)); }
 
 int kq_quantize_layer(float* W, int64_t m64, int64_t n64, const float* U, int bits, int group,
-                      int block, uint8_t* codes, float* scales, uint8_t* zeros, float* W_hat,
-                      int32_t* info, void* ws, size_t ws_bytes, cudaStream_t st) {
+                      int block, int options, uint8_t* codes, float* scales, uint8_t* zeros,
+                      float* W_hat, int32_t* info, void* ws, size_t ws_bytes, cudaStream_t st) {
   if (!W || !U || !codes || !scales || !zeros || m64 <= 0 || n64 <= 0) return KRONQ_ERR_INVALID_ARG;
+  if (options & ~KRONQ_QUANT_CLIP) return KRONQ_ERR_INVALID_ARG;
+  const bool clip = (options & KRONQ_QUANT_CLIP) != 0;
   if (bits != 2 && bits != 3 && bits != 4 && bits != 8) return KRONQ_ERR_INVALID_ARG;
   if (group != -1 && (group <= 0 || n64 % group)) return KRONQ_ERR_INVALID_ARG;
   if (block != QB) return KRONQ_ERR_UNSUPPORTED;
@@ -460,7 +566,10 @@ int kq_quantize_layer(float* W, int64_t m64, int64_t n64, const float* U, int bi
     }
   }
 
-  if (group == -1) {
+  if (group == -1 && clip) {
+    row_clip_params_kernel<<<m, 256, 0, st>>>(W, m, n, bits, scales, zeros);
+    KQ_CHECK_LAUNCH();
+  } else if (group == -1) {
     row_params_kernel<<<(m + 7) / 8, 256, 0, st>>>(W, m, n, bits, scales, zeros);
     KQ_CHECK_LAUNCH();
   }
@@ -469,12 +578,14 @@ int kq_quantize_layer(float* W, int64_t m64, int64_t n64, const float* U, int bi
     const int slab_end = B2 > QB ? sb_end : n;
     for (int i1 = sb; i1 < sb_end; i1 += QB) {
       int s;
+#define KQ_BLOCK(G, C) launch_block<G, C>(W, m, n, U, i1, bits, codes, scales, zeros, W_hat, sc, sb, slab_end, st)
       switch (group) {
-        case -1: s = launch_block<0>(W, m, n, U, i1, bits, codes, scales, zeros, W_hat, sc, sb, slab_end, st); break;
-        case 32: s = launch_block<32>(W, m, n, U, i1, bits, codes, scales, zeros, W_hat, sc, sb, slab_end, st); break;
-        case 64: s = launch_block<64>(W, m, n, U, i1, bits, codes, scales, zeros, W_hat, sc, sb, slab_end, st); break;
-        default: s = launch_block<128>(W, m, n, U, i1, bits, codes, scales, zeros, W_hat, sc, sb, slab_end, st); break;
+        case -1: s = KQ_BLOCK(0, false); break;   // per-channel: the clip search ran before the loop
+        case 32: s = clip ? KQ_BLOCK(32, true) : KQ_BLOCK(32, false); break;
+        case 64: s = clip ? KQ_BLOCK(64, true) : KQ_BLOCK(64, false); break;
+        default: s = clip ? KQ_BLOCK(128, true) : KQ_BLOCK(128, false); break;
       }
+#undef KQ_BLOCK
       if (s != KRONQ_OK) return s;
       const int i2 = i1 + QB;
       if (i2 < sb_end) {
@@ -622,6 +733,6 @@ int kq_quantize_layer_noalloc(float* W, int64_t m, int64_t n, const float* U, in
   if (m > kNoAllocMaxRows || n > kNoAllocMaxCols) return KRONQ_ERR_UNSUPPORTED;
   float* scratch = noalloc_scratch();
   if (!scratch) return KRONQ_ERR_CUDA;
-  return kq_quantize_layer(W, m, n, U, bits, group, block, codes, scales, zeros, W_hat, info,
+  return kq_quantize_layer(W, m, n, U, bits, group, block, 0, codes, scales, zeros, W_hat, info,
                            scratch, sizeof(g_noalloc_scratch), st);
 }

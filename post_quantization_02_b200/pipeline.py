@@ -32,8 +32,9 @@ class LayerResult:
     W_hat: torch.Tensor | None
     H_X: torch.Tensor            # rotated H_X'
     H_G: torch.Tensor            # rotated H_G'
-    U_c: torch.Tensor
+    U_c: torch.Tensor            # factor of the (permuted, with act_order) damped H_X'
     info: torch.Tensor           # device int32 status word
+    perm: torch.Tensor | None = None   # --act_order column order (int32), None without
 
 
 def covariance(A: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
@@ -48,11 +49,15 @@ def quantize_sublayer(W: torch.Tensor, HX: torch.Tensor, HG: torch.Tensor,
                       sign_u: torch.Tensor, sign_v: torch.Tensor, bits: int, group: int = -1,
                       alpha: float = 0.25, mode: str = "full", damp: float = 0.01,
                       block: int = 128, keep: bool = False, ws: torch.Tensor | None = None,
-                      in_place: bool = False, stream=None) -> LayerResult:
+                      in_place: bool = False, act_order: bool = False, clip: bool = False,
+                      stream=None) -> LayerResult:
     """BiIP -> sensitivity -> inverse Cholesky -> OBS -> pack for one sublayer.
 
     W (m x n fp32), HX (n x n fp32), HG (m x m fp32) are device tensors.  They
-    are cloned unless in_place is set (then W, HX, HG are overwritten)."""
+    are cloned unless in_place is set (then W, HX, HG are overwritten).
+    act_order / clip: the README's --act_order and --w_clip (readings in
+    include/kronq.h); codes, W_hat and W_rot come back in the original column
+    order, scales / zeros by groups of the permuted order."""
     m, n = W.shape
     dev = W.device
     if not in_place:
@@ -66,20 +71,37 @@ def quantize_sublayer(W: torch.Tensor, HX: torch.Tensor, HG: torch.Tensor,
     sens = torch.empty(3, dtype=torch.float64, device=dev)
     abi.kronq_sensitivity(HX, HG, sens, stream=stream)
     U = torch.empty((n, n), dtype=torch.float32, device=dev)
-    abi.kronq_cholesky_inv(HX, damp, U, info, ws, stream=stream)
     W_rot = W.clone() if keep else None
+    perm = None
+    Hs, Ws = HX, W
+    if act_order:
+        perm = torch.empty(n, dtype=torch.int32, device=dev)
+        abi.kronq_act_order(HX, perm, stream=stream)
+        Hs, Ws = torch.empty_like(HX), torch.empty_like(W)
+        abi.kronq_permute(HX, Hs, perm, abi.PERM_SYM, info, stream=stream)
+        abi.kronq_permute(W, Ws, perm, abi.PERM_COLS, info, stream=stream)
+    abi.kronq_cholesky_inv(Hs, damp, U, info, ws, stream=stream)
     G = 1 if group == -1 else n // group
     codes = torch.empty((m, n), dtype=torch.uint8, device=dev)
     scales = torch.empty((m, G), dtype=torch.float32, device=dev)
     zeros = torch.empty((m, G), dtype=torch.uint8, device=dev)
     W_hat = torch.empty((m, n), dtype=torch.float32, device=dev) if keep else None
-    abi.kronq_quantize_layer(W, U, bits, group, block, codes, scales, zeros, W_hat, info, ws,
-                             stream=stream)
+    abi.kronq_quantize_layer_opt(Ws, U, bits, group, block, abi.QUANT_CLIP if clip else 0,
+                                 codes, scales, zeros, W_hat, info, ws, stream=stream)
+    if act_order:
+        c_back = torch.empty_like(codes)
+        abi.kronq_permute(codes, c_back, perm, abi.UNPERM_COLS, info, stream=stream)
+        codes = c_back
+        if W_hat is not None:
+            h_back = torch.empty_like(W_hat)
+            abi.kronq_permute(W_hat, h_back, perm, abi.UNPERM_COLS, info, stream=stream)
+            W_hat = h_back
     packed = None
     if bits in (2, 4):
         packed = torch.empty((m, abi.packed_words(n, bits)), dtype=torch.int32, device=dev)
         abi.kronq_pack(codes, bits, packed, stream=stream)
-    return LayerResult(codes, scales, zeros, packed, sens, SX, SG, W_rot, W_hat, HX, HG, U, info)
+    return LayerResult(codes, scales, zeros, packed, sens, SX, SG, W_rot, W_hat, HX, HG, U, info,
+                       perm)
 
 
 def covariance_from_host(A_host: torch.Tensor, H: torch.Tensor, chunk_rows: int = 16384,

@@ -94,6 +94,28 @@ def test_host_side_argument_errors(L):
                               ctypes.c_float(0.0), null, null) == 0
 
 
+def test_host_side_argument_errors_act_order_clip(L):
+    null = None
+    ptr = ctypes.c_void_p(16)  # never dereferenced: rejected before any launch
+    # unknown option bits
+    assert L.kronq_quantize_layer_opt(ptr, 4, 256, ptr, 4, -1, 128, 2, ptr, ptr, ptr, null, null,
+                                      null, 0, null) == -1
+    # the clip option passes the argument checks up to the workspace
+    assert L.kronq_quantize_layer_opt(ptr, 4, 256, ptr, 4, -1, 128, 1, ptr, ptr, ptr, null, null,
+                                      null, 0, null) == -6
+    # act_order: empty is a no-op, null pointers invalid
+    assert L.kronq_act_order(null, 0, null, null) == 0
+    assert L.kronq_act_order(null, 8, ptr, null) == -1
+    # permute: bad mode, aliasing, symmetric needs a square fp32 matrix, bad element size
+    q = ctypes.c_void_p(32)
+    assert L.kronq_permute(ptr, q, 4, 8, 4, ptr, 7, null, null) == -1
+    assert L.kronq_permute(ptr, ptr, 4, 8, 4, ptr, 0, null, null) == -1
+    assert L.kronq_permute(ptr, q, 4, 8, 4, ptr, 2, null, null) == -1
+    assert L.kronq_permute(ptr, q, 8, 8, 1, ptr, 2, null, null) == -1
+    assert L.kronq_permute(ptr, q, 4, 8, 2, ptr, 0, null, null) == -1
+    assert L.kronq_permute(null, null, 0, 8, 4, null, 0, null, null) == 0
+
+
 def test_binding_refuses_host_tensors():
     import torch
     from post_quantization_02_b200 import abi

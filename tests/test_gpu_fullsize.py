@@ -299,3 +299,60 @@ def test_llama3_8b_block_ranking_allocation_and_down_proj(cuda):
         del HG[name]
     torch.cuda.empty_cache()
     _sublayer_chain(cfg, sub, HX[sub.site], HG[sub.name], bits[-1], r)
+
+
+def test_llama2_7b_q_proj_act_order_and_clip_solver_full_size(cuda):
+    """The README's --act_order and --w_clip (readings in include/kronq.h) on
+    the benchmarked layer, in the launch sequence bench.py times with
+    --act-order --w-clip: covariances -> BiIP -> act_order -> permute H_X',
+    W' -> inverse Cholesky of the permuted damped H_X' -> solver with the
+    clip search -> codes back to the original order.  Stage-isolated like
+    the chain above: the oracle takes the GPU's fp32 H_X' and W' (so the
+    permutation is compared bit-exact), factors the permuted damped matrix
+    itself and re-runs the column loop on 1024 seeded rows."""
+    cfg = synth.get_config("llama2-7b-q_proj")
+    sub = cfg.sublayers[0]
+    m, n, bits, group = sub.m, sub.n, sub.bits, sub.group
+    r = np.random.default_rng(303)
+    HXs, HGs, _, _ = _covariances(cfg, cuda, r)
+    HX, HG = HXs[sub.site], HGs[sub.name]
+    dev = cuda
+    su, sv = synth.make_signs(cfg, sub)
+    Wd = torch.from_numpy(synth.make_w(cfg, sub)).to(dev)
+    ws = abi.workspace(m, n, bits, group, device=dev)
+    SX, SG = torch.empty(n, device=dev), torch.empty(m, device=dev)
+    abi.kronq_biip_rotate(Wd, HX, HG, torch.from_numpy(su).to(dev), torch.from_numpy(sv).to(dev),
+                          cfg.alpha, cfg.mode, 0, SX, SG, ws)
+    info = torch.zeros(1, dtype=torch.int32, device=dev)
+    perm = torch.empty(n, dtype=torch.int32, device=dev)
+    abi.kronq_act_order(HX, perm)
+    Hp, Wp = torch.empty_like(HX), torch.empty_like(Wd)
+    abi.kronq_permute(HX, Hp, perm, abi.PERM_SYM, info)
+    abi.kronq_permute(Wd, Wp, perm, abi.PERM_COLS, info)
+    U = torch.empty_like(HX)
+    abi.kronq_cholesky_inv(Hp, cfg.damp, U, info, ws)
+    cp = torch.empty((m, n), dtype=torch.uint8, device=dev)
+    scales = torch.empty((m, 1), device=dev)
+    zeros = torch.empty((m, 1), dtype=torch.uint8, device=dev)
+    Whp = torch.empty((m, n), device=dev)
+    abi.kronq_quantize_layer_opt(Wp, U, bits, group, cfg.block, abi.QUANT_CLIP, cp, scales, zeros,
+                                 Whp, info, ws)
+    codes, What = torch.empty_like(cp), torch.empty_like(Whp)
+    abi.kronq_permute(cp, codes, perm, abi.UNPERM_COLS, info)
+    abi.kronq_permute(Whp, What, perm, abi.UNPERM_COLS, info)
+    torch.cuda.synchronize()
+    assert info.item() == 0
+    HXr, Wrot = HX.cpu().numpy(), Wd.cpu().numpy()
+    p_ref = oq.act_order_perm(HXr)
+    np.testing.assert_array_equal(perm.cpu().numpy(), p_ref)
+    rows = np.sort(r.choice(m, 1024, replace=False))
+    Hd = ochol.damp(HXr, cfg.damp)
+    ref = oq.obs_quantize_act_order(Wrot[rows], Hd, p_ref, bits, group, clip=True)
+    cg = codes.cpu().numpy()[rows]
+    same = (cg == ref["codes"]).mean()
+    assert same >= 0.999, same
+    np.testing.assert_array_equal(scales.cpu().numpy()[rows], ref["scale"])
+    np.testing.assert_array_equal(zeros.cpu().numpy()[rows], ref["zero"])
+    lg = oq.row_losses(Wrot[rows] - What.cpu().numpy()[rows], HXr, cfg.damp).sum()
+    lr = oq.row_losses(Wrot[rows] - ref["W_hat"], HXr, cfg.damp).sum()
+    assert abs(lg / lr - 1) <= 0.01, (lg, lr)
