@@ -26,4 +26,4 @@ brute force on tiny inputs, textbook matrices) -- except where a docstring
 says "parity unpinned".
 """
 
-from . import covariance, transform, biip, sensitivity, cholesky, quantizer, pack, pipeline, diagnostics  # noqa: F401
+from . import covariance, transform, biip, sensitivity, cholesky, quantizer, pack, pipeline, diagnostics, deploy  # noqa: F401
