@@ -50,6 +50,9 @@ def parse():
                     help="quantize columns in descending H_X' diagonal order (README --act_order)")
     ap.add_argument("--w-clip", action="store_true",
                     help="clip-ratio search for every grid (README --w_clip)")
+    ap.add_argument("--deploy", action="store_true",
+                    help="time the deployment matvec (kronq_deploy_matvec, batch 1) of the "
+                         "quantized layer instead of the quantization step")
     ap.add_argument("--tokens", type=int, default=None,
                     help="calibration tokens per X/G (default: the workload's; smaller only for "
                          "profiler captures)")
@@ -383,8 +386,93 @@ def gpu_step(cfg, layers, X, ws, stream, cov_events=None, act_order=False, clip=
                            stream=stream)
 
 
+def run_deploy(args):
+    """Batch-1 decode through the packed layer: y = W_hat x with the BiIP
+    transforms applied to x and y (kronq_deploy_matvec).  The layer is
+    quantized once on the GPU; `copies` distinct copies of its packed codes
+    (more bytes than L2) are cycled so that every matvec reads its weights
+    from HBM; the calls are captured in one CUDA graph (one replay = all
+    copies) and timed with CUDA events."""
+    import dataclasses
+    import numpy as np
+    import torch
+    import synth
+    from post_quantization_02_b200 import abi
+    from post_quantization_02_b200 import pipeline as gpipe
+    dev = torch.device("cuda", 0)
+    cfg = dataclasses.replace(synth.get_config(args.config), tokens=args.tokens or 16384)
+    sub = cfg.sublayers[0]
+    m, n, bits, group = sub.m, sub.n, (sub.bits if sub.bits in (2, 4) else 4), sub.group
+    site = cfg.site(sub.site)
+    X = torch.from_numpy(synth.make_x(cfg, site).view(np.int16)).to(dev).view(torch.bfloat16)
+    G_ = torch.from_numpy(synth.make_g(cfg, sub).view(np.int16)).to(dev).view(torch.bfloat16)
+    HX, HG = gpipe.covariance(X), gpipe.covariance(G_)
+    del X, G_
+    su, sv = synth.make_signs(cfg, sub)
+    su_d, sv_d = torch.from_numpy(su).to(dev), torch.from_numpy(sv).to(dev)
+    W = torch.from_numpy(synth.make_w(cfg, sub)).to(dev)
+    res = gpipe.quantize_sublayer(W, HX, HG, su_d, sv_d, bits, group, cfg.alpha, cfg.mode,
+                                  cfg.damp, cfg.block)
+    torch.cuda.synchronize()
+    layer_bytes = res.packed.numel() * 4 + res.scales.numel() * 4 + res.zeros.numel()
+    copies = max(2, int(4 * 126 * 2 ** 20 // layer_bytes) + 1)
+    packs = [res.packed.clone() for _ in range(copies)]
+    x = torch.randn((1, n), device=dev)
+    ys = [torch.empty((1, m), device=dev) for _ in range(copies)]
+    ws = abi.deploy_workspace(m, n, 1, dev)
+    stream = torch.cuda.Stream(dev)
+
+    def call(k):
+        abi.kronq_deploy_matvec(packs[k], n, bits, group, res.scales, res.zeros, res.S_X, res.S_G,
+                                su_d, sv_d, cfg.mode, x, ys[k], ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for k in range(copies):
+            call(k)
+    torch.cuda.synchronize()
+    launches0 = abi.kronq_launch_count()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for k in range(copies):
+            call(k)
+    launches_per_replay = abi.kronq_launch_count() - launches0
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):          # replay() runs on the current stream
+        for _ in range(max(3, args.warmup)):
+            g.replay()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.steps):
+            g.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / (args.steps * copies)
+    peaks, src = load_peaks()
+    algo = layer_bytes + (n + m) * 4
+    achieved = algo / (us * 1e-6) / 1e9
+    line = {
+        "metric": "deploy matvec us per layer (batch 1, packed weights from HBM)", "value": us,
+        "unit": "us", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": us * copies / 1e3, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded generator)",
+        "config": {"workload": f"{cfg.name} {sub.name} {m}x{n} W{bits} "
+                               f"{'per-channel' if group == -1 else f'g{group}'} BiIP {cfg.mode}",
+                   "copies_cycled": copies, "bytes_per_layer": int(algo),
+                   "l2": "distinct copies larger than L2 in total, no flush"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": float(peaks["hbm_gbs"]),
+                     "unit": "GB/s", "frac": achieved / float(peaks["hbm_gbs"]), "traffic": None,
+                     "kernel": "kronq_deploy_matvec (transforms + dequant_matvec_kernel)",
+                     "peak_source": src},
+        "gpu_launches": launches_per_replay * args.steps,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
+    if args.deploy:
+        run_deploy(args)
+        return
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))

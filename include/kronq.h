@@ -234,6 +234,33 @@ int kronq_permute(const void* src, void* dst, int64_t m, int64_t n, int elem_byt
                   const int32_t* perm, int mode, int32_t* info, void* stream);
 
 /*
+ * Deployment matvec of a quantized layer: y = W_hat x in the original space,
+ * straight from the packed codes, with the BiIP transforms applied to the
+ * vectors (KronQ README (GitHub): the fused dequant + BiIP matvec of the
+ * deploy path, batch-1 decode).  With W' = U S_G W S_X V^T (KronQ summary
+ * (hyper.ai), "Method", Eqs. 11-12):
+ *     y = S_G^-1 U^T ( W_hat' ( V S_X^-1 x ) ),
+ *     W_hat'[i][j] = scale[i][g(j)] (code[i][j] - zero[i][g(j)]).
+ *
+ * packed : m x (n bits/32) uint32 from kronq_pack, 16-byte aligned.
+ * bits   : 2 or 4.  group: -1 (per-channel), 32, 64 or 128.
+ * scales, zeros : m x G as written by kronq_quantize_layer (no act_order:
+ *          the columns of the codes are in the transform's order).
+ * S_X (n), S_G (m), sign_u (m), sign_v (n), mode : as used and written by
+ *          kronq_biip_rotate (S_X, S_G 16-byte, the signs 4-byte aligned).
+ * x      : batch x n fp32, y: batch x m fp32 (16-byte aligned); batch 1, 2,
+ *          4 or 8.  n a multiple of 64, m of 16.
+ * ws     : at least kronq_deploy_workspace_size(m, n, batch) bytes.
+ */
+size_t kronq_deploy_workspace_size(int64_t m, int64_t n, int64_t batch);
+int kronq_deploy_matvec(const uint32_t* packed, int64_t m, int64_t n, int bits, int group,
+                        const float* scales, const uint8_t* zeros,
+                        const float* S_X, const float* S_G,
+                        const int8_t* sign_u, const int8_t* sign_v, int mode,
+                        const float* x, int64_t batch, float* y,
+                        void* ws, size_t ws_bytes, void* stream);
+
+/*
  * kronq_quantize_layer without a workspace: for callers that cannot allocate
  * device memory while they run (a host framework that owns the allocator,
  * memory planned once at start-up, or a loop where cudaMalloc/cudaFree would

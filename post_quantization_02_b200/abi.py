@@ -57,6 +57,8 @@ def lib() -> ctypes.CDLL:
         "kronq_quantize_layer_opt": ([P, I64, I64, P, I32, I32, I32, I32, P, P, P, P, P, P, SZ, P], I32),
         "kronq_act_order": ([P, I64, P, P], I32),
         "kronq_permute": ([P, P, I64, I64, I32, P, I32, P, P], I32),
+        "kronq_deploy_workspace_size": ([I64, I64, I64], SZ),
+        "kronq_deploy_matvec": ([P, I64, I64, I32, I32, P, P, P, P, P, P, I32, P, I64, P, P, SZ, P], I32),
         "kronq_pack": ([P, I64, I64, I32, P, P], I32),
         "kronq_unpack": ([P, I64, I64, I32, P, P], I32),
         "kronq_layer_loss": ([P, P, I64, I64, P, P, P, P, SZ, P], I32),
@@ -228,6 +230,33 @@ def kronq_permute(src, dst, perm, mode: int, info=None, stream=None):
     m, n = src.shape
     _check("kronq_permute", lib().kronq_permute(_p(src), _p(dst), m, n, src.element_size(),
                                                 _p(perm), mode, _p(info), _s(stream)))
+
+
+def kronq_deploy_workspace_size(m: int, n: int, batch: int) -> int:
+    return lib().kronq_deploy_workspace_size(m, n, batch)
+
+
+def deploy_workspace(m: int, n: int, batch: int, device=None) -> torch.Tensor:
+    nbytes = kronq_deploy_workspace_size(m, n, batch)
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def kronq_deploy_matvec(packed, n: int, bits: int, group: int, scales, zeros, SX, SG, sign_u, sign_v,
+                        mode, x, y, ws, stream=None):
+    """y (batch x m) = W_hat x for x (batch x n) from the packed layer (see kronq.h)."""
+    _dev(packed, (torch.int32, torch.uint32), "packed", 2)
+    _dev(x, torch.float32, "x", 2)
+    _dev(y, torch.float32, "y", 2)
+    for t_, nm in ((packed, "packed"), (scales, "scales"), (zeros, "zeros"), (x, "x"), (y, "y")):
+        _contig(t_, nm)
+    m = packed.shape[0]
+    batch = x.shape[0]
+    if x.shape[1] != n or y.shape != (batch, m):
+        raise ValueError("kronq_deploy_matvec: shapes do not match")
+    md = MODES[mode] if isinstance(mode, str) else int(mode)
+    _check("kronq_deploy_matvec", lib().kronq_deploy_matvec(
+        _p(packed), m, n, bits, group, _p(scales), _p(zeros), _p(SX), _p(SG), _p(sign_u),
+        _p(sign_v), md, _p(x), batch, _p(y), _p(ws), ws.numel() * ws.element_size(), _s(stream)))
 
 
 def kronq_quantize_layer_noalloc(W, U, bits: int, group: int, block: int, codes, scales, zeros,

@@ -22,6 +22,11 @@ int kq_quantize_layer(float* W, int64_t m, int64_t n, const float* U, int bits, 
                       int block, int options, uint8_t* codes, float* scales, uint8_t* zeros,
                       float* W_hat, int32_t* info, void* ws, size_t ws_bytes, cudaStream_t st);
 int kq_act_order(const float* H, int64_t n, int32_t* perm, cudaStream_t st);
+size_t kq_deploy_ws(int64_t m, int64_t n, int64_t batch);
+int kq_deploy_matvec(const uint32_t* packed, int64_t m, int64_t n, int bits, int group,
+                     const float* scales, const uint8_t* zeros, const float* SX, const float* SG,
+                     const int8_t* su, const int8_t* sv, int mode, const float* x, int64_t batch,
+                     float* y, void* ws, size_t ws_bytes, cudaStream_t st);
 int kq_permute(const void* src, void* dst, int64_t m, int64_t n, int elem_bytes,
                const int32_t* perm, int mode, int32_t* info, cudaStream_t st);
 int kq_quantize_layer_noalloc(float* W, int64_t m, int64_t n, const float* U, int bits, int group,
@@ -160,6 +165,19 @@ int kronq_act_order(const float* H, int64_t n, int32_t* perm, void* stream) {
 int kronq_permute(const void* src, void* dst, int64_t m, int64_t n, int elem_bytes,
                   const int32_t* perm, int mode, int32_t* info, void* stream) {
   return kq_permute(src, dst, m, n, elem_bytes, perm, mode, info, S(stream));
+}
+
+size_t kronq_deploy_workspace_size(int64_t m, int64_t n, int64_t batch) {
+  return kq_deploy_ws(m, n, batch);
+}
+
+int kronq_deploy_matvec(const uint32_t* packed, int64_t m, int64_t n, int bits, int group,
+                        const float* scales, const uint8_t* zeros, const float* S_X,
+                        const float* S_G, const int8_t* sign_u, const int8_t* sign_v, int mode,
+                        const float* x, int64_t batch, float* y, void* ws, size_t ws_bytes,
+                        void* stream) {
+  return kq_deploy_matvec(packed, m, n, bits, group, scales, zeros, S_X, S_G, sign_u, sign_v, mode,
+                          x, batch, y, ws, ws_bytes, S(stream));
 }
 
 int kronq_quantize_layer_noalloc(float* W, int64_t m, int64_t n, const float* U_c, int bits,

@@ -403,10 +403,13 @@ int set_attrs() {
 
 // Apply T D along rows (row pass, with scaling) of an R x C matrix.
 int row_pass(float* X, int R, int C, const float* rs, const float* cs, const int8_t* sign,
-             const Split& sp, const float* M, int inverse, float* cf, cudaStream_t st) {
+             const Split& sp, const float* M, int inverse, float* cf, cudaStream_t st,
+             bool cf_ready = false) {
   if (sp.Q == 1 && sp.L2 >= 512) {
-    col_factor_kernel<<<(C + 255) / 256, 256, 0, st>>>(cs, sign, C, cf);
-    KQ_CHECK_LAUNCH();
+    if (!cf_ready) {
+      col_factor_kernel<<<(C + 255) / 256, 256, 0, st>>>(cs, sign, C, cf);
+      KQ_CHECK_LAUNCH();
+    }
     const dim3 g((R + 1) / 2, C / sp.L2);
     switch (sp.L2) {
       case 512: row_fht_kernel<4><<<g, 128, 0, st>>>(X, R, C, rs, cf, inverse); break;
@@ -584,3 +587,61 @@ int kq_biip_rotate(float* W, int64_t m64, int64_t n64, float* HX, float* HG, con
   }
   return KRONQ_OK;
 }
+
+// ---------------------------------------------------------------------------
+// Vectors through one side of BiIP (the deployment path): each row x of the
+// R x C matrix X becomes V diag(1/S) x (forward) or diag(1/S) V^T x
+// (inverse), V = T_C D (rotate = 1), or only the scaling (rotate = 0).
+// Scratch: kq_vec_transform_ws(C) bytes.
+size_t kq_vec_transform_ws(int64_t C) {
+  return 2 * a256((size_t)C * sizeof(float)) + a256(64 * 64 * sizeof(float));
+}
+
+namespace {
+// rS[c] = 1 / S[c] and cf[c] = sign[c] / S[c] (the row pass's column factor).
+__global__ void recip_factor_kernel(const float* __restrict__ S, const int8_t* __restrict__ sign,
+                                    int C, float* __restrict__ rS, float* __restrict__ cf) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c < C) {
+    const float r = 1.f / S[c];
+    rS[c] = r;
+    if (sign) cf[c] = r * (float)sign[c];
+  }
+}
+
+__global__ void vec_scale_kernel(float* __restrict__ X, int64_t R, int C, const float* __restrict__ rS) {
+  const int64_t total = R * C;
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
+       e += (int64_t)gridDim.x * blockDim.x)
+    X[e] *= rS[e % C];
+}
+}  // namespace
+
+int kq_vec_transform(float* X, int64_t R, int64_t C, const float* S, const int8_t* sign, int rotate,
+                     int inverse, void* ws, cudaStream_t st) {
+  if (!X || !S || (rotate && !sign) || R <= 0 || C <= 0) return KRONQ_ERR_INVALID_ARG;
+  Split sp;
+  if (!split_width(C, sp) || C > 65536 || R > (1 << 30)) return KRONQ_ERR_UNSUPPORTED;
+  int s0 = set_attrs();
+  if (s0 != KRONQ_OK) return s0;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  float* rS = reinterpret_cast<float*>(w);
+  w += a256((size_t)C * sizeof(float));
+  float* cf = reinterpret_cast<float*>(w);
+  w += a256((size_t)C * sizeof(float));
+  float* M = reinterpret_cast<float*>(w);
+  recip_factor_kernel<<<(int)((C + 255) / 256), 256, 0, st>>>(S, rotate ? sign : nullptr, (int)C,
+                                                               rS, cf);
+  KQ_CHECK_LAUNCH();
+  if (!rotate) {
+    vec_scale_kernel<<<2 * kqh::num_sms(), 256, 0, st>>>(X, R, (int)C, rS);
+    KQ_CHECK_LAUNCH();
+    return KRONQ_OK;
+  }
+  if (sp.Q > 1) {
+    make_mix_kernel<<<1, 256, 0, st>>>(M, sp.q, sp.k1);
+    KQ_CHECK_LAUNCH();
+  }
+  return row_pass(X, (int)R, (int)C, nullptr, rS, sign, sp, M, inverse, cf, st, /*cf_ready=*/true);
+}
+
