@@ -63,6 +63,7 @@ __global__ void colnorm_kernel(const float* __restrict__ W, int m, int n, double
   const int rows_per = (m + gridDim.y - 1) / gridDim.y;
   const int r0 = blockIdx.y * rows_per, r1 = min(m, r0 + rows_per);
   double s = 0.0;
+#pragma unroll 8
   for (int i = r0; i < r1; ++i) {
     const double v = W[(int64_t)i * n + j];
     s += v * v;
@@ -364,16 +365,21 @@ col_fht_reg_kernel(float* __restrict__ X, int C, int L2, int st, const int8_t* _
   }
 }
 
-__global__ void sensitivity_kernel(const float* __restrict__ HX, int n, const float* __restrict__ HG,
-                                   int m, double* __restrict__ out) {
-  __shared__ double sx[256], sg[256];
+__global__ void __launch_bounds__(1024) sensitivity_kernel(const float* __restrict__ HX, int n,
+                                                           const float* __restrict__ HG, int m,
+                                                           double* __restrict__ out) {
+  // one CTA of 1024 threads: every diagonal entry is a separate cache line,
+  // so the loads are spread over as many threads as possible
+  __shared__ double sx[1024], sg[1024];
   double a = 0.0, b = 0.0;
+#pragma unroll 4
   for (int i = threadIdx.x; i < n; i += blockDim.x) a += (double)HX[(int64_t)i * n + i];
+#pragma unroll 4
   for (int i = threadIdx.x; i < m; i += blockDim.x) b += (double)HG[(int64_t)i * m + i];
   sx[threadIdx.x] = a;
   sg[threadIdx.x] = b;
   __syncthreads();
-  for (int w = 128; w > 0; w >>= 1) {
+  for (int w = blockDim.x / 2; w > 0; w >>= 1) {
     if (threadIdx.x < w) {
       sx[threadIdx.x] += sx[threadIdx.x + w];
       sg[threadIdx.x] += sg[threadIdx.x + w];
@@ -479,7 +485,7 @@ int kq_sensitivity(const float* HX, int64_t n, const float* HG, int64_t m, doubl
                    cudaStream_t st) {
   if (!HX || !HG || !out || n <= 0 || m <= 0 || n > INT32_MAX || m > INT32_MAX)
     return KRONQ_ERR_INVALID_ARG;
-  sensitivity_kernel<<<1, 256, 0, st>>>(HX, (int)n, HG, (int)m, out);
+  sensitivity_kernel<<<1, 1024, 0, st>>>(HX, (int)n, HG, (int)m, out);
   KQ_CHECK_LAUNCH();
   return KRONQ_OK;
 }
@@ -541,7 +547,7 @@ int kq_biip_rotate(float* W, int64_t m64, int64_t n64, float* HX, float* HG, con
   // ---- rescale factors
   if (cudaMemsetAsync(cn, 0, (size_t)n * sizeof(double), st) != cudaSuccess) return KRONQ_ERR_CUDA;
   if (in_s) {
-    colnorm_kernel<<<dim3((n + 255) / 256, 32), 256, 0, st>>>(W, m, n, cn);
+    colnorm_kernel<<<dim3((n + 255) / 256, (m + 31) / 32), 256, 0, st>>>(W, m, n, cn);
     KQ_CHECK_LAUNCH();
   }
   scale_from_diag_kernel<<<(n + 255) / 256, 256, 0, st>>>(HX, n, cn, alpha, SX, rSX, in_s);

@@ -41,13 +41,15 @@ constexpr int SM_AS = SM_P + 32 * LDX;
 constexpr int SM_YT = SM_AS + 32 * LDA;
 constexpr int SM_FLOATS = SM_YT + 32 * LDY;
 
-__global__ void diag_sum_kernel(const float* __restrict__ H, int n, double* out) {
-  __shared__ double red[256];
+__global__ void __launch_bounds__(1024) diag_sum_kernel(const float* __restrict__ H, int n,
+                                                        double* out) {
+  __shared__ double red[1024];
   double s = 0.0;
+#pragma unroll 4
   for (int i = threadIdx.x; i < n; i += blockDim.x) s += (double)H[(int64_t)i * n + i];
   red[threadIdx.x] = s;
   __syncthreads();
-  for (int w = 128; w > 0; w >>= 1) {
+  for (int w = blockDim.x / 2; w > 0; w >>= 1) {
     if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
     __syncthreads();
   }
@@ -62,19 +64,22 @@ __global__ void reverse_damp_kernel(const float* __restrict__ H, int n, int np,
                                     float* __restrict__ R, float* __restrict__ Z, float damp_rel,
                                     const double* __restrict__ diag_sum) {
   const float delta = (float)((double)damp_rel * (*diag_sum / (double)n));
-  const int64_t total = (int64_t)np * np;
-  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
-       e += (int64_t)gridDim.x * blockDim.x) {
-    const int a = (int)(e / np), b = (int)(e % np);
-    float v;
-    if (a < n && b < n) {
-      v = H[(int64_t)(n - 1 - a) * n + (n - 1 - b)];
-      if (a == b) v += delta;
-    } else {
-      v = (a == b) ? 1.f : 0.f;
+  // one row of R (and Z) per CTA iteration, its columns across the threads
+  for (int a = blockIdx.x; a < np; a += gridDim.x) {
+    float* Ra = R + (int64_t)a * np;
+    float* Za = Z + (int64_t)a * np;
+    const float* Hr = H + (int64_t)(n - 1 - a) * n + (n - 1);   // H[n-1-a][n-1-b] = Hr[-b]
+    for (int b = threadIdx.x; b < np; b += blockDim.x) {
+      float v;
+      if (a < n && b < n) {
+        v = Hr[-b];
+        if (a == b) v += delta;
+      } else {
+        v = (a == b) ? 1.f : 0.f;
+      }
+      Ra[b] = v;
+      Za[b] = 0.f;
     }
-    R[e] = v;
-    Z[e] = 0.f;
   }
 }
 
@@ -468,7 +473,7 @@ int kq_cholesky_inv(const float* H, int64_t n64, float damp_rel, float* U, int32
   float *Lh = planes[0], *Ll = planes[1], *Zh = planes[2], *Zl = planes[3];
 
   const int sms = kqh::num_sms();
-  diag_sum_kernel<<<1, 256, 0, st>>>(H, n, dsum);
+  diag_sum_kernel<<<1, 1024, 0, st>>>(H, n, dsum);
   KQ_CHECK_LAUNCH();
   reverse_damp_kernel<<<4 * sms, 256, 0, st>>>(H, n, np, R, Z, damp_rel, dsum);
   KQ_CHECK_LAUNCH();

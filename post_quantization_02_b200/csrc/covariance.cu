@@ -327,8 +327,9 @@ cov_tc_kernel(const __grid_constant__ CUtensorMap tmap, float* __restrict__ H, i
 // otherwise sit idle take the last C - k* chunks of g = ceil(R / (P - R))
 // tiles each, k* balancing the two: k* = ceil(g C / (g + 1)).  Only two token
 // offsets are then in flight.  A tile split that way is added into H by its
-// two pairs with fp32 reductions, onto an H the host has zeroed (or scaled by
-// beta) first; with beta = 0 the sum 0 + a + b does not depend on the order.
+// two pairs with fp32 reductions, onto its region of H zeroed (or scaled by
+// beta) by a pass over the split tiles first; with beta = 0 the sum
+// 0 + a + b does not depend on the order.
 //
 // Barriers: full[s] of the even CTA counts the bytes of both CTAs' loads
 // (its producer arms it for 2 x 32 KB; the odd CTA's loads complete on it
@@ -596,6 +597,27 @@ __global__ void __launch_bounds__(256) mirror_tiles_kernel(float* __restrict__ H
   }
 }
 
+// H = beta H (zeros when beta = 0) on the listed 256 x 256 tiles only: the
+// tiles whose parts arrive by reductions.  blockIdx.x = listed tile * 64 +
+// 32 x 32 block.
+__global__ void __launch_bounds__(256) scale_tiles_kernel(float* __restrict__ H, int64_t ldh, int d,
+                                                          float beta,
+                                                          const __grid_constant__ SharedTiles st) {
+  const int li = blockIdx.x >> 6, sb = blockIdx.x & 63;
+  int rb, cb;
+  pair_tile_coords(st.tile[li], rb, cb);
+  const int i0 = rb * P_TILE + (sb >> 3) * 32, j0 = cb * P_TILE + (sb & 7) * 32;
+  if (i0 >= d || j0 >= d) return;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  for (int r = ty; r < 32; r += 8) {
+    const int i = i0 + r, j = j0 + tx;
+    if (i < d && j < d) {
+      float* p = H + (int64_t)i * ldh + j;
+      *p = (beta == 0.f) ? 0.f : beta * *p;
+    }
+  }
+}
+
 // H = beta H over d x d (ldh), zeros when beta = 0 (no read).
 __global__ void scale_kernel(float* __restrict__ H, int64_t ldh, int d, float beta) {
   const bool vec = (d % 4) == 0 && (ldh % 4) == 0;
@@ -701,12 +723,12 @@ int kq_covariance(const uint16_t* A, int64_t N, int64_t d, int64_t lda, float* H
     const bool shared = list.count > 0;
     const int pairs = (sc.waves == 0 && !shared) ? sc.rest : P;
     if (shared && beta != 1.f) {
-      // shared tiles add into H: start from beta H (zeros when beta = 0); the
-      // tiles a single pair owns then store alpha sum + 1 * (beta H)
-      scale_kernel<<<2 * kqh::num_sms(), 256, 0, st>>>(H, ldh, (int)d, beta);
+      // the split tiles add into H: they start from beta H (zeros when beta = 0);
+      // the tiles a single pair owns apply beta themselves
+      scale_tiles_kernel<<<list.count * 64, 256, 0, st>>>(H, ldh, (int)d, beta, list);
       KQ_CHECK_LAUNCH();
     }
-    const float beta_owned = shared ? (beta == 0.f ? 0.f : 1.f) : beta;
+    const float beta_owned = beta;
     cov_pair_kernel<<<2 * pairs, THREADS, P_SMEM_BYTES, st>>>(tmap, H, ldh, (int)d, k_iters, sc,
                                                              alpha, beta_owned, info);
     KQ_CHECK_LAUNCH();
