@@ -76,6 +76,29 @@ def l2_note(cfg) -> str:
             f"({cfg.tokens} tokens, bf16)")
 
 
+# ---------------------------------------------------- ranks (N > 1)
+def rank_config(cfg0, rank: int):
+    """Each rank quantizes its own layer (weak scaling): the seed is offset
+    by the rank, so no two ranks draw the same inputs."""
+    import dataclasses
+    return dataclasses.replace(cfg0, seed=cfg0.seed + rank)
+
+
+def reduce_max_ms(ms: float, world: int, device) -> float:
+    """The job's time: the slowest rank's (a MAX all-reduce; every rank calls it)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(weights: int, world: int, steps: int, ms: float) -> float:
+    """Whole-job Mweights/s: every rank's layer, all timed steps, over the max time."""
+    return weights * world * steps / (ms / 1e3) / 1e6
+
+
 # ------------------------------------------------------------- clocks
 class ClockSampler:
     """nvidia-smi samples every 200 ms while running (clocks and throttle reasons)."""
@@ -497,7 +520,7 @@ def main():
     cfg0 = synth.get_config(args.config)
     if args.tokens:
         cfg0 = dataclasses.replace(cfg0, tokens=args.tokens)
-    cfg = dataclasses.replace(cfg0, seed=cfg0.seed + rank)   # each rank: its own layer (weak scaling)
+    cfg = rank_config(cfg0, rank)   # each rank: its own layer (weak scaling)
 
     # ---- seeded inputs on the host (pinned for the end-to-end leg), then HBM
     t_gen = time.perf_counter()
@@ -540,11 +563,7 @@ def main():
     if world > 1:
         dist.barrier()
     launches = abi.kronq_launch_count() - launches0
-    ms = start.elapsed_time(end)
-    ms_t = torch.tensor([ms], device=dev)
-    if world > 1:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms = float(ms_t.item())
+    ms = reduce_max_ms(start.elapsed_time(end), world, dev)
     cov_ms = [ev[2 * i].elapsed_time(ev[2 * i + 1]) for ev in cov_events for i in range(ncov)]
 
     # ---- end to end through the public API with pinned host buffers
@@ -610,19 +629,15 @@ def main():
             h2d, d2h = e2e_step()
         s1.record(stream)
         torch.cuda.synchronize()
-        e_ms = s0.elapsed_time(s1)
-        et = torch.tensor([e_ms], device=dev)
-        if world > 1:
-            dist.all_reduce(et, op=dist.ReduceOp.MAX)
-        e_ms = float(et.item())
-        e2e = {"value": weights * world * args.e2e_steps / (e_ms / 1e3) / 1e6, "unit": UNIT,
+        e_ms = reduce_max_ms(s0.elapsed_time(s1), world, dev)
+        e2e = {"value": job_throughput(weights, world, args.e2e_steps, e_ms), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": e_ms / args.e2e_steps}
     time.sleep(0.3)
     sampler.stop()
     clocks = sampler.summary()
 
-    value = weights * world * args.steps / (ms / 1e3) / 1e6
+    value = job_throughput(weights, world, args.steps, ms)
     peaks, peak_src = load_peaks()
     timed_s = ms / 1e3
     peak_kind = "bf16_tflops_sustained" if timed_s >= 1.0 else "bf16_tflops"

@@ -39,7 +39,9 @@ constexpr int SM_X = SM_D + NB * LDD;
 constexpr int SM_P = SM_X + NB * LDX;
 constexpr int SM_AS = SM_P + 32 * LDX;
 constexpr int SM_YT = SM_AS + 32 * LDA;
-constexpr int SM_FLOATS = SM_YT + 32 * LDY;
+constexpr int SM_LB = SM_YT + 32 * LDY;       // the leaf's broadcast buffers (2 x 32)
+constexpr int SM_FLOATS = SM_LB + 64;
+static_assert(SM_LB % 4 == 0, "leaf buffers must allow 16-byte loads");
 
 __global__ void __launch_bounds__(1024) diag_sum_kernel(const float* __restrict__ H, int n,
                                                         double* out) {
@@ -86,15 +88,19 @@ __global__ void reverse_damp_kernel(const float* __restrict__ H, int n, int np,
 // One warp factors the 32 x 32 diagonal block at offset o of D (lower part
 // valid, already updated) and inverts the factor: on return D holds L_oo,
 // X holds Y_oo = L_oo^-1 and YT its transpose.  Lane i keeps row i of the
-// block and row i of the accumulating inverse in registers; pivot step j
-// needs no barrier, the pivot, the column L[:, j] and the finished row j of
-// the inverse travel by shuffles:
+// block and row i of the accumulating inverse in registers; pivot step j:
 //   L[i][j] = a_i[j] r,  r = 1 / sqrt(a_j[j]),   a_i[c] -= L[i][j] L[c][j]  (c > j)
 //   Y[j][:] = y_j[:] r,  y_i[:] -= L[i][j] Y[j][:]                          (i > j)
+// The pivot travels by one shuffle; the column L[:, j] and the finished row
+// Y[j][:] are broadcast through shared memory (lb: 2 x 32 floats), read by
+// every lane with 16-byte loads, which keeps the chain from one pivot to the
+// next short.  The arithmetic (and its order) is that of the plain update.
 __device__ __forceinline__ void warp_leaf32(float* D, float* X, float* YT, int o, int kb,
-                                            int* bad) {
+                                            int* bad, float* lb) {
   const int i = threadIdx.x & 31;
   constexpr unsigned FULL = 0xffffffffu;
+  float* colb = lb;         // L[:, j] of the current pivot
+  float* rowb = lb + 32;    // Y[j][:] of the current pivot
   float a[32], y[32];
 #pragma unroll
   for (int c = 0; c < 32; ++c) {
@@ -111,14 +117,22 @@ __device__ __forceinline__ void warp_leaf32(float* D, float* X, float* YT, int o
     const float r = rsqrtf(d);
     const float l = (i >= j) ? a[j] * r : 0.f;
     a[j] = l;
-    // the next pivot's column first: it is on the critical path
+    colb[i] = l;
+    if (i == j) {
 #pragma unroll
-    for (int c = j + 1; c < 32; ++c) a[c] = fmaf(-l, __shfl_sync(FULL, l, c), a[c]);
-#pragma unroll
-    for (int c = 0; c <= j; ++c) {
-      const float yj = __shfl_sync(FULL, y[c], j) * r;
-      y[c] = (i == j) ? yj : fmaf(-l, yj, y[c]);
+      for (int c = 0; c <= j; ++c) {
+        y[c] = y[c] * r;
+        rowb[c] = y[c];
+      }
     }
+    __syncwarp();
+#pragma unroll
+    for (int c = j + 1; c < 32; ++c) a[c] = fmaf(-l, colb[c], a[c]);
+    if (i != j) {
+#pragma unroll
+      for (int c = 0; c <= j; ++c) y[c] = fmaf(-l, rowb[c], y[c]);
+    }
+    __syncwarp();
   }
 #pragma unroll
   for (int c = 0; c < 32; ++c) {
@@ -147,11 +161,12 @@ __device__ __forceinline__ void warp_leaf32(float* D, float* X, float* YT, int o
 // memory whose wide operands are read as contiguous rows (YT, As, rows of X).
 constexpr int PANEL_THREADS = 256;
 
-__device__ void factor_and_invert(float* D, float* X, float* As, float* YT, int kb, int* bad) {
+__device__ void factor_and_invert(float* D, float* X, float* As, float* YT, float* LB, int kb,
+                                  int* bad) {
   const int tid = threadIdx.x;
   for (int e = tid; e < NB * LDX; e += blockDim.x) X[e] = 0.f;
   __syncthreads();
-  if (tid < 32) warp_leaf32(D, X, YT, 0, kb, bad);
+  if (tid < 32) warp_leaf32(D, X, YT, 0, kb, bad, LB);
   __syncthreads();
   for (int b = 0; b < NB / 32; ++b) {
     const int o = 32 * b;
@@ -238,7 +253,7 @@ __device__ void factor_and_invert(float* D, float* X, float* As, float* YT, int 
     __syncthreads();
     // ---- step 3b on warps 1.., the next diagonal block on warp 0
     if (tid < 32) {
-      warp_leaf32(D, X, YT, o2, kb, bad);
+      warp_leaf32(D, X, YT, o2, kb, bad, LB);
     } else {
       // item = 4 rows x 8 columns; 12 column groups: 8 g < o2 (Acc), else past the next block
       const int items = (R1 / 4) * 12;
@@ -318,6 +333,7 @@ __global__ void __launch_bounds__(PANEL_THREADS, 1) panel_kernel(const float* R,
   float* P = sm + SM_P;
   float* As = sm + SM_AS;
   float* YT = sm + SM_YT;
+  float* LB = sm + SM_LB;
   __shared__ int bad;
   __shared__ int abort_flag;
   __shared__ __align__(8) uint64_t pbar;
@@ -343,7 +359,7 @@ __global__ void __launch_bounds__(PANEL_THREADS, 1) panel_kernel(const float* R,
     D[i * LDD + c] = (c <= i) ? R[(int64_t)(k + i) * np + (k + c)] : 0.f;
   }
   __syncthreads();
-  factor_and_invert(D, X, As, YT, NB, &bad);
+  factor_and_invert(D, X, As, YT, LB, NB, &bad);
   if (blockIdx.x == 0 && tid == 0 && bad) kq::record_error(info, KRONQ_ERR_NOT_PD);
 
   if (!has_tile) {

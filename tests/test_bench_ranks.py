@@ -1,0 +1,55 @@
+"""The host side of bench.py --gpus N (one process per GPU, replicas): two
+gloo ranks on the CPU check that the job time is the slowest rank's on every
+rank, that the throughput counts every rank's layer, and that the ranks draw
+different layers (weak scaling, no data-path collective)."""
+
+import os
+import socket
+import sys
+
+import numpy as np
+import pytest
+import torch.multiprocessing as mp
+
+from conftest import ROOT
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank(rank, world, port, out):
+    import torch.distributed as dist
+    sys.path.insert(0, str(ROOT))
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    import bench
+    import synth
+    ms = bench.reduce_max_ms([5.0, 7.5][rank], world, "cpu")
+    cfg = bench.rank_config(synth.get_config("toy-256"), rank)
+    w = synth.make_w(cfg, cfg.sublayers[0])
+    out.put((rank, ms, bench.job_throughput(cfg.weights, world, 4, ms), float(w[0, 0]), cfg.seed))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_reduce_max_and_draw_distinct_layers():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    (r0, ms0, v0, w0, s0), (r1, ms1, v1, w1, s1) = res
+    assert ms0 == ms1 == 7.5                       # the slowest rank's time on both
+    assert v0 == v1 == pytest.approx(65536 * 2 * 4 / 7.5e-3 / 1e6)
+    assert s1 == s0 + 1 and w0 != w1                # different seeds, different layers
