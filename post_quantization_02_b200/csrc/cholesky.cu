@@ -354,9 +354,29 @@ __global__ void __launch_bounds__(PANEL_THREADS, 1) panel_kernel(const float* R,
     kq::mbar_arrive_expect_tx(&pbar, PR * NB * 4);
     for (int r = 0; r < PR; ++r) bulk_copy_row(P + r * LDX, src + (int64_t)r * np, NB * 4, &pbar);
   }
-  for (int e = tid; e < NB * NB; e += blockDim.x) {
-    const int i = e / NB, c = e % NB;
-    D[i * LDD + c] = (c <= i) ? R[(int64_t)(k + i) * np + (k + c)] : 0.f;
+  // the diagonal block, lower triangle: 16-byte loads, a half of them
+  // requested before any is stored (one CTA per SM leaves few warps to hide
+  // the latency of one load at a time)
+  static_assert(NB * NB / 4 == 16 * PANEL_THREADS, "diagonal block load assumes 256 threads");
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    float4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int e4 = tid + PANEL_THREADS * (8 * h + u);
+      const int i = e4 >> 5, c = (e4 & 31) * 4;
+      v[u] = *reinterpret_cast<const float4*>(R + (int64_t)(k + i) * np + k + c);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int e4 = tid + PANEL_THREADS * (8 * h + u);
+      const int i = e4 >> 5, c = (e4 & 31) * 4;
+      float* d = D + i * LDD + c;
+      d[0] = (c <= i) ? v[u].x : 0.f;
+      d[1] = (c + 1 <= i) ? v[u].y : 0.f;
+      d[2] = (c + 2 <= i) ? v[u].z : 0.f;
+      d[3] = (c + 3 <= i) ? v[u].w : 0.f;
+    }
   }
   __syncthreads();
   factor_and_invert(D, X, As, YT, LB, NB, &bad);
