@@ -40,7 +40,8 @@ constexpr int SM_P = SM_X + NB * LDX;
 constexpr int SM_AS = SM_P + 32 * LDX;
 constexpr int SM_YT = SM_AS + 32 * LDA;
 constexpr int SM_LB = SM_YT + 32 * LDY;       // the leaf's broadcast buffers (2 x 32)
-constexpr int SM_FLOATS = SM_LB + 64;
+constexpr int SM_P2 = SM_LB + 64;             // second slice buffer (double buffering)
+constexpr int SM_FLOATS = SM_P2 + 32 * LDX;
 static_assert(SM_LB % 4 == 0, "leaf buffers must allow 16-byte loads");
 
 __global__ void __launch_bounds__(1024) diag_sum_kernel(const float* __restrict__ H, int n,
@@ -314,46 +315,52 @@ KQ_DEV void put_split(float* hi_plane, float* lo_plane, int64_t idx, float v) {
 }
 
 // Panel step p (rows / columns k = 128 p ...) of the padded np x np matrices,
-// in 32-row slices (PR rows per CTA):
-//   CTA b < tiles_L:        L_ip = R_ip L_pp^-T for rows k+128+32b ..
-//                           -> the hi / lo planes Lh, Ll (np x 128, row 0 = row k+128)
-//   CTA tiles_L + j, j < 4p: Z_jp = B_jp L_pp^-T for Z rows 32j .. -> Z and the
-//                           planes Zh, Zl (row = Z row)
-//   CTA tiles_L + 4p:       Z_pp = L_pp^-T      -> Z and the planes
-// Every CTA first factors and inverts the diagonal block in shared memory;
-// the 32 x 128 slice it multiplies is fetched by bulk copies meanwhile.
+// in 32-row slices ("tiles", PR rows each):
+//   tile t < tiles_L:          L_ip = R_ip L_pp^-T for rows k+128+32t ..
+//                              -> the hi / lo planes Lh, Ll (np x 128, row 0 = row k+128)
+//   tile tiles_L + j, j < 4p:  Z_jp = B_jp L_pp^-T for Z rows 32j .. -> Z and the
+//                              planes Zh, Zl (row = Z row)
+//   tile tiles_L + 4p (last):  Z_pp = L_pp^-T      -> Z and the planes
+// At most one CTA per SM: each factors and inverts the diagonal block once in
+// shared memory, then takes tiles t = blockIdx.x, + gridDim.x, ... (the
+// first slice is fetched by bulk copies during the factorisation, each
+// following one while the previous is multiplied: two slice buffers).
 constexpr int PR = 32;
 
 __global__ void __launch_bounds__(PANEL_THREADS, 1) panel_kernel(const float* R, float* Z, float* Lh,
                                                     float* Ll, float* Zh, float* Zl, int np, int k,
-                                                    int p, int tiles_L, int32_t* info) {
+                                                    int p, int tiles_L, int tiles_total,
+                                                    int32_t* info) {
   extern __shared__ __align__(16) float sm[];
   float* D = sm + SM_D;
   float* X = sm + SM_X;
-  float* P = sm + SM_P;
   float* As = sm + SM_AS;
   float* YT = sm + SM_YT;
   float* LB = sm + SM_LB;
+  float* Pbuf[2] = {sm + SM_P, sm + SM_P2};
   __shared__ int bad;
   __shared__ int abort_flag;
-  __shared__ __align__(8) uint64_t pbar;
+  __shared__ __align__(8) uint64_t pbar[2];
   const int tid = threadIdx.x;
-  const int role_L = (int)blockIdx.x < tiles_L;
-  const int j = (int)blockIdx.x - tiles_L;
-  const bool has_tile = role_L || j < 4 * p;
-  const float* src = role_L ? R + (int64_t)(k + NB + PR * blockIdx.x) * np + k
-                            : Z + (int64_t)(PR * (j < 4 * p ? j : 0)) * np + k;
+  const int z_pp = tiles_L + 4 * p;   // the tile without a slice to fetch (the last one)
+  auto slice_src = [&](int t) -> const float* {
+    return t < tiles_L ? R + (int64_t)(k + NB + PR * t) * np + k
+                       : Z + (int64_t)(PR * (t - tiles_L)) * np + k;
+  };
+  auto fetch = [&](int t, int b) {
+    const float* src = slice_src(t);
+    kq::mbar_arrive_expect_tx(&pbar[b], PR * NB * 4);
+    for (int r = 0; r < PR; ++r) bulk_copy_row(Pbuf[b] + r * LDX, src + (int64_t)r * np, NB * 4, &pbar[b]);
+  };
   if (tid == 0) {
     bad = 0;
     abort_flag = 0;
-    kq::mbar_init(&pbar, 1);
+    kq::mbar_init(&pbar[0], 1);
+    kq::mbar_init(&pbar[1], 1);
     kq::fence_barrier_init();
   }
   __syncthreads();
-  if (tid == 0 && has_tile) {
-    kq::mbar_arrive_expect_tx(&pbar, PR * NB * 4);
-    for (int r = 0; r < PR; ++r) bulk_copy_row(P + r * LDX, src + (int64_t)r * np, NB * 4, &pbar);
-  }
+  if (tid == 0 && (int)blockIdx.x < z_pp) fetch(blockIdx.x, 0);
   // the diagonal block, lower triangle: 16-byte loads, a half of them
   // requested before any is stored (one CTA per SM leaves few warps to hide
   // the latency of one load at a time)
@@ -382,64 +389,77 @@ __global__ void __launch_bounds__(PANEL_THREADS, 1) panel_kernel(const float* R,
   factor_and_invert(D, X, As, YT, LB, NB, &bad);
   if (blockIdx.x == 0 && tid == 0 && bad) kq::record_error(info, KRONQ_ERR_NOT_PD);
 
-  if (!has_tile) {
-    // Z_pp = X^T (upper; X is zero above its diagonal)
-    for (int e = tid; e < NB * NB; e += blockDim.x) {
-      const int a = e / NB, c = e % NB;
-      const float v = X[c * LDX + a];
-      Z[(int64_t)(k + a) * np + k + c] = v;
-      put_split(Zh, Zl, (int64_t)(k + a) * NB + c, v);
-    }
-    return;
-  }
-  if (!kq::mbar_wait(&pbar, 0, &abort_flag, info)) {
-    // give the copies in flight a bounded time to land before the CTA exits
-    kq::tf32x3::drain_wait(&pbar, 0, info);
-    return;
-  }
-  // C = P X^T (32 x 128): thread (ty, tx) owns rows ty, ty + 16 and columns tx + 16 jj
   const int ty = tid >> 4, tx = tid & 15;
-  float acc[2][8];
-#pragma unroll
-  for (int i = 0; i < 2; ++i)
-#pragma unroll
-    for (int jj = 0; jj < 8; ++jj) acc[i][jj] = 0.f;
-#pragma unroll 4
-  for (int kk = 0; kk < NB; kk += 4) {
-    float4 pa[2], xb[8];
-#pragma unroll
-    for (int i = 0; i < 2; ++i) pa[i] = *reinterpret_cast<const float4*>(&P[(ty + 16 * i) * LDX + kk]);
-#pragma unroll
-    for (int jj = 0; jj < 8; ++jj)
-      xb[jj] = *reinterpret_cast<const float4*>(&X[(tx + 16 * jj) * LDX + kk]);
+  int n_it = 0;
+  for (int t = blockIdx.x; t < tiles_total; t += gridDim.x, ++n_it) {
+    const int b = n_it & 1;
+    const uint32_t ph = (uint32_t)(n_it >> 1) & 1u;
+    const int tn = t + gridDim.x;
+    // the next slice into the other buffer (its last reader finished at the
+    // barrier that ended the previous iteration)
+    if (tid == 0 && tn < z_pp) fetch(tn, b ^ 1);
+    if (t == z_pp) {
+      // Z_pp = X^T (upper; X is zero above its diagonal)
+      for (int e = tid; e < NB * NB; e += blockDim.x) {
+        const int a = e / NB, c = e % NB;
+        const float v = X[c * LDX + a];
+        Z[(int64_t)(k + a) * np + k + c] = v;
+        put_split(Zh, Zl, (int64_t)(k + a) * NB + c, v);
+      }
+      break;                          // the last tile
+    }
+    if (!kq::mbar_wait(&pbar[b], ph, &abort_flag, info)) {
+      // give the copies in flight a bounded time to land before the CTA exits
+      kq::tf32x3::drain_wait(&pbar[b], ph, info);
+      if (tn < z_pp) kq::tf32x3::drain_wait(&pbar[b ^ 1], (uint32_t)((n_it + 1) >> 1) & 1u, info);
+      return;
+    }
+    const float* P = Pbuf[b];
+    // C = P X^T (32 x 128): thread (ty, tx) owns rows ty, ty + 16 and columns tx + 16 jj
+    float acc[2][8];
 #pragma unroll
     for (int i = 0; i < 2; ++i)
 #pragma unroll
-      for (int jj = 0; jj < 8; ++jj) {
-        acc[i][jj] = fmaf(pa[i].x, xb[jj].x, acc[i][jj]);
-        acc[i][jj] = fmaf(pa[i].y, xb[jj].y, acc[i][jj]);
-        acc[i][jj] = fmaf(pa[i].z, xb[jj].z, acc[i][jj]);
-        acc[i][jj] = fmaf(pa[i].w, xb[jj].w, acc[i][jj]);
-      }
-  }
-  if (role_L) {
+      for (int jj = 0; jj < 8; ++jj) acc[i][jj] = 0.f;
+#pragma unroll 4
+    for (int kk = 0; kk < NB; kk += 4) {
+      float4 pa[2], xb[8];
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int64_t r = (int64_t)PR * blockIdx.x + ty + 16 * i;   // plane row
+      for (int i = 0; i < 2; ++i) pa[i] = *reinterpret_cast<const float4*>(&P[(ty + 16 * i) * LDX + kk]);
 #pragma unroll
-      for (int jj = 0; jj < 8; ++jj) put_split(Lh, Ll, r * NB + tx + 16 * jj, acc[i][jj]);
+      for (int jj = 0; jj < 8; ++jj)
+        xb[jj] = *reinterpret_cast<const float4*>(&X[(tx + 16 * jj) * LDX + kk]);
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          acc[i][jj] = fmaf(pa[i].x, xb[jj].x, acc[i][jj]);
+          acc[i][jj] = fmaf(pa[i].y, xb[jj].y, acc[i][jj]);
+          acc[i][jj] = fmaf(pa[i].z, xb[jj].z, acc[i][jj]);
+          acc[i][jj] = fmaf(pa[i].w, xb[jj].w, acc[i][jj]);
+        }
     }
-  } else {
+    if (t < tiles_L) {
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int64_t r = (int64_t)PR * j + ty + 16 * i;
+      for (int i = 0; i < 2; ++i) {
+        const int64_t r = (int64_t)PR * t + ty + 16 * i;   // plane row
 #pragma unroll
-      for (int jj = 0; jj < 8; ++jj) {
-        const int c = tx + 16 * jj;
-        Z[r * np + k + c] = acc[i][jj];
-        put_split(Zh, Zl, r * NB + c, acc[i][jj]);
+        for (int jj = 0; jj < 8; ++jj) put_split(Lh, Ll, r * NB + tx + 16 * jj, acc[i][jj]);
+      }
+    } else {
+      const int j = t - tiles_L;
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int64_t r = (int64_t)PR * j + ty + 16 * i;
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          const int c = tx + 16 * jj;
+          Z[r * np + k + c] = acc[i][jj];
+          put_split(Zh, Zl, r * NB + c, acc[i][jj]);
+        }
       }
     }
+    __syncthreads();                  // P[b] is read; it may be refilled two tiles on
   }
 }
 
@@ -518,8 +538,10 @@ int kq_cholesky_inv(const float* H, int64_t n64, float damp_rel, float* U, int32
     const int k = p * NB;
     const int rest = np - k - NB;
     const int tiles_L = rest / PR;
-    panel_kernel<<<tiles_L + 4 * p + 1, PANEL_THREADS, kPanelSmem, st>>>(R, Z, Lh, Ll, Zh, Zl, np, k, p,
-                                                               tiles_L, info);
+    const int tiles_total = tiles_L + 4 * p + 1;
+    const int grid = tiles_total < sms ? tiles_total : sms;
+    panel_kernel<<<grid, PANEL_THREADS, kPanelSmem, st>>>(R, Z, Lh, Ll, Zh, Zl, np, k, p, tiles_L,
+                                                          tiles_total, info);
     KQ_CHECK_LAUNCH();
     if (rest > 0) {
       // trailing update on the tensor cores, B = the panel rows L_ip (planes):
