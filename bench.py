@@ -345,32 +345,61 @@ class Layer:
             self.codes_p = torch.empty((m, n), dtype=torch.uint8, device=dev)
 
 
-def solve_layer(cfg, L, ws, stream, act_order=False, clip=False):
+class StageMarks:
+    """CUDA events at stage boundaries of one step; each mark closes the
+    stage named by it (the time since the previous mark)."""
+
+    def __init__(self, stream):
+        self.stream = stream
+        self.events = []
+
+    def mark(self, name):
+        import torch
+        e = torch.cuda.Event(enable_timing=True)
+        e.record(self.stream)
+        self.events.append((name, e))
+
+    def totals(self):
+        out = {}
+        for (_, e0), (name, e1) in zip(self.events, self.events[1:]):
+            out[name] = out.get(name, 0.0) + e0.elapsed_time(e1)
+        return out
+
+
+def solve_layer(cfg, L, ws, stream, act_order=False, clip=False, mark=None):
     """Damped inverse Cholesky and the column loop of one sublayer, with the
     README's --act_order (column order by the H_X' diagonal, results back in
     the original order) and --w_clip (clip-ratio search) when asked for."""
     from post_quantization_02_b200 import abi
     opts = abi.QUANT_CLIP if clip else 0
+    mark = mark or (lambda name: None)
     if not act_order:
         abi.kronq_cholesky_inv(L.HX, cfg.damp, L.U, L.info, ws, stream=stream)
+        mark("inverse_cholesky")
         abi.kronq_quantize_layer_opt(L.W, L.U, L.bits, L.sub.group, cfg.block, opts, L.codes,
                                      L.scales, L.zeros, None, L.info, ws, stream=stream)
+        mark("solver")
         return
     abi.kronq_act_order(L.HX, L.perm, stream=stream)
     abi.kronq_permute(L.HX, L.Hp, L.perm, abi.PERM_SYM, L.info, stream=stream)
     abi.kronq_permute(L.W, L.Wp, L.perm, abi.PERM_COLS, L.info, stream=stream)
     abi.kronq_cholesky_inv(L.Hp, cfg.damp, L.U, L.info, ws, stream=stream)
+    mark("inverse_cholesky")
     abi.kronq_quantize_layer_opt(L.Wp, L.U, L.bits, L.sub.group, cfg.block, opts, L.codes_p,
                                  L.scales, L.zeros, None, L.info, ws, stream=stream)
     abi.kronq_permute(L.codes_p, L.codes, L.perm, abi.UNPERM_COLS, L.info, stream=stream)
+    mark("solver")
 
 
-def gpu_step(cfg, layers, X, ws, stream, cov_events=None, act_order=False, clip=False):
+def gpu_step(cfg, layers, X, ws, stream, cov_events=None, act_order=False, clip=False,
+             marks=None):
     """One pass of the whole path over every sublayer of the config."""
     import torch
     from post_quantization_02_b200 import abi, alloc
     N = cfg.tokens
     ev = iter(cov_events) if cov_events is not None else None
+    mark = marks.mark if marks is not None else (lambda name: None)
+    mark("start")
 
     def cov(A, H):
         if ev is not None:
@@ -391,6 +420,7 @@ def gpu_step(cfg, layers, X, ws, stream, cov_events=None, act_order=False, clip=
             L.HX.copy_(hx_site[L.sub.site])
     for L in layers:
         L.W.copy_(L.W0)
+    mark("covariance")
     # H_X of a shared site is rotated per sublayer: rotate copies, the site's own last
     for L in layers:
         abi.kronq_biip_rotate(L.W, L.HX, L.HG, L.su, L.sv, cfg.alpha, cfg.mode, 0, L.SX, L.SG, ws,
@@ -401,12 +431,14 @@ def gpu_step(cfg, layers, X, ws, stream, cov_events=None, act_order=False, clip=
         bits = alloc.allocate_bits(scores, [L.sub.m * L.sub.n for L in layers], cfg.mixed_avg_bits)
         for L, b in zip(layers, bits):
             L.bits = b
+    mark("biip_sensitivity")
     for L in layers:
-        solve_layer(cfg, L, ws, stream, act_order, clip)
+        solve_layer(cfg, L, ws, stream, act_order, clip, mark)
         if L.bits in (2, 4):
             pk = L.packed[:, : abi.packed_words(L.sub.n, L.bits)]
             abi.kronq_pack(L.codes, L.bits, pk.contiguous() if not pk.is_contiguous() else pk,
                            stream=stream)
+        mark("pack")
 
 
 def run_deploy(args):
@@ -550,6 +582,7 @@ def main():
     sampler.start()
     time.sleep(0.3)
     cov_events = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * ncov)] for _ in range(args.steps)]
+    stage_marks = [StageMarks(stream) for _ in range(args.steps)]
     launches0 = abi.kronq_launch_count()
     if world > 1:
         dist.barrier()
@@ -557,7 +590,8 @@ def main():
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record(stream)
     for k in range(args.steps):
-        gpu_step(cfg, layers, X, ws, stream, cov_events[k], args.act_order, args.w_clip)
+        gpu_step(cfg, layers, X, ws, stream, cov_events[k], args.act_order, args.w_clip,
+                 stage_marks[k])
     end.record(stream)
     torch.cuda.synchronize()
     if world > 1:
@@ -565,6 +599,10 @@ def main():
     launches = abi.kronq_launch_count() - launches0
     ms = reduce_max_ms(start.elapsed_time(end), world, dev)
     cov_ms = [ev[2 * i].elapsed_time(ev[2 * i + 1]) for ev in cov_events for i in range(ncov)]
+    stages = {}
+    for sm_ in stage_marks:
+        for name, t in sm_.totals().items():
+            stages[name] = stages.get(name, 0.0) + t / args.steps
 
     # ---- end to end through the public API with pinned host buffers
     e2e = None
@@ -675,6 +713,7 @@ def main():
                        "act_order": args.act_order, "w_clip": args.w_clip},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
             "clocks": clocks,
+            "stages_ms": {k: round(v, 4) for k, v in stages.items()},
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -53,3 +53,22 @@ def test_two_gloo_ranks_reduce_max_and_draw_distinct_layers():
     assert ms0 == ms1 == 7.5                       # the slowest rank's time on both
     assert v0 == v1 == pytest.approx(65536 * 2 * 4 / 7.5e-3 / 1e6)
     assert s1 == s0 + 1 and w0 != w1                # different seeds, different layers
+
+
+def test_stage_marks_attribute_each_interval_to_the_stage_it_closes():
+    sys.path.insert(0, str(ROOT))
+    import bench
+
+    class Ev:
+        def __init__(self, t):
+            self.t = t
+
+        def elapsed_time(self, other):
+            return other.t - self.t
+
+    m = bench.StageMarks(stream=None)
+    m.events = [("start", Ev(0.0)), ("covariance", Ev(7.0)), ("biip_sensitivity", Ev(7.5)),
+                ("inverse_cholesky", Ev(10.0)), ("solver", Ev(11.25)), ("pack", Ev(11.5)),
+                ("inverse_cholesky", Ev(12.0)), ("solver", Ev(12.5)), ("pack", Ev(12.75))]
+    assert m.totals() == {"covariance": 7.0, "biip_sensitivity": 0.5, "inverse_cholesky": 3.0,
+                          "solver": 1.75, "pack": 0.5}
