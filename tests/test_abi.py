@@ -116,6 +116,23 @@ def test_host_side_argument_errors_act_order_clip(L):
     assert L.kronq_permute(null, null, 0, 8, 4, null, 0, null, null) == 0
 
 
+def test_host_side_argument_errors_deploy(L):
+    null = None
+    ptr = ctypes.c_void_p(256)  # never dereferenced: rejected before any launch
+    args = lambda m, n, bits, group, mode, batch, ws_bytes: (
+        ptr, m, n, bits, group, ptr, ptr, ptr, ptr, ptr, ptr, mode, ptr, batch, ptr, ptr, ws_bytes, null)
+    assert L.kronq_deploy_matvec(null, 64, 128, 4, -1, ptr, ptr, ptr, ptr, ptr, ptr, 0, ptr, 1, ptr,
+                                 ptr, 1 << 20, null) == -1          # null packed codes
+    assert L.kronq_deploy_matvec(*args(64, 128, 3, -1, 0, 1, 1 << 20)) == -2   # 3-bit is not packed
+    assert L.kronq_deploy_matvec(*args(64, 96, 4, -1, 0, 1, 1 << 20)) == -1    # n not a multiple of 64
+    assert L.kronq_deploy_matvec(*args(64, 128, 4, 48, 0, 1, 1 << 20)) == -2   # group 48
+    assert L.kronq_deploy_matvec(*args(64, 128, 4, -1, 5, 1, 1 << 20)) == -1   # unknown incoh mode
+    assert L.kronq_deploy_matvec(*args(64, 128, 4, -1, 0, 3, 1 << 20)) == -2   # batch 3
+    assert L.kronq_deploy_matvec(*args(64, 128, 4, -1, 0, 1, 0)) == -6         # workspace too small
+    assert L.kronq_deploy_workspace_size(64, 128, 1) > 64 * 128
+    assert L.kronq_deploy_workspace_size(0, 128, 1) == 0
+
+
 def test_binding_refuses_host_tensors():
     import torch
     from post_quantization_02_b200 import abi
