@@ -258,3 +258,33 @@ def test_row_losses_damping_argument_and_fp32_input():
     H32 = H.astype(np.float32)
     np.testing.assert_allclose(Q.row_losses(dW, H32), np.einsum("ij,jk,ik->i", dW, H32.astype(np.float64), dW),
                                rtol=1e-11)
+
+
+def test_ldlq_quarter_bound_table9():
+    """KronQ review (pith.science), reference-list fragment of the appendix,
+    Table 9 (worst-case proxy loss under LDLQ rounding, GPTQ-LDLQ with
+    H_G = I): with rounding errors of at most half a grid step, a row's loss
+    under the column loop is at most 1/4 step^2 tr(D_X), D_X the diagonal of
+    the LDL factorisation of H in the loop's order.  D_X is taken here from a
+    Cholesky factor of the index-reversed H (not from the oracle's factor):
+    it must equal 1 / U[j, j]^2, and the loop's loss sum_j e_j^2 must respect
+    the bound on every row whose rounding errors stayed within half a step
+    (a value pushed past the grid's end is clamped and may err by more)."""
+    r = np.random.default_rng(41)
+    m, n, bits = 24, 64, 8
+    W = r.standard_normal((m, n))
+    Hd = C.damp(_spd(r, n, cond=200.0), 0.01)
+    U = C.inverse_cholesky(Hd)
+    Lr = np.linalg.cholesky(Hd[::-1, ::-1])
+    D = (np.diag(Lr) ** 2)[::-1]
+    np.testing.assert_allclose(1.0 / np.diag(U) ** 2, D, rtol=1e-9)
+    res = Q.obs_quantize(W, U, bits)
+    checked = 0
+    for i in range(m):
+        step = float(res["scale"][i, 0])
+        rerr = res["E"][i] * np.diag(U)              # w_j - w_hat_j at quantization time
+        if np.max(np.abs(rerr)) > 0.5 * step * (1 + 1e-6):
+            continue
+        assert np.sum(res["E"][i] ** 2) <= 0.25 * step ** 2 * np.sum(D) * (1 + 1e-9)
+        checked += 1
+    assert checked >= m // 2, checked
