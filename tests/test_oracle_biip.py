@@ -88,6 +88,21 @@ def test_alpha_quarter_equalisation():
     np.testing.assert_array_equal(W0, W)
 
 
+def test_alpha_half_exchanges_diagonal_and_norms():
+    """KronQ README (GitHub), "Mapping paper results to flags": the
+    weight-and-activation setting uses --alpha 0.5.  At alpha = 1/2 the input
+    rescale S_X = (H_jj / ||W_j||^2)^(1/2) exchanges the two: the rescaled
+    diagonal H_jj / S_j^2 is the old squared column norm and the rescaled
+    squared column norm ||W_j||^2 S_j^2 is the old diagonal (closed form)."""
+    r = np.random.default_rng(19)
+    m, n = 12, 24
+    W = r.standard_normal((m, n)) * np.exp(r.uniform(-2, 2, n))[None, :]
+    HX, HG = _spd(r, n), _spd(r, m)
+    W1, HX1, _, SX, _ = biip.rescale(W, HX, HG, 0.5, "sv_only")
+    np.testing.assert_allclose(np.diag(HX1), (W ** 2).sum(0), rtol=1e-12)
+    np.testing.assert_allclose((W1 ** 2).sum(0), np.diag(HX), rtol=1e-12)
+
+
 def test_modes_touch_only_their_side():
     r = np.random.default_rng(10)
     m, n = 8, 16
