@@ -714,7 +714,7 @@ def main():
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
             "clocks": clocks,
             "stages_ms": {k: round(v, 4) for k, v in stages.items()},
-            # the solver given H_X' (SURVEY's "solver-only" figure): inverse Cholesky + OBS loop
+            # the solver alone, given H_X': inverse Cholesky + OBS loop
             "solver_only_mweights_s": (
                 weights / ((stages.get("inverse_cholesky", 0.0) + stages.get("solver", 0.0)) / 1e3) / 1e6
                 if stages.get("inverse_cholesky", 0.0) + stages.get("solver", 0.0) > 0 else None),

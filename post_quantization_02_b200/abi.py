@@ -89,17 +89,69 @@ def _check(fn: str, code: int):
 def _dev(t, dtype, name, ndim=None):
     if t is None:
         return
-    if not t.is_cuda:
-        raise ValueError(f"{name} must be a CUDA tensor")
+    if not isinstance(t, torch.Tensor):
+        raise ValueError(f"{name} must be a torch tensor")
     if dtype is not None and t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
     if ndim is not None and t.dim() != ndim:
         raise ValueError(f"{name} must have {ndim} dims")
 
 
+def _shape(t, shape, name):
+    """t must have exactly this shape (None: no tensor given, nothing to check)."""
+    if t is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _numel(t, count, name):
+    if t is not None and t.numel() != count:
+        raise ValueError(f"{name} has {t.numel()} elements, expected {count}")
+
+
+def _on_current_device(*named):
+    """Every tensor lives on the current CUDA device: the kernels launch there
+    (and per-device library state is looked up there)."""
+    tensors = [(t, nm) for t, nm in named if t is not None]
+    for t, nm in tensors:
+        if not t.is_cuda:
+            raise ValueError(f"{nm} must be a CUDA tensor")
+    if tensors:
+        cur = torch.cuda.current_device()
+        for t, nm in tensors:
+            if t.device.index != cur:
+                raise ValueError(f"{nm} is on cuda:{t.device.index}, the current device is cuda:{cur}")
+
+
 def _contig(t, name):
     if t is not None and not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+
+
+def _groups(n: int, group: int) -> int:
+    return 1 if group == -1 or group <= 0 else max(1, n // group)
+
+
+def _quant_args(W, U, codes, scales, zeros, W_hat, group):
+    """Types, shapes and placement of the solver's tensors for an m x n layer."""
+    _dev(W, torch.float32, "W", 2)
+    _dev(U, torch.float32, "U_c", 2)
+    _dev(codes, torch.uint8, "codes", 2)
+    _dev(scales, torch.float32, "scales")
+    _dev(zeros, torch.uint8, "zeros")
+    _dev(W_hat, torch.float32, "W_hat", 2)
+    m, n = W.shape
+    G = _groups(n, group)
+    _shape(U, (n, n), "U_c")
+    _shape(codes, (m, n), "codes")
+    _numel(scales, m * G, "scales")
+    _numel(zeros, m * G, "zeros")
+    _shape(W_hat, (m, n), "W_hat")
+    named = ((W, "W"), (U, "U_c"), (codes, "codes"), (scales, "scales"), (zeros, "zeros"),
+             (W_hat, "W_hat"))
+    _on_current_device(*named)
+    for t, nm in named:
+        _contig(t, nm)
+    return m, n
 
 
 def kronq_status_string(code: int) -> str:
@@ -129,11 +181,12 @@ def kronq_covariance(A, H, alpha: float, beta: float = 0.0, info=None, stream=No
     stride); H: (d, d) fp32 with unit column stride."""
     _dev(A, (torch.bfloat16, torch.int16, torch.uint16), "A", 2)
     _dev(H, torch.float32, "H", 2)
+    _dev(info, torch.int32, "info")
+    N, d = A.shape
+    _shape(H, (d, d), "H")
+    _on_current_device((A, "A"), (H, "H"), (info, "info"))
     if A.stride(1) != 1 or H.stride(1) != 1:
         raise ValueError("A and H need unit stride along their last dimension")
-    N, d = A.shape
-    if H.shape != (d, d):
-        raise ValueError("H must be d x d")
     _check("kronq_covariance", lib().kronq_covariance(
         _p(A), N, d, A.stride(0) if N > 0 else d, _p(H), H.stride(0), alpha, beta, _p(info), _s(stream)))
 
@@ -143,6 +196,11 @@ def kronq_sensitivity(HX, HG, out, stream=None):
     _dev(HX, torch.float32, "H_X", 2)
     _dev(HG, torch.float32, "H_G", 2)
     _dev(out, torch.float64, "out")
+    _shape(HX, (HX.shape[0], HX.shape[0]), "H_X")
+    _shape(HG, (HG.shape[0], HG.shape[0]), "H_G")
+    if out.numel() < 3:
+        raise ValueError("out needs 3 fp64 elements")
+    _on_current_device((HX, "H_X"), (HG, "H_G"), (out, "out"))
     _contig(HX, "H_X"); _contig(HG, "H_G")
     _check("kronq_sensitivity", lib().kronq_sensitivity(
         _p(HX), HX.shape[0], _p(HG), HG.shape[0], _p(out), _s(stream)))
@@ -157,36 +215,46 @@ def kronq_biip_rotate(W, HX, HG, sign_u, sign_v, alpha: float, mode, inverse: in
     _dev(sign_v, torch.int8, "sign_v")
     _dev(SX, torch.float32, "S_X")
     _dev(SG, torch.float32, "S_G")
-    for t, nm in ((W, "W"), (HX, "H_X"), (HG, "H_G"), (ws, "ws")):
-        _contig(t, nm)
+    _dev(ws, None, "ws")
     m, n = W.shape
+    _shape(HX, (n, n), "H_X")
+    _shape(HG, (m, m), "H_G")
+    _numel(sign_u, m, "sign_u")
+    _numel(sign_v, n, "sign_v")
+    _numel(SX, n, "S_X")
+    _numel(SG, m, "S_G")
+    named = ((W, "W"), (HX, "H_X"), (HG, "H_G"), (sign_u, "sign_u"), (sign_v, "sign_v"),
+             (SX, "S_X"), (SG, "S_G"), (ws, "ws"))
+    _on_current_device(*named)
+    for t, nm in named:
+        _contig(t, nm)
     mode = MODES[mode] if isinstance(mode, str) else int(mode)
     _check("kronq_biip_rotate", lib().kronq_biip_rotate(
         _p(W), m, n, _p(HX), _p(HG), _p(sign_u), _p(sign_v), alpha, mode, int(inverse),
-        _p(SX), _p(SG), _p(ws), ws.numel() * ws.element_size(), _s(stream)))
+        _p(SX), _p(SG), _p(ws), 0 if ws is None else ws.numel() * ws.element_size(), _s(stream)))
 
 
 def kronq_cholesky_inv(H, damp_rel: float, U, info, ws, stream=None):
     _dev(H, torch.float32, "H", 2)
     _dev(U, torch.float32, "U_c", 2)
-    _contig(H, "H"); _contig(U, "U_c")
+    _dev(info, torch.int32, "info")
+    _dev(ws, None, "ws")
+    n = H.shape[0]
+    _shape(H, (n, n), "H")
+    _shape(U, (n, n), "U_c")
+    _on_current_device((H, "H"), (U, "U_c"), (info, "info"), (ws, "ws"))
+    _contig(H, "H"); _contig(U, "U_c"); _contig(ws, "ws")
     _check("kronq_cholesky_inv", lib().kronq_cholesky_inv(
-        _p(H), H.shape[0], damp_rel, _p(U), _p(info), _p(ws), ws.numel() * ws.element_size(),
-        _s(stream)))
+        _p(H), n, damp_rel, _p(U), _p(info), _p(ws),
+        0 if ws is None else ws.numel() * ws.element_size(), _s(stream)))
 
 
 def kronq_quantize_layer(W, U, bits: int, group: int, block: int, codes, scales, zeros,
                          W_hat=None, info=None, ws=None, stream=None):
-    _dev(W, torch.float32, "W", 2)
-    _dev(U, torch.float32, "U_c", 2)
-    _dev(codes, torch.uint8, "codes", 2)
-    _dev(scales, torch.float32, "scales")
-    _dev(zeros, torch.uint8, "zeros")
-    _dev(W_hat, torch.float32, "W_hat", 2)
-    for t, nm in ((W, "W"), (U, "U_c"), (codes, "codes"), (scales, "scales"), (zeros, "zeros"),
-                  (W_hat, "W_hat")):
-        _contig(t, nm)
-    m, n = W.shape
+    m, n = _quant_args(W, U, codes, scales, zeros, W_hat, group)
+    _dev(info, torch.int32, "info")
+    _dev(ws, None, "ws")
+    _on_current_device((info, "info"), (ws, "ws"))
     _check("kronq_quantize_layer", lib().kronq_quantize_layer(
         _p(W), m, n, _p(U), bits, group, block, _p(codes), _p(scales), _p(zeros), _p(W_hat),
         _p(info), _p(ws), 0 if ws is None else ws.numel() * ws.element_size(), _s(stream)))
@@ -195,16 +263,10 @@ def kronq_quantize_layer(W, U, bits: int, group: int, block: int, codes, scales,
 def kronq_quantize_layer_opt(W, U, bits: int, group: int, block: int, options: int, codes, scales,
                              zeros, W_hat=None, info=None, ws=None, stream=None):
     """kronq_quantize_layer with option flags (QUANT_CLIP: the --w_clip search)."""
-    _dev(W, torch.float32, "W", 2)
-    _dev(U, torch.float32, "U_c", 2)
-    _dev(codes, torch.uint8, "codes", 2)
-    _dev(scales, torch.float32, "scales")
-    _dev(zeros, torch.uint8, "zeros")
-    _dev(W_hat, torch.float32, "W_hat", 2)
-    for t, nm in ((W, "W"), (U, "U_c"), (codes, "codes"), (scales, "scales"), (zeros, "zeros"),
-                  (W_hat, "W_hat")):
-        _contig(t, nm)
-    m, n = W.shape
+    m, n = _quant_args(W, U, codes, scales, zeros, W_hat, group)
+    _dev(info, torch.int32, "info")
+    _dev(ws, None, "ws")
+    _on_current_device((info, "info"), (ws, "ws"))
     _check("kronq_quantize_layer_opt", lib().kronq_quantize_layer_opt(
         _p(W), m, n, _p(U), bits, group, block, options, _p(codes), _p(scales), _p(zeros),
         _p(W_hat), _p(info), _p(ws), 0 if ws is None else ws.numel() * ws.element_size(),
@@ -215,8 +277,12 @@ def kronq_act_order(H, perm, stream=None):
     """perm (int32, n) = the --act_order column order from diag(H)."""
     _dev(H, torch.float32, "H", 2)
     _dev(perm, torch.int32, "perm", 1)
+    n = H.shape[0]
+    _shape(H, (n, n), "H")
+    _numel(perm, n, "perm")
+    _on_current_device((H, "H"), (perm, "perm"))
     _contig(H, "H")
-    _check("kronq_act_order", lib().kronq_act_order(_p(H), H.shape[0], _p(perm), _s(stream)))
+    _check("kronq_act_order", lib().kronq_act_order(_p(H), n, _p(perm), _s(stream)))
 
 
 def kronq_permute(src, dst, perm, mode: int, info=None, stream=None):
@@ -224,9 +290,11 @@ def kronq_permute(src, dst, perm, mode: int, info=None, stream=None):
     _dev(src, (torch.float32, torch.uint8), "src", 2)
     _dev(dst, src.dtype, "dst", 2)
     _dev(perm, torch.int32, "perm", 1)
-    _contig(src, "src"); _contig(dst, "dst")
+    _dev(info, torch.int32, "info")
     if dst.shape != src.shape or perm.numel() != src.shape[1]:
         raise ValueError("kronq_permute: shapes do not match")
+    _on_current_device((src, "src"), (dst, "dst"), (perm, "perm"), (info, "info"))
+    _contig(src, "src"); _contig(dst, "dst")
     m, n = src.shape
     _check("kronq_permute", lib().kronq_permute(_p(src), _p(dst), m, n, src.element_size(),
                                                 _p(perm), mode, _p(info), _s(stream)))
@@ -247,12 +315,29 @@ def kronq_deploy_matvec(packed, n: int, bits: int, group: int, scales, zeros, SX
     _dev(packed, (torch.int32, torch.uint32), "packed", 2)
     _dev(x, torch.float32, "x", 2)
     _dev(y, torch.float32, "y", 2)
-    for t_, nm in ((packed, "packed"), (scales, "scales"), (zeros, "zeros"), (x, "x"), (y, "y")):
-        _contig(t_, nm)
+    _dev(scales, torch.float32, "scales")
+    _dev(zeros, torch.uint8, "zeros")
+    _dev(SX, torch.float32, "S_X")
+    _dev(SG, torch.float32, "S_G")
+    _dev(sign_u, torch.int8, "sign_u")
+    _dev(sign_v, torch.int8, "sign_v")
     m = packed.shape[0]
     batch = x.shape[0]
     if x.shape[1] != n or y.shape != (batch, m):
         raise ValueError("kronq_deploy_matvec: shapes do not match")
+    G = _groups(n, group)
+    _shape(packed, (m, packed_words(n, bits)), "packed")
+    _numel(scales, m * G, "scales")
+    _numel(zeros, m * G, "zeros")
+    _numel(SX, n, "S_X")
+    _numel(SG, m, "S_G")
+    _numel(sign_u, m, "sign_u")
+    _numel(sign_v, n, "sign_v")
+    named = ((packed, "packed"), (scales, "scales"), (zeros, "zeros"), (SX, "S_X"), (SG, "S_G"),
+             (sign_u, "sign_u"), (sign_v, "sign_v"), (x, "x"), (y, "y"), (ws, "ws"))
+    _on_current_device(*named)
+    for t_, nm in named:
+        _contig(t_, nm)
     md = MODES[mode] if isinstance(mode, str) else int(mode)
     _check("kronq_deploy_matvec", lib().kronq_deploy_matvec(
         _p(packed), m, n, bits, group, _p(scales), _p(zeros), _p(SX), _p(SG), _p(sign_u),
@@ -262,17 +347,13 @@ def kronq_deploy_matvec(packed, n: int, bits: int, group: int, scales, zeros, SX
 def kronq_quantize_layer_noalloc(W, U, bits: int, group: int, block: int, codes, scales, zeros,
                                  W_hat=None, info=None, stream=None):
     """kronq_quantize_layer with its scratch in the library's static device
-    array (no workspace, nothing allocated; at most 32768 rows and 32768 columns)."""
-    _dev(W, torch.float32, "W", 2)
-    _dev(U, torch.float32, "U_c", 2)
-    _dev(codes, torch.uint8, "codes", 2)
-    _dev(scales, torch.float32, "scales")
-    _dev(zeros, torch.uint8, "zeros")
-    _dev(W_hat, torch.float32, "W_hat", 2)
-    for t, nm in ((W, "W"), (U, "U_c"), (codes, "codes"), (scales, "scales"), (zeros, "zeros"),
-                  (W_hat, "W_hat")):
-        _contig(t, nm)
-    m, n = W.shape
+    array (no workspace, nothing allocated; at most 32768 rows and 32768
+    columns).  Layers whose two-level lazy-update scratch exceeds the array's
+    64 MiB run the one-level update (K = 128 trailing updates): the same
+    codes up to floating-point summation order, at a lower speed."""
+    m, n = _quant_args(W, U, codes, scales, zeros, W_hat, group)
+    _dev(info, torch.int32, "info")
+    _on_current_device((info, "info"))
     _check("kronq_quantize_layer_noalloc", lib().kronq_quantize_layer_noalloc(
         _p(W), m, n, _p(U), bits, group, block, _p(codes), _p(scales), _p(zeros), _p(W_hat),
         _p(info), _s(stream)))
@@ -281,25 +362,39 @@ def kronq_quantize_layer_noalloc(W, U, bits: int, group: int, block: int, codes,
 def kronq_pack(codes, bits: int, packed, stream=None):
     _dev(codes, torch.uint8, "codes", 2)
     _dev(packed, (torch.int32, torch.uint32), "packed", 2)
-    _contig(codes, "codes"); _contig(packed, "packed")
     m, n = codes.shape
+    if bits in (2, 4):
+        _shape(packed, (m, packed_words(n, bits)), "packed")
+    _on_current_device((codes, "codes"), (packed, "packed"))
+    _contig(codes, "codes"); _contig(packed, "packed")
     _check("kronq_pack", lib().kronq_pack(_p(codes), m, n, bits, _p(packed), _s(stream)))
 
 
 def kronq_unpack(packed, n: int, bits: int, codes, stream=None):
     _dev(codes, torch.uint8, "codes", 2)
     _dev(packed, (torch.int32, torch.uint32), "packed", 2)
-    _contig(codes, "codes"); _contig(packed, "packed")
     m = codes.shape[0]
+    _shape(codes, (m, n), "codes")
+    if bits in (2, 4):
+        _shape(packed, (m, packed_words(n, bits)), "packed")
+    _on_current_device((codes, "codes"), (packed, "packed"))
+    _contig(codes, "codes"); _contig(packed, "packed")
     _check("kronq_unpack", lib().kronq_unpack(_p(packed), m, n, bits, _p(codes), _s(stream)))
 
 
 def kronq_layer_loss(W_ref, W_hat, HX, HG, out, ws, stream=None):
     for t, nm in ((W_ref, "W_ref"), (W_hat, "W_hat"), (HX, "H_X"), (HG, "H_G")):
         _dev(t, torch.float32, nm, 2)
-        _contig(t, nm)
     _dev(out, torch.float64, "loss_out")
     m, n = W_ref.shape
+    _shape(W_hat, (m, n), "W_hat")
+    _shape(HX, (n, n), "H_X")
+    _shape(HG, (m, m), "H_G")
+    named = ((W_ref, "W_ref"), (W_hat, "W_hat"), (HX, "H_X"), (HG, "H_G"), (out, "loss_out"),
+             (ws, "ws"))
+    _on_current_device(*named)
+    for t, nm in named[:4]:
+        _contig(t, nm)
     _check("kronq_layer_loss", lib().kronq_layer_loss(
         _p(W_ref), _p(W_hat), m, n, _p(HX), _p(HG), _p(out), _p(ws),
         ws.numel() * ws.element_size(), _s(stream)))
@@ -307,6 +402,7 @@ def kronq_layer_loss(W_ref, W_hat, HX, HG, out, ws, stream=None):
 
 def kronq_selftest_wait(info, limit_ns: int, stream=None):
     _dev(info, torch.int32, "info")
+    _on_current_device((info, "info"))
     _check("kronq_selftest_wait", lib().kronq_selftest_wait(_p(info), int(limit_ns), _s(stream)))
 
 

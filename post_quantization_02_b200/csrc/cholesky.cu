@@ -505,13 +505,8 @@ int kq_cholesky_inv(const float* H, int64_t n64, float damp_rel, float* U, int32
   if (!H || !U || H == U) return KRONQ_ERR_INVALID_ARG;
   if (n64 > 65536) return KRONQ_ERR_UNSUPPORTED;
   if (!ws || ws_bytes < kq_cholesky_ws(n64) || !kqh::aligned(ws, 256)) return KRONQ_ERR_WORKSPACE;
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(panel_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kPanelSmem) != cudaSuccess)
-      return KRONQ_ERR_CUDA;
-    attr = true;
-  }
+  static kqh::PerDevice attr;
+  if (kqh::smem_attr_once(attr, panel_kernel, (int)kPanelSmem) <= 0) return KRONQ_ERR_CUDA;
   const int n = (int)n64;
   const int np = (int)padded(n64);
   uint8_t* w = static_cast<uint8_t*>(ws);

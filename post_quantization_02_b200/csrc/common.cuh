@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "../../include/kronq.h"
 
 #define KQ_DEV __device__ __forceinline__
@@ -294,6 +296,46 @@ bool aligned(const void* p, size_t a);
 unsigned long long launches();
 int launch_status();        // KRONQ_ERR_CUDA if the last launch failed, else KRONQ_OK;
                             // also counts the launch (kronq_launch_count)
+
+// One-time set-up per device (a kernel's shared-memory attribute, an
+// occupancy figure): cudaFuncSetAttribute and occupancy queries apply to the
+// current device only, so a process that drives several GPUs needs each
+// done once on every one of them.
+struct PerDevice {
+  std::mutex mu;
+  int value[64] = {};
+  bool set[64] = {};
+};
+
+// The value init() returns on the current device, computed the first time
+// this device is seen (under the lock) and cached; init() returns a positive
+// value on success and <= 0 on failure (then nothing is cached).  Returns 0
+// if the current device cannot be determined.
+template <class F>
+int per_device(PerDevice& pd, F&& init) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  std::lock_guard<std::mutex> lock(pd.mu);
+  if (!pd.set[dev]) {
+    const int v = init();
+    if (v <= 0) return v;
+    pd.value[dev] = v;
+    pd.set[dev] = true;
+  }
+  return pd.value[dev];
+}
+
+// 1 after cudaFuncSetAttribute(MaxDynamicSharedMemorySize) succeeded on the
+// current device (once per device), else 0.
+template <class K>
+int smem_attr_once(PerDevice& pd, K kernel, int bytes) {
+  return per_device(pd, [&] {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
+                   cudaSuccess
+               ? 1
+               : 0;
+  });
+}
 
 }  // namespace kqh
 

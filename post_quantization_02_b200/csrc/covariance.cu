@@ -687,11 +687,12 @@ int kq_covariance(const uint16_t* A, int64_t N, int64_t d, int64_t lda, float* H
     // CTA pairs on 256 x 256 tiles
     const int ncb2 = (int)((d + P_TILE - 1) / P_TILE);
     const int tiles2 = ncb2 * (ncb2 + 1) / 2;
-    static int max_pairs = 0;
-    if (max_pairs == 0) {
+    // the shared-memory attribute and the number of co-resident pairs, once per device
+    static kqh::PerDevice pairs_of_device;
+    const int P = kqh::per_device(pairs_of_device, [] {
       if (cudaFuncSetAttribute(cov_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                P_SMEM_BYTES) != cudaSuccess)
-        return KRONQ_ERR_CUDA;
+        return 0;
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(2 * (kqh::num_sms() / 2), 1, 1);
       cfg.blockDim = dim3(THREADS, 1, 1);
@@ -701,9 +702,9 @@ int kq_covariance(const uint16_t* A, int64_t N, int64_t d, int64_t lda, float* H
         cudaGetLastError();
         n = kqh::num_sms() / 2;
       }
-      max_pairs = n < kMaxSharedTiles ? n : kMaxSharedTiles;
-    }
-    const int P = max_pairs;
+      return n < kMaxSharedTiles ? n : kMaxSharedTiles;
+    });
+    if (P <= 0) return KRONQ_ERR_CUDA;
     PairSchedule sc;
     sc.tiles = tiles2;
     sc.chunks = (k_iters + KC_ITERS - 1) / KC_ITERS;
@@ -743,13 +744,8 @@ int kq_covariance(const uint16_t* A, int64_t N, int64_t d, int64_t lda, float* H
   int num_tiles = 0;
   for (int cb = 0; cb < ncb; ++cb) num_tiles += (2 * cb + 2 < nrb) ? 2 * cb + 2 : nrb;
 
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(cov_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             SMEM_BYTES) != cudaSuccess)
-      return KRONQ_ERR_CUDA;
-    attr_set = true;
-  }
+  static kqh::PerDevice attr;
+  if (kqh::smem_attr_once(attr, cov_tc_kernel, SMEM_BYTES) <= 0) return KRONQ_ERR_CUDA;
   const int grid = num_tiles < kqh::num_sms() ? num_tiles : kqh::num_sms();
   cov_tc_kernel<<<grid, THREADS, SMEM_BYTES, st>>>(tmap, H, ldh, (int)d, k_iters, ncb, num_tiles,
                                                    alpha, beta, info);

@@ -163,13 +163,9 @@ int launch_mv(const uint32_t* packed, int m, int n, int lg_group, int G, const f
   const int nb4 = n / 4;
   const size_t smem = (size_t)BATCH * (nb4 + nb4 / F4L) * sizeof(float4);
   if (smem > 200 * 1024) return KRONQ_ERR_UNSUPPORTED;
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(dequant_matvec_kernel<BITS, BATCH>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) != cudaSuccess)
-      return KRONQ_ERR_CUDA;
-    attr = true;
-  }
+  static kqh::PerDevice attr;
+  if (kqh::smem_attr_once(attr, dequant_matvec_kernel<BITS, BATCH>, 200 * 1024) <= 0)
+    return KRONQ_ERR_CUDA;
   const int warps = MV_THREADS / 32;
   const int grid = (m + warps - 1) / warps;
   dequant_matvec_kernel<BITS, BATCH><<<grid, MV_THREADS, smem, st>>>(

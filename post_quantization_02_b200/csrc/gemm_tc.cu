@@ -316,13 +316,8 @@ int kq_gemm_nt_tc(const kq::GemmNT* probs, int count, int32_t* info, cudaStream_
   }
   if (P.count == 0) return KRONQ_OK;
   if (P.count == 1) P.p[1] = P.p[0];
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(gemm_nt_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             SMEM_BYTES) != cudaSuccess)
-      return KRONQ_ERR_CUDA;
-    attr = true;
-  }
+  static kqh::PerDevice attr;
+  if (kqh::smem_attr_once(attr, gemm_nt_tc_kernel, SMEM_BYTES) <= 0) return KRONQ_ERR_CUDA;
   int grid = P.total_tiles < kqh::num_sms() ? P.total_tiles : kqh::num_sms();
   if (max_ctas > 0 && grid > max_ctas) grid = max_ctas;
   gemm_nt_tc_kernel<<<grid, THREADS, SMEM_BYTES, st>>>(maps, P, info);

@@ -490,14 +490,10 @@ template <int GROUP, bool CLIP>
 int launch_block(const float* W, int m, int n, const float* U, int i1, int bits, uint8_t* codes,
                  float* scales, uint8_t* zeros, float* W_hat, const SolverScratch& sc, int sb,
                  int slab_end, cudaStream_t st) {
-  static bool attr = false;
+  static kqh::PerDevice attr;
   const size_t smem = (size_t)(QB * US_LD + QB + QB * TT_LD) * sizeof(float);
-  if (!attr) {
-    if (cudaFuncSetAttribute(obs_block_kernel<GROUP, CLIP>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-      return KRONQ_ERR_CUDA;
-    attr = true;
-  }
+  if (kqh::smem_attr_once(attr, obs_block_kernel<GROUP, CLIP>, (int)smem) <= 0)
+    return KRONQ_ERR_CUDA;
   const int grid = (m + ROWS_PER_CTA - 1) / ROWS_PER_CTA;
   obs_block_kernel<GROUP, CLIP><<<grid, OBS_THREADS, smem, st>>>(W, m, n, U, i1, bits, codes, scales, zeros,
                                                    W_hat, sc.Eh + (i1 - sb), sc.El + (i1 - sb),

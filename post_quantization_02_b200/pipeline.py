@@ -11,6 +11,7 @@ of the computation is a libkronq kernel.
 
 from __future__ import annotations
 
+import contextlib
 from dataclasses import dataclass
 
 import torch
@@ -57,7 +58,18 @@ def quantize_sublayer(W: torch.Tensor, HX: torch.Tensor, HG: torch.Tensor,
     are cloned unless in_place is set (then W, HX, HG are overwritten).
     act_order / clip: the README's --act_order and --w_clip (readings in
     include/kronq.h); codes, W_hat and W_rot come back in the original column
-    order, scales / zeros by groups of the permuted order."""
+    order, scales / zeros by groups of the permuted order.
+
+    Every temporary is allocated while `stream` is the current stream, so the
+    caching allocator ties its memory to the stream the kernels run on."""
+    ctx = torch.cuda.stream(stream) if stream is not None else contextlib.nullcontext()
+    with ctx:
+        return _quantize_sublayer(W, HX, HG, sign_u, sign_v, bits, group, alpha, mode, damp, block,
+                                  keep, ws, in_place, act_order, clip, stream)
+
+
+def _quantize_sublayer(W, HX, HG, sign_u, sign_v, bits, group, alpha, mode, damp, block, keep, ws,
+                       in_place, act_order, clip, stream) -> LayerResult:
     m, n = W.shape
     dev = W.device
     if not in_place:
@@ -114,12 +126,18 @@ def covariance_from_host(A_host: torch.Tensor, H: torch.Tensor, chunk_rows: int 
     stream = stream or torch.cuda.current_stream(dev)
     copy_stream = copy_stream or torch.cuda.Stream(dev)
     if staging is None:
-        staging = [torch.empty((chunk_rows, d), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+        # allocated on the compute stream and also used by the copy stream
+        with torch.cuda.stream(stream):
+            staging = [torch.empty((chunk_rows, d), dtype=torch.bfloat16, device=dev)
+                       for _ in range(2)]
+        for t in staging:
+            t.record_stream(copy_stream)
     done = [torch.cuda.Event(), torch.cuda.Event()]
     used = [torch.cuda.Event(), torch.cuda.Event()]
     nchunks = (N + chunk_rows - 1) // chunk_rows
     if nchunks == 0:
-        abi.kronq_covariance(A_host[:0].to(dev), H, 0.0, 0.0, stream=stream)
+        with torch.cuda.stream(stream):
+            abi.kronq_covariance(A_host[:0].to(dev), H, 0.0, 0.0, stream=stream)
         return 0
     copied = 0
     for c in range(nchunks):

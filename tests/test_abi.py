@@ -146,3 +146,57 @@ def test_product_never_imports_the_oracle():
     for f in list(pkg.glob("*.py")) + list((pkg / "csrc").glob("*")):
         text = f.read_text(errors="ignore")
         assert "oracle" not in re.findall(r"\b(?:import|from)\s+(\w+)", text), f
+
+
+def _quant_tensors(m=8, n=256, G=1):
+    import torch
+    return dict(W=torch.zeros(m, n), U=torch.zeros(n, n),
+                codes=torch.zeros(m, n, dtype=torch.uint8), scales=torch.zeros(m, G),
+                zeros=torch.zeros(m, G, dtype=torch.uint8), W_hat=torch.zeros(m, n))
+
+
+@pytest.mark.parametrize("bad", ["U", "codes", "scales", "zeros", "W_hat"])
+@pytest.mark.parametrize("entry", ["kronq_quantize_layer", "kronq_quantize_layer_opt",
+                                   "kronq_quantize_layer_noalloc"])
+def test_binding_checks_solver_shapes(bad, entry):
+    """Every solver tensor is checked against (m, n, G) before anything is
+    passed on (a wrong shape would let the kernels run past its end)."""
+    import torch
+    from post_quantization_02_b200 import abi
+    t = _quant_tensors(G=2)
+    t[bad] = torch.zeros((3,) + tuple(t[bad].shape[1:]), dtype=t[bad].dtype)
+    fn = getattr(abi, entry)
+    extra = (0,) if entry.endswith("_opt") else ()
+    with pytest.raises(ValueError, match="shape|elements"):
+        fn(t["W"], t["U"], 4, 128, 128, *extra, t["codes"], t["scales"], t["zeros"], t["W_hat"])
+
+
+def test_binding_checks_other_shapes():
+    import torch
+    from post_quantization_02_b200 import abi
+    f32 = lambda *s: torch.zeros(*s)
+    i8 = lambda n: torch.ones(n, dtype=torch.int8)
+    with pytest.raises(ValueError, match="shape"):          # H_X must be n x n
+        abi.kronq_biip_rotate(f32(8, 64), f32(32, 32), f32(8, 8), i8(8), i8(64), 0.25, "full", 0,
+                              f32(64), f32(8), None)
+    with pytest.raises(ValueError, match="elements"):       # sign_v has n entries
+        abi.kronq_biip_rotate(f32(8, 64), f32(64, 64), f32(8, 8), i8(8), i8(32), 0.25, "full", 0,
+                              f32(64), f32(8), None)
+    with pytest.raises(ValueError, match="shape"):          # U_c must match H
+        abi.kronq_cholesky_inv(f32(64, 64), 0.01, f32(32, 32), None, None)
+    with pytest.raises(ValueError, match="shape"):          # H must be d x d
+        abi.kronq_covariance(torch.zeros(4, 64, dtype=torch.bfloat16), f32(32, 32), 1.0)
+    with pytest.raises(ValueError, match="shape"):          # packed words per row
+        abi.kronq_pack(torch.zeros(4, 64, dtype=torch.uint8), 4, torch.zeros(4, 4, dtype=torch.int32))
+    with pytest.raises(ValueError, match="shape"):          # W_hat matches W_ref
+        abi.kronq_layer_loss(f32(8, 64), f32(8, 32), f32(64, 64), f32(8, 8),
+                             torch.zeros(1, dtype=torch.float64), None)
+    with pytest.raises(ValueError, match="elements"):       # perm has n entries
+        abi.kronq_act_order(f32(64, 64), torch.zeros(32, dtype=torch.int32))
+
+
+def test_binding_refuses_host_tensors_of_the_right_shape():
+    from post_quantization_02_b200 import abi
+    t = _quant_tensors()
+    with pytest.raises(ValueError, match="CUDA"):
+        abi.kronq_quantize_layer(t["W"], t["U"], 4, -1, 128, t["codes"], t["scales"], t["zeros"])

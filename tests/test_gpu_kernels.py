@@ -137,6 +137,47 @@ def test_biip_matches_oracle(cuda, m, n, mode):
     assert rel_fro(Wd.cpu().numpy(), W) <= 1e-5
 
 
+@pytest.mark.parametrize("m,n", [(256, 256), (64, 112), (688, 96), (1024, 512), (112, 1376)])
+@pytest.mark.parametrize("mode", ["full", "no_rescale", "su_only", "sv_only"])
+def test_biip_alpha_half_matches_oracle(cuda, m, n, mode):
+    """The weight-and-activation setting, --alpha 0.5 (KronQ README (GitHub),
+    "Mapping paper results to flags"): the same kernels with the exponent
+    1/2, against the oracle in every incoh mode."""
+    r = np.random.default_rng(7 * m + n)
+    W, HX, HG, su, sv = _biip_case(r, m, n)
+    Wd, HXd, HGd = t(W, cuda), t(HX, cuda), t(HG, cuda)
+    SX = torch.empty(n, device=cuda)
+    SG = torch.empty(m, device=cuda)
+    ws = abi.workspace(m, n, device=cuda)
+    abi.kronq_biip_rotate(Wd, HXd, HGd, t(su, cuda), t(sv, cuda), 0.5, mode, 0, SX, SG, ws)
+    Wr, HXr, HGr, SXr, SGr = obiip.biip(W, HX, HG, su, sv, 0.5, mode)
+    np.testing.assert_allclose(SX.cpu().numpy(), SXr, rtol=2e-6)
+    np.testing.assert_allclose(SG.cpu().numpy(), SGr, rtol=2e-6)
+    assert rel_fro(Wd.cpu().numpy(), Wr) <= 1e-5
+    assert rel_fro(HXd.cpu().numpy(), HXr) <= 1e-5
+    assert rel_fro(HGd.cpu().numpy(), HGr) <= 1e-5
+
+
+def test_biip_alpha_half_exchanges_diagonal_and_norms_on_gpu(cuda):
+    """At alpha = 1/2 the input rescale swaps diag(H_X) and the squared
+    column norms of W (closed form), checked on the GPU's own S_X: the
+    rescaled diagonal H_jj / S_j^2 equals ||W_j||^2 and ||W_j||^2 S_j^2
+    equals H_jj."""
+    r = np.random.default_rng(23)
+    m, n = 96, 512
+    W, HX, HG, su, sv = _biip_case(r, m, n)
+    SX = torch.empty(n, device=cuda)
+    SG = torch.empty(m, device=cuda)
+    ws = abi.workspace(m, n, device=cuda)
+    abi.kronq_biip_rotate(t(W, cuda), t(HX, cuda), t(HG, cuda), t(su, cuda), t(sv, cuda), 0.5,
+                          "sv_only", 0, SX, SG, ws)
+    sx = SX.cpu().numpy().astype(np.float64)
+    col2 = (W.astype(np.float64) ** 2).sum(0)
+    hd = np.diag(HX).astype(np.float64)
+    np.testing.assert_allclose(hd / sx ** 2, col2, rtol=1e-5)
+    np.testing.assert_allclose(col2 * sx ** 2, hd, rtol=1e-5)
+
+
 # ---------------------------------------------------------- inverse Cholesky
 @pytest.mark.parametrize("n", [64, 72, 200, 256, 1000])
 def test_cholesky_inv_matches_oracle(cuda, n):

@@ -80,3 +80,22 @@ def test_score_from_diagonals_equals_score_after_biip():
         _, HXt, HGt, SX, SG = biip.biip(W, HX, HG, su, sv, 0.25, mode)
         np.testing.assert_allclose(S.sensitivity_from_diagonals(np.diag(HX), np.diag(HG), SX, SG),
                                    S.sensitivity(HXt, HGt), rtol=1e-12)
+
+
+def test_oracle_allocation_is_the_lexicographic_maximum():
+    """The greedy rule equals an exhaustive search: among all vectors in
+    {2,3,4}^k whose parameter-weighted average stays at or below the target,
+    the largest when read in descending score order."""
+    import itertools
+    r = np.random.default_rng(12)
+    for _ in range(200):
+        k = int(r.integers(1, 6))
+        params = [int(p) for p in r.integers(1, 30, k)]
+        scores = [float(s) for s in r.integers(0, 4, k)]
+        target = float(r.choice([2.5, 3.0, 3.4]))
+        order = S.ranking(scores)
+        budget = round(target * sum(params))
+        feas = [b for b in itertools.product((2, 3, 4), repeat=k)
+                if sum(x * p for x, p in zip(b, params)) <= budget]
+        best = max(feas, key=lambda b: tuple(b[i] for i in order))
+        assert S.allocate_bits(scores, params, target) == list(best)

@@ -28,9 +28,16 @@ def _outputs(cuda, m, n, bits, group):
             torch.empty((m, n), device=cuda))
 
 
-@pytest.mark.parametrize("case", [0])
-def test_noalloc_matches_workspace_entry_point_twice(cuda, case):
-    for call, (m, n, bits, group) in enumerate([(300, 512, 4, -1), (520, 384, 2, 128)]):
+# Two shapes whose two-level lazy-update scratch fits the static array (the
+# same path as the workspace call) and, for the second pair of calls, a
+# 4096 x 4096 layer whose two-level scratch does not (68 MiB > 64 MiB): the
+# static-array call then runs the one-level update while the workspace call
+# runs two levels, so only the summation order differs.
+@pytest.mark.parametrize("shapes", [[(300, 512, 4, -1), (520, 384, 2, 128)],
+                                    [(4096, 4096, 4, -1), (4096, 4096, 2, 128)]],
+                         ids=["two-level", "one-level-fallback"])
+def test_noalloc_matches_workspace_entry_point_twice(cuda, shapes):
+    for call, (m, n, bits, group) in enumerate(shapes):
         r = np.random.default_rng(100 + call)
         W = (r.standard_normal((m, n)) * 0.02).astype(np.float32)
         U = ochol.inverse_cholesky(ochol.damp(spd(r, n, spread=1.0), 0.01)).astype(np.float32)
@@ -47,7 +54,12 @@ def test_noalloc_matches_workspace_entry_point_twice(cuda, case):
         assert info.item() == 0
         rc, gc = ref[0].cpu().numpy(), got[0].cpu().numpy()
         assert (rc == gc).mean() >= 0.999              # the codes bar the parity tests use
-        np.testing.assert_allclose(got[1].cpu().numpy(), ref[1].cpu().numpy(), rtol=1e-6)
+        # grids: on rows whose codes all agree (a group grid is taken from the
+        # updated weights, which carry the lazy update's summation order)
+        rows = (rc == gc).all(axis=1)
+        assert rows.mean() >= 0.9
+        np.testing.assert_allclose(got[1].cpu().numpy()[rows], ref[1].cpu().numpy()[rows],
+                                   rtol=1e-5)
         assert (got[2].cpu().numpy() == ref[2].cpu().numpy()).mean() >= 0.999
         same = rc == gc
         np.testing.assert_allclose(got[3].cpu().numpy()[same], ref[3].cpu().numpy()[same],
