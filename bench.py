@@ -33,7 +33,7 @@ sys.path.insert(0, str(ROOT))
 
 METRIC = "layer quantize Mweights/s end-to-end; H_X/H_G GEMM % of bf16 tensor peak"
 UNIT = "Mweights/s"
-DEFAULT_CONFIG = "llama2-7b-q_proj"
+DEFAULT_CONFIG = "llama3-70b-mlp"
 
 
 def parse():
@@ -56,6 +56,9 @@ def parse():
     ap.add_argument("--tokens", type=int, default=None,
                     help="calibration tokens per X/G (default: the workload's; smaller only for "
                          "profiler captures)")
+    ap.add_argument("--oracle-full-chain", action="store_true",
+                    help="time the fp64 oracle's whole chain once on the host cores (every "
+                         "token, every row) for the configuration and print one line; no GPU")
     return ap.parse_args()
 
 
@@ -197,34 +200,41 @@ def load_traffic(workload: str):
 
 
 # ---------------------------------------------------------- oracle side
-def oracle_sample(cfg, budget_s: float = 20.0):
+# The fixed oracle sample both CPU legs time (the cpu_baseline of the GPU
+# run and every step of --impl reference): the same stages on the same
+# sample sizes, scaled to the whole layer the same way, so the two agree.
+SAMPLE_TOKENS = 512        # covariance rows, scaled by tokens
+SAMPLE_ROT_ROWS = 64       # rows through each rotation, scaled by rows
+SAMPLE_CHOL_N = 1024       # inverse Cholesky size, scaled by n^3
+SAMPLE_OBS_COLS = 4096     # column-loop width, scaled by cols^2 above it
+
+
+def oracle_sample(cfg):
     """Time the fp64 oracle, as it stands, on a bounded sample of the workload
     and extrapolate to the whole job.  Returns (seconds_full, sample_text)."""
     import numpy as np
     import synth
-    from oracle import biip as obiip, cholesky as ochol, quantizer as oq, pack as opack
+    from oracle import cholesky as ochol, quantizer as oq, pack as opack
+    from oracle import covariance as ocov
     from oracle import transform as otr
 
-    f = max(0.1, min(1.0, budget_s / 20.0))
-    tok = max(256, int(1024 * f)) // 256 * 256
-    rows_rot = max(32, int(256 * f))
-    rows_obs = max(4, int(16 * f))
+    tok = SAMPLE_TOKENS
+    rows_rot = SAMPLE_ROT_ROWS
     total = 0.0
     parts = []
+    r = np.random.default_rng(0)
     for sub in cfg.sublayers:
         site = cfg.site(sub.site)
         m, n = sub.m, sub.n
         # covariances: tok tokens of X and G, scaled to all tokens
         xb = synth.x_chunk(cfg, site, 0, tokens=tok)
         gb = synth.g_chunk(cfg, sub, 0, tokens=tok)
-        from oracle import covariance as ocov
         t0 = time.perf_counter()
         ocov.covariance(synth.bf16_bits_to_f32(xb).astype(np.float64))
         ocov.covariance(synth.bf16_bits_to_f32(gb).astype(np.float64))
         t_cov = (time.perf_counter() - t0) * cfg.tokens / tok
-        # BiIP: the row transform on rows_rot rows of each matrix, scaled to the
+        # BiIP: the transform on rows_rot rows of each width, scaled to the
         # row and column passes of W (m x n), H_X (n x n), H_G (m x m)
-        r = np.random.default_rng(0)
         su, sv = synth.make_signs(cfg, sub)
         t0 = time.perf_counter()
         otr.apply(r.standard_normal((rows_rot, n)), sv)
@@ -233,23 +243,22 @@ def oracle_sample(cfg, budget_s: float = 20.0):
         otr.apply(r.standard_normal((rows_rot, m)), su)
         t_rm = (time.perf_counter() - t0) / rows_rot
         t_rot = t_rn * (m + 2 * n) + t_rm * (n + 2 * m)
-        # damped inverse Cholesky, n x n (on a smaller n if large, scaled n^3)
-        nc = min(n, 2048)
+        # damped inverse Cholesky at SAMPLE_CHOL_N, scaled by n^3
+        nc = min(n, SAMPLE_CHOL_N)
         A = r.standard_normal((nc, nc))
         H = A @ A.T / nc + np.eye(nc)
         t0 = time.perf_counter()
         ochol.inverse_cholesky(ochol.damp(H, cfg.damp))
         t_chol = (time.perf_counter() - t0) * (n / nc) ** 3
-        # column loop: one wave of the oracle's threaded 64-row chunks, at the
-        # layer's width up to 4096 columns (scaled by rows, and by cols^2 beyond)
-        nn = min(n, 4096)
-        # the loop's cost does not depend on the factor's values: any upper
-        # triangular matrix with a positive diagonal serves for timing
+        # column loop: one 64-row chunk per host thread at up to 4096 columns,
+        # scaled by rows and by cols^2 beyond (the loop's cost does not depend
+        # on the factor's values: any upper triangular matrix with a positive
+        # diagonal serves for timing)
+        nn = min(n, SAMPLE_OBS_COLS)
         U = np.triu(r.standard_normal((nn, nn)) * 0.01) + np.eye(nn)
         bits = sub.bits or 3
         grp = sub.group if sub.group == -1 or nn % sub.group == 0 else -1
-        rows_obs = min(m, 16 * max(1, min(32, os.cpu_count() or 1)))
-        rows_obs = max(4, int(rows_obs * f))
+        rows_obs = min(m, 64 * max(1, min(32, os.cpu_count() or 1)))
         Wr = r.standard_normal((rows_obs, nn)) * 0.02
         t0 = time.perf_counter()
         res = oq.obs_quantize_rows(Wr, U, bits, grp)
@@ -261,9 +270,46 @@ def oracle_sample(cfg, budget_s: float = 20.0):
         total += t_cov + t_rot + t_chol + t_obs + t_pack
         parts.append(f"{sub.name}: cov {tok} of {cfg.tokens} tokens, rotation {rows_rot} rows, "
                      f"inverse Cholesky n={nc}, OBS {rows_obs} of {m} rows x {nn} cols")
-    sample = ("fp64 oracle stages timed on samples and scaled to the whole layer (covariance x tokens, "
-              "rotation x rows, inverse Cholesky x n^3, OBS x rows, x cols^2 above 4096): " + "; ".join(parts))
+    sample = ("fp64 oracle stages timed on a fixed sample and scaled to the whole layer (covariance "
+              "x tokens, rotation x rows, inverse Cholesky x n^3, OBS x rows, x cols^2 above "
+              f"{SAMPLE_OBS_COLS}): " + "; ".join(parts))
     return total, sample
+
+
+def host_cpu_model() -> str:
+    try:
+        for ln in open("/proc/cpuinfo"):
+            if ln.lower().startswith("model name"):
+                return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def oracle_full_chain(args):
+    """The whole fp64 oracle chain of the configuration, timed once on the
+    host cores: covariances over every token, BiIP, s, damped inverse
+    Cholesky, the unblocked column loop on every row, packing."""
+    import synth
+    from oracle import pipeline as opipe
+    cfg = synth.get_config(args.config)
+    t0 = time.perf_counter()
+    stages = {}
+    for sub in cfg.sublayers:
+        t = time.perf_counter()
+        hx = opipe.x_covariance(cfg, cfg.site(sub.site))
+        hg = opipe.g_covariance(cfg, sub)
+        stages["covariance"] = stages.get("covariance", 0.0) + time.perf_counter() - t
+        t = time.perf_counter()
+        opipe.quantize_sublayer(cfg, sub, hx, hg, sub.bits or 3)
+        stages["biip_to_pack"] = stages.get("biip_to_pack", 0.0) + time.perf_counter() - t
+    wall = time.perf_counter() - t0
+    line = {"impl": "reference", "kind": "oracle full chain", "metric": METRIC,
+            "value": cfg.weights / wall / 1e6, "unit": UNIT, "seconds": wall,
+            "stages_s": {k: round(v, 2) for k, v in stages.items()},
+            "config": {"workload": workload_desc(cfg)}, "cores": blas_threads(),
+            "host_cpus": os.cpu_count(), "cpu_model": host_cpu_model(), "dtype": "f64"}
+    print(json.dumps(line), flush=True)
 
 
 def blas_threads() -> int:
@@ -281,14 +327,13 @@ def run_reference(args, rank, world):
         return
     cfg = synth.get_config(args.config)
     weights = cfg.weights
-    per_step = max(3.0, min(30.0, 150.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
-        oracle_sample(cfg, per_step)
+        oracle_sample(cfg)
     t0 = time.perf_counter()
     ests = []
     sample = ""
     for _ in range(args.steps):
-        est, sample = oracle_sample(cfg, per_step)
+        est, sample = oracle_sample(cfg)
         ests.append(est)
     wall = time.perf_counter() - t0
     full = statistics.mean(ests)
@@ -300,7 +345,8 @@ def run_reference(args, rank, world):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded generator)",
         "config": {"workload": workload_desc(cfg), "sample_wall_s_per_step": wall / max(1, args.steps)},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
+                         "host_cpus": os.cpu_count(), "cpu_model": host_cpu_model()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -335,7 +381,9 @@ class Layer:
         G = 1 if sub.group == -1 else n // sub.group
         self.scales = torch.empty((m, G), dtype=torch.float32, device=dev)
         self.zeros = torch.empty((m, G), dtype=torch.uint8, device=dev)
-        self.packed = torch.empty((m, abi.packed_words(n, 4)), dtype=torch.int32, device=dev)
+        # room for 4-bit words; 2-bit codes use the first m x n/16 words as one
+        # contiguous m x (n/16) matrix (packed_view)
+        self.packed_store = torch.empty(m * abi.packed_words(n, 4), dtype=torch.int32, device=dev)
         self.bits = sub.bits
         self.perm = self.Hp = self.Wp = self.codes_p = None
         if act_order:
@@ -343,6 +391,16 @@ class Layer:
             self.Hp = torch.empty((n, n), dtype=torch.float32, device=dev)
             self.Wp = torch.empty((m, n), dtype=torch.float32, device=dev)
             self.codes_p = torch.empty((m, n), dtype=torch.uint8, device=dev)
+
+
+def packed_view(L, bits):
+    words = abi_packed_words(L.sub.n, bits)
+    return L.packed_store[: L.sub.m * words].view(L.sub.m, words)
+
+
+def abi_packed_words(n, bits):
+    from post_quantization_02_b200 import abi
+    return abi.packed_words(n, bits)
 
 
 class StageMarks:
@@ -435,9 +493,7 @@ def gpu_step(cfg, layers, X, ws, stream, cov_events=None, act_order=False, clip=
     for L in layers:
         solve_layer(cfg, L, ws, stream, act_order, clip, mark)
         if L.bits in (2, 4):
-            pk = L.packed[:, : abi.packed_words(L.sub.n, L.bits)]
-            abi.kronq_pack(L.codes, L.bits, pk.contiguous() if not pk.is_contiguous() else pk,
-                           stream=stream)
+            abi.kronq_pack(L.codes, L.bits, packed_view(L, L.bits), stream=stream)
         mark("pack")
 
 
@@ -523,10 +579,67 @@ def run_deploy(args):
     print(json.dumps(line), flush=True)
 
 
+# fp32 CUDA-core peak of a B200 (no measured figure exists for it): 148 SMs x
+# 128 fp32 lanes x 2 flops per FMA x the 1965 MHz maximum SM clock.
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1965e6 / 1e12
+
+
+def stage_rooflines(cfg, layers, steps, stages, inner, peaks, peak_src, peak, peak_kind):
+    """Per-kernel roofline entries from the live CUDA-event timings of the
+    timed region: the lazy-update GEMMs and the inverse Cholesky (library
+    event pairs around their launches), BiIP (the stage marks).  Algorithmic
+    work: lazy update m n (n - 128) flops per sublayer; inverse Cholesky
+    2 n^3 / 3 flops; BiIP 8 bytes per element per pass, two passes over each
+    of W, H_X, H_G (16 (m n + n^2 + m^2) bytes)."""
+    out = {}
+    ms, cnt = inner["lazy_update"]
+    lazy_flops = sum(L.sub.m * L.sub.n * max(0, L.sub.n - 128) for L in layers)
+    if cnt and ms > 0:
+        ach = lazy_flops * steps / (ms / 1e3) / 1e12
+        out["lazy_update"] = {
+            "bound": "tensor", "kernel": "gemm_nt_tc_kernel (solver lazy updates)",
+            "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
+            "peak_source": f"{peak_src} {peak_kind}", "flops_per_step": lazy_flops,
+            "ms_per_step": ms / steps, "launches_per_step": cnt / steps,
+            "avg_launch_ms": ms / cnt,
+            "note": "fp32-accurate products as three tf32 tensor-core MMAs (hi*hi + hi*lo + lo*hi)"}
+    chol_ms = stages.get("inverse_cholesky", 0.0)
+    chol_flops = sum(2 * L.sub.n ** 3 / 3 for L in layers)
+    if chol_ms > 0:
+        ach = chol_flops / (chol_ms / 1e3) / 1e12
+        out["inverse_cholesky"] = {
+            "bound": "alu", "kernel": "panel_kernel + gemm_nt_tc_kernel (kronq_cholesky_inv)",
+            "achieved": ach, "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s",
+            "frac": ach / FP32_ALU_TFLOPS,
+            "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1965 MHz",
+            "flops_per_step": chol_flops, "ms_per_step": chol_ms,
+            "panel_ms_per_step": inner["chol_panel"][0] / steps,
+            "update_ms_per_step": inner["chol_update"][0] / steps,
+            "panels_per_step": inner["chol_panel"][1] / steps}
+    biip_ms = stages.get("biip_sensitivity", 0.0)
+    biip_bytes = sum(16 * (L.sub.m * L.sub.n + L.sub.n ** 2 + L.sub.m ** 2) for L in layers)
+    if biip_ms > 0:
+        hbm = float(peaks["hbm_gbs"])
+        ach = biip_bytes / (biip_ms / 1e3) / 1e9
+        out["biip"] = {"bound": "hbm", "kernel": "row / column transform passes (kronq_biip_rotate)",
+                       "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+                       "peak_source": f"{peak_src} hbm_gbs", "bytes_per_step": biip_bytes,
+                       "ms_per_step": biip_ms,
+                       "note": "stage time includes the norm reductions and the trace sums"}
+    obs_ms, obs_cnt = inner["obs_block"]
+    if obs_cnt:
+        out["obs_block"] = {"bound": "latency", "ms_per_step": obs_ms / steps,
+                            "launches_per_step": obs_cnt / steps}
+    return out
+
+
 def main():
     args = parse()
     if args.deploy:
         run_deploy(args)
+        return
+    if args.oracle_full_chain:
+        oracle_full_chain(args)
         return
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -587,6 +700,7 @@ def main():
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    abi.kronq_timing_enable(True)       # event pairs around the library's inner launches
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record(stream)
     for k in range(args.steps):
@@ -597,6 +711,8 @@ def main():
     if world > 1:
         dist.barrier()
     launches = abi.kronq_launch_count() - launches0
+    inner = {k: abi.kronq_timing_read(k) for k in abi.TIMERS}
+    abi.kronq_timing_enable(False)
     ms = reduce_max_ms(start.elapsed_time(end), world, dev)
     cov_ms = [ev[2 * i].elapsed_time(ev[2 * i + 1]) for ev in cov_events for i in range(ncov)]
     stages = {}
@@ -612,7 +728,7 @@ def main():
                "G": {s: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).pin_memory()
                      for s, v in host["G"].items()},
                "W": {L.sub.name: L.W0.cpu().pin_memory() for L in layers}}
-        outs = {L.sub.name: (torch.empty(L.packed.shape, dtype=torch.int32).pin_memory(),
+        outs = {L.sub.name: (torch.empty(L.packed_store.shape, dtype=torch.int32).pin_memory(),
                              torch.empty(L.scales.shape).pin_memory(),
                              torch.empty(L.zeros.shape, dtype=torch.uint8).pin_memory()) for L in layers}
         copy_stream = torch.cuda.Stream(dev)
@@ -647,11 +763,10 @@ def main():
                 solve_layer(cfg, L, ws, stream, args.act_order, args.w_clip)
                 pk, sc, zr = outs[L.sub.name]
                 if L.bits in (2, 4):
-                    words = abi.packed_words(L.sub.n, L.bits)
-                    abi.kronq_pack(L.codes, L.bits, L.packed[:, :words].contiguous()
-                                   if words != L.packed.shape[1] else L.packed, stream=stream)
-                    pk.copy_(L.packed, non_blocking=True)
-                    d2h += L.packed.numel() * 4
+                    pv = packed_view(L, L.bits)
+                    abi.kronq_pack(L.codes, L.bits, pv, stream=stream)
+                    pk[: pv.numel()].copy_(pv.view(-1), non_blocking=True)
+                    d2h += pv.numel() * 4
                 sc.copy_(L.scales, non_blocking=True)
                 zr.copy_(L.zeros, non_blocking=True)
                 d2h += L.scales.numel() * 4 + L.zeros.numel()
@@ -694,12 +809,17 @@ def main():
                 "peak_source": f"{peak_src} {peak_kind}",
                 "flops_per_launch": statistics.mean(cov_flops), "avg_launch_ms": avg_ms,
                 "launches_timed": len(cov_ms)}
+    rooflines = stage_rooflines(cfg0, layers, args.steps, stages, inner, peaks, peak_src, peak,
+                                peak_kind)
+    rooflines["covariance"] = {k: roofline[k] for k in ("bound", "achieved", "peak", "unit", "frac",
+                                                        "avg_launch_ms", "flops_per_launch")}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        est, sample = oracle_sample(cfg0, 20.0)
+        est, sample = oracle_sample(cfg0)
         cpu = {"value": cfg0.weights / est / 1e6, "unit": UNIT, "cores": blas_threads(),
-               "kind": "oracle", "sample": sample, "host_cpus": os.cpu_count()}
+               "kind": "oracle", "sample": sample, "host_cpus": os.cpu_count(),
+               "cpu_model": host_cpu_model()}
 
     if rank == 0:
         line = {
@@ -711,7 +831,8 @@ def main():
                        "l2": l2_note(cfg0),
                        "solver_dtype": "fp32", "input_gen_s": round(t_gen, 1),
                        "act_order": args.act_order, "w_clip": args.w_clip},
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
+            "roofline": roofline, "rooflines": rooflines, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": launches,
             "clocks": clocks,
             "stages_ms": {k: round(v, 4) for k, v in stages.items()},
             # the solver alone, given H_X': inverse Cholesky + OBS loop

@@ -66,6 +66,28 @@ int kronq_abi_version(void);
 uint64_t kronq_launch_count(void);
 
 /*
+ * Launch timing, a measurement helper (the pages have no counterpart; it
+ * lets a benchmark attribute time to kernels that run inside one call).
+ * While enabled, the library records a CUDA event pair on the launching
+ * stream around every launch of the categories below; kronq_timing_read
+ * waits for the recorded events of the current device and returns the
+ * summed device time in ms and the number of launches of one category.
+ * kronq_timing_enable(on) clears the records (on = 0 also stops recording).
+ * Events are created by the library (cudaEventCreate) and reused; do not
+ * enable timing while a stream is being captured into a CUDA graph.
+ * Recording adds a few microseconds of host time per timed launch.
+ */
+enum kronq_timer {
+  KRONQ_TIMER_LAZY_UPDATE = 0,  /* the solver's lazy block updates (tensor-core GEMMs) */
+  KRONQ_TIMER_CHOL_UPDATE = 1,  /* the inverse Cholesky's trailing updates (tensor-core GEMMs) */
+  KRONQ_TIMER_CHOL_PANEL = 2,   /* the inverse Cholesky's panel factorisations */
+  KRONQ_TIMER_OBS_BLOCK = 3,    /* the solver's 128-column block kernels */
+  KRONQ_TIMER_COUNT = 4
+};
+int kronq_timing_enable(int on);
+int kronq_timing_read(int category, double* total_ms, uint64_t* launches);
+
+/*
  * Workspace, in bytes, that kronq_biip_rotate, kronq_cholesky_inv,
  * kronq_quantize_layer and kronq_layer_loss need for a layer of m x n.
  * Returns 0 for invalid sizes.

@@ -53,13 +53,15 @@ def g_covariance(cfg, sub, tokens=None, threads=None) -> np.ndarray:
                        sub.m, tokens, threads)
 
 
-def quantize_sublayer(cfg, sub, HX, HG, bits, rows=None, W=None, act_order=False, clip=False):
+def quantize_sublayer(cfg, sub, HX, HG, bits, rows=None, W=None, act_order=False, clip=False,
+                      loop="numpy"):
     """Steps 2-6 for one sublayer given its two covariances.
 
     rows: the rows of W' to run the column loop on (all when None); the loop
     treats rows independently, so a subset gives those rows' exact results.
     act_order / clip: the README's --act_order and --w_clip (readings in
-    oracle/quantizer.py)."""
+    oracle/quantizer.py).  loop="c": the column loop through its plain-C
+    restatement (bit-identical results; no act_order / clip there)."""
     if W is None:
         W = synth.make_w(cfg, sub)
     su, sv = synth.make_signs(cfg, sub)
@@ -73,7 +75,10 @@ def quantize_sublayer(cfg, sub, HX, HG, bits, rows=None, W=None, act_order=False
     else:
         perm = None
         Uc = cholesky.inverse_cholesky(Hd)
-        res = quantizer.obs_quantize_rows(Wp, Uc, bits, sub.group, rows=rows, clip=clip)
+        if loop == "c" and not clip:
+            res = quantizer.obs_quantize_rows_c(Wp, Uc, bits, sub.group, rows=rows)
+        else:
+            res = quantizer.obs_quantize_rows(Wp, Uc, bits, sub.group, rows=rows, clip=clip)
     out = {"W_rot": Wp, "HX_rot": HXt, "HG_rot": HGt, "S_X": SX, "S_G": SG, "s": s,
            "U_c": Uc, "perm": perm, "rows": np.arange(sub.m) if rows is None else np.asarray(rows)}
     out.update(res)

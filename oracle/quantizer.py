@@ -197,6 +197,42 @@ def obs_quantize_rows(W: np.ndarray, U: np.ndarray, bits: int, group: int = -1,
     return {k: np.concatenate([r[k] for r in res], axis=0) for k in res[0]}
 
 
+def obs_quantize_rows_c(W: np.ndarray, U: np.ndarray, bits: int, group: int = -1, rows=None,
+                        threads: int | None = None):
+    """obs_quantize on a subset of rows through the plain-C restatement of
+    the same loop (oracle/c/obs_rows.c: the same fp32 decisions and fp64
+    updates in the same order, without floating-point contraction), for
+    wide layers where the numpy loop is too slow.  Results are bit-identical
+    to obs_quantize (pinned in the oracle tests).  No --w_clip here."""
+    import ctypes
+    from . import build_c
+    lib = ctypes.CDLL(str(build_c.build()))
+    f = lib.kronq_oracle_obs_rows
+    P = ctypes.c_void_p
+    f.argtypes = [P, ctypes.c_int64, ctypes.c_int64, P, ctypes.c_int, ctypes.c_int, P, P, P, P,
+                  ctypes.c_int]
+    f.restype = ctypes.c_int
+    W = np.asarray(W)
+    rows = np.arange(W.shape[0]) if rows is None else np.asarray(rows)
+    n = W.shape[1]
+    _check(n, group, bits)
+    Wr = np.ascontiguousarray(W[rows], dtype=np.float64)
+    U = np.ascontiguousarray(U, dtype=np.float64)
+    m = Wr.shape[0]
+    ng = 1 if group == -1 else n // group
+    codes = np.zeros((m, n), dtype=np.uint8)
+    scales = np.zeros((m, ng), dtype=F32)
+    zeros = np.zeros((m, ng), dtype=np.uint8)
+    What = np.zeros((m, n))
+    if m:
+        st = f(Wr.ctypes.data, m, n, U.ctypes.data, bits, group, codes.ctypes.data,
+               scales.ctypes.data, zeros.ctypes.data, What.ctypes.data,
+               int(threads or (os.cpu_count() or 1)))
+        if st != 0:
+            raise ValueError("oracle C loop rejected its arguments")
+    return {"codes": codes, "scale": scales, "zero": zeros, "W_hat": What}
+
+
 def act_order_perm(H: np.ndarray) -> np.ndarray:
     """--act_order (reading): the columns are quantized in descending order
     of the diagonal of the (rotated, undamped) H_X handed to the solver, equal

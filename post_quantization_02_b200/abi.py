@@ -63,6 +63,8 @@ def lib() -> ctypes.CDLL:
         "kronq_unpack": ([P, I64, I64, I32, P, P], I32),
         "kronq_layer_loss": ([P, P, I64, I64, P, P, P, P, SZ, P], I32),
         "kronq_selftest_wait": ([P, I64, P], I32),
+        "kronq_timing_enable": ([I32], I32),
+        "kronq_timing_read": ([I32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_uint64)], I32),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -398,6 +400,23 @@ def kronq_layer_loss(W_ref, W_hat, HX, HG, out, ws, stream=None):
     _check("kronq_layer_loss", lib().kronq_layer_loss(
         _p(W_ref), _p(W_hat), m, n, _p(HX), _p(HG), _p(out), _p(ws),
         ws.numel() * ws.element_size(), _s(stream)))
+
+
+TIMERS = {"lazy_update": 0, "chol_update": 1, "chol_panel": 2, "obs_block": 3}
+
+
+def kronq_timing_enable(on: bool = True):
+    """Start (and clear) or stop the library's event timing of its inner launches."""
+    _check("kronq_timing_enable", lib().kronq_timing_enable(1 if on else 0))
+
+
+def kronq_timing_read(category) -> tuple:
+    """(summed device ms, launches) of one timer category on the current device."""
+    cat = TIMERS[category] if isinstance(category, str) else int(category)
+    ms = ctypes.c_double(0.0)
+    cnt = ctypes.c_uint64(0)
+    _check("kronq_timing_read", lib().kronq_timing_read(cat, ctypes.byref(ms), ctypes.byref(cnt)))
+    return ms.value, int(cnt.value)
 
 
 def kronq_selftest_wait(info, limit_ns: int, stream=None):

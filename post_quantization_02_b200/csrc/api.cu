@@ -2,6 +2,8 @@
 // Host-side argument checks live next to each launcher; this file only maps
 // the ABI onto them and provides the shared host helpers.
 #include <atomic>
+#include <mutex>
+#include <vector>
 
 #include "common.cuh"
 
@@ -65,6 +67,47 @@ int launch_status() {
 
 unsigned long long launches() { return g_launches.load(std::memory_order_relaxed); }
 
+// ---- launch timing: event pairs per device, reused after every enable
+namespace {
+struct TimerSlot {
+  cudaEvent_t start, end;
+  int category;
+};
+std::mutex g_timer_mu;
+std::atomic<bool> g_timer_on{false};
+std::vector<TimerSlot> g_timer_slots[64];
+size_t g_timer_used[64] = {};
+}  // namespace
+
+int timer_begin(int category, cudaStream_t st) {
+  if (!g_timer_on.load(std::memory_order_relaxed)) return -1;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
+  std::lock_guard<std::mutex> lock(g_timer_mu);
+  std::vector<TimerSlot>& slots = g_timer_slots[dev];
+  if (g_timer_used[dev] == slots.size()) {
+    TimerSlot t;
+    if (cudaEventCreate(&t.start) != cudaSuccess) return -1;
+    if (cudaEventCreate(&t.end) != cudaSuccess) {
+      cudaEventDestroy(t.start);
+      return -1;
+    }
+    slots.push_back(t);
+  }
+  const size_t i = g_timer_used[dev]++;
+  slots[i].category = category;
+  if (cudaEventRecord(slots[i].start, st) != cudaSuccess) return -1;
+  return dev * (1 << 24) + (int)i;
+}
+
+void timer_end(int slot, cudaStream_t st) {
+  if (slot < 0) return;
+  std::lock_guard<std::mutex> lock(g_timer_mu);
+  const int dev = slot >> 24;
+  const size_t i = (size_t)(slot & ((1 << 24) - 1));
+  if (dev < 64 && i < g_timer_used[dev]) cudaEventRecord(g_timer_slots[dev][i].end, st);
+}
+
 }  // namespace kqh
 
 static cudaStream_t S(void* s) { return static_cast<cudaStream_t>(s); }
@@ -102,6 +145,35 @@ const char* kronq_status_string(int st) {
 int kronq_abi_version(void) { return 100; }
 
 uint64_t kronq_launch_count(void) { return kqh::launches(); }
+
+int kronq_timing_enable(int on) {
+  std::lock_guard<std::mutex> lock(kqh::g_timer_mu);
+  for (int d = 0; d < 64; ++d) kqh::g_timer_used[d] = 0;
+  kqh::g_timer_on.store(on != 0);
+  return KRONQ_OK;
+}
+
+int kronq_timing_read(int category, double* total_ms, uint64_t* launches) {
+  if (!total_ms || !launches || category < 0 || category >= KRONQ_TIMER_COUNT)
+    return KRONQ_ERR_INVALID_ARG;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return KRONQ_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(kqh::g_timer_mu);
+  double ms = 0.0;
+  uint64_t count = 0;
+  for (size_t i = 0; i < kqh::g_timer_used[dev]; ++i) {
+    const kqh::TimerSlot& t = kqh::g_timer_slots[dev][i];
+    if (t.category != category) continue;
+    if (cudaEventSynchronize(t.end) != cudaSuccess) return KRONQ_ERR_CUDA;
+    float e = 0.f;
+    if (cudaEventElapsedTime(&e, t.start, t.end) != cudaSuccess) return KRONQ_ERR_CUDA;
+    ms += e;
+    ++count;
+  }
+  *total_ms = ms;
+  *launches = count;
+  return KRONQ_OK;
+}
 
 int kronq_selftest_wait(int32_t* info, int64_t limit_ns, void* stream) {
   if (!info || limit_ns <= 0 || limit_ns > 2000000000ll) return KRONQ_ERR_INVALID_ARG;

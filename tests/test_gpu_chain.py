@@ -49,7 +49,16 @@ def test_toy_layer_full_chain(cuda):
     assert rel_fro(res.H_X.cpu().numpy(), ref["HX_rot"]) <= 1e-4
     assert rel_fro(res.H_G.cpu().numpy(), ref["HG_rot"]) <= 1e-4
     np.testing.assert_allclose(res.sens[0].item(), ref["s"], rtol=1e-4)
-    assert rel_fro(res.U_c.cpu().numpy(), ref["U_c"]) <= 1e-3
+    # U_c: stage-isolated (the oracle factors the GPU's own H_X') at 1e-4;
+    # end to end it also carries the difference of its input H_X', which the
+    # factor of the damped matrix amplifies by at most about kappa(H_d)
+    # (first-order perturbation of the factorisation)
+    from oracle import cholesky as ochol
+    Ug, HXr = res.U_c.cpu().numpy(), res.H_X.cpu().numpy()
+    assert rel_fro(Ug, ochol.inverse_cholesky(ochol.damp(HXr, cfg.damp))) <= 1e-4
+    ev = np.linalg.eigvalsh(ochol.damp(ref["HX_rot"], cfg.damp))
+    bound = 1e-4 + 2 * (ev[-1] / ev[0]) * rel_fro(HXr, ref["HX_rot"])
+    assert rel_fro(Ug, ref["U_c"]) <= bound, (rel_fro(Ug, ref["U_c"]), bound)
     codes = res.codes.cpu().numpy()
     same = (codes == ref["codes"]).mean()
     assert same >= 0.999, same

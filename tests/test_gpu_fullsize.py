@@ -15,9 +15,10 @@ sampled outputs, each computed from its definition on the same inputs:
 * inverse Cholesky (review, Algorithm 2, steps 1-2): the trailing 2048 x 2048
   block of U_c exactly (it depends on the trailing block of H only), and
   U_c^T U_c H_d = I on sampled columns.
-* OBS (Prop. 1: rows are independent given U_c): a seeded row subset through
-  the unblocked oracle loop; >= 99.9 % identical codes, equal grids, and the
-  subset's loss within 1 %.
+* OBS (Prop. 1: rows are independent given U_c): a seeded subset of 1024
+  rows (all rows of narrower layers) through the unblocked oracle loop (its
+  plain-C restatement, bit-identical to the numpy loop); >= 99.9 % identical
+  codes, equal grids, and the subset's loss within 1 %.
 * packing: every word, bit-exact.
 """
 
@@ -88,10 +89,10 @@ def _check_cov(H, diag_ref, blk_ref, idx):
 
 
 def _rows_for(n):
-    """Solver rows the oracle re-runs: its unblocked fp64 loop costs
-    rows * n^2 / 2 updates, memory-bound on the host (about 20 s at
-    n = 28672 for 64 rows)."""
-    return 1024 if n <= 8192 else (256 if n <= 16384 else 64)
+    """Solver rows the oracle re-runs at every width: its unblocked fp64
+    loop costs rows * n^2 / 2 updates (the C restatement runs about 1e10
+    of them per second on the host's cores: tens of seconds at n = 28672)."""
+    return 1024
 
 
 def _sublayer_chain(cfg, sub, HX, HG, bits, r, rows=None, full_loss=False):
@@ -160,7 +161,7 @@ def _sublayer_chain(cfg, sub, HX, HG, bits, r, rows=None, full_loss=False):
     rows = np.sort(r.choice(m, min(m, rows or _rows_for(n)), replace=False))
     U64 = Uh.astype(np.float64)
     del Uh
-    ref = oq.obs_quantize_rows(Wrot[rows], U64, bits, group, chunk=16 if n > 8192 else 64)
+    ref = oq.obs_quantize_rows_c(Wrot[rows], U64, bits, group)
     del U64
     cg = codes.cpu().numpy()
     same = (cg[rows] == ref["codes"]).mean()
@@ -259,12 +260,13 @@ def test_llama3_70b_mlp_full_size(cuda, name):
     _sublayer_chain(cfg, sub, HX[sub.site], HG[sub.name], sub.bits, r)
 
 
-def test_llama3_8b_block_ranking_allocation_and_down_proj(cuda):
+def test_llama3_8b_block_ranking_allocation_and_all_sublayers(cuda):
     """Seven sublayers on four input sites: every covariance at full size,
     s for each sublayer after BiIP, the ranking and the 2/3/4-bit allocation
     at a 3-bit average identical to the oracle's (whose s comes from its own
-    fp64 covariance diagonals and its own S_X, S_G); then the widest
-    sublayer (down_proj, 4096 x 14336) through the solver at its bits."""
+    fp64 covariance diagonals and its own S_X, S_G); then every sublayer
+    through the rest of the chain at its allocated bits (3-bit codes stay
+    unpacked)."""
     cfg = synth.get_config("llama3-8b-block")
     r = np.random.default_rng(303)
     HX, HG, dx, dg = _covariances(cfg, cuda, r)
@@ -293,12 +295,14 @@ def test_llama3_8b_block_ranking_allocation_and_down_proj(cuda):
     assert bits == osens.allocate_bits(s_ref, params, cfg.mixed_avg_bits)
     assert sorted(set(bits)) != [3], bits          # a real mix, not all 3-bit
     assert sum(b * p for b, p in zip(bits, params)) <= 3 * sum(params)
-    # the widest sublayer through the rest of the chain, at its allocated bits
-    sub = cfg.sublayers[-1]
-    for name in [s.name for s in cfg.sublayers[:-1]]:
-        del HG[name]
-    torch.cuda.empty_cache()
-    _sublayer_chain(cfg, sub, HX[sub.site], HG[sub.name], bits[-1], r)
+    # every sublayer through the rest of the chain, at its allocated bits; a
+    # shared input site's H_X is rotated per sublayer, so each gets a copy
+    for sub, b in zip(cfg.sublayers, bits):
+        hx = HX[sub.site].clone()
+        out = _sublayer_chain(cfg, sub, hx, HG.pop(sub.name), b, r)
+        assert out["same"] >= 0.999
+        del hx
+        torch.cuda.empty_cache()
 
 
 def test_llama2_7b_q_proj_act_order_and_clip_solver_full_size(cuda):

@@ -137,6 +137,41 @@ def test_biip_matches_oracle(cuda, m, n, mode):
     assert rel_fro(Wd.cpu().numpy(), W) <= 1e-5
 
 
+@pytest.mark.parametrize("m,n", [(64, 14336), (14336, 64), (32, 28672), (28672, 32)])
+def test_biip_odd_factor_seven_wide(cuda, m, n):
+    """Widths 7 x 2^11 and 7 x 2^12 (the LLaMA-3 MLP widths 14336 and 28672)
+    take the fused passes: every segment's Walsh-Hadamard transform and the
+    7-segment mix in one pass over the rows, and the column pass in two.
+    Sampled entries of W', H_X', H_G' (64 x 64 blocks, every segment
+    represented) and the scales in full, against the oracle."""
+    r = np.random.default_rng(m + 5 * n)
+    W = (r.standard_normal((m, n)) * 0.02 * np.exp(r.uniform(-1, 1, n))[None, :]).astype(np.float32)
+
+    def wide(d):
+        H = r.standard_normal((d, d), dtype=np.float32)
+        H[np.arange(d), np.arange(d)] = np.abs(H[np.arange(d), np.arange(d)]) + 1.0
+        return H
+
+    HX, HG = wide(n), wide(m)
+    su, sv = signs(r, m), signs(r, n)
+    Wd, HXd, HGd = t(W, cuda), t(HX, cuda), t(HG, cuda)
+    SX = torch.empty(n, device=cuda)
+    SG = torch.empty(m, device=cuda)
+    ws = abi.workspace(m, n, device=cuda)
+    abi.kronq_biip_rotate(Wd, HXd, HGd, t(su, cuda), t(sv, cuda), 0.25, "full", 0, SX, SG, ws)
+    torch.cuda.synchronize()
+    pick = lambda d, k: np.sort(r.choice(d, min(d, k), replace=False))
+    wr, wc, hxi, hgi = pick(m, 64), pick(n, 64), pick(n, 64), pick(m, 64)
+    Wb, HXb, HGb, SXr, SGr = obiip.biip_entries(W, HX, HG, su, sv, 0.25, "full", wr, wc, hxi, hgi)
+    np.testing.assert_allclose(SX.cpu().numpy(), SXr, rtol=2e-6)
+    np.testing.assert_allclose(SG.cpu().numpy(), SGr, rtol=2e-6)
+    assert rel_fro(Wd.cpu().numpy()[np.ix_(wr, wc)], Wb) <= 1e-5
+    ix = torch.as_tensor(hxi, device=cuda)
+    assert rel_fro(HXd[ix][:, ix].cpu().numpy(), HXb) <= 1e-5
+    ig = torch.as_tensor(hgi, device=cuda)
+    assert rel_fro(HGd[ig][:, ig].cpu().numpy(), HGb) <= 1e-5
+
+
 @pytest.mark.parametrize("m,n", [(256, 256), (64, 112), (688, 96), (1024, 512), (112, 1376)])
 @pytest.mark.parametrize("mode", ["full", "no_rescale", "su_only", "sv_only"])
 def test_biip_alpha_half_matches_oracle(cuda, m, n, mode):

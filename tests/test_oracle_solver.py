@@ -288,3 +288,25 @@ def test_ldlq_quarter_bound_table9():
         assert np.sum(res["E"][i] ** 2) <= 0.25 * step ** 2 * np.sum(D) * (1 + 1e-9)
         checked += 1
     assert checked >= m // 2, checked
+
+
+@pytest.mark.parametrize("m,n,bits,group", [(37, 256, 4, -1), (20, 384, 2, 128), (9, 128, 3, 32),
+                                            (17, 512, 2, 64), (1, 128, 4, 128), (0, 128, 4, -1)])
+def test_c_loop_is_bit_identical_to_the_numpy_loop(m, n, bits, group):
+    """oracle/c/obs_rows.c restates obs_quantize in C for wide layers: the
+    same fp32 decisions and fp64 updates in the same order, so every code,
+    grid and W_hat entry must agree bit for bit, on rows with outliers and
+    an all-zero row too."""
+    from oracle import cholesky as ochol
+    r = np.random.default_rng(m * 7 + n)
+    A = r.standard_normal((2 * n, n)) * np.exp(r.uniform(-1, 1, n))
+    U = ochol.inverse_cholesky(ochol.damp(A.T @ A / (2 * n), 0.01))
+    W = r.standard_normal((m, n)) * 0.02
+    if m > 2:
+        W[1] = 0.0
+        W[2, :: max(1, n // 5)] *= 40.0
+    a = Q.obs_quantize(W, U, bits, group)
+    rows = np.arange(m)[::-1].copy()
+    b = Q.obs_quantize_rows_c(W, U, bits, group, rows=rows)
+    for k in ("codes", "scale", "zero", "W_hat"):
+        assert np.array_equal(a[k][rows], b[k]), k
