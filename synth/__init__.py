@@ -19,8 +19,10 @@ from .gen import (
     make_signs,
     make_w,
     make_x,
+    make_xq,
     g_chunk,
     x_chunk,
+    xq_chunk,
     n_chunks,
     CHUNK_TOKENS,
 )
@@ -28,5 +30,5 @@ from .gen import (
 __all__ = [
     "CONFIGS", "Config", "Sublayer", "XSite", "get_config",
     "bf16_bits_to_f32", "f32_to_bf16_bits", "make_g", "make_signs", "make_w",
-    "make_x", "g_chunk", "x_chunk", "n_chunks", "CHUNK_TOKENS",
+    "make_x", "make_xq", "g_chunk", "x_chunk", "xq_chunk", "n_chunks", "CHUNK_TOKENS",
 ]

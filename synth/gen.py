@@ -25,6 +25,12 @@ SLAB_ROWS = 1024
 
 # tensor ids of the generator keys
 T_W, T_X, T_G, T_SIGN_U, T_SIGN_V, T_OUTLIER, T_GSCALE, T_WROW, T_XAUX = 1, 2, 3, 4, 5, 6, 7, 8, 9
+T_XDRIFT = 10
+
+# Drift of the quantized model's layer input against the full-precision one
+# (the asymmetric-calibration inputs): noise of this standard deviation per
+# unit of the channel's scale.
+DRIFT_SIGMA = 0.05
 
 
 def _rng(seed: int, tensor_id: int, index: int, chunk: int = 0) -> np.random.Generator:
@@ -119,6 +125,38 @@ def x_chunk(cfg: Config, site: XSite, c: int, tokens: int | None = None,
             zz[:, oc] *= np.float32(cfg.x_outlier_scale)
         out[r0:r1] = f32_to_bf16_bits(zz)
     return out
+
+
+def xq_chunk(cfg: Config, site: XSite, c: int, tokens: int | None = None,
+             sigma: float = DRIFT_SIGMA, out: np.ndarray | None = None) -> np.ndarray:
+    """Rows [c*CHUNK_TOKENS, ...) of X~, the input the same site sees in the
+    partly quantized model, as bf16 bits: the bf16 values of X plus seeded
+    Gaussian noise of standard deviation sigma times the channel's scale
+    (x_outlier_scale on the outlier channels, 1 elsewhere), rounded to bf16."""
+    xb = x_chunk(cfg, site, c, tokens)
+    rows, d = xb.shape
+    if out is None:
+        out = np.empty((rows, d), dtype=np.uint16)
+    scale = np.ones(d, dtype=np.float32)
+    oc = outlier_channels(cfg, site)
+    if len(oc):
+        scale[oc] = np.float32(cfg.x_outlier_scale)
+    gz = _rng(cfg.seed, T_XDRIFT, site.index, c)
+    for r0 in range(0, rows, SLAB_ROWS):
+        r1 = min(rows, r0 + SLAB_ROWS)
+        z = gz.standard_normal((r1 - r0, d), dtype=np.float32)
+        z *= np.float32(sigma) * scale[None, :]
+        z += bf16_bits_to_f32(xb[r0:r1])
+        out[r0:r1] = f32_to_bf16_bits(z)
+    return out
+
+
+def make_xq(cfg: Config, site: XSite, tokens: int | None = None, threads: int | None = None,
+            sigma: float = DRIFT_SIGMA, out: np.ndarray | None = None) -> np.ndarray:
+    """Whole X~ (tokens x width) for one site, bf16 bits."""
+    tokens = cfg.tokens if tokens is None else tokens
+    return _assemble(lambda c, o: xq_chunk(cfg, site, c, tokens, sigma, out=o), tokens,
+                     site.width, threads, out)
 
 
 def g_scales(cfg: Config, sub: Sublayer) -> np.ndarray:
