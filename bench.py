@@ -56,6 +56,11 @@ def parse():
     ap.add_argument("--tokens", type=int, default=None,
                     help="calibration tokens per X/G (default: the workload's; smaller only for "
                          "profiler captures)")
+    ap.add_argument("--kernel", choices=["covariance"], default=None,
+                    help="time one kernel alone (for profiler captures on small cases): "
+                         "kronq_covariance of a --tokens x --width bf16 matrix")
+    ap.add_argument("--width", type=int, default=None,
+                    help="feature width for --kernel (default: the workload's widest)")
     ap.add_argument("--oracle-full-chain", action="store_true",
                     help="time the fp64 oracle's whole chain once on the host cores (every "
                          "token, every row) for the configuration and print one line; no GPU")
@@ -633,8 +638,48 @@ def stage_rooflines(cfg, layers, steps, stages, inner, peaks, peak_src, peak, pe
     return out
 
 
+def run_kernel(args):
+    """One kernel alone on a seeded input: --kernel covariance times
+    kronq_covariance of a (tokens x width) bf16 matrix (X drawn like the
+    workload's widest input site), after untimed warm-up launches."""
+    import numpy as np
+    import torch
+    import dataclasses
+    import synth
+    from post_quantization_02_b200 import abi
+    dev = torch.device("cuda", 0)
+    cfg = synth.get_config(args.config)
+    site = max(cfg.sites, key=lambda s_: s_.width)
+    if args.width:
+        site = dataclasses.replace(site, width=args.width)
+    tokens = args.tokens or 16384
+    cfg = dataclasses.replace(cfg, tokens=tokens)
+    X = torch.from_numpy(synth.make_x(cfg, site).view(np.int16)).to(dev).view(torch.bfloat16)
+    d = site.width
+    H = torch.empty((d, d), dtype=torch.float32, device=dev)
+    for _ in range(max(1, args.warmup)):
+        abi.kronq_covariance(X, H, 1.0 / tokens, 0.0)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        abi.kronq_covariance(X, H, 1.0 / tokens, 0.0)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    flops = tokens * d * d
+    peaks, src = load_peaks()
+    tf = flops / (ms / 1e3) / 1e12
+    print(json.dumps({"kernel": "kronq_covariance", "tokens": tokens, "width": d, "ms": ms,
+                      "tflops": tf, "frac_of_burst_peak": tf / float(peaks["bf16_tflops"]),
+                      "peak_source": src}), flush=True)
+
+
 def main():
     args = parse()
+    if args.kernel:
+        run_kernel(args)
+        return
     if args.deploy:
         run_deploy(args)
         return

@@ -301,6 +301,162 @@ row_fht_kernel(float* __restrict__ X, int R, int C, const float* __restrict__ rs
   }
 }
 
+// Row pass for widths with an odd factor (forward only), one row per CTA:
+// segment g of the row (L2 = 128 E entries) belongs to threads
+// [128 g, 128 g + 128), which transform it in registers exactly as
+// row_fht_kernel does (scaling and signs fused into the load), then leave it
+// in shared memory; after one barrier every thread mixes the Q segments at
+// its positions r (y[s L2 + r] = sum_t M[s][t] x[t L2 + r]) straight into
+// global memory.  One read and one write of the row, like the power-of-two
+// rows.
+template <int Q, int E>
+__global__ void __launch_bounds__(128 * Q, 1)
+row_fht_mix_kernel(float* __restrict__ X, int C, const float* __restrict__ rs,
+                   const float* __restrict__ cf, const float* __restrict__ M) {
+  constexpr int L2 = 128 * E;
+  constexpr int LD = L2 + L2 / 32;            // padded segment in shared memory
+  extern __shared__ float sm[];               // [Q][LD], then M (Q x Q)
+  float* Ms = sm + Q * LD;
+  const int tid = threadIdx.x, g = tid >> 7, t = tid & 127;
+  const int64_t row = blockIdx.x;
+  float* base = X + row * C;
+  if (tid < Q * Q) Ms[tid] = M[tid];
+  {
+    const int c0 = g * L2;
+    const float rsc = rs ? rs[row] : 1.f;
+    float v[E];
+#pragma unroll
+    for (int k = 0; k < E; ++k) {
+      const int c = c0 + t + 128 * k;
+      v[k] = base[c] * (rsc * cf[c]);
+    }
+#pragma unroll
+    for (int h = 1; h < E; h <<= 1)
+#pragma unroll
+      for (int k = 0; k < E; ++k)
+        if (!(k & h)) {
+          const float a = v[k], b = v[k + h];
+          v[k] = a + b;
+          v[k + h] = a - b;
+        }
+    float* seg = sm + g * LD;
+#pragma unroll
+    for (int k = 0; k < E; ++k) {
+      const int i = t + 128 * k;
+      seg[i + (i >> 5)] = v[k];
+    }
+    // the stages E <= h < L2 among the segment's 128 threads: a transpose
+    // within the segment (named barrier per segment: 4 warps)
+    asm volatile("bar.sync %0, 128;" ::"r"(g + 1) : "memory");
+#pragma unroll
+    for (int k = 0; k < E; ++k) {
+      const int i = E * t + k;
+      v[k] = seg[i + (i >> 5)];
+    }
+#pragma unroll
+    for (int h = 1; h < E; h <<= 1)
+#pragma unroll
+      for (int k = 0; k < E; ++k)
+        if (!(k & h)) {
+          const float a = v[k], b = v[k + h];
+          v[k] = a + b;
+          v[k + h] = a - b;
+        }
+#pragma unroll
+    for (int m = 1; m < 128 / E; m <<= 1) {
+      const bool upper = (t & m) != 0;
+#pragma unroll
+      for (int k = 0; k < E; ++k) {
+        const float o = __shfl_xor_sync(0xffffffffu, v[k], m);
+        v[k] = upper ? (o - v[k]) : (v[k] + o);
+      }
+    }
+    asm volatile("bar.sync %0, 128;" ::"r"(g + 1) : "memory");
+#pragma unroll
+    for (int k = 0; k < E; ++k) {
+      const int i = E * t + k;
+      seg[i + (i >> 5)] = v[k];
+    }
+  }
+  __syncthreads();
+  const float norm = rsqrtf((float)L2);
+  for (int r = tid; r < L2; r += 128 * Q) {
+    const int ri = r + (r >> 5);
+    float x[Q];
+#pragma unroll
+    for (int u = 0; u < Q; ++u) x[u] = sm[u * LD + ri];
+#pragma unroll
+    for (int s2 = 0; s2 < Q; ++s2) {
+      float acc = 0.f;
+#pragma unroll
+      for (int u = 0; u < Q; ++u) acc = fmaf(Ms[s2 * Q + u], x[u], acc);
+      base[s2 * L2 + r] = acc * norm;
+    }
+  }
+}
+
+// Column pass, last launch for heights with an odd factor (forward only): the
+// Walsh-Hadamard factor H_{NR} on the rows with stride st (as
+// col_fht_reg_kernel) for each of the Q segments, then the Q-mix across the
+// segments, in one read and one write.  Warp s of the CTA owns segment s
+// (32 columns, coalesced 128-byte row pieces); the transformed values meet in
+// shared memory for the mix.  first: the row signs before (when this launch
+// is the whole Walsh-Hadamard part); the 1/sqrt(L2) normalisation is applied.
+template <int Q, int LG>
+__global__ void __launch_bounds__(32 * Q)
+col_fht_mix_kernel(float* __restrict__ X, int C, int L2, int st, const int8_t* __restrict__ sign,
+                   const float* __restrict__ M, int first) {
+  constexpr int NR = 1 << LG;
+  extern __shared__ float dyn[];
+  float(*buf)[NR][33] = reinterpret_cast<float(*)[NR][33]>(dyn);   // [Q][NR][33]
+  float* Ms = dyn + Q * NR * 33;
+  const int lane = threadIdx.x & 31, s = threadIdx.x >> 5;
+  if (threadIdx.x < Q * Q) Ms[threadIdx.x] = M[threadIdx.x];
+  const int c = blockIdx.x * 32 + lane;
+  const bool live = c < C;
+  const int g = blockIdx.y;
+  const int hi = g / st, lo = g % st;
+  const int64_t r0 = (int64_t)hi * st * NR + lo;      // row within the segment
+  const int64_t step = (int64_t)st * C;
+  float v[NR];
+  {
+    const float* p = X + ((int64_t)s * L2 + r0) * C + (live ? c : 0);
+#pragma unroll
+    for (int j = 0; j < NR; ++j) {
+      v[j] = live ? *p : 0.f;
+      p += step;
+    }
+  }
+  if (first) {
+    const int8_t* sg = sign + (int64_t)s * L2 + r0;
+#pragma unroll
+    for (int j = 0; j < NR; ++j) v[j] = (sg[(int64_t)j * st] < 0) ? -v[j] : v[j];
+  }
+#pragma unroll
+  for (int h = 1; h < NR; h <<= 1)
+#pragma unroll
+    for (int j = 0; j < NR; ++j)
+      if (!(j & h)) {
+        const float a = v[j], b = v[j + h];
+        v[j] = a + b;
+        v[j + h] = a - b;
+      }
+#pragma unroll
+  for (int j = 0; j < NR; ++j) buf[s][j][lane] = v[j];
+  __syncthreads();
+  if (!live) return;
+  const float norm = rsqrtf((float)L2);
+  float* p = X + ((int64_t)s * L2 + r0) * C + c;
+#pragma unroll 4
+  for (int j = 0; j < NR; ++j) {
+    float acc = 0.f;
+#pragma unroll
+    for (int u = 0; u < Q; ++u) acc = fmaf(Ms[s * Q + u], buf[u][j][lane], acc);
+    *p = acc * norm;
+    p += step;
+  }
+}
+
 // cf[c] = cs[c] sign[c] (cs may be null: 1).
 __global__ void col_factor_kernel(const float* __restrict__ cs, const int8_t* __restrict__ sign,
                                   int C, float* __restrict__ cf) {
@@ -395,15 +551,22 @@ __global__ void __launch_bounds__(1024) sensitivity_kernel(const float* __restri
 
 size_t a256(size_t b) { return (b + 255) & ~(size_t)255; }
 
-bool g_row_attr = false;
+kqh::PerDevice g_row_attr;
 
 int set_attrs() {
-  if (!g_row_attr) {
-    if (cudaFuncSetAttribute(row_transform_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             200 * 1024) != cudaSuccess)
-      return KRONQ_ERR_CUDA;
-    g_row_attr = true;
-  }
+  return kqh::smem_attr_once(g_row_attr, row_transform_kernel, 200 * 1024) > 0 ? KRONQ_OK
+                                                                                : KRONQ_ERR_CUDA;
+}
+
+template <int Q, int E>
+int launch_row_fht_mix(float* X, int R, int C, const float* rs, const float* cf, const float* M,
+                       cudaStream_t st) {
+  constexpr int LD = 128 * E + 4 * E;
+  const int smem = (Q * LD + Q * Q) * (int)sizeof(float);
+  static kqh::PerDevice attr;
+  if (kqh::smem_attr_once(attr, row_fht_mix_kernel<Q, E>, smem) <= 0) return KRONQ_ERR_CUDA;
+  row_fht_mix_kernel<Q, E><<<R, 128 * Q, smem, st>>>(X, C, rs, cf, M);
+  KQ_CHECK_LAUNCH();
   return KRONQ_OK;
 }
 
@@ -425,6 +588,19 @@ int row_pass(float* X, int R, int C, const float* rs, const float* cs, const int
     }
     KQ_CHECK_LAUNCH();
     return KRONQ_OK;
+  }
+  if (!inverse && (sp.Q == 7 || sp.Q == 2) && (sp.L2 == 2048 || sp.L2 == 4096)) {
+    // a factor 7 (widths 14336, 28672) or a second 4096 segment (8192): one
+    // fused pass (for Q = 2 the "mix" is the last Walsh-Hadamard stage)
+    if (!cf_ready) {
+      col_factor_kernel<<<(C + 255) / 256, 256, 0, st>>>(cs, sign, C, cf);
+      KQ_CHECK_LAUNCH();
+    }
+    if (sp.Q == 7)
+      return sp.L2 == 4096 ? launch_row_fht_mix<7, 32>(X, R, C, rs, cf, M, st)
+                           : launch_row_fht_mix<7, 16>(X, R, C, rs, cf, M, st);
+    return sp.L2 == 4096 ? launch_row_fht_mix<2, 32>(X, R, C, rs, cf, M, st)
+                         : launch_row_fht_mix<2, 16>(X, R, C, rs, cf, M, st);
   }
   const size_t smem = (size_t)C * sizeof(float);
   if (smem > 200 * 1024) return KRONQ_ERR_UNSUPPORTED;
@@ -453,8 +629,40 @@ int col_fht_launch(float* X, int R, int C, int L2, int lg, int stride, const int
 // Apply T D along columns of an R x C matrix (R = Q * L2): the Hadamard part
 // as H_{2^a} within groups of 2^a consecutive rows, then (when L2 > 64)
 // H_{L2 / 2^a} across them; the odd factor as a Q x Q mix of the segments.
+template <int Q, int LG>
+int col_fht_mix_launch_lg(float* X, int C, int L2, int stride, const int8_t* sign, const float* M,
+                          int first, cudaStream_t st) {
+  const int smem = (Q * (1 << LG) * 33 + Q * Q) * (int)sizeof(float);
+  static kqh::PerDevice attr;
+  if (kqh::smem_attr_once(attr, col_fht_mix_kernel<Q, LG>, smem) <= 0) return KRONQ_ERR_CUDA;
+  const dim3 g((C + 31) / 32, L2 >> LG);
+  col_fht_mix_kernel<Q, LG><<<g, 32 * Q, smem, st>>>(X, C, L2, stride, sign, M, first);
+  KQ_CHECK_LAUNCH();
+  return KRONQ_OK;
+}
+
+template <int Q>
+int col_fht_mix_launch(float* X, int C, int L2, int lg, int stride, const int8_t* sign,
+                       const float* M, int first, cudaStream_t st) {
+  switch (lg) {
+    case 5: return col_fht_mix_launch_lg<Q, 5>(X, C, L2, stride, sign, M, first, st);
+    case 6: return col_fht_mix_launch_lg<Q, 6>(X, C, L2, stride, sign, M, first, st);
+    default: return KRONQ_ERR_UNSUPPORTED;
+  }
+}
+
 int col_pass(float* X, int R, int C, const int8_t* sign, const Split& sp, const float* M,
              int inverse, cudaStream_t st) {
+  if (!inverse && (sp.Q == 7 || sp.Q == 2) && (sp.L2 == 2048 || sp.L2 == 4096)) {
+    // heights 14336, 28672 (factor 7) and 8192 (two 4096 segments): H_64 on
+    // consecutive rows, then H_{L2/64} with stride 64 fused with the mix of
+    // the segments
+    const int k2 = 31 - __builtin_clz((unsigned)sp.L2);
+    int s = col_fht_launch(X, R, C, sp.L2, 6, 1, sign, 1, 0, 0, st);
+    if (s != KRONQ_OK) return s;
+    return sp.Q == 7 ? col_fht_mix_launch<7>(X, C, sp.L2, k2 - 6, 64, sign, M, 0, st)
+                     : col_fht_mix_launch<2>(X, C, sp.L2, k2 - 6, 64, sign, M, 0, st);
+  }
   if (inverse && sp.Q > 1) {
     col_mix_kernel<<<dim3((C + 63) / 64, sp.L2), 64, 0, st>>>(X, C, sp.L2, sp.Q, M, 1);
     KQ_CHECK_LAUNCH();
@@ -651,3 +859,44 @@ int kq_vec_transform(float* X, int64_t R, int64_t C, const float* S, const int8_
   return row_pass(X, (int)R, (int)C, nullptr, rS, sign, sp, M, inverse, cf, st, /*cf_ready=*/true);
 }
 
+
+// ---------------------------------------------------------------------------
+// The input side of BiIP applied to another n x n matrix built from input
+// vectors (the drift covariance of the asymmetric calibration):
+// A <- V S_X^-1 A S_X^-1 V^T with the S_X and V of H_X; mode as in
+// kq_biip_rotate (the output side is not touched).
+int kq_biip_rotate_input(float* A, int64_t n64, const float* SX, const int8_t* sv, int mode,
+                         void* ws, size_t ws_bytes, cudaStream_t st) {
+  if (mode < 0 || mode > 3 || !A || !SX || !sv || n64 <= 0) return KRONQ_ERR_INVALID_ARG;
+  if (n64 % 16) return KRONQ_ERR_INVALID_ARG;
+  if (n64 > 65536) return KRONQ_ERR_UNSUPPORTED;
+  Split spn;
+  if (!split_width(n64, spn)) return KRONQ_ERR_UNSUPPORTED;
+  if (!ws || ws_bytes < kq_biip_ws(n64, n64) || !kqh::aligned(ws, 256)) return KRONQ_ERR_WORKSPACE;
+  int s0 = set_attrs();
+  if (s0 != KRONQ_OK) return s0;
+  const int n = (int)n64;
+  const bool in_s = mode == 0 || mode == 3, in_r = mode != 2;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  float* rSX = reinterpret_cast<float*>(w);
+  w += a256((size_t)n * sizeof(float));
+  float* cf = reinterpret_cast<float*>(w);
+  w += a256((size_t)n * sizeof(float));
+  float* Mn = reinterpret_cast<float*>(w);
+  recip_kernel<<<(n + 255) / 256, 256, 0, st>>>(SX, rSX, n);
+  KQ_CHECK_LAUNCH();
+  if (in_r) {
+    if (spn.Q > 1) {
+      make_mix_kernel<<<1, 256, 0, st>>>(Mn, spn.q, spn.k1);
+      KQ_CHECK_LAUNCH();
+    }
+    int s = row_pass(A, n, n, in_s ? rSX : nullptr, in_s ? rSX : nullptr, sv, spn, Mn, 0, cf, st);
+    if (s) return s;
+    return col_pass(A, n, n, sv, spn, Mn, 0, st);
+  }
+  if (in_s) {
+    scale_only_kernel<<<4 * kqh::num_sms(), 256, 0, st>>>(A, n, n, rSX, rSX);
+    KQ_CHECK_LAUNCH();
+  }
+  return KRONQ_OK;
+}

@@ -317,10 +317,12 @@ KQ_DEV void put_split(float* hi_plane, float* lo_plane, int64_t idx, float v) {
 // Panel step p (rows / columns k = 128 p ...) of the padded np x np matrices,
 // in 32-row slices ("tiles", PR rows each):
 //   tile t < tiles_L:          L_ip = R_ip L_pp^-T for rows k+128+32t ..
-//                              -> the hi / lo planes Lh, Ll (np x 128, row 0 = row k+128)
+//                              -> the hi / lo planes Lh, Ll
 //   tile tiles_L + j, j < 4p:  Z_jp = B_jp L_pp^-T for Z rows 32j .. -> Z and the
-//                              planes Zh, Zl (row = Z row)
+//                              planes Zh, Zl
 //   tile tiles_L + 4p (last):  Z_pp = L_pp^-T      -> Z and the planes
+// The planes are np x ldp, indexed by matrix row; the panel's 128 columns go
+// to plane columns pc .. pc + 127 (its place in the current super-block).
 // At most one CTA per SM: each factors and inverts the diagonal block once in
 // shared memory, then takes tiles t = blockIdx.x, + gridDim.x, ... (the
 // first slice is fetched by bulk copies during the factorisation, each
@@ -329,8 +331,8 @@ constexpr int PR = 32;
 
 __global__ void __launch_bounds__(PANEL_THREADS, 1) panel_kernel(const float* R, float* Z, float* Lh,
                                                     float* Ll, float* Zh, float* Zl, int np, int k,
-                                                    int p, int tiles_L, int tiles_total,
-                                                    int32_t* info) {
+                                                    int p, int tiles_L, int tiles_total, int ldp,
+                                                    int pc, int32_t* info) {
   extern __shared__ __align__(16) float sm[];
   float* D = sm + SM_D;
   float* X = sm + SM_X;
@@ -404,7 +406,7 @@ __global__ void __launch_bounds__(PANEL_THREADS, 1) panel_kernel(const float* R,
         const int a = e / NB, c = e % NB;
         const float v = X[c * LDX + a];
         Z[(int64_t)(k + a) * np + k + c] = v;
-        put_split(Zh, Zl, (int64_t)(k + a) * NB + c, v);
+        put_split(Zh, Zl, (int64_t)(k + a) * ldp + pc + c, v);
       }
       break;                          // the last tile
     }
@@ -442,9 +444,9 @@ __global__ void __launch_bounds__(PANEL_THREADS, 1) panel_kernel(const float* R,
     if (t < tiles_L) {
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
-        const int64_t r = (int64_t)PR * t + ty + 16 * i;   // plane row
+        const int64_t r = (int64_t)k + NB + PR * t + ty + 16 * i;   // matrix row
 #pragma unroll
-        for (int jj = 0; jj < 8; ++jj) put_split(Lh, Ll, r * NB + tx + 16 * jj, acc[i][jj]);
+        for (int jj = 0; jj < 8; ++jj) put_split(Lh, Ll, r * ldp + pc + tx + 16 * jj, acc[i][jj]);
       }
     } else {
       const int j = t - tiles_L;
@@ -455,7 +457,7 @@ __global__ void __launch_bounds__(PANEL_THREADS, 1) panel_kernel(const float* R,
         for (int jj = 0; jj < 8; ++jj) {
           const int c = tx + 16 * jj;
           Z[r * np + k + c] = acc[i][jj];
-          put_split(Zh, Zl, r * NB + c, acc[i][jj]);
+          put_split(Zh, Zl, r * ldp + pc + c, acc[i][jj]);
         }
       }
     }
@@ -492,10 +494,16 @@ int64_t padded(int64_t n) { return (n + NB - 1) / NB * NB; }
 
 }  // namespace
 
+// Super-block width of the two-level sweep: its panels update only the
+// super-block's own columns; the trailing matrix gets one K = SBW update.
+constexpr int SBW = 1024;
+
+int64_t plane_ld(int64_t np) { return np < SBW ? np : SBW; }
+
 size_t kq_cholesky_ws(int64_t n) {
   const int64_t np = padded(n);
   return align256(sizeof(double)) + 2 * align256((size_t)np * np * sizeof(float)) +
-         4 * align256((size_t)np * NB * sizeof(float));
+         4 * align256((size_t)np * plane_ld(np) * sizeof(float));
 }
 
 int kq_cholesky_inv(const float* H, int64_t n64, float damp_rel, float* U, int32_t* info, void* ws,
@@ -517,9 +525,10 @@ int kq_cholesky_inv(const float* H, int64_t n64, float damp_rel, float* U, int32
   float* Z = reinterpret_cast<float*>(w);
   w += align256((size_t)np * np * sizeof(float));
   float* planes[4];
+  const int ldp = (int)plane_ld(np);
   for (int i = 0; i < 4; ++i) {
     planes[i] = reinterpret_cast<float*>(w);
-    w += align256((size_t)np * NB * sizeof(float));
+    w += align256((size_t)np * ldp * sizeof(float));
   }
   float *Lh = planes[0], *Ll = planes[1], *Zh = planes[2], *Zl = planes[3];
 
@@ -528,25 +537,57 @@ int kq_cholesky_inv(const float* H, int64_t n64, float damp_rel, float* U, int32
   KQ_CHECK_LAUNCH();
   reverse_damp_kernel<<<4 * sms, 256, 0, st>>>(H, n, np, R, Z, damp_rel, dsum);
   KQ_CHECK_LAUNCH();
-  const int nblk = np / NB;
-  for (int p = 0; p < nblk; ++p) {
-    const int k = p * NB;
-    const int rest = np - k - NB;
-    const int tiles_L = rest / PR;
-    const int tiles_total = tiles_L + 4 * p + 1;
-    const int grid = tiles_total < sms ? tiles_total : sms;
-    panel_kernel<<<grid, PANEL_THREADS, kPanelSmem, st>>>(R, Z, Lh, Ll, Zh, Zl, np, k, p, tiles_L,
-                                                          tiles_total, info);
-    KQ_CHECK_LAUNCH();
+  for (int kb = 0; kb < np; kb += ldp) {
+    const int kb_end = kb + ldp < np ? kb + ldp : np;
+    // the Z planes of the super-block's columns are read down to row kb_end
+    // by its trailing update: the rows below each panel's block are zero
+    const size_t zrows = (size_t)(kb_end - kb) * ldp * sizeof(float);
+    if (cudaMemsetAsync(Zh + (size_t)kb * ldp, 0, zrows, st) != cudaSuccess ||
+        cudaMemsetAsync(Zl + (size_t)kb * ldp, 0, zrows, st) != cudaSuccess)
+      return KRONQ_ERR_CUDA;
+    for (int k = kb; k < kb_end; k += NB) {
+      const int p = k / NB, pc = k - kb;
+      const int below = np - k - NB;
+      const int tiles_L = below / PR;
+      const int tiles_total = tiles_L + 4 * p + 1;
+      const int grid = tiles_total < sms ? tiles_total : sms;
+      const int tp = kqh::timer_begin(KRONQ_TIMER_CHOL_PANEL, st);
+      panel_kernel<<<grid, PANEL_THREADS, kPanelSmem, st>>>(R, Z, Lh, Ll, Zh, Zl, np, k, p,
+                                                            tiles_L, tiles_total, ldp, pc, info);
+      kqh::timer_end(tp, st);
+      KQ_CHECK_LAUNCH();
+      const int inner = kb_end - k - NB;      // the super-block's columns after this panel
+      if (inner > 0) {
+        // inside the super-block, on the tensor cores (B = the panel rows L_ip):
+        //   R[k+128:, k+128:kb_end] -= L L[k+128:kb_end]^T   (every row below; the
+        //                                                      part above the diagonal is unused)
+        //   Z[:k+128, k+128:kb_end] -= Z[:k+128, k:k+128] L[k+128:kb_end]^T
+        const int64_t lr = (int64_t)(k + NB) * ldp + pc;
+        kq::GemmNT g[2];
+        g[0] = {Lh + lr, Ll + lr, ldp, Lh + lr, Ll + lr, ldp, R + (int64_t)(k + NB) * np + (k + NB),
+                np, below, inner, NB, -1.f, 0};
+        g[1] = {Zh + pc, Zl + pc, ldp, Lh + lr, Ll + lr, ldp, Z + (k + NB), np, k + NB, inner, NB,
+                -1.f, 0};
+        const int tu = kqh::timer_begin(KRONQ_TIMER_CHOL_UPDATE, st);
+        const int s = kq_gemm_nt_tc(g, 2, info, st);
+        kqh::timer_end(tu, st);
+        if (s != KRONQ_OK) return s;
+      }
+    }
+    const int rest = np - kb_end;
     if (rest > 0) {
-      // trailing update on the tensor cores, B = the panel rows L_ip (planes):
-      //   R[k+128:, k+128:] -= L L^T                 (lower triangle)
-      //   Z[:k+128, k+128:] -= Z[:k+128, k:k+128] L^T
+      // the trailing matrix, once per super-block (K = kb_end - kb):
+      //   R[kb_end:, kb_end:] -= L L^T (lower triangle),  L = L[kb_end:, kb:kb_end]
+      //   Z[:kb_end, kb_end:] -= Z[:kb_end, kb:kb_end] L^T
+      const int K = kb_end - kb;
+      const int64_t lr = (int64_t)kb_end * ldp;
       kq::GemmNT g[2];
-      g[0] = {Lh, Ll, NB, Lh, Ll, NB, R + (int64_t)(k + NB) * np + (k + NB), np, rest, rest, NB,
-              -1.f, 1};
-      g[1] = {Zh, Zl, NB, Lh, Ll, NB, Z + (k + NB), np, k + NB, rest, NB, -1.f, 0};
+      g[0] = {Lh + lr, Ll + lr, ldp, Lh + lr, Ll + lr, ldp, R + (int64_t)kb_end * np + kb_end, np,
+              rest, rest, K, -1.f, 1};
+      g[1] = {Zh, Zl, ldp, Lh + lr, Ll + lr, ldp, Z + kb_end, np, kb_end, rest, K, -1.f, 0};
+      const int tu = kqh::timer_begin(KRONQ_TIMER_CHOL_UPDATE, st);
       const int s = kq_gemm_nt_tc(g, 2, info, st);
+      kqh::timer_end(tu, st);
       if (s != KRONQ_OK) return s;
     }
   }

@@ -297,6 +297,13 @@ unsigned long long launches();
 int launch_status();        // KRONQ_ERR_CUDA if the last launch failed, else KRONQ_OK;
                             // also counts the launch (kronq_launch_count)
 
+// Optional CUDA-event timing of selected launches (kronq_timing_enable):
+// timer_begin records a start event on `st` for the category (a
+// kronq_timer value) and returns a slot, or -1 when timing is off or an event
+// cannot be had; timer_end records the slot's end event on the same stream.
+int timer_begin(int category, cudaStream_t st);
+void timer_end(int slot, cudaStream_t st);
+
 // One-time set-up per device (a kernel's shared-memory attribute, an
 // occupancy figure): cudaFuncSetAttribute and occupancy queries apply to the
 // current device only, so a process that drives several GPUs needs each

@@ -356,17 +356,44 @@ struct PairBars {
   int abort;
 };
 
-// Square tiles in the upper triangle, ordered by column block: column block
-// cb holds the row blocks 0 .. cb, i.e. cb (cb + 1) / 2 tiles precede it.
-__device__ __forceinline__ void pair_tile_coords(int t, int& rb, int& cb) {
-  int c = (int)((sqrt(8.0 * (double)t + 1.0) - 1.0) * 0.5);
-  while ((long long)(c + 1) * (c + 2) / 2 <= t) ++c;
-  while ((long long)c * (c + 1) / 2 > t) --c;
-  cb = c;
-  rb = t - c * (c + 1) / 2;
+// Tiles per side of a super-block of the tile order below.
+constexpr int P_SB = 8;
+
+// Square tiles (rb <= cb) of the upper triangle of an nb x nb tile grid, in
+// super-blocks of P_SB x P_SB tiles: super-columns J in order; in each, the
+// super-blocks I = 0 .. J -- row-major inside an off-diagonal one, column by
+// column inside the diagonal one.  The pairs of one wave take consecutive
+// tiles at the same token offset, so with this order a wave's tiles span
+// about 2 P_SB row and column panels (instead of a whole column of the
+// triangle, i.e. most of the panels): each token slab a wave needs leaves
+// DRAM once for a few panels, which L2 then serves to every pair.
+__device__ __forceinline__ void pair_tile_coords(int t, int nb, int& rb, int& cb) {
+  const int nsb = (nb + P_SB - 1) / P_SB;
+  int J = 0, base = 0, w = 0;
+  for (;; ++J) {
+    w = min(P_SB, nb - J * P_SB);
+    const int cnt = J * P_SB * w + w * (w + 1) / 2;
+    if (t < base + cnt || J >= nsb - 1) break;
+    base += cnt;
+  }
+  int u = t - base;
+  const int off = J * P_SB * w;
+  if (u < off) {
+    const int I = u / (P_SB * w), v = u - I * (P_SB * w);
+    rb = I * P_SB + v / w;
+    cb = J * P_SB + v % w;
+  } else {
+    u -= off;
+    int c = (int)((sqrtf(8.f * (float)u + 1.f) - 1.f) * 0.5f);
+    while ((c + 1) * (c + 2) / 2 <= u) ++c;
+    while (c * (c + 1) / 2 > u) --c;
+    rb = J * P_SB + (u - c * (c + 1) / 2);
+    cb = J * P_SB + c;
+  }
 }
 
 struct PairSchedule {
+  int nb;              // tiles per side of the tile grid
   int tiles, chunks;   // T, C
   int waves, rest;     // W = T / P, R = T mod P
   int per_helper;      // g
@@ -440,7 +467,7 @@ cov_pair_kernel(const __grid_constant__ CUtensorMap tmap, float* __restrict__ H,
       int t, c0, c1;
       for (int sg = 0; pair_segment(sched, cid, ncl, sg, t, c0, c1); ++sg) {
         int rb, cb;
-        pair_tile_coords(t, rb, cb);
+        pair_tile_coords(t, sched.nb, rb, cb);
         const int i0 = rb * P_TILE + P_BM * (int)rank;          // this CTA's rows of the tile
         const int j0 = cb * P_TILE + (P_TILE / 2) * (int)rank;  // this CTA's half of the columns
         bool ok = true;
@@ -513,7 +540,7 @@ cov_pair_kernel(const __grid_constant__ CUtensorMap tmap, float* __restrict__ H,
     for (int sg = 0; ok && pair_segment(sched, cid, ncl, sg, t, c0, c1); ++sg) {
       const bool shared_tile = c0 > 0 || c1 < sched.chunks;   // another pair adds the rest
       int rb, cb;
-      pair_tile_coords(t, rb, cb);
+      pair_tile_coords(t, sched.nb, rb, cb);
       const int i0 = rb * P_TILE + P_BM * (int)rank, j0 = cb * P_TILE;
       const int row0 = i0 + q * 32;
       const int row = row0 + lane;
@@ -570,6 +597,7 @@ cov_pair_kernel(const __grid_constant__ CUtensorMap tmap, float* __restrict__ H,
 // The square tiles several pairs shared (at most one per pair boundary).
 constexpr int kMaxSharedTiles = 256;
 struct SharedTiles {
+  int nb;      // tiles per side of the tile grid
   int count;
   int tile[kMaxSharedTiles];
 };
@@ -582,7 +610,7 @@ __global__ void __launch_bounds__(256) mirror_tiles_kernel(float* __restrict__ H
   __shared__ float tile[32][33];
   const int li = blockIdx.x >> 6, sb = blockIdx.x & 63;
   int rb, cb;
-  pair_tile_coords(st.tile[li], rb, cb);
+  pair_tile_coords(st.tile[li], st.nb, rb, cb);
   const int i0 = rb * P_TILE + (sb >> 3) * 32, j0 = cb * P_TILE + (sb & 7) * 32;   // source block
   if (i0 >= d || j0 >= d || j0 + 31 < i0) return;                                  // nothing above the diagonal
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
@@ -605,7 +633,7 @@ __global__ void __launch_bounds__(256) scale_tiles_kernel(float* __restrict__ H,
                                                           const __grid_constant__ SharedTiles st) {
   const int li = blockIdx.x >> 6, sb = blockIdx.x & 63;
   int rb, cb;
-  pair_tile_coords(st.tile[li], rb, cb);
+  pair_tile_coords(st.tile[li], st.nb, rb, cb);
   const int i0 = rb * P_TILE + (sb >> 3) * 32, j0 = cb * P_TILE + (sb & 7) * 32;
   if (i0 >= d || j0 >= d) return;
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
@@ -706,6 +734,7 @@ int kq_covariance(const uint16_t* A, int64_t N, int64_t d, int64_t lda, float* H
     });
     if (P <= 0) return KRONQ_ERR_CUDA;
     PairSchedule sc;
+    sc.nb = ncb2;
     sc.tiles = tiles2;
     sc.chunks = (k_iters + KC_ITERS - 1) / KC_ITERS;
     sc.waves = tiles2 / P;
@@ -716,6 +745,7 @@ int kq_covariance(const uint16_t* A, int64_t N, int64_t d, int64_t lda, float* H
     if (sc.kstar > sc.chunks) sc.kstar = sc.chunks;
     // the split tiles: the R tiles of the last, partial wave when helpers take their tail
     SharedTiles list;
+    list.nb = ncb2;
     list.count = 0;
     if (sc.rest > 0 && sc.kstar < sc.chunks) {
       if (sc.rest > kMaxSharedTiles) return KRONQ_ERR_UNSUPPORTED;

@@ -319,7 +319,7 @@ def test_bounded_wait_times_out_and_context_survives(cuda):
     assert info.item() == -5
     # the context is still usable
     codes = torch.ones((2, 16), dtype=torch.uint8, device=cuda)
-    packed = torch.zeros((2, 2), dtype=torch.int32, device=cuda)
+    packed = torch.zeros((2, 1), dtype=torch.int32, device=cuda)
     abi.kronq_pack(codes, 2, packed)
     torch.cuda.synchronize()
     assert packed[0, 0].item() == 0x55555555
