@@ -313,6 +313,57 @@ int kronq_quantize_layer_noalloc(float* W, int64_t m, int64_t n, const float* U_
                                  int32_t* info, void* stream);
 
 /*
+ * GPTAQ asymmetric calibration (optional: the drift-corrected objective).
+ *
+ * KronQ summary (hyper.ai), "Method": building on GPTAQ, the objective is
+ * corrected for input drift -- the quantized layer sees X~ (its input in
+ * the partly quantized model) while its target is the full-precision W X.
+ * KronQ review (pith.science), appendix, Algorithm 2, step 3:
+ * P = alpha (Delta X X^T L) (.) M_U L^T, L <- InverseCholesky(H_X), M_U the
+ * upper-triangular mask.  Readings: Delta X = X - X~; the solver's H_X is
+ * the covariance of X~; L = U_c^T (H_d^-1 = L L^T); M_U keeps the diagonal;
+ * after column p is quantized, each later column k receives
+ * -delta_p U_c[p][k] + w_p P[p][k] with w_p the value the quantizer saw.
+ * Sequence: kronq_drift_covariance -> kronq_biip_rotate (on W, H~, H_G) ->
+ * kronq_biip_rotate_input (on Delta X X^T, with that call's S_X) ->
+ * kronq_cholesky_inv (on H~') -> kronq_gptaq_correction ->
+ * kronq_quantize_layer_gptaq.  Workspace: kronq_gptaq_workspace_size bytes
+ * (it covers every call of the sequence).
+ */
+size_t kronq_gptaq_workspace_size(int64_t m, int64_t n);
+
+/* H = X~^T X~ / N and A = (X - X~)^T X~ / N (both n x n fp32, full) from the
+ * two calibration inputs side by side: XqX is N x 2n bf16 (row stride ld
+ * >= 2n elements, 16-byte aligned rows), row t = [x~_t, x_t].  One
+ * covariance of the 2n-wide rows (into the workspace), then the two blocks;
+ * A is the difference of two fp32 sums, so its absolute error is that of H
+ * (about 1e-5 of |H|).  Errors as kronq_covariance. */
+int kronq_drift_covariance(const void* XqX, int64_t N, int64_t n, int64_t ld, float* H, float* A,
+                           int32_t* info, void* ws, size_t ws_bytes, void* stream);
+
+/* The input side of BiIP applied to A (n x n fp32, in place):
+ * A <- V S_X^-1 A S_X^-1 V^T with the S_X a kronq_biip_rotate call returned
+ * and its sign_v; mode as there (SU_ONLY leaves A unchanged, NO_RESCALE
+ * only rotates, SV_ONLY and FULL rescale and rotate). */
+int kronq_biip_rotate_input(float* A, int64_t n, const float* S_X, const int8_t* sign_v, int mode,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/* P (n x n fp32 out, upper triangular) = alpha ((A U_c^T) (.) M_U) U_c, i.e.
+ * alpha (Delta X X^T L) (.) M_U L^T with L = U_c^T; tensor-core products at
+ * fp32 accuracy.  n a multiple of 4, at most 32768; pointers 16-byte
+ * aligned; P must not alias A or U_c. */
+int kronq_gptaq_correction(const float* A, const float* U_c, int64_t n, float alpha, float* P,
+                           int32_t* info, void* ws, size_t ws_bytes, void* stream);
+
+/* kronq_quantize_layer with the GPTAQ term P (n x n fp32, from
+ * kronq_gptaq_correction): same arguments otherwise; group -1 or 128;
+ * n <= 32768.  With P = 0 the codes are those of kronq_quantize_layer. */
+int kronq_quantize_layer_gptaq(float* W, int64_t m, int64_t n, const float* U_c, const float* P,
+                               int bits, int group, int block,
+                               uint8_t* codes, float* scales, uint8_t* zeros, float* W_hat,
+                               int32_t* info, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * Pack b-bit codes into 32-bit words (b = 2 or 4).
  *
  * KronQ README (GitHub), "Model zoo": W4 / W2 stored as packed int4 / int2;

@@ -63,6 +63,11 @@ def lib() -> ctypes.CDLL:
         "kronq_unpack": ([P, I64, I64, I32, P, P], I32),
         "kronq_layer_loss": ([P, P, I64, I64, P, P, P, P, SZ, P], I32),
         "kronq_selftest_wait": ([P, I64, P], I32),
+        "kronq_gptaq_workspace_size": ([I64, I64], SZ),
+        "kronq_drift_covariance": ([P, I64, I64, I64, P, P, P, P, SZ, P], I32),
+        "kronq_biip_rotate_input": ([P, I64, P, P, I32, P, SZ, P], I32),
+        "kronq_gptaq_correction": ([P, P, I64, F32, P, P, P, SZ, P], I32),
+        "kronq_quantize_layer_gptaq": ([P, I64, I64, P, P, I32, I32, I32, P, P, P, P, P, P, SZ, P], I32),
         "kronq_timing_enable": ([I32], I32),
         "kronq_timing_read": ([I32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_uint64)], I32),
     }
@@ -400,6 +405,82 @@ def kronq_layer_loss(W_ref, W_hat, HX, HG, out, ws, stream=None):
     _check("kronq_layer_loss", lib().kronq_layer_loss(
         _p(W_ref), _p(W_hat), m, n, _p(HX), _p(HG), _p(out), _p(ws),
         ws.numel() * ws.element_size(), _s(stream)))
+
+
+# ------------------------------------------------ GPTAQ asymmetric calibration
+def kronq_gptaq_workspace_size(m: int, n: int) -> int:
+    return int(lib().kronq_gptaq_workspace_size(m, n))
+
+
+def gptaq_workspace(m: int, n: int, device=None):
+    return torch.empty(max(kronq_gptaq_workspace_size(m, n), 256), dtype=torch.uint8,
+                       device=device or "cuda")
+
+
+def kronq_drift_covariance(XqX, H, A, info=None, ws=None, stream=None):
+    """H = X~^T X~ / N, A = (X - X~)^T X~ / N from XqX = [X~ | X] (N x 2n bf16)."""
+    _dev(XqX, (torch.bfloat16, torch.int16, torch.uint16), "XqX", 2)
+    _dev(H, torch.float32, "H", 2)
+    _dev(A, torch.float32, "A", 2)
+    _dev(info, torch.int32, "info")
+    N, w2 = XqX.shape
+    if w2 % 2:
+        raise ValueError("XqX must have an even width (X~ then X)")
+    n = w2 // 2
+    _shape(H, (n, n), "H")
+    _shape(A, (n, n), "A")
+    _on_current_device((XqX, "XqX"), (H, "H"), (A, "A"), (info, "info"), (ws, "ws"))
+    if XqX.stride(1) != 1:
+        raise ValueError("XqX needs unit stride along its last dimension")
+    _contig(H, "H"); _contig(A, "A")
+    _check("kronq_drift_covariance", lib().kronq_drift_covariance(
+        _p(XqX), N, n, XqX.stride(0) if N > 0 else w2, _p(H), _p(A), _p(info), _p(ws),
+        0 if ws is None else ws.numel() * ws.element_size(), _s(stream)))
+
+
+def kronq_biip_rotate_input(A, SX, sign_v, mode, ws, stream=None):
+    _dev(A, torch.float32, "A", 2)
+    _dev(SX, torch.float32, "S_X")
+    _dev(sign_v, torch.int8, "sign_v")
+    n = A.shape[0]
+    _shape(A, (n, n), "A")
+    _numel(SX, n, "S_X")
+    _numel(sign_v, n, "sign_v")
+    _on_current_device((A, "A"), (SX, "S_X"), (sign_v, "sign_v"), (ws, "ws"))
+    _contig(A, "A")
+    md = MODES[mode] if isinstance(mode, str) else int(mode)
+    _check("kronq_biip_rotate_input", lib().kronq_biip_rotate_input(
+        _p(A), n, _p(SX), _p(sign_v), md, _p(ws),
+        0 if ws is None else ws.numel() * ws.element_size(), _s(stream)))
+
+
+def kronq_gptaq_correction(A, U, alpha: float, P, info=None, ws=None, stream=None):
+    for t, nm in ((A, "A"), (U, "U_c"), (P, "P")):
+        _dev(t, torch.float32, nm, 2)
+    n = A.shape[0]
+    for t, nm in ((A, "A"), (U, "U_c"), (P, "P")):
+        _shape(t, (n, n), nm)
+    _dev(info, torch.int32, "info")
+    _on_current_device((A, "A"), (U, "U_c"), (P, "P"), (info, "info"), (ws, "ws"))
+    for t, nm in ((A, "A"), (U, "U_c"), (P, "P")):
+        _contig(t, nm)
+    _check("kronq_gptaq_correction", lib().kronq_gptaq_correction(
+        _p(A), _p(U), n, alpha, _p(P), _p(info), _p(ws),
+        0 if ws is None else ws.numel() * ws.element_size(), _s(stream)))
+
+
+def kronq_quantize_layer_gptaq(W, U, P, bits: int, group: int, block: int, codes, scales, zeros,
+                               W_hat=None, info=None, ws=None, stream=None):
+    m, n = _quant_args(W, U, codes, scales, zeros, W_hat, group)
+    _dev(P, torch.float32, "P", 2)
+    _shape(P, (n, n), "P")
+    _dev(info, torch.int32, "info")
+    _on_current_device((P, "P"), (info, "info"), (ws, "ws"))
+    _contig(P, "P")
+    _check("kronq_quantize_layer_gptaq", lib().kronq_quantize_layer_gptaq(
+        _p(W), m, n, _p(U), _p(P), bits, group, block, _p(codes), _p(scales), _p(zeros),
+        _p(W_hat), _p(info), _p(ws), 0 if ws is None else ws.numel() * ws.element_size(),
+        _s(stream)))
 
 
 TIMERS = {"lazy_update": 0, "chol_update": 1, "chol_panel": 2, "obs_block": 3}

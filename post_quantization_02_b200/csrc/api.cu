@@ -36,6 +36,19 @@ int kq_quantize_layer_noalloc(float* W, int64_t m, int64_t n, const float* U, in
                               float* W_hat, int32_t* info, cudaStream_t st);
 int kq_pack(const uint8_t* codes, int64_t m, int64_t n, int bits, uint32_t* packed,
             cudaStream_t st);
+size_t kq_drift_ws(int64_t n);
+size_t kq_correction_ws(int64_t n);
+size_t kq_quantize_asym_ws(int64_t m, int64_t n);
+int kq_drift_covariance(const uint16_t* XqX, int64_t N, int64_t n, int64_t ld, float* H, float* A,
+                        int32_t* info, void* ws, size_t ws_bytes, cudaStream_t st);
+int kq_biip_rotate_input(float* A, int64_t n, const float* SX, const int8_t* sv, int mode,
+                         void* ws, size_t ws_bytes, cudaStream_t st);
+int kq_gptaq_correction(const float* A, const float* U, int64_t n, float alpha, float* P,
+                        int32_t* info, void* ws, size_t ws_bytes, cudaStream_t st);
+int kq_quantize_layer_asym(float* W, int64_t m, int64_t n, const float* U, const float* P,
+                           int bits, int group, int block, uint8_t* codes, float* scales,
+                           uint8_t* zeros, float* W_hat, int32_t* info, void* ws, size_t ws_bytes,
+                           cudaStream_t st);
 int kq_unpack(const uint32_t* packed, int64_t m, int64_t n, int bits, uint8_t* codes,
               cudaStream_t st);
 int kq_layer_loss(const float* Wr, const float* Wh, int64_t m, int64_t n, const float* HX,
@@ -273,6 +286,39 @@ int kronq_layer_loss(const float* W_ref, const float* W_hat, int64_t m, int64_t 
                      const float* H_X, const float* H_G, double* loss_out, void* ws,
                      size_t ws_bytes, void* stream) {
   return kq_layer_loss(W_ref, W_hat, m, n, H_X, H_G, loss_out, ws, ws_bytes, S(stream));
+}
+
+size_t kronq_gptaq_workspace_size(int64_t m, int64_t n) {
+  if (m <= 0 || n <= 0) return 0;
+  size_t s = kronq_workspace_size(m, n, 4, -1, 128);
+  const size_t parts[3] = {kq_drift_ws(n), kq_correction_ws(n), kq_quantize_asym_ws(m, n)};
+  for (size_t p : parts)
+    if (p > s) s = p;
+  return s;
+}
+
+int kronq_drift_covariance(const void* XqX, int64_t N, int64_t n, int64_t ld, float* H, float* A,
+                           int32_t* info, void* ws, size_t ws_bytes, void* stream) {
+  return kq_drift_covariance(static_cast<const uint16_t*>(XqX), N, n, ld, H, A, info, ws, ws_bytes,
+                             S(stream));
+}
+
+int kronq_biip_rotate_input(float* A, int64_t n, const float* S_X, const int8_t* sign_v, int mode,
+                            void* ws, size_t ws_bytes, void* stream) {
+  return kq_biip_rotate_input(A, n, S_X, sign_v, mode, ws, ws_bytes, S(stream));
+}
+
+int kronq_gptaq_correction(const float* A, const float* U_c, int64_t n, float alpha, float* P,
+                           int32_t* info, void* ws, size_t ws_bytes, void* stream) {
+  return kq_gptaq_correction(A, U_c, n, alpha, P, info, ws, ws_bytes, S(stream));
+}
+
+int kronq_quantize_layer_gptaq(float* W, int64_t m, int64_t n, const float* U_c, const float* P,
+                               int bits, int group, int block, uint8_t* codes, float* scales,
+                               uint8_t* zeros, float* W_hat, int32_t* info, void* ws,
+                               size_t ws_bytes, void* stream) {
+  return kq_quantize_layer_asym(W, m, n, U_c, P, bits, group, block, codes, scales, zeros, W_hat,
+                                info, ws, ws_bytes, S(stream));
 }
 
 }  // extern "C"

@@ -175,13 +175,19 @@ __global__ void row_params_kernel(const float* __restrict__ W, int m, int n, int
   }
 }
 
-template <int GROUP, bool CLIP>  // GROUP 0: per-channel grid; else 32, 64 or 128.  CLIP: --w_clip
+// GROUP 0: per-channel grid; else 32, 64 or 128.  CLIP: --w_clip.  ASYM: the
+// GPTAQ term (P != null): after column j, later columns k also receive
+// v_j P[j][k] (v_j: column j's value the quantizer saw); the kernel then
+// also writes -v_j next to e_j (columns QB .. 2 QB - 1 of the block's part of
+// the E planes) and P's slab next to U's (columns QB .. 2 QB - 1 of the slab
+// planes), so that the lazy update is one product with K = 2 QB per block.
+template <int GROUP, bool CLIP, bool ASYM = false>
 __global__ void __launch_bounds__(OBS_THREADS)
 obs_block_kernel(const float* __restrict__ W, int m, int n, const float* __restrict__ U, int i1,
                  int bits, uint8_t* __restrict__ codes, float* __restrict__ scales,
                  uint8_t* __restrict__ zeros, float* __restrict__ W_hat, float* __restrict__ Eh,
                  float* __restrict__ El, int ld_e, float* __restrict__ Uth,
-                 float* __restrict__ Utl, int slab_end) {
+                 float* __restrict__ Utl, int slab_end, const float* __restrict__ P = nullptr) {
   // Thread `chunk` (0..7) of a row owns the 16 columns 32 s + 4 chunk + t
   // (s, t in 0..3), held in w[4 s + t]: for a fixed s the 8 threads of a row
   // read 8 consecutive float4 of a U row, so the shared-memory reads are
@@ -190,7 +196,9 @@ obs_block_kernel(const float* __restrict__ W, int m, int n, const float* __restr
   float* Us = smem;                    // [QB][US_LD]
   float* rdiag = smem + QB * US_LD;    // [QB]
   float* Tt = rdiag + QB;              // [QB][TT_LD]
+  float* Ps = Tt + QB * TT_LD;         // [QB][US_LD] (ASYM only)
   const int tid = threadIdx.x, lane = tid & 31;
+  constexpr int LDU = ASYM ? 2 * QB : QB;     // slab plane row length
 
   // The lazy update's B operand: Ut[c - i2][k] = U[i1 + k][c] for
   // i2 <= c < slab_end (the rest of the super-block, or of the matrix with
@@ -199,22 +207,26 @@ obs_block_kernel(const float* __restrict__ W, int m, int n, const float* __restr
   {
     const int i2 = i1 + QB;
     const int slices = (slab_end - i2) / TT_W;
-    for (int sl = blockIdx.x; sl < slices; sl += gridDim.x) {
-      const int c0 = i2 + TT_W * sl;
-      for (int e = tid; e < QB * TT_W; e += blockDim.x) {
-        const int k = e / TT_W, cc = e % TT_W;
-        Tt[k * TT_LD + cc] = U[(int64_t)(i1 + k) * n + c0 + cc];
+#pragma unroll 1
+    for (int which = 0; which < (ASYM ? 2 : 1); ++which) {
+      const float* S = which ? P : U;
+      for (int sl = blockIdx.x; sl < slices; sl += gridDim.x) {
+        const int c0 = i2 + TT_W * sl;
+        for (int e = tid; e < QB * TT_W; e += blockDim.x) {
+          const int k = e / TT_W, cc = e % TT_W;
+          Tt[k * TT_LD + cc] = S[(int64_t)(i1 + k) * n + c0 + cc];
+        }
+        __syncthreads();
+        for (int e = tid; e < QB * TT_W; e += blockDim.x) {
+          const int cc = e >> 7, k = e & (QB - 1);
+          const float v = Tt[k * TT_LD + cc];
+          const float h = kq::tf32x3::hi(v);
+          const int64_t o = (int64_t)(c0 - i2 + cc) * LDU + which * QB + k;
+          Uth[o] = h;
+          Utl[o] = v - h;
+        }
+        __syncthreads();
       }
-      __syncthreads();
-      for (int e = tid; e < QB * TT_W; e += blockDim.x) {
-        const int cc = e >> 7, k = e & (QB - 1);
-        const float v = Tt[k * TT_LD + cc];
-        const float h = kq::tf32x3::hi(v);
-        const int64_t o = (int64_t)(c0 - i2 + cc) * QB + k;
-        Uth[o] = h;
-        Utl[o] = v - h;
-      }
-      __syncthreads();
     }
   }
   const int chunk = tid & 7;
@@ -229,6 +241,13 @@ obs_block_kernel(const float* __restrict__ W, int m, int n, const float* __restr
     *reinterpret_cast<float4*>(Us + r * US_LD + c4 * 4) = u;
   }
   for (int j = tid; j < QB; j += blockDim.x) rdiag[j] = 1.f / U[(int64_t)(i1 + j) * n + i1 + j];
+  if (ASYM) {
+    for (int e = tid; e < QB * QB / 4; e += blockDim.x) {
+      const int r = e / (QB / 4), c4 = e % (QB / 4);
+      const float4 u = *reinterpret_cast<const float4*>(P + (int64_t)(i1 + r) * n + i1 + c4 * 4);
+      *reinterpret_cast<float4*>(Ps + r * US_LD + c4 * 4) = u;
+    }
+  }
 
   float w[16];
   {
@@ -248,6 +267,7 @@ obs_block_kernel(const float* __restrict__ W, int m, int n, const float* __restr
   __syncthreads();
 
   float qv[16], ev[16], hv[16];
+  float vv[ASYM ? 16 : 1];
 #pragma unroll
   for (int sg = 0; sg < 4; ++sg) {
 #pragma unroll 1
@@ -312,16 +332,31 @@ obs_block_kernel(const float* __restrict__ W, int m, int n, const float* __restr
         qv[4 * sg + t] = own ? q : qv[4 * sg + t];
         hv[4 * sg + t] = own ? wh : hv[4 * sg + t];
         ev[4 * sg + t] = own ? e_own : ev[4 * sg + t];
-        // w_k -= e U[j][k] for this thread's columns k > j (groups left of sg are done)
+        float v = 0.f;
+        if (ASYM) {
+          const float v_bc = __shfl_sync(0xffffffffu, x, src);
+          v = own ? x : v_bc;
+          vv[(4 * sg + t) % (ASYM ? 16 : 1)] = own ? x : vv[(4 * sg + t) % (ASYM ? 16 : 1)];
+        }
+        // w_k -= e U[j][k] (and, ASYM, += v P[j][k]) for this thread's
+        // columns k > j (groups left of sg are done)
         const float* ur = Us + j * US_LD + 4 * chunk;
+        const float* pr = Ps + j * US_LD + 4 * chunk;
 #pragma unroll
         for (int s2 = sg; s2 < 4; ++s2) {
           const float4 u = *reinterpret_cast<const float4*>(ur + 32 * s2);
           const float uu[4] = {u.x, u.y, u.z, u.w};
+          float pp[4] = {0.f, 0.f, 0.f, 0.f};
+          if (ASYM) {
+            const float4 p4 = *reinterpret_cast<const float4*>(pr + 32 * s2);
+            pp[0] = p4.x; pp[1] = p4.y; pp[2] = p4.z; pp[3] = p4.w;
+          }
 #pragma unroll
           for (int t2 = 0; t2 < 4; ++t2) {
-            const float coef = (s2 > sg || 4 * chunk + t2 > 4 * c + t) ? uu[t2] : 0.f;
+            const bool later = s2 > sg || 4 * chunk + t2 > 4 * c + t;
+            const float coef = later ? uu[t2] : 0.f;
             w[4 * s2 + t2] = fmaf(-e, coef, w[4 * s2 + t2]);
+            if (ASYM) w[4 * s2 + t2] = fmaf(v, later ? pp[t2] : 0.f, w[4 * s2 + t2]);
           }
         }
       }
@@ -347,6 +382,21 @@ obs_block_kernel(const float* __restrict__ W, int m, int n, const float* __restr
       const int64_t eo = (int64_t)row * ld_e + 32 * sg + 4 * chunk;
       *reinterpret_cast<float4*>(Eh + eo) = eh;
       *reinterpret_cast<float4*>(El + eo) = el;
+      if (ASYM) {
+        // -v next to e: the lazy update subtracts [E | -V] [U ; P]
+        float4 vh, vl;
+        const int b = (4 * sg) % (ASYM ? 16 : 1);
+        vh.x = kq::tf32x3::hi(-vv[b]);
+        vh.y = kq::tf32x3::hi(-vv[b + 1]);
+        vh.z = kq::tf32x3::hi(-vv[b + 2]);
+        vh.w = kq::tf32x3::hi(-vv[b + 3]);
+        vl.x = -vv[b] - vh.x;
+        vl.y = -vv[b + 1] - vh.y;
+        vl.z = -vv[b + 2] - vh.z;
+        vl.w = -vv[b + 3] - vh.w;
+        *reinterpret_cast<float4*>(Eh + eo + QB) = vh;
+        *reinterpret_cast<float4*>(El + eo + QB) = vl;
+      }
     }
     if (W_hat)
       *reinterpret_cast<float4*>(W_hat + off) =
@@ -486,20 +536,54 @@ __global__ void __launch_bounds__(256) slab_transpose_kernel(const float* __rest
   }
 }
 
-template <int GROUP, bool CLIP>
+template <int GROUP, bool CLIP, bool ASYM = false>
 int launch_block(const float* W, int m, int n, const float* U, int i1, int bits, uint8_t* codes,
                  float* scales, uint8_t* zeros, float* W_hat, const SolverScratch& sc, int sb,
-                 int slab_end, cudaStream_t st) {
+                 int slab_end, cudaStream_t st, const float* P = nullptr) {
   static kqh::PerDevice attr;
-  const size_t smem = (size_t)(QB * US_LD + QB + QB * TT_LD) * sizeof(float);
-  if (kqh::smem_attr_once(attr, obs_block_kernel<GROUP, CLIP>, (int)smem) <= 0)
+  const size_t smem = (size_t)(QB * US_LD + QB + QB * TT_LD + (ASYM ? QB * US_LD : 0)) * sizeof(float);
+  if (kqh::smem_attr_once(attr, obs_block_kernel<GROUP, CLIP, ASYM>, (int)smem) <= 0)
     return KRONQ_ERR_CUDA;
   const int grid = (m + ROWS_PER_CTA - 1) / ROWS_PER_CTA;
-  obs_block_kernel<GROUP, CLIP><<<grid, OBS_THREADS, smem, st>>>(W, m, n, U, i1, bits, codes, scales, zeros,
-                                                   W_hat, sc.Eh + (i1 - sb), sc.El + (i1 - sb),
-                                                   sc.B2, sc.Uth, sc.Utl, slab_end);
+  constexpr int KM = ASYM ? 2 : 1;               // E planes: [E | -V] per block with ASYM
+  const int ts = kqh::timer_begin(KRONQ_TIMER_OBS_BLOCK, st);
+  obs_block_kernel<GROUP, CLIP, ASYM><<<grid, OBS_THREADS, smem, st>>>(
+      W, m, n, U, i1, bits, codes, scales, zeros, W_hat, sc.Eh + KM * (i1 - sb),
+      sc.El + KM * (i1 - sb), KM * sc.B2, sc.Uth, sc.Utl, slab_end, P);
+  kqh::timer_end(ts, st);
   KQ_CHECK_LAUNCH();
   return KRONQ_OK;
+}
+
+// The GPTAQ variant of slab_transpose_kernel: rows row0 .. row0 + rows - 1 of
+// U and of P, transposed, interleaved per 128-row block b as the K layout of
+// the asymmetric lazy update: T[c - col0][2 QB b + k] = U[row0 + QB b + k][c]
+// and T[c - col0][2 QB b + QB + k] = P[row0 + QB b + k][c].
+__global__ void __launch_bounds__(256) slab_transpose2_kernel(const float* __restrict__ U,
+                                                              const float* __restrict__ P, int n,
+                                                              int row0, int rows, int col0,
+                                                              float* __restrict__ Th,
+                                                              float* __restrict__ Tl, int ld) {
+  __shared__ float t[32][33];
+  const float* S = blockIdx.z ? P : U;
+  const int kb = blockIdx.y * 32, cb = col0 + blockIdx.x * 32;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  for (int r = ty; r < 32; r += 8) {
+    const int k = kb + r, c = cb + tx;
+    t[r][tx] = (k < rows && c < n) ? S[(int64_t)(row0 + k) * n + c] : 0.f;
+  }
+  __syncthreads();
+  for (int r = ty; r < 32; r += 8) {
+    const int c = cb + r, k = kb + tx;
+    if (c < n && k < rows) {
+      const float v = t[tx][r];
+      const float h = kq::tf32x3::hi(v);
+      const int kk = 2 * QB * (k / QB) + (int)blockIdx.z * QB + k % QB;
+      const int64_t o = (int64_t)(c - col0) * ld + kk;
+      Th[o] = h;
+      Tl[o] = v - h;
+    }
+  }
 }
 
 constexpr int QB2 = 1024;        // outer super-block of the two-level lazy update
@@ -588,7 +672,9 @@ int kq_quantize_layer(float* W, int64_t m64, int64_t n64, const float* U, int bi
         // inner: W[:, i2:sb_end] -= E_blk U[i1:i2, i2:sb_end]
         const kq::GemmNT g = {sc.Eh + (i1 - sb), sc.El + (i1 - sb), B2, sc.Uth, sc.Utl, QB,
                               W + i2, n, m, sb_end - i2, QB, -1.f, 0};
+        const int ts = kqh::timer_begin(KRONQ_TIMER_LAZY_UPDATE, st);
         s = kq_gemm_nt_tc(&g, 1, info, st);
+        kqh::timer_end(ts, st);
         if (s != KRONQ_OK) return s;
       }
     }
@@ -609,7 +695,112 @@ int kq_quantize_layer(float* W, int64_t m64, int64_t n64, const float* U, int bi
       // (one level: the block kernel already wrote U[sb:sb_end, sb_end:]^T into Ut)
       const kq::GemmNT g = {sc.Eh, sc.El, B2, Bh, Bl, ldb, W + sb_end, n, m, n - sb_end, K,
                             -1.f, 0};
+      const int ts = kqh::timer_begin(KRONQ_TIMER_LAZY_UPDATE, st);
       const int s = kq_gemm_nt_tc(&g, 1, info, st);
+      kqh::timer_end(ts, st);
+      if (s != KRONQ_OK) return s;
+    }
+  }
+  return KRONQ_OK;
+}
+
+// ---------------------------------------------------------------------------
+// The solver with the GPTAQ term (asymmetric calibration): the block kernel
+// adds v_j P[j][k] next to -e_j U[j][k], and every lazy update subtracts
+// [E | -V] [U ; P] with K = 2 QB per block (E and -V interleaved per block,
+// U's and P's slabs likewise), as one tensor-core product.
+namespace {
+size_t solver_ws_asym(int64_t m, int64_t n, int B2) {
+  size_t b = 2 * a256((size_t)m * 2 * B2 * sizeof(float)) + 2 * a256((size_t)n * 2 * QB * sizeof(float));
+  if (B2 > QB) b += 2 * a256((size_t)n * 2 * B2 * sizeof(float));
+  return b;
+}
+}  // namespace
+
+size_t kq_quantize_asym_ws(int64_t m, int64_t n) { return solver_ws_asym(m, n, QB2); }
+
+int kq_quantize_layer_asym(float* W, int64_t m64, int64_t n64, const float* U, const float* P,
+                           int bits, int group, int block, uint8_t* codes, float* scales,
+                           uint8_t* zeros, float* W_hat, int32_t* info, void* ws, size_t ws_bytes,
+                           cudaStream_t st) {
+  if (!W || !U || !P || !codes || !scales || !zeros || m64 <= 0 || n64 <= 0)
+    return KRONQ_ERR_INVALID_ARG;
+  if (bits != 2 && bits != 3 && bits != 4 && bits != 8) return KRONQ_ERR_INVALID_ARG;
+  if (group != -1 && (group <= 0 || n64 % group)) return KRONQ_ERR_INVALID_ARG;
+  if (block != QB) return KRONQ_ERR_UNSUPPORTED;
+  if (group != -1 && group != 128) return KRONQ_ERR_UNSUPPORTED;
+  if (n64 % QB) return KRONQ_ERR_UNSUPPORTED;
+  if (m64 > INT32_MAX || n64 > 32768) return KRONQ_ERR_UNSUPPORTED;
+  if (!kqh::aligned(W, 16) || !kqh::aligned(U, 16) || !kqh::aligned(P, 16) ||
+      !kqh::aligned(codes, 16) || (W_hat && !kqh::aligned(W_hat, 16)))
+    return KRONQ_ERR_INVALID_ARG;
+  if (!ws || !kqh::aligned(ws, 256)) return KRONQ_ERR_WORKSPACE;
+  const int B2 = (n64 > QB && ws_bytes >= solver_ws_asym(m64, n64, QB2)) ? QB2 : QB;
+  if (ws_bytes < solver_ws_asym(m64, n64, B2)) return KRONQ_ERR_WORKSPACE;
+  const int m = (int)m64, n = (int)n64;
+  SolverScratch sc;
+  {
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    sc.B2 = B2;
+    sc.Eh = reinterpret_cast<float*>(w);
+    w += a256((size_t)m * 2 * B2 * sizeof(float));
+    sc.El = reinterpret_cast<float*>(w);
+    w += a256((size_t)m * 2 * B2 * sizeof(float));
+    sc.Uth = reinterpret_cast<float*>(w);
+    w += a256((size_t)n * 2 * QB * sizeof(float));
+    sc.Utl = reinterpret_cast<float*>(w);
+    w += a256((size_t)n * 2 * QB * sizeof(float));
+    sc.Voh = sc.Vol = nullptr;
+    if (B2 > QB) {
+      sc.Voh = reinterpret_cast<float*>(w);
+      w += a256((size_t)n * 2 * B2 * sizeof(float));
+      sc.Vol = reinterpret_cast<float*>(w);
+    }
+  }
+  if (group == -1) {
+    row_params_kernel<<<(m + 7) / 8, 256, 0, st>>>(W, m, n, bits, scales, zeros);
+    KQ_CHECK_LAUNCH();
+  }
+  for (int sb = 0; sb < n; sb += B2) {
+    const int sb_end = sb + B2 < n ? sb + B2 : n;
+    const int slab_end = B2 > QB ? sb_end : n;
+    for (int i1 = sb; i1 < sb_end; i1 += QB) {
+      const int s = group == -1
+          ? launch_block<0, false, true>(W, m, n, U, i1, bits, codes, scales, zeros, W_hat, sc, sb,
+                                         slab_end, st, P)
+          : launch_block<128, false, true>(W, m, n, U, i1, bits, codes, scales, zeros, W_hat, sc,
+                                           sb, slab_end, st, P);
+      if (s != KRONQ_OK) return s;
+      const int i2 = i1 + QB;
+      if (i2 < sb_end) {
+        // inner: W[:, i2:sb_end] -= [E_blk | -V_blk] [U ; P][i1:i2, i2:sb_end]
+        const kq::GemmNT g = {sc.Eh + 2 * (i1 - sb), sc.El + 2 * (i1 - sb), 2 * B2, sc.Uth, sc.Utl,
+                              2 * QB, W + i2, n, m, sb_end - i2, 2 * QB, -1.f, 0};
+        const int ts = kqh::timer_begin(KRONQ_TIMER_LAZY_UPDATE, st);
+        const int s2 = kq_gemm_nt_tc(&g, 1, info, st);
+        kqh::timer_end(ts, st);
+        if (s2 != KRONQ_OK) return s2;
+      }
+    }
+    if (sb_end < n) {
+      // outer: W[:, sb_end:] -= [E | -V]_sb [U ; P][sb:sb_end, sb_end:]
+      const int K = sb_end - sb;
+      const float* Bh = sc.Uth;
+      const float* Bl = sc.Utl;
+      int ldb = 2 * QB;
+      if (B2 > QB) {
+        const dim3 g((n - sb_end + 31) / 32, (K + 31) / 32, 2);
+        slab_transpose2_kernel<<<g, 256, 0, st>>>(U, P, n, sb, K, sb_end, sc.Voh, sc.Vol, 2 * B2);
+        KQ_CHECK_LAUNCH();
+        Bh = sc.Voh;
+        Bl = sc.Vol;
+        ldb = 2 * B2;
+      }
+      const kq::GemmNT g = {sc.Eh, sc.El, 2 * B2, Bh, Bl, ldb, W + sb_end, n, m, n - sb_end, 2 * K,
+                            -1.f, 0};
+      const int ts = kqh::timer_begin(KRONQ_TIMER_LAZY_UPDATE, st);
+      const int s = kq_gemm_nt_tc(&g, 1, info, st);
+      kqh::timer_end(ts, st);
       if (s != KRONQ_OK) return s;
     }
   }

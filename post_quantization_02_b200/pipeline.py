@@ -153,3 +153,61 @@ def covariance_from_host(A_host: torch.Tensor, H: torch.Tensor, chunk_rows: int 
         abi.kronq_covariance(staging[b][: r1 - r0], H, 1.0 / N, 0.0 if c == 0 else 1.0, stream=stream)
         used[b].record(stream)
     return copied
+
+
+@dataclass
+class GptaqResult:
+    codes: torch.Tensor
+    scales: torch.Tensor
+    zeros: torch.Tensor
+    packed: torch.Tensor | None
+    S_X: torch.Tensor
+    S_G: torch.Tensor
+    W_rot: torch.Tensor | None
+    W_hat: torch.Tensor | None
+    H_X: torch.Tensor            # rotated covariance of the drifted input X~
+    H_G: torch.Tensor
+    A: torch.Tensor              # rotated drift covariance (X - X~)^T X~ / N
+    U_c: torch.Tensor
+    P: torch.Tensor
+    info: torch.Tensor
+
+
+def quantize_sublayer_gptaq(W: torch.Tensor, HX: torch.Tensor, A: torch.Tensor, HG: torch.Tensor,
+                            sign_u: torch.Tensor, sign_v: torch.Tensor, bits: int, group: int = -1,
+                            alpha: float = 0.25, mode: str = "full", damp: float = 0.01,
+                            block: int = 128, alpha_asym: float = 0.25, keep: bool = False,
+                            ws: torch.Tensor | None = None, stream=None) -> GptaqResult:
+    """The layer path with GPTAQ's asymmetric calibration: HX = X~^T X~ / N and
+    A = (X - X~)^T X~ / N (kronq_drift_covariance), HG = G^T G / N.  BiIP ->
+    the drift covariance rotated like H_X -> inverse Cholesky -> P -> the
+    column loop with the P term -> pack.  Inputs are cloned."""
+    ctx = torch.cuda.stream(stream) if stream is not None else contextlib.nullcontext()
+    with ctx:
+        m, n = W.shape
+        dev = W.device
+        W, HX, A, HG = W.clone(), HX.clone(), A.clone(), HG.clone()
+        if ws is None:
+            ws = abi.gptaq_workspace(m, n, dev)
+        info = torch.zeros(1, dtype=torch.int32, device=dev)
+        SX = torch.empty(n, dtype=torch.float32, device=dev)
+        SG = torch.empty(m, dtype=torch.float32, device=dev)
+        abi.kronq_biip_rotate(W, HX, HG, sign_u, sign_v, alpha, mode, 0, SX, SG, ws, stream=stream)
+        abi.kronq_biip_rotate_input(A, SX, sign_v, mode, ws, stream=stream)
+        U = torch.empty((n, n), dtype=torch.float32, device=dev)
+        abi.kronq_cholesky_inv(HX, damp, U, info, ws, stream=stream)
+        P = torch.empty((n, n), dtype=torch.float32, device=dev)
+        abi.kronq_gptaq_correction(A, U, alpha_asym, P, info, ws, stream=stream)
+        W_rot = W.clone() if keep else None
+        G = 1 if group == -1 else n // group
+        codes = torch.empty((m, n), dtype=torch.uint8, device=dev)
+        scales = torch.empty((m, G), dtype=torch.float32, device=dev)
+        zeros = torch.empty((m, G), dtype=torch.uint8, device=dev)
+        W_hat = torch.empty((m, n), dtype=torch.float32, device=dev) if keep else None
+        abi.kronq_quantize_layer_gptaq(W, U, P, bits, group, block, codes, scales, zeros, W_hat,
+                                       info, ws, stream=stream)
+        packed = None
+        if bits in (2, 4):
+            packed = torch.empty((m, abi.packed_words(n, bits)), dtype=torch.int32, device=dev)
+            abi.kronq_pack(codes, bits, packed, stream=stream)
+        return GptaqResult(codes, scales, zeros, packed, SX, SG, W_rot, W_hat, HX, HG, A, U, P, info)
