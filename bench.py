@@ -56,9 +56,13 @@ def parse():
     ap.add_argument("--tokens", type=int, default=None,
                     help="calibration tokens per X/G (default: the workload's; smaller only for "
                          "profiler captures)")
-    ap.add_argument("--kernel", choices=["covariance"], default=None,
-                    help="time one kernel alone (for profiler captures on small cases): "
-                         "kronq_covariance of a --tokens x --width bf16 matrix")
+    ap.add_argument("--kernel", choices=["covariance", "cholesky", "solver", "biip"], default=None,
+                    help="time one stage alone (for profiler captures on small cases): "
+                         "kronq_covariance of a --tokens x --width bf16 matrix, "
+                         "kronq_cholesky_inv of a --width x --width covariance, "
+                         "kronq_quantize_layer of a --rows x --width layer, or "
+                         "kronq_biip_rotate of that layer with its two covariances")
+    ap.add_argument("--rows", type=int, default=4096, help="layer rows for --kernel solver")
     ap.add_argument("--width", type=int, default=None,
                     help="feature width for --kernel (default: the workload's widest)")
     ap.add_argument("--oracle-full-chain", action="store_true",
@@ -607,7 +611,8 @@ def stage_rooflines(cfg, layers, steps, stages, inner, peaks, peak_src, peak, pe
             "peak_source": f"{peak_src} {peak_kind}", "flops_per_step": lazy_flops,
             "ms_per_step": ms / steps, "launches_per_step": cnt / steps,
             "avg_launch_ms": ms / cnt,
-            "note": "fp32-accurate products as three tf32 tensor-core MMAs (hi*hi + hi*lo + lo*hi)"}
+            "note": "each product as three bf16 tensor-core MMAs of hi / lo planes (hi*hi + hi*lo + "
+                    "lo*hi, ~2^-17 relative), so the algorithmic ceiling is 1/3 of the bf16 peak"}
     chol_ms = stages.get("inverse_cholesky", 0.0)
     chol_flops = sum(2 * L.sub.n ** 3 / 3 for L in layers)
     if chol_ms > 0:
@@ -657,22 +662,82 @@ def run_kernel(args):
     X = torch.from_numpy(synth.make_x(cfg, site).view(np.int16)).to(dev).view(torch.bfloat16)
     d = site.width
     H = torch.empty((d, d), dtype=torch.float32, device=dev)
+    abi.kronq_covariance(X, H, 1.0 / tokens, 0.0)
+    info = torch.zeros(1, dtype=torch.int32, device=dev)
+    if args.kernel == "covariance":
+        def call():
+            abi.kronq_covariance(X, H, 1.0 / tokens, 0.0)
+        flops, what = tokens * d * d, "kronq_covariance"
+    elif args.kernel == "cholesky":
+        del X
+        U = torch.empty_like(H)
+        ws = abi.workspace(d, d, device=dev)
+
+        def call():
+            abi.kronq_cholesky_inv(H, 0.01, U, info, ws)
+        flops, what = 2 * d ** 3 / 3, "kronq_cholesky_inv"
+    elif args.kernel == "biip":
+        del X
+        m = args.rows
+        G_ = torch.randn((tokens, m), generator=torch.Generator(device=dev).manual_seed(1),
+                         device=dev).to(torch.bfloat16)
+        HG = torch.empty((m, m), dtype=torch.float32, device=dev)
+        abi.kronq_covariance(G_, HG, 1.0 / tokens, 0.0)
+        del G_
+        W0 = torch.randn((m, d), generator=torch.Generator(device=dev).manual_seed(0),
+                         device=dev) * 0.02
+        W, HXr, HGr = torch.empty_like(W0), torch.empty_like(H), torch.empty_like(HG)
+        su = (torch.randint(0, 2, (m,), device=dev, dtype=torch.int8) * 2 - 1).to(torch.int8)
+        sv = (torch.randint(0, 2, (d,), device=dev, dtype=torch.int8) * 2 - 1).to(torch.int8)
+        SX = torch.empty(d, device=dev)
+        SG = torch.empty(m, device=dev)
+        ws = abi.workspace(m, d, device=dev)
+
+        def call():
+            W.copy_(W0)
+            HXr.copy_(H)
+            HGr.copy_(HG)
+            abi.kronq_biip_rotate(W, HXr, HGr, su, sv, 0.25, "full", 0, SX, SG, ws)
+        flops, what = 16 * (m * d + d * d + m * m), "kronq_biip_rotate (algorithmic bytes)"
+    else:
+        del X
+        U = torch.empty_like(H)
+        ws = abi.workspace(args.rows, d, device=dev)
+        abi.kronq_cholesky_inv(H, 0.01, U, info, ws)
+        sub = cfg.sublayers[0]
+        W0 = torch.randn((args.rows, d), generator=torch.Generator(device=dev).manual_seed(0),
+                         device=dev) * 0.02
+        W = torch.empty_like(W0)
+        codes = torch.empty((args.rows, d), dtype=torch.uint8, device=dev)
+        G = 1 if sub.group == -1 else d // sub.group
+        scales = torch.empty((args.rows, G), device=dev)
+        zeros = torch.empty((args.rows, G), dtype=torch.uint8, device=dev)
+
+        def call():
+            W.copy_(W0)
+            abi.kronq_quantize_layer(W, U, sub.bits or 4, sub.group, 128, codes, scales, zeros,
+                                     None, info, ws)
+        flops, what = args.rows * d * (d - 128), "kronq_quantize_layer (lazy-update flops)"
     for _ in range(max(1, args.warmup)):
-        abi.kronq_covariance(X, H, 1.0 / tokens, 0.0)
+        call()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(args.steps):
-        abi.kronq_covariance(X, H, 1.0 / tokens, 0.0)
+        call()
     e1.record()
     torch.cuda.synchronize()
+    if info.item() != 0:
+        raise RuntimeError(f"device status {info.item()}")
     ms = e0.elapsed_time(e1) / args.steps
-    flops = tokens * d * d
     peaks, src = load_peaks()
-    tf = flops / (ms / 1e3) / 1e12
-    print(json.dumps({"kernel": "kronq_covariance", "tokens": tokens, "width": d, "ms": ms,
-                      "tflops": tf, "frac_of_burst_peak": tf / float(peaks["bf16_tflops"]),
-                      "peak_source": src}), flush=True)
+    rate = flops / (ms / 1e3) / 1e12
+    if args.kernel == "biip":
+        out = {"tb_per_s": rate, "frac_of_hbm": rate * 1e3 / float(peaks["hbm_gbs"])}
+    else:
+        out = {"tflops": rate, "frac_of_burst_peak": rate / float(peaks["bf16_tflops"])}
+    print(json.dumps({"kernel": what, "tokens": tokens, "width": d, "rows": args.rows, "ms": ms,
+                      **out, "peak_source": src}), flush=True)
 
 
 def main():

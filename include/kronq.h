@@ -291,14 +291,15 @@ int kronq_deploy_matvec(const uint32_t* packed, int64_t m, int64_t n, int bits, 
  *
  * Same arguments and meaning as kronq_quantize_layer, minus (ws, ws_bytes).
  * The solver's scratch (its m x 128 error block and the current block's
- * n x 128 slab of U_c, both as tf32 hi / lo planes) lives in a static 64 MiB
+ * n x 128 slab of U_c, both as bf16 hi / lo planes) lives in a static 64 MiB
  * device array inside the library (every GPU that loads the library holds it
  * until the process exits), so m and n may each be at most 32768
  * (KRONQ_ERR_UNSUPPORTED above that).  That array always holds the one-level
  * lazy update's scratch; when the two-level update's (1024-column
- * super-blocks, 2 (m + n) 1024 x 4 bytes more) does not also fit in it -- e.g.
- * m = n = 4096, or any n of 7296 or more -- the call runs the one-level update
- * (K = 128 trailing updates after every block).  The codes agree with
+ * super-blocks, about 4 (m + n) KiB) does not also fit in it -- e.g.
+ * m = n = 8192, or m = 16384 with n = 4096, or any n of 14592 or more --
+ * the call runs the one-level update (K = 128 trailing updates after every
+ * block).  The codes agree with
  * kronq_quantize_layer's up to floating-point summation order (the parity
  * bar, >= 99.9 % identical); the one-level update is slower on wide layers.  The library looks up the array's device
  * address once per device, during the first call made on that device; make

@@ -356,8 +356,9 @@ def kronq_quantize_layer_noalloc(W, U, bits: int, group: int, block: int, codes,
     """kronq_quantize_layer with its scratch in the library's static device
     array (no workspace, nothing allocated; at most 32768 rows and 32768
     columns).  Layers whose two-level lazy-update scratch exceeds the array's
-    64 MiB run the one-level update (K = 128 trailing updates): the same
-    codes up to floating-point summation order, at a lower speed."""
+    64 MiB (e.g. 8192 x 8192) run the one-level update (K = 128 trailing
+    updates): the same codes up to floating-point summation order, at a
+    lower speed."""
     m, n = _quant_args(W, U, codes, scales, zeros, W_hat, group)
     _dev(info, torch.int32, "info")
     _on_current_device((info, "info"))

@@ -1,8 +1,12 @@
-// C += alpha * A B^T on the 5th-generation tensor cores with fp32-level
-// accuracy (tf32, three-term split: tf32x3.cuh), for up to two problems
-// per launch.  A (M x K) and B (N x K) come pre-split: each as a hi plane
-// (tf32-exact) and a lo plane (the fp32 remainder), all row-major, so all
-// four reach the tensor core K-major straight from TMA.  C is M x N
+// C += alpha * A B^T on the 5th-generation tensor cores from operands split
+// into hi / lo planes, three products per K step (hi*hi + hi*lo + lo*hi),
+// for up to two problems per launch.  Two plane types (one per launch):
+//   tf32: hi tf32-exact, lo the fp32 remainder (fp32-level accuracy; the
+//         inverse Cholesky's updates and the GPTAQ correction),
+//   bf16: hi = RN_bf16(x), lo = RN_bf16(x - hi) (~2^-17 relative, twice the
+//         tf32 rate and half the bytes; the solver's lazy updates).
+// All planes row-major, so all four reach the tensor core K-major straight
+// from TMA, 128-byte rows (32 tf32 or 64 bf16 K values).  C is M x N
 // row-major, updated in place.  A problem may ask for its lower triangle
 // only (M = N, tiles with tile column > tile row skipped, diagonal tiles
 // written on and below the diagonal): the symmetric rank-K update of a
@@ -23,11 +27,9 @@
 
 namespace {
 
-using kq::tf32x3::KC;
-
 constexpr int TM = 128, TN = 128;
 constexpr int STAGES = 3;
-constexpr int CHUNK = TM * KC * 4;             // 16 KB: 128 rows x 32 fp32
+constexpr int CHUNK = TM * 128;                // 16 KB: 128 rows x 128 bytes (32 fp32 / 64 bf16)
 constexpr int STAGE_BYTES = 4 * CHUNK;         // A hi, A lo, B hi, B lo
 constexpr int THREADS = 320;
 constexpr int EPI_WARP0 = 2;
@@ -84,6 +86,7 @@ struct Tile {
   int prob, tm, tn, kchunks;
 };
 
+template <int KC>
 __device__ __forceinline__ Tile tile_of(const Problems& P, int t) {
   Tile r;
   r.prob = (P.count > 1 && t >= P.p[0].tiles) ? 1 : 0;
@@ -104,9 +107,13 @@ __device__ __forceinline__ Tile tile_of(const Problems& P, int t) {
   return r;
 }
 
+// BF16 = false: tf32 planes (32 fp32 K values per 128-byte row);
+// true: bf16 planes (64 bf16 K values per row).
+template <bool BF16>
 __global__ void __launch_bounds__(THREADS, 1)
 gemm_nt_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Problems P,
                   int32_t* info) {
+  constexpr int KC = BF16 ? 64 : 32;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* stages = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -149,7 +156,7 @@ gemm_nt_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Pro
       int it = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < P.total_tiles && ok; t += gridDim.x) {
-        const Tile tl = tile_of(P, t);
+        const Tile tl = tile_of<KC>(P, t);
         for (int kc = 0; kc < tl.kchunks; ++kc, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
@@ -175,7 +182,7 @@ gemm_nt_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Pro
       int it = 0, tcount = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < P.total_tiles && ok; t += gridDim.x, ++tcount) {
-        const Tile tl = tile_of(P, t);
+        const Tile tl = tile_of<KC>(P, t);
         const int buf = tcount & 1;
         const uint32_t aph = (uint32_t)(tcount >> 1) & 1u;
         if (!kq::mbar_wait(&bars->tempty[buf], aph ^ 1u, abort, info)) break;
@@ -188,9 +195,14 @@ gemm_nt_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Pro
           kq::tc_fence_after();
           const uint32_t a = kq::smem_u32(stages + s * STAGE_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < KC / 8; ++kk)
-            kq::tf32x3::mma3(d_tmem, a, a + CHUNK, a + 2 * CHUNK, a + 3 * CHUNK, kk,
-                             (kc == 0 && kk == 0) ? 0u : 1u);
+          for (int kk = 0; kk < 4; ++kk) {     // four 32-byte K steps per 128-byte row
+            if (BF16)
+              kq::tf32x3::mma3_bf16(d_tmem, a, a + CHUNK, a + 2 * CHUNK, a + 3 * CHUNK, kk,
+                                    (kc == 0 && kk == 0) ? 0u : 1u);
+            else
+              kq::tf32x3::mma3(d_tmem, a, a + CHUNK, a + 2 * CHUNK, a + 3 * CHUNK, kk,
+                               (kc == 0 && kk == 0) ? 0u : 1u);
+          }
           kq::mma_commit(&bars->empty[s]);
         }
         if (ok) kq::mma_commit(&bars->tfull[buf]);
@@ -209,7 +221,7 @@ gemm_nt_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Pro
     int tcount = 0;
     bool pending = false;
     for (int t = blockIdx.x; t < P.total_tiles; t += gridDim.x, ++tcount) {
-      const Tile tl = tile_of(P, t);
+      const Tile tl = tile_of<KC>(P, t);
       const Problem& pr = P.p[tl.prob];
       const int buf = tcount & 1;
       const uint32_t aph = (uint32_t)(tcount >> 1) & 1u;
@@ -280,21 +292,32 @@ int kq_gemm_nt_tc(const kq::GemmNT* probs, int count, int32_t* info, cudaStream_
   Problems P;
   P.count = 0;
   P.total_tiles = 0;
+  const int bf16 = probs[0].bf16;
+  const int KC = bf16 ? 64 : 32;
+  const int64_t lda_align = bf16 ? 8 : 4;          // 16-byte rows
   for (int i = 0; i < count; ++i) {
     const kq::GemmNT& g = probs[i];
     if (g.M <= 0 || g.N <= 0 || g.K <= 0) continue;
-    if (!g.A_hi || !g.A_lo || !g.B_hi || !g.B_lo || !g.C || g.lda % 4 || g.ldb % 4 || g.ldc % 4 ||
-        !kqh::aligned(g.A_hi, 16) || !kqh::aligned(g.A_lo, 16) || !kqh::aligned(g.B_hi, 16) ||
-        !kqh::aligned(g.B_lo, 16) || !kqh::aligned(g.C, 16))
+    if (g.bf16 != bf16) return KRONQ_ERR_INVALID_ARG;
+    if (!g.A_hi || !g.A_lo || !g.B_hi || !g.B_lo || !g.C || g.lda % lda_align ||
+        g.ldb % lda_align || g.ldc % 4 || !kqh::aligned(g.A_hi, 16) ||
+        !kqh::aligned(g.A_lo, 16) || !kqh::aligned(g.B_hi, 16) || !kqh::aligned(g.B_lo, 16) ||
+        !kqh::aligned(g.C, 16))
       return KRONQ_ERR_INVALID_ARG;
     if (g.lower && g.M != g.N) return KRONQ_ERR_INVALID_ARG;
     const int j = P.count;
-    if (!kqh::make_map_f32(&maps.a_hi[j], g.A_hi, g.K, g.M, g.lda, KC, TM) ||
-        !kqh::make_map_f32(&maps.a_lo[j], g.A_lo, g.K, g.M, g.lda, KC, TM) ||
-        !kqh::make_map_f32(&maps.b_hi[j], g.B_hi, g.K, g.N, g.ldb, KC, TN) ||
-        !kqh::make_map_f32(&maps.b_lo[j], g.B_lo, g.K, g.N, g.ldb, KC, TN) ||
-        !kqh::make_map_f32(&maps.c[j], g.C, g.N, g.M, g.ldc, 32, 32))
-      return KRONQ_ERR_CUDA;
+    bool ok;
+    if (bf16)
+      ok = kqh::make_map_bf16(&maps.a_hi[j], g.A_hi, g.K, g.M, g.lda, KC, TM) &&
+           kqh::make_map_bf16(&maps.a_lo[j], g.A_lo, g.K, g.M, g.lda, KC, TM) &&
+           kqh::make_map_bf16(&maps.b_hi[j], g.B_hi, g.K, g.N, g.ldb, KC, TN) &&
+           kqh::make_map_bf16(&maps.b_lo[j], g.B_lo, g.K, g.N, g.ldb, KC, TN);
+    else
+      ok = kqh::make_map_f32(&maps.a_hi[j], static_cast<const float*>(g.A_hi), g.K, g.M, g.lda, KC, TM) &&
+           kqh::make_map_f32(&maps.a_lo[j], static_cast<const float*>(g.A_lo), g.K, g.M, g.lda, KC, TM) &&
+           kqh::make_map_f32(&maps.b_hi[j], static_cast<const float*>(g.B_hi), g.K, g.N, g.ldb, KC, TN) &&
+           kqh::make_map_f32(&maps.b_lo[j], static_cast<const float*>(g.B_lo), g.K, g.N, g.ldb, KC, TN);
+    if (!ok || !kqh::make_map_f32(&maps.c[j], g.C, g.N, g.M, g.ldc, 32, 32)) return KRONQ_ERR_CUDA;
     Problem& q = P.p[j];
     q.C = g.C;
     q.ldc = g.ldc;
@@ -316,11 +339,16 @@ int kq_gemm_nt_tc(const kq::GemmNT* probs, int count, int32_t* info, cudaStream_
   }
   if (P.count == 0) return KRONQ_OK;
   if (P.count == 1) P.p[1] = P.p[0];
-  static kqh::PerDevice attr;
-  if (kqh::smem_attr_once(attr, gemm_nt_tc_kernel, SMEM_BYTES) <= 0) return KRONQ_ERR_CUDA;
+  static kqh::PerDevice attr_tf32, attr_bf16;
+  if (bf16 ? kqh::smem_attr_once(attr_bf16, gemm_nt_tc_kernel<true>, SMEM_BYTES) <= 0
+           : kqh::smem_attr_once(attr_tf32, gemm_nt_tc_kernel<false>, SMEM_BYTES) <= 0)
+    return KRONQ_ERR_CUDA;
   int grid = P.total_tiles < kqh::num_sms() ? P.total_tiles : kqh::num_sms();
   if (max_ctas > 0 && grid > max_ctas) grid = max_ctas;
-  gemm_nt_tc_kernel<<<grid, THREADS, SMEM_BYTES, st>>>(maps, P, info);
+  if (bf16)
+    gemm_nt_tc_kernel<true><<<grid, THREADS, SMEM_BYTES, st>>>(maps, P, info);
+  else
+    gemm_nt_tc_kernel<false><<<grid, THREADS, SMEM_BYTES, st>>>(maps, P, info);
   KQ_CHECK_LAUNCH();
   return KRONQ_OK;
 }

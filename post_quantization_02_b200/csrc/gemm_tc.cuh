@@ -7,18 +7,21 @@
 namespace kq {
 
 // C (M x N, row-major, ldc) += alpha * A B^T with A M x K and B N x K, both
-// row-major and given pre-split: A = A_hi + A_lo with A_hi exactly a tf32
-// value (the low 13 mantissa bits clear) and A_lo the fp32 remainder, the
-// two planes sharing the leading dimension lda (B likewise, ldb).
+// row-major and given pre-split into a hi and a lo plane sharing the leading
+// dimension (lda / ldb elements):
+//   bf16 = 0: fp32 planes, A_hi exactly a tf32 value (the low 13 mantissa
+//             bits clear) and A_lo the fp32 remainder;
+//   bf16 = 1: bf16 planes, A_hi = RN_bf16(A) and A_lo = RN_bf16(A - A_hi)
+//             (A = A_hi + A_lo to about 2^-17 relative).
 // lower = 1: M == N and only the lower triangle of C (tile by tile, the
 // diagonal tiles on and below the diagonal) is updated.  Pointers 16-byte
-// aligned, leading dimensions multiples of 4.
+// aligned, leading dimensions multiples of 16 bytes.
 struct GemmNT {
-  const float* A_hi;
-  const float* A_lo;
+  const void* A_hi;
+  const void* A_lo;
   int64_t lda;
-  const float* B_hi;
-  const float* B_lo;
+  const void* B_hi;
+  const void* B_lo;
   int64_t ldb;
   float* C;
   int64_t ldc;
@@ -30,12 +33,13 @@ struct GemmNT {
   // the diagonal); tile_end < 0: to the last tile
   int tile_begin = 0;
   int tile_end = -1;
+  int bf16 = 0;
 };
 
 }  // namespace kq
 
-// One launch for up to two independent problems (count 1 or 2); empty
-// problems are skipped.  Returns KRONQ_OK, KRONQ_ERR_INVALID_ARG or
+// One launch for up to two independent problems (count 1 or 2, both with
+// the same plane type); empty problems are skipped.  Returns KRONQ_OK, KRONQ_ERR_INVALID_ARG or
 // KRONQ_ERR_CUDA.
 // max_ctas > 0 caps the persistent grid (to leave SMs to concurrent work).
 int kq_gemm_nt_tc(const kq::GemmNT* probs, int count, int32_t* info, cudaStream_t st,

@@ -185,9 +185,9 @@ template <int GROUP, bool CLIP, bool ASYM = false>
 __global__ void __launch_bounds__(OBS_THREADS)
 obs_block_kernel(const float* __restrict__ W, int m, int n, const float* __restrict__ U, int i1,
                  int bits, uint8_t* __restrict__ codes, float* __restrict__ scales,
-                 uint8_t* __restrict__ zeros, float* __restrict__ W_hat, float* __restrict__ Eh,
-                 float* __restrict__ El, int ld_e, float* __restrict__ Uth,
-                 float* __restrict__ Utl, int slab_end, const float* __restrict__ P = nullptr) {
+                 uint8_t* __restrict__ zeros, float* __restrict__ W_hat, uint16_t* __restrict__ Eh,
+                 uint16_t* __restrict__ El, int ld_e, uint16_t* __restrict__ Uth,
+                 uint16_t* __restrict__ Utl, int slab_end, const float* __restrict__ P = nullptr) {
   // Thread `chunk` (0..7) of a row owns the 16 columns 32 s + 4 chunk + t
   // (s, t in 0..3), held in w[4 s + t]: for a fixed s the 8 threads of a row
   // read 8 consecutive float4 of a U row, so the shared-memory reads are
@@ -219,11 +219,8 @@ obs_block_kernel(const float* __restrict__ W, int m, int n, const float* __restr
         __syncthreads();
         for (int e = tid; e < QB * TT_W; e += blockDim.x) {
           const int cc = e >> 7, k = e & (QB - 1);
-          const float v = Tt[k * TT_LD + cc];
-          const float h = kq::tf32x3::hi(v);
           const int64_t o = (int64_t)(c0 - i2 + cc) * LDU + which * QB + k;
-          Uth[o] = h;
-          Utl[o] = v - h;
+          kq::tf32x3::split_bf16(Tt[k * TT_LD + cc], Uth[o], Utl[o]);
         }
         __syncthreads();
       }
@@ -370,32 +367,20 @@ obs_block_kernel(const float* __restrict__ W, int m, int n, const float* __restr
                         ((uint32_t)qv[4 * sg + 2] << 16) | ((uint32_t)qv[4 * sg + 3] << 24);
     *reinterpret_cast<uint32_t*>(codes + off) = pk;
     {
-      float4 eh, el;
-      eh.x = kq::tf32x3::hi(ev[4 * sg]);
-      eh.y = kq::tf32x3::hi(ev[4 * sg + 1]);
-      eh.z = kq::tf32x3::hi(ev[4 * sg + 2]);
-      eh.w = kq::tf32x3::hi(ev[4 * sg + 3]);
-      el.x = ev[4 * sg] - eh.x;
-      el.y = ev[4 * sg + 1] - eh.y;
-      el.z = ev[4 * sg + 2] - eh.z;
-      el.w = ev[4 * sg + 3] - eh.w;
+      // E as bf16 hi / lo planes (four values: one 8-byte store per plane)
+      uint16_t h[4], l[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) kq::tf32x3::split_bf16(ev[4 * sg + u], h[u], l[u]);
       const int64_t eo = (int64_t)row * ld_e + 32 * sg + 4 * chunk;
-      *reinterpret_cast<float4*>(Eh + eo) = eh;
-      *reinterpret_cast<float4*>(El + eo) = el;
+      *reinterpret_cast<uint2*>(Eh + eo) = make_uint2(h[0] | ((uint32_t)h[1] << 16), h[2] | ((uint32_t)h[3] << 16));
+      *reinterpret_cast<uint2*>(El + eo) = make_uint2(l[0] | ((uint32_t)l[1] << 16), l[2] | ((uint32_t)l[3] << 16));
       if (ASYM) {
         // -v next to e: the lazy update subtracts [E | -V] [U ; P]
-        float4 vh, vl;
         const int b = (4 * sg) % (ASYM ? 16 : 1);
-        vh.x = kq::tf32x3::hi(-vv[b]);
-        vh.y = kq::tf32x3::hi(-vv[b + 1]);
-        vh.z = kq::tf32x3::hi(-vv[b + 2]);
-        vh.w = kq::tf32x3::hi(-vv[b + 3]);
-        vl.x = -vv[b] - vh.x;
-        vl.y = -vv[b + 1] - vh.y;
-        vl.z = -vv[b + 2] - vh.z;
-        vl.w = -vv[b + 3] - vh.w;
-        *reinterpret_cast<float4*>(Eh + eo + QB) = vh;
-        *reinterpret_cast<float4*>(El + eo + QB) = vl;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) kq::tf32x3::split_bf16(-vv[b + u], h[u], l[u]);
+        *reinterpret_cast<uint2*>(Eh + eo + QB) = make_uint2(h[0] | ((uint32_t)h[1] << 16), h[2] | ((uint32_t)h[3] << 16));
+        *reinterpret_cast<uint2*>(El + eo + QB) = make_uint2(l[0] | ((uint32_t)l[1] << 16), l[2] | ((uint32_t)l[3] << 16));
       }
     }
     if (W_hat)
@@ -503,19 +488,21 @@ __global__ void unpack_kernel(const uint32_t* __restrict__ packed, int64_t m, in
 
 size_t a256(size_t b) { return (b + 255) & ~(size_t)255; }
 
+// The lazy update's operands are bf16 hi / lo planes (x = hi + lo to about
+// 2^-17 relative; three bf16 tensor-core products per fp32 product).
 struct SolverScratch {
   int B2;                  // outer (super-)block width: 128 (one level) or 1024
-  float *Eh, *El;          // E of the super-block, m x B2 each
-  float *Uth, *Utl;        // inner slab U[i1:i1+128, i1+128:sb_end]^T, n x 128 each
-  float *Voh, *Vol;        // outer slab U[sb:sb_end, sb_end:]^T, n x B2 each (two levels only)
+  uint16_t *Eh, *El;       // E of the super-block, m x B2 each
+  uint16_t *Uth, *Utl;     // inner slab U[i1:i1+128, i1+128:sb_end]^T, n x 128 each
+  uint16_t *Voh, *Vol;     // outer slab U[sb:sb_end, sb_end:]^T, n x B2 each (two levels only)
 };
 
 // Ut[c - col0][k] = U[row0 + k][c] for k < rows, col0 <= c < n, as tf32
 // hi / lo planes with leading dimension ld: one 32 x 32 tile per CTA.
 __global__ void __launch_bounds__(256) slab_transpose_kernel(const float* __restrict__ U, int n,
                                                              int row0, int rows, int col0,
-                                                             float* __restrict__ Th,
-                                                             float* __restrict__ Tl, int ld) {
+                                                             uint16_t* __restrict__ Th,
+                                                             uint16_t* __restrict__ Tl, int ld) {
   __shared__ float t[32][33];
   const int kb = blockIdx.y * 32, cb = col0 + blockIdx.x * 32;
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
@@ -527,11 +514,8 @@ __global__ void __launch_bounds__(256) slab_transpose_kernel(const float* __rest
   for (int r = ty; r < 32; r += 8) {
     const int c = cb + r, k = kb + tx;
     if (c < n && k < rows) {
-      const float v = t[tx][r];
-      const float h = kq::tf32x3::hi(v);
       const int64_t o = (int64_t)(c - col0) * ld + k;
-      Th[o] = h;
-      Tl[o] = v - h;
+      kq::tf32x3::split_bf16(t[tx][r], Th[o], Tl[o]);
     }
   }
 }
@@ -562,8 +546,8 @@ int launch_block(const float* W, int m, int n, const float* U, int i1, int bits,
 __global__ void __launch_bounds__(256) slab_transpose2_kernel(const float* __restrict__ U,
                                                               const float* __restrict__ P, int n,
                                                               int row0, int rows, int col0,
-                                                              float* __restrict__ Th,
-                                                              float* __restrict__ Tl, int ld) {
+                                                              uint16_t* __restrict__ Th,
+                                                              uint16_t* __restrict__ Tl, int ld) {
   __shared__ float t[32][33];
   const float* S = blockIdx.z ? P : U;
   const int kb = blockIdx.y * 32, cb = col0 + blockIdx.x * 32;
@@ -576,12 +560,9 @@ __global__ void __launch_bounds__(256) slab_transpose2_kernel(const float* __res
   for (int r = ty; r < 32; r += 8) {
     const int c = cb + r, k = kb + tx;
     if (c < n && k < rows) {
-      const float v = t[tx][r];
-      const float h = kq::tf32x3::hi(v);
       const int kk = 2 * QB * (k / QB) + (int)blockIdx.z * QB + k % QB;
       const int64_t o = (int64_t)(c - col0) * ld + kk;
-      Th[o] = h;
-      Tl[o] = v - h;
+      kq::tf32x3::split_bf16(t[tx][r], Th[o], Tl[o]);
     }
   }
 }
@@ -592,8 +573,8 @@ constexpr int QB2 = 1024;        // outer super-block of the two-level lazy upda
 // planes (m x B2 each), the inner U_c slab transposed (n x 128 each) and,
 // with two levels, the outer slab transposed (n x B2 each).
 size_t solver_ws(int64_t m, int64_t n, int B2) {
-  size_t b = 2 * a256((size_t)m * B2 * sizeof(float)) + 2 * a256((size_t)n * QB * sizeof(float));
-  if (B2 > QB) b += 2 * a256((size_t)n * B2 * sizeof(float));
+  size_t b = 2 * a256((size_t)m * B2 * sizeof(uint16_t)) + 2 * a256((size_t)n * QB * sizeof(uint16_t));
+  if (B2 > QB) b += 2 * a256((size_t)n * B2 * sizeof(uint16_t));
   return b;
 }
 
@@ -630,19 +611,19 @@ int kq_quantize_layer(float* W, int64_t m64, int64_t n64, const float* U, int bi
   {
     uint8_t* w = static_cast<uint8_t*>(ws);
     sc.B2 = B2;
-    sc.Eh = reinterpret_cast<float*>(w);
-    w += a256((size_t)m * B2 * sizeof(float));
-    sc.El = reinterpret_cast<float*>(w);
-    w += a256((size_t)m * B2 * sizeof(float));
-    sc.Uth = reinterpret_cast<float*>(w);
-    w += a256((size_t)n * QB * sizeof(float));
-    sc.Utl = reinterpret_cast<float*>(w);
-    w += a256((size_t)n * QB * sizeof(float));
+    sc.Eh = reinterpret_cast<uint16_t*>(w);
+    w += a256((size_t)m * B2 * sizeof(uint16_t));
+    sc.El = reinterpret_cast<uint16_t*>(w);
+    w += a256((size_t)m * B2 * sizeof(uint16_t));
+    sc.Uth = reinterpret_cast<uint16_t*>(w);
+    w += a256((size_t)n * QB * sizeof(uint16_t));
+    sc.Utl = reinterpret_cast<uint16_t*>(w);
+    w += a256((size_t)n * QB * sizeof(uint16_t));
     sc.Voh = sc.Vol = nullptr;
     if (B2 > QB) {
-      sc.Voh = reinterpret_cast<float*>(w);
-      w += a256((size_t)n * B2 * sizeof(float));
-      sc.Vol = reinterpret_cast<float*>(w);
+      sc.Voh = reinterpret_cast<uint16_t*>(w);
+      w += a256((size_t)n * B2 * sizeof(uint16_t));
+      sc.Vol = reinterpret_cast<uint16_t*>(w);
     }
   }
 
@@ -670,8 +651,9 @@ int kq_quantize_layer(float* W, int64_t m64, int64_t n64, const float* U, int bi
       const int i2 = i1 + QB;
       if (i2 < sb_end) {
         // inner: W[:, i2:sb_end] -= E_blk U[i1:i2, i2:sb_end]
-        const kq::GemmNT g = {sc.Eh + (i1 - sb), sc.El + (i1 - sb), B2, sc.Uth, sc.Utl, QB,
-                              W + i2, n, m, sb_end - i2, QB, -1.f, 0};
+        kq::GemmNT g = {sc.Eh + (i1 - sb), sc.El + (i1 - sb), B2, sc.Uth, sc.Utl, QB,
+                        W + i2, n, m, sb_end - i2, QB, -1.f, 0};
+        g.bf16 = 1;
         const int ts = kqh::timer_begin(KRONQ_TIMER_LAZY_UPDATE, st);
         s = kq_gemm_nt_tc(&g, 1, info, st);
         kqh::timer_end(ts, st);
@@ -681,8 +663,8 @@ int kq_quantize_layer(float* W, int64_t m64, int64_t n64, const float* U, int bi
     if (sb_end < n) {
       // outer: W[:, sb_end:] -= E_sb U[sb:sb_end, sb_end:]   (K = sb_end - sb)
       const int K = sb_end - sb;
-      const float* Bh = sc.Uth;
-      const float* Bl = sc.Utl;
+      const uint16_t* Bh = sc.Uth;
+      const uint16_t* Bl = sc.Utl;
       int ldb = QB;
       if (B2 > QB) {
         const dim3 g((n - sb_end + 31) / 32, (K + 31) / 32);
@@ -693,8 +675,8 @@ int kq_quantize_layer(float* W, int64_t m64, int64_t n64, const float* U, int bi
         ldb = B2;
       }
       // (one level: the block kernel already wrote U[sb:sb_end, sb_end:]^T into Ut)
-      const kq::GemmNT g = {sc.Eh, sc.El, B2, Bh, Bl, ldb, W + sb_end, n, m, n - sb_end, K,
-                            -1.f, 0};
+      kq::GemmNT g = {sc.Eh, sc.El, B2, Bh, Bl, ldb, W + sb_end, n, m, n - sb_end, K, -1.f, 0};
+      g.bf16 = 1;
       const int ts = kqh::timer_begin(KRONQ_TIMER_LAZY_UPDATE, st);
       const int s = kq_gemm_nt_tc(&g, 1, info, st);
       kqh::timer_end(ts, st);
@@ -711,8 +693,9 @@ int kq_quantize_layer(float* W, int64_t m64, int64_t n64, const float* U, int bi
 // U's and P's slabs likewise), as one tensor-core product.
 namespace {
 size_t solver_ws_asym(int64_t m, int64_t n, int B2) {
-  size_t b = 2 * a256((size_t)m * 2 * B2 * sizeof(float)) + 2 * a256((size_t)n * 2 * QB * sizeof(float));
-  if (B2 > QB) b += 2 * a256((size_t)n * 2 * B2 * sizeof(float));
+  size_t b = 2 * a256((size_t)m * 2 * B2 * sizeof(uint16_t)) +
+             2 * a256((size_t)n * 2 * QB * sizeof(uint16_t));
+  if (B2 > QB) b += 2 * a256((size_t)n * 2 * B2 * sizeof(uint16_t));
   return b;
 }
 }  // namespace
@@ -742,19 +725,19 @@ int kq_quantize_layer_asym(float* W, int64_t m64, int64_t n64, const float* U, c
   {
     uint8_t* w = static_cast<uint8_t*>(ws);
     sc.B2 = B2;
-    sc.Eh = reinterpret_cast<float*>(w);
-    w += a256((size_t)m * 2 * B2 * sizeof(float));
-    sc.El = reinterpret_cast<float*>(w);
-    w += a256((size_t)m * 2 * B2 * sizeof(float));
-    sc.Uth = reinterpret_cast<float*>(w);
-    w += a256((size_t)n * 2 * QB * sizeof(float));
-    sc.Utl = reinterpret_cast<float*>(w);
-    w += a256((size_t)n * 2 * QB * sizeof(float));
+    sc.Eh = reinterpret_cast<uint16_t*>(w);
+    w += a256((size_t)m * 2 * B2 * sizeof(uint16_t));
+    sc.El = reinterpret_cast<uint16_t*>(w);
+    w += a256((size_t)m * 2 * B2 * sizeof(uint16_t));
+    sc.Uth = reinterpret_cast<uint16_t*>(w);
+    w += a256((size_t)n * 2 * QB * sizeof(uint16_t));
+    sc.Utl = reinterpret_cast<uint16_t*>(w);
+    w += a256((size_t)n * 2 * QB * sizeof(uint16_t));
     sc.Voh = sc.Vol = nullptr;
     if (B2 > QB) {
-      sc.Voh = reinterpret_cast<float*>(w);
-      w += a256((size_t)n * 2 * B2 * sizeof(float));
-      sc.Vol = reinterpret_cast<float*>(w);
+      sc.Voh = reinterpret_cast<uint16_t*>(w);
+      w += a256((size_t)n * 2 * B2 * sizeof(uint16_t));
+      sc.Vol = reinterpret_cast<uint16_t*>(w);
     }
   }
   if (group == -1) {
@@ -774,8 +757,9 @@ int kq_quantize_layer_asym(float* W, int64_t m64, int64_t n64, const float* U, c
       const int i2 = i1 + QB;
       if (i2 < sb_end) {
         // inner: W[:, i2:sb_end] -= [E_blk | -V_blk] [U ; P][i1:i2, i2:sb_end]
-        const kq::GemmNT g = {sc.Eh + 2 * (i1 - sb), sc.El + 2 * (i1 - sb), 2 * B2, sc.Uth, sc.Utl,
-                              2 * QB, W + i2, n, m, sb_end - i2, 2 * QB, -1.f, 0};
+        kq::GemmNT g = {sc.Eh + 2 * (i1 - sb), sc.El + 2 * (i1 - sb), 2 * B2, sc.Uth, sc.Utl,
+                        2 * QB, W + i2, n, m, sb_end - i2, 2 * QB, -1.f, 0};
+        g.bf16 = 1;
         const int ts = kqh::timer_begin(KRONQ_TIMER_LAZY_UPDATE, st);
         const int s2 = kq_gemm_nt_tc(&g, 1, info, st);
         kqh::timer_end(ts, st);
@@ -785,8 +769,8 @@ int kq_quantize_layer_asym(float* W, int64_t m64, int64_t n64, const float* U, c
     if (sb_end < n) {
       // outer: W[:, sb_end:] -= [E | -V]_sb [U ; P][sb:sb_end, sb_end:]
       const int K = sb_end - sb;
-      const float* Bh = sc.Uth;
-      const float* Bl = sc.Utl;
+      const uint16_t* Bh = sc.Uth;
+      const uint16_t* Bl = sc.Utl;
       int ldb = 2 * QB;
       if (B2 > QB) {
         const dim3 g((n - sb_end + 31) / 32, (K + 31) / 32, 2);
@@ -796,8 +780,9 @@ int kq_quantize_layer_asym(float* W, int64_t m64, int64_t n64, const float* U, c
         Bl = sc.Vol;
         ldb = 2 * B2;
       }
-      const kq::GemmNT g = {sc.Eh, sc.El, 2 * B2, Bh, Bl, ldb, W + sb_end, n, m, n - sb_end, 2 * K,
-                            -1.f, 0};
+      kq::GemmNT g = {sc.Eh, sc.El, 2 * B2, Bh, Bl, ldb, W + sb_end, n, m, n - sb_end, 2 * K,
+                      -1.f, 0};
+      g.bf16 = 1;
       const int ts = kqh::timer_begin(KRONQ_TIMER_LAZY_UPDATE, st);
       const int s = kq_gemm_nt_tc(&g, 1, info, st);
       kqh::timer_end(ts, st);
@@ -875,13 +860,14 @@ int kq_layer_loss(const float* Wr, const float* Wh, int64_t m64, int64_t n64, co
 // a process that plans all of its memory at start-up and must not grow it
 // later, or a latency-sensitive loop in which cudaMalloc / cudaFree would
 // synchronise the device and stall other streams.  For them the solver's
-// scratch (the error block and the transposed U_c slab, each as tf32 hi / lo
+// scratch (the error block and the transposed U_c slab, each as bf16 hi / lo
 // planes) lives in the static device array below instead of a caller
 // workspace.
 //
 // The array is part of the library image: every GPU that loads libkronq holds
-// its 64 MiB until the process exits; it fits m <= 32768 rows and
-// n <= 32768 columns.  Host code cannot use the symbol as a device address,
+// its 64 MiB until the process exits; it holds the one-level scratch of up
+// to m = 32768 rows and n = 32768 columns (half of it), and the two-level
+// scratch whenever that fits too.  Host code cannot use the symbol as a device address,
 // so its address is looked up with cudaGetSymbolAddress once per device (with
 // that device current), on the first call made on that device.  All calls
 // share the one array and it keeps the previous call's contents: nothing in

@@ -15,6 +15,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
@@ -78,6 +79,29 @@ KQ_DEV void mma3(uint32_t d_tmem, uint32_t a_h, uint32_t a_l, uint32_t b_h, uint
   mma(d_tmem, ah, bh, 1u);
 }
 
+// The same three products from bf16 planes (kind::f16 with bf16 operands,
+// K = 16 per instruction: a K step is again 32 bytes of the 128-byte row).
+constexpr uint32_t kIdescBf16_128 = idesc_f16(128, 128, /*bf16*/ 1, /*A K-major*/ 0, /*B K-major*/ 0);
+
+KQ_DEV void mma3_bf16(uint32_t d_tmem, uint32_t a_h, uint32_t a_l, uint32_t b_h, uint32_t b_l,
+                      int kk, uint32_t accumulate) {
+  const uint64_t ah = smem_desc(a_h + kk * 32, 16, 1024, kLayoutSwizzle128B);
+  const uint64_t al = smem_desc(a_l + kk * 32, 16, 1024, kLayoutSwizzle128B);
+  const uint64_t bh = smem_desc(b_h + kk * 32, 16, 1024, kLayoutSwizzle128B);
+  const uint64_t bl = smem_desc(b_l + kk * 32, 16, 1024, kLayoutSwizzle128B);
+  mma_f16(d_tmem, al, bh, kIdescBf16_128, accumulate);
+  mma_f16(d_tmem, ah, bl, kIdescBf16_128, 1u);
+  mma_f16(d_tmem, ah, bh, kIdescBf16_128, 1u);
+}
+
+// Split x into bf16 hi = RN(x) and lo = RN(x - hi), as raw bits.
+KQ_DEV void split_bf16(float x, uint16_t& h, uint16_t& l) {
+  const __nv_bfloat16 hb = __float2bfloat16_rn(x);
+  const __nv_bfloat16 lb = __float2bfloat16_rn(x - __bfloat162float(hb));
+  h = __bfloat16_as_ushort(hb);
+  l = __bfloat16_as_ushort(lb);
+}
+
 // Bounded wait used while winding down (records a timeout, never aborts).
 KQ_DEV void drain_wait(uint64_t* bar, uint32_t parity, int32_t* info) {
   if (mbar_try_wait(bar, parity)) return;
@@ -115,6 +139,27 @@ inline bool make_map_f32(CUtensorMap* map, const float* ptr, int64_t cols, int64
   cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(ptr), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The same for a bf16 matrix (2-byte elements; ld in elements).
+inline bool make_map_bf16(CUtensorMap* map, const void* ptr, int64_t cols, int64_t rows, int64_t ld,
+                          uint32_t box_cols, uint32_t box_rows) {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return false;
+    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }

@@ -128,12 +128,14 @@ def x_chunk(cfg: Config, site: XSite, c: int, tokens: int | None = None,
 
 
 def xq_chunk(cfg: Config, site: XSite, c: int, tokens: int | None = None,
-             sigma: float = DRIFT_SIGMA, out: np.ndarray | None = None) -> np.ndarray:
+             sigma: float = DRIFT_SIGMA, out: np.ndarray | None = None,
+             x_bits: np.ndarray | None = None) -> np.ndarray:
     """Rows [c*CHUNK_TOKENS, ...) of X~, the input the same site sees in the
     partly quantized model, as bf16 bits: the bf16 values of X plus seeded
     Gaussian noise of standard deviation sigma times the channel's scale
-    (x_outlier_scale on the outlier channels, 1 elsewhere), rounded to bf16."""
-    xb = x_chunk(cfg, site, c, tokens)
+    (x_outlier_scale on the outlier channels, 1 elsewhere), rounded to bf16.
+    x_bits: the same chunk of X when the caller has drawn it already."""
+    xb = x_chunk(cfg, site, c, tokens) if x_bits is None else x_bits
     rows, d = xb.shape
     if out is None:
         out = np.empty((rows, d), dtype=np.uint16)

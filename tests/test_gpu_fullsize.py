@@ -172,10 +172,16 @@ def _sublayer_chain(cfg, sub, HX, HG, bits, r, rows=None, full_loss=False):
         np.testing.assert_array_equal(zr, ref["zero"])
     else:
         # group grids come from the already-updated weights: a code that
-        # flipped earlier in the row (equally valid, fp order) moves them a
-        # little, so the bar is the same 99.9 % as for the codes
+        # flipped earlier in the row (equally valid, fp order) moves every
+        # later grid of that row, so grids are compared on the groups with no
+        # differing code before them; those carry only the rounding of the
+        # lazy updates (bf16 hi / lo products, ~2^-17 relative)
         assert (zr == ref["zero"]).mean() >= 0.999
-        assert (np.abs(sc / ref["scale"] - 1) <= 1e-5).mean() >= 0.999
+        diff = cg[rows] != ref["codes"]
+        first_diff = np.where(diff.any(axis=1), diff.argmax(axis=1), n)
+        clean = np.arange(sc.shape[1])[None, :] * group < first_diff[:, None]
+        assert clean.mean() >= 0.9
+        assert (np.abs(sc / ref["scale"] - 1)[clean] <= 1e-5).mean() >= 0.999
     Wh = What.cpu().numpy()
     lg = oq.row_losses(Wrot[rows] - Wh[rows], HXr, cfg.damp).sum()
     lr = oq.row_losses(Wrot[rows] - ref["W_hat"], HXr, cfg.damp).sum()

@@ -14,6 +14,8 @@ oracle's values); P is checked against the oracle's P of the GPU's own A' and U_
 """
 
 import dataclasses
+import os
+from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
 import pytest
@@ -141,10 +143,15 @@ def test_llama2_7b_q_proj_gptaq_rows(cuda):
     sub, site = cfg.sublayers[0], cfg.site("attn_in")
     N, n, m = cfg.tokens, sub.n, sub.m
     XqX = torch.empty((N, 2 * n), dtype=torch.bfloat16, device=cuda)
-    for c in range(synth.n_chunks(N)):
-        r0 = c * synth.CHUNK_TOKENS
-        xb, xqb = synth.x_chunk(cfg, site, c), synth.xq_chunk(cfg, site, c)
-        XqX[r0:r0 + len(xb)].copy_(bf16_dev(_side_by_side(xqb, xb), "cpu"))
+
+    def pair(c):
+        xb = synth.x_chunk(cfg, site, c)
+        return c, _side_by_side(synth.xq_chunk(cfg, site, c, x_bits=xb), xb)
+
+    with ThreadPoolExecutor(max(1, min(16, os.cpu_count() or 1))) as ex:
+        for c, bits in ex.map(pair, range(synth.n_chunks(N))):
+            r0 = c * synth.CHUNK_TOKENS
+            XqX[r0:r0 + len(bits)].copy_(bf16_dev(bits, "cpu"))
     HX = torch.empty((n, n), device=cuda)
     A = torch.empty((n, n), device=cuda)
     ws = abi.gptaq_workspace(m, n, cuda)

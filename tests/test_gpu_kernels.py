@@ -360,7 +360,8 @@ def test_quantize_two_level_lazy_update_matches_one_level_and_oracle(cuda):
     def a256(b):
         return (b + 255) // 256 * 256
 
-    one_level = 2 * a256(m * 128 * 4) + 2 * a256(n * 128 * 4)
+    # the one-level scratch: E (m x 128) and the U_c slab (n x 128) as bf16 hi / lo planes
+    one_level = 2 * a256(m * 128 * 2) + 2 * a256(n * 128 * 2)
     outs = []
     for ws in (abi.workspace(m, n, bits, -1, device=cuda),
                torch.empty(one_level, dtype=torch.uint8, device=cuda)):

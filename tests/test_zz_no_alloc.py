@@ -30,11 +30,11 @@ def _outputs(cuda, m, n, bits, group):
 
 # Two shapes whose two-level lazy-update scratch fits the static array (the
 # same path as the workspace call) and, for the second pair of calls, a
-# 4096 x 4096 layer whose two-level scratch does not (68 MiB > 64 MiB): the
+# 16384 x 4096 layer whose two-level scratch does not (82 MiB > 64 MiB): the
 # static-array call then runs the one-level update while the workspace call
 # runs two levels, so only the summation order differs.
 @pytest.mark.parametrize("shapes", [[(300, 512, 4, -1), (520, 384, 2, 128)],
-                                    [(4096, 4096, 4, -1), (4096, 4096, 2, 128)]],
+                                    [(16384, 4096, 4, -1), (16384, 4096, 2, 128)]],
                          ids=["two-level", "one-level-fallback"])
 def test_noalloc_matches_workspace_entry_point_twice(cuda, shapes):
     for call, (m, n, bits, group) in enumerate(shapes):
