@@ -65,6 +65,9 @@ def parse():
     ap.add_argument("--rows", type=int, default=4096, help="layer rows for --kernel solver")
     ap.add_argument("--width", type=int, default=None,
                     help="feature width for --kernel (default: the workload's widest)")
+    ap.add_argument("--gptaq", action="store_true",
+                    help="time the step with GPTAQ's asymmetric calibration: the drift covariance "
+                         "of [X~ | X] in place of H_X, the correction P and the solver with it")
     ap.add_argument("--oracle-full-chain", action="store_true",
                     help="time the fp64 oracle's whole chain once on the host cores (every "
                          "token, every row) for the configuration and print one line; no GPU")
@@ -740,8 +743,123 @@ def run_kernel(args):
                       **out, "peak_source": src}), flush=True)
 
 
+def run_gptaq(args):
+    """One step per sublayer: H~, Delta X X^T = kronq_drift_covariance([X~ | X]),
+    H_G, BiIP, the drift covariance rotated like H~, inverse Cholesky, P,
+    the column loop with the P term, packing.  Inputs resident in HBM."""
+    import dataclasses
+    import numpy as np
+    import torch
+    import synth
+    from post_quantization_02_b200 import abi
+    from concurrent.futures import ThreadPoolExecutor
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    cfg = synth.get_config(args.config)
+    if args.tokens:
+        cfg = dataclasses.replace(cfg, tokens=args.tokens)
+    N = cfg.tokens
+    t_gen = time.perf_counter()
+    xqx, gs = {}, {}
+    for site in cfg.sites:
+        buf = torch.empty((N, 2 * site.width), dtype=torch.bfloat16, device=dev)
+
+        def pair(c, site=site):
+            xb = synth.x_chunk(cfg, site, c)
+            return c, np.concatenate([synth.xq_chunk(cfg, site, c, x_bits=xb), xb], axis=1)
+
+        with ThreadPoolExecutor(max(1, min(16, os.cpu_count() or 1))) as ex:
+            for c, bits in ex.map(pair, range(synth.n_chunks(N))):
+                r0 = c * synth.CHUNK_TOKENS
+                buf[r0:r0 + len(bits)].copy_(torch.from_numpy(np.ascontiguousarray(bits).view(np.int16))
+                                             .view(torch.bfloat16))
+        xqx[site.name] = buf
+    for sub in cfg.sublayers:
+        gs[sub.name] = torch.from_numpy(synth.make_g(cfg, sub).view(np.int16)).to(dev).view(torch.bfloat16)
+    t_gen = time.perf_counter() - t_gen
+    L = []
+    for sub in cfg.sublayers:
+        m, n = sub.m, sub.n
+        su, sv = synth.make_signs(cfg, sub)
+        G = 1 if sub.group == -1 else n // sub.group
+        L.append(dict(sub=sub, W0=torch.from_numpy(synth.make_w(cfg, sub)).to(dev),
+                      W=torch.empty((m, n), device=dev), HX=torch.empty((n, n), device=dev),
+                      A=torch.empty((n, n), device=dev), HG=torch.empty((m, m), device=dev),
+                      U=torch.empty((n, n), device=dev), P=torch.empty((n, n), device=dev),
+                      SX=torch.empty(n, device=dev), SG=torch.empty(m, device=dev),
+                      su=torch.from_numpy(su).to(dev), sv=torch.from_numpy(sv).to(dev),
+                      codes=torch.empty((m, n), dtype=torch.uint8, device=dev),
+                      scales=torch.empty((m, G), device=dev),
+                      zeros=torch.empty((m, G), dtype=torch.uint8, device=dev),
+                      packed=torch.empty((m, abi.packed_words(n, sub.bits or 4)), dtype=torch.int32,
+                                         device=dev)))
+    ws = abi.gptaq_workspace(max(s.m for s in cfg.sublayers), max(s.n for s in cfg.sublayers), dev)
+    info = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    ev = {}
+
+    def step(marks=None):
+        def mark(k):
+            if marks is not None:
+                e = torch.cuda.Event(enable_timing=True)
+                e.record(stream)
+                marks.append((k, e))
+        mark("start")
+        for d in L:
+            sub = d["sub"]
+            abi.kronq_drift_covariance(xqx[sub.site], d["HX"], d["A"], info, ws)
+            abi.kronq_covariance(gs[sub.name], d["HG"], 1.0 / N, 0.0)
+        mark("covariances")
+        for d in L:
+            sub = d["sub"]
+            d["W"].copy_(d["W0"])
+            abi.kronq_biip_rotate(d["W"], d["HX"], d["HG"], d["su"], d["sv"], cfg.alpha, cfg.mode, 0,
+                                  d["SX"], d["SG"], ws)
+            abi.kronq_biip_rotate_input(d["A"], d["SX"], d["sv"], cfg.mode, ws)
+            abi.kronq_cholesky_inv(d["HX"], cfg.damp, d["U"], info, ws)
+            abi.kronq_gptaq_correction(d["A"], d["U"], 0.25, d["P"], info, ws)
+        mark("biip_cholesky_correction")
+        for d in L:
+            sub = d["sub"]
+            abi.kronq_quantize_layer_gptaq(d["W"], d["U"], d["P"], sub.bits, sub.group, cfg.block,
+                                           d["codes"], d["scales"], d["zeros"], None, info, ws)
+            if sub.bits in (2, 4):
+                abi.kronq_pack(d["codes"], sub.bits, d["packed"])
+        mark("solver_pack")
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if info.item() != 0:
+        raise RuntimeError(f"device status {info.item()} in warm-up")
+    marks_all = []
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        marks = []
+        step(marks)
+        marks_all.append(marks)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    stages = {}
+    for marks in marks_all:
+        for (_, a), (k, b2) in zip(marks, marks[1:]):
+            stages[k] = stages.get(k, 0.0) + a.elapsed_time(b2) / args.steps
+    print(json.dumps({"metric": METRIC + " (GPTAQ asymmetric calibration)", "value":
+                      cfg.weights / (ms / 1e3) / 1e6, "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+                      "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+                      "dtype": "bf16", "data": "synthetic (seeded generator; drifted X~ = X + noise)",
+                      "config": {"workload": workload_desc(cfg) + "; GPTAQ alpha 0.25",
+                                 "input_gen_s": round(t_gen, 1)},
+                      "stages_ms": {k: round(v, 3) for k, v in stages.items()}}), flush=True)
+
+
 def main():
     args = parse()
+    if args.gptaq:
+        run_gptaq(args)
+        return
     if args.kernel:
         run_kernel(args)
         return

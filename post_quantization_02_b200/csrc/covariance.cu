@@ -343,6 +343,12 @@ constexpr int P_A_BYTES = P_BM * BK * 2;             // 16 KB
 constexpr int P_B_BYTES = (P_TILE / 2) * BK * 2;     // 16 KB
 constexpr int P_STAGE_BYTES = P_A_BYTES + P_B_BYTES; // 32 KB
 constexpr int P_SMEM_BYTES = P_STAGES * P_STAGE_BYTES + 1024 + 256;
+// warps 0-3: TMA producer, MMA issuer, TMEM allocator, idle; warps 4-11: the
+// epilogue, two per TMEM lane quadrant (128 columns each), so that folding
+// the accumulator into the master (which the next chunk's MMAs wait for)
+// takes few round trips to TMEM
+constexpr int P_THREADS = 384;
+constexpr int P_EPI_WARPS = 8;
 constexpr uint32_t P_IDESC = kq::idesc_f16(2 * P_BM, P_TILE, /*bf16*/ 1, /*A MN-major*/ 1, /*B MN-major*/ 1);
 static_assert(P_SMEM_BYTES <= 227 * 1024, "pair ring exceeds the shared-memory limit");
 
@@ -429,7 +435,7 @@ __device__ __forceinline__ bool pair_segment(const PairSchedule& S, int p, int n
   return true;
 }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
 cov_pair_kernel(const __grid_constant__ CUtensorMap tmap, float* __restrict__ H, int64_t ldh, int d,
                 int k_iters, const PairSchedule sched, float alpha, float beta, int32_t* info) {
   extern __shared__ uint8_t smem_raw[];
@@ -448,7 +454,7 @@ cov_pair_kernel(const __grid_constant__ CUtensorMap tmap, float* __restrict__ H,
       kq::mbar_init(&bars->empty[s], 1);
     }
     kq::mbar_init(&bars->tfull, 1);
-    kq::mbar_init(&bars->tempty, 8);
+    kq::mbar_init(&bars->tempty, 2 * P_EPI_WARPS);   // every epilogue warp of both CTAs
     kq::mbar_init(&bars->drain, 1);
     bars->abort = 0;
     kq::fence_barrier_init();
@@ -531,7 +537,9 @@ cov_pair_kernel(const __grid_constant__ CUtensorMap tmap, float* __restrict__ H,
     }
   } else if (warp >= 4) {
     // -------------------------------------------------- epilogue (both CTAs)
-    const int q = warp & 3;
+    // warp 4 + 4 h + q: TMEM lane quadrant q (a warp may only read its own
+    // quadrant), tile columns [128 h, 128 h + 128)
+    const int q = warp & 3, cbeg = 128 * ((warp - 4) >> 2);
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     const uint32_t tempty_leader = kq::map_to_rank(kq::smem_u32(&bars->tempty), 0);
     int cc = 0;
@@ -548,8 +556,9 @@ cov_pair_kernel(const __grid_constant__ CUtensorMap tmap, float* __restrict__ H,
         const bool first = ch == c0, last = ch == c1 - 1;
         if (!kq::mbar_wait(&bars->tfull, (uint32_t)cc & 1u, abort, info)) { ok = false; break; }
         kq::tc_fence_after();
+        // fold: master = acc (first chunk) or master + acc (rounded to nearest)
 #pragma unroll 1
-        for (int c = 0; c < P_TILE; c += 32) {
+        for (int c = cbeg; c < cbeg + 128; c += 32) {
           if (j0 + c >= d) break;
           if (j0 + c + 31 < row0) continue;
           float v[32], mst[32];
@@ -569,7 +578,7 @@ cov_pair_kernel(const __grid_constant__ CUtensorMap tmap, float* __restrict__ H,
         if (lane == 0) kq::mbar_arrive_cluster(tempty_leader);
         if (!last) continue;
 #pragma unroll 1
-        for (int c = 0; c < P_TILE; c += 32) {
+        for (int c = cbeg; c < cbeg + 128; c += 32) {
           const int jc = j0 + c;
           if (jc >= d) break;
           if (jc + 31 < row0) continue;
@@ -723,7 +732,7 @@ int kq_covariance(const uint16_t* A, int64_t N, int64_t d, int64_t lda, float* H
         return 0;
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(2 * (kqh::num_sms() / 2), 1, 1);
-      cfg.blockDim = dim3(THREADS, 1, 1);
+      cfg.blockDim = dim3(P_THREADS, 1, 1);
       cfg.dynamicSmemBytes = P_SMEM_BYTES;
       int n = 0;
       if (cudaOccupancyMaxActiveClusters(&n, cov_pair_kernel, &cfg) != cudaSuccess || n <= 0) {
@@ -760,7 +769,7 @@ int kq_covariance(const uint16_t* A, int64_t N, int64_t d, int64_t lda, float* H
       KQ_CHECK_LAUNCH();
     }
     const float beta_owned = beta;
-    cov_pair_kernel<<<2 * pairs, THREADS, P_SMEM_BYTES, st>>>(tmap, H, ldh, (int)d, k_iters, sc,
+    cov_pair_kernel<<<2 * pairs, P_THREADS, P_SMEM_BYTES, st>>>(tmap, H, ldh, (int)d, k_iters, sc,
                                                              alpha, beta_owned, info);
     KQ_CHECK_LAUNCH();
     if (shared) {
