@@ -22,6 +22,8 @@
 //                  R[k+128:, k+128:] -= L L^T (lower triangle) and
 //                  Z[:k+128, k+128:] -= Z[:k+128, k:k+128] L^T, L = the panel rows.
 // Then U_c[a][b] = Z[n-1-b][n-1-a] (a <= b).
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 #include "gemm_tc.cuh"
 #include "tf32x3.cuh"
@@ -486,6 +488,67 @@ __global__ void __launch_bounds__(256) reverse_out_kernel(const float* __restric
   }
 }
 
+// Rows of the fp32 values held as tf32 hi / lo planes (x = hi + lo exactly;
+// rows * K values from column 0, leading dimension ld) as fp16 hi / lo planes
+// of x * 2^e_i with e_i chosen so that the row's largest |x| * 2^e_i lies in
+// [2^13, 2^14): fp16 keeps 11 + 11 bits of every entry within 2^-17 of the
+// row's largest, smaller ones lose only absolute precision far below that
+// entry's contribution.  inv[i] = 2^-e_i (1 for an all-zero row).  One warp
+// per row, K a multiple of 128 (up to 1024).
+__global__ void __launch_bounds__(256) fp16_rows_kernel(const float* __restrict__ Sh,
+                                                        const float* __restrict__ Sl, int rows,
+                                                        int K, int ld, __half* __restrict__ Dh,
+                                                        __half* __restrict__ Dl,
+                                                        float* __restrict__ inv) {
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const float* h = Sh + (int64_t)row * ld;
+  const float* l = Sl + (int64_t)row * ld;
+  float x[32];
+  float mx = 0.f;
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const int c = 4 * lane + 128 * u;
+    if (c < K) {
+      const float4 a = *reinterpret_cast<const float4*>(h + c);
+      const float4 b = *reinterpret_cast<const float4*>(l + c);
+      x[4 * u] = a.x + b.x;
+      x[4 * u + 1] = a.y + b.y;
+      x[4 * u + 2] = a.z + b.z;
+      x[4 * u + 3] = a.w + b.w;
+    } else {
+      x[4 * u] = x[4 * u + 1] = x[4 * u + 2] = x[4 * u + 3] = 0.f;
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) mx = fmaxf(mx, fabsf(x[4 * u + q]));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  int e2 = 0;
+  if (mx > 0.f) {
+    frexpf(mx, &e2);                     // mx = f 2^e2, f in [0.5, 1)
+    e2 = 14 - e2;                        // mx 2^e2 in [2^13, 2^14)
+  }
+  if (lane == 0) inv[row] = ldexpf(1.f, -e2);
+  __half* dh = Dh + (int64_t)row * ld;
+  __half* dl = Dl + (int64_t)row * ld;
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const int c = 4 * lane + 128 * u;
+    if (c < K) {
+      __half hh[4], ll[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float v = ldexpf(x[4 * u + q], e2);
+        hh[q] = __float2half_rn(v);
+        ll[q] = __float2half_rn(v - __half2float(hh[q]));
+      }
+      *reinterpret_cast<uint2*>(dh + c) = *reinterpret_cast<const uint2*>(hh);
+      *reinterpret_cast<uint2*>(dl + c) = *reinterpret_cast<const uint2*>(ll);
+    }
+  }
+}
+
 size_t align256(size_t b) { return (b + 255) & ~(size_t)255; }
 
 constexpr size_t kPanelSmem = (size_t)SM_FLOATS * sizeof(float);
@@ -503,7 +566,9 @@ int64_t plane_ld(int64_t np) { return np < SBW ? np : SBW; }
 size_t kq_cholesky_ws(int64_t n) {
   const int64_t np = padded(n);
   return align256(sizeof(double)) + 2 * align256((size_t)np * np * sizeof(float)) +
-         4 * align256((size_t)np * plane_ld(np) * sizeof(float));
+         4 * align256((size_t)np * plane_ld(np) * sizeof(float)) +
+         4 * align256((size_t)np * plane_ld(np) * sizeof(__half)) +
+         2 * align256((size_t)np * sizeof(float));
 }
 
 int kq_cholesky_inv(const float* H, int64_t n64, float damp_rel, float* U, int32_t* info, void* ws,
@@ -531,6 +596,15 @@ int kq_cholesky_inv(const float* H, int64_t n64, float damp_rel, float* U, int32
     w += align256((size_t)np * ldp * sizeof(float));
   }
   float *Lh = planes[0], *Ll = planes[1], *Zh = planes[2], *Zl = planes[3];
+  // the outer updates' operands: fp16 planes of row-scaled L and Z, and the rows' factors
+  __half* p16[4];
+  for (int i = 0; i < 4; ++i) {
+    p16[i] = reinterpret_cast<__half*>(w);
+    w += align256((size_t)np * ldp * sizeof(__half));
+  }
+  float* sL = reinterpret_cast<float*>(w);
+  w += align256((size_t)np * sizeof(float));
+  float* sZ = reinterpret_cast<float*>(w);
 
   const int sms = kqh::num_sms();
   diag_sum_kernel<<<1, 1024, 0, st>>>(H, n, dsum);
@@ -576,16 +650,27 @@ int kq_cholesky_inv(const float* H, int64_t n64, float damp_rel, float* U, int32
     }
     const int rest = np - kb_end;
     if (rest > 0) {
-      // the trailing matrix, once per super-block (K = kb_end - kb):
+      // the trailing matrix, once per super-block (K = kb_end - kb), on fp16
+      // planes of row-scaled operands (twice the tf32 rate, ~2^-22 relative):
       //   R[kb_end:, kb_end:] -= L L^T (lower triangle),  L = L[kb_end:, kb:kb_end]
       //   Z[:kb_end, kb_end:] -= Z[:kb_end, kb:kb_end] L^T
       const int K = kb_end - kb;
       const int64_t lr = (int64_t)kb_end * ldp;
-      kq::GemmNT g[2];
-      g[0] = {Lh + lr, Ll + lr, ldp, Lh + lr, Ll + lr, ldp, R + (int64_t)kb_end * np + kb_end, np,
-              rest, rest, K, -1.f, 1};
-      g[1] = {Zh, Zl, ldp, Lh + lr, Ll + lr, ldp, Z + kb_end, np, kb_end, rest, K, -1.f, 0};
       const int tu = kqh::timer_begin(KRONQ_TIMER_CHOL_UPDATE, st);
+      fp16_rows_kernel<<<(rest + 7) / 8, 256, 0, st>>>(Lh + lr, Ll + lr, rest, K, ldp, p16[0] + lr,
+                                                       p16[1] + lr, sL + kb_end);
+      KQ_CHECK_LAUNCH();
+      fp16_rows_kernel<<<(kb_end + 7) / 8, 256, 0, st>>>(Zh, Zl, kb_end, K, ldp, p16[2], p16[3], sZ);
+      KQ_CHECK_LAUNCH();
+      kq::GemmNT g[2];
+      g[0] = {p16[0] + lr, p16[1] + lr, ldp, p16[0] + lr, p16[1] + lr, ldp,
+              R + (int64_t)kb_end * np + kb_end, np, rest, rest, K, -1.f, 1};
+      g[1] = {p16[2], p16[3], ldp, p16[0] + lr, p16[1] + lr, ldp, Z + kb_end, np, kb_end, rest, K,
+              -1.f, 0};
+      g[0].fp16 = g[1].fp16 = 1;
+      g[0].a_scale = g[0].b_scale = sL + kb_end;
+      g[1].a_scale = sZ;
+      g[1].b_scale = sL + kb_end;
       const int s = kq_gemm_nt_tc(g, 2, info, st);
       kqh::timer_end(tu, st);
       if (s != KRONQ_OK) return s;

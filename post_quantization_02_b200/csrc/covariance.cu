@@ -28,6 +28,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <mutex>
+
 #include "common.cuh"
 
 namespace {
@@ -435,9 +437,30 @@ __device__ __forceinline__ bool pair_segment(const PairSchedule& S, int p, int n
   return true;
 }
 
+// Keeping the pairs of a launch at the same token offset.  Every pair
+// streams all N tokens for each of its tiles, so the pairs of one wave share
+// each token slab through L2 only while they stay together; left alone they
+// drift apart over many waves (measured: ~1.2 TB of DRAM reads for one
+// 28672-wide launch over 262144 tokens, ~80x the input).  Before its next
+// wave's tile, a producer waits until every producer of the launch has
+// issued the loads of the current wave (the counter reaches target).  The
+// wait is a timing hint, not a guard: it gives up after kWaveGateNs without
+// recording anything, and nothing depends on it for correctness.
+constexpr unsigned long long kWaveGateNs = 2000000ull;  // 2 ms
+
+__device__ __forceinline__ void wave_gate(const unsigned int* ctr, unsigned int target) {
+  if (*reinterpret_cast<const volatile unsigned int*>(ctr) >= target) return;
+  const unsigned long long t0 = kq::globaltimer();
+  while (*reinterpret_cast<const volatile unsigned int*>(ctr) < target) {
+    if (kq::globaltimer() - t0 > kWaveGateNs) return;
+    __nanosleep(256);
+  }
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
 cov_pair_kernel(const __grid_constant__ CUtensorMap tmap, float* __restrict__ H, int64_t ldh, int d,
-                int k_iters, const PairSchedule sched, float alpha, float beta, int32_t* info) {
+                int k_iters, const PairSchedule sched, float alpha, float beta, int32_t* info,
+                unsigned int* wave_ctr) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* tiles = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -476,6 +499,7 @@ cov_pair_kernel(const __grid_constant__ CUtensorMap tmap, float* __restrict__ H,
         pair_tile_coords(t, sched.nb, rb, cb);
         const int i0 = rb * P_TILE + P_BM * (int)rank;          // this CTA's rows of the tile
         const int j0 = cb * P_TILE + (P_TILE / 2) * (int)rank;  // this CTA's half of the columns
+        if (wave_ctr && sg > 0 && sg < sched.waves) wave_gate(wave_ctr, 2u * (unsigned)ncl * (unsigned)sg);
         bool ok = true;
         const int kb_end = min(k_iters, c1 * KC_ITERS);
         for (int kb = c0 * KC_ITERS; kb < kb_end; ++kb, ++it) {
@@ -493,6 +517,8 @@ cov_pair_kernel(const __grid_constant__ CUtensorMap tmap, float* __restrict__ H,
           kq::tma_load_2d_pair(b + BOX_BYTES, &tmap, fb, j0 + 64, y);
         }
         if (!ok) break;
+        // this producer has issued its whole tile of the wave
+        if (wave_ctr && sg < sched.waves) atomicAdd(wave_ctr, 1u);
       }
       // wind down (even CTA): every armed phase has landed, the odd CTA's
       // bytes included, before the pair may exit
@@ -691,6 +717,32 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
 
 }  // namespace
 
+// The wave counter of cov_pair_kernel: one word per device (a static device
+// variable of the library), reset before every launch on the launch's stream.
+// Launches that overlap on the GPU share it; then a gate may open early or
+// give up after its time limit -- only the timing changes.
+static __device__ unsigned int g_cov_wave_ctr;
+
+namespace {
+std::mutex g_wave_mutex;
+unsigned int* g_wave_ptr[64] = {};
+
+unsigned int* wave_counter() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(g_wave_mutex);
+  if (!g_wave_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_cov_wave_ctr) != cudaSuccess || !p) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    g_wave_ptr[dev] = static_cast<unsigned int*>(p);
+  }
+  return g_wave_ptr[dev];
+}
+}  // namespace
+
 int kq_covariance(const uint16_t* A, int64_t N, int64_t d, int64_t lda, float* H, int64_t ldh,
                   float alpha, float beta, int32_t* info, cudaStream_t st) {
   if (d < 0 || N < 0) return KRONQ_ERR_INVALID_ARG;
@@ -769,8 +821,10 @@ int kq_covariance(const uint16_t* A, int64_t N, int64_t d, int64_t lda, float* H
       KQ_CHECK_LAUNCH();
     }
     const float beta_owned = beta;
+    unsigned int* wctr = sc.waves > 1 ? wave_counter() : nullptr;
+    if (wctr && cudaMemsetAsync(wctr, 0, sizeof(unsigned int), st) != cudaSuccess) return KRONQ_ERR_CUDA;
     cov_pair_kernel<<<2 * pairs, P_THREADS, P_SMEM_BYTES, st>>>(tmap, H, ldh, (int)d, k_iters, sc,
-                                                             alpha, beta_owned, info);
+                                                             alpha, beta_owned, info, wctr);
     KQ_CHECK_LAUNCH();
     if (shared) {
       mirror_tiles_kernel<<<list.count * 64, 256, 0, st>>>(H, ldh, (int)d, list);

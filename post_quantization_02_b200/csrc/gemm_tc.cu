@@ -67,6 +67,8 @@ KQ_DEV void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "me
 
 struct Problem {
   float* C;
+  const float* a_scale;   // fp16 planes only: per-row and per-column factors of the product
+  const float* b_scale;
   int64_t ldc;
   int M, N, K;
   float alpha;
@@ -107,13 +109,14 @@ __device__ __forceinline__ Tile tile_of(const Problems& P, int t) {
   return r;
 }
 
-// BF16 = false: tf32 planes (32 fp32 K values per 128-byte row);
-// true: bf16 planes (64 bf16 K values per row).
-template <bool BF16>
+// KIND 0: tf32 planes (32 fp32 K values per 128-byte row); 1: bf16 planes;
+// 2: fp16 planes of scaled rows (64 K values per row; the epilogue applies
+// the rows' and columns' factors).
+template <int KIND>
 __global__ void __launch_bounds__(THREADS, 1)
 gemm_nt_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Problems P,
                   int32_t* info) {
-  constexpr int KC = BF16 ? 64 : 32;
+  constexpr int KC = KIND ? 64 : 32;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* stages = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -196,9 +199,12 @@ gemm_nt_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Pro
           const uint32_t a = kq::smem_u32(stages + s * STAGE_BYTES);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {     // four 32-byte K steps per 128-byte row
-            if (BF16)
-              kq::tf32x3::mma3_bf16(d_tmem, a, a + CHUNK, a + 2 * CHUNK, a + 3 * CHUNK, kk,
-                                    (kc == 0 && kk == 0) ? 0u : 1u);
+            if (KIND == 1)
+              kq::tf32x3::mma3_16(d_tmem, a, a + CHUNK, a + 2 * CHUNK, a + 3 * CHUNK, kk,
+                                  (kc == 0 && kk == 0) ? 0u : 1u, kq::tf32x3::kIdescBf16_128);
+            else if (KIND == 2)
+              kq::tf32x3::mma3_16(d_tmem, a, a + CHUNK, a + 2 * CHUNK, a + 3 * CHUNK, kk,
+                                  (kc == 0 && kk == 0) ? 0u : 1u, kq::tf32x3::kIdescFp16_128);
             else
               kq::tf32x3::mma3(d_tmem, a, a + CHUNK, a + 2 * CHUNK, a + 3 * CHUNK, kk,
                                (kc == 0 && kk == 0) ? 0u : 1u);
@@ -237,7 +243,9 @@ gemm_nt_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Pro
       kq::tc_fence_before();
       __syncwarp();
       if (lane == 0) kq::mbar_arrive(&bars->tempty[buf]);
-      const float al = pr.alpha;
+      // the row's factor (fp16 planes), else alpha alone
+      const int grow = tl.tm * TM + rt;
+      const float al = (KIND == 2 && grow < pr.M) ? pr.alpha * pr.a_scale[grow] : pr.alpha;
       const bool diag = pr.lower && tl.tm == tl.tn;
 #pragma unroll
       for (int c2 = 0; c2 < 2; ++c2) {
@@ -253,6 +261,14 @@ gemm_nt_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Pro
           o.y = al * v[c2][4 * ch + 1];
           o.z = al * v[c2][4 * ch + 2];
           o.w = al * v[c2][4 * ch + 3];
+          if (KIND == 2) {
+            // the columns' factors (B rows); beyond N the box is clipped anyway
+            const int gc = tl.tn * TN + ct + 4 * ch;
+            o.x *= gc < pr.N ? pr.b_scale[gc] : 0.f;
+            o.y *= gc + 1 < pr.N ? pr.b_scale[gc + 1] : 0.f;
+            o.z *= gc + 2 < pr.N ? pr.b_scale[gc + 2] : 0.f;
+            o.w *= gc + 3 < pr.N ? pr.b_scale[gc + 3] : 0.f;
+          }
           if (diag) {                                 // keep the strict upper triangle untouched
             const int c = ct + 4 * ch;
             if (c > rt) o.x = 0.f;
@@ -292,13 +308,15 @@ int kq_gemm_nt_tc(const kq::GemmNT* probs, int count, int32_t* info, cudaStream_
   Problems P;
   P.count = 0;
   P.total_tiles = 0;
-  const int bf16 = probs[0].bf16;
-  const int KC = bf16 ? 64 : 32;
-  const int64_t lda_align = bf16 ? 8 : 4;          // 16-byte rows
+  const int bf16 = probs[0].bf16, fp16 = probs[0].fp16;
+  const int kind = fp16 ? 2 : (bf16 ? 1 : 0);
+  const int KC = kind ? 64 : 32;
+  const int64_t lda_align = kind ? 8 : 4;          // 16-byte rows
   for (int i = 0; i < count; ++i) {
     const kq::GemmNT& g = probs[i];
     if (g.M <= 0 || g.N <= 0 || g.K <= 0) continue;
-    if (g.bf16 != bf16) return KRONQ_ERR_INVALID_ARG;
+    if (g.bf16 != bf16 || g.fp16 != fp16 || (bf16 && fp16)) return KRONQ_ERR_INVALID_ARG;
+    if (fp16 && (!g.a_scale || !g.b_scale)) return KRONQ_ERR_INVALID_ARG;
     if (!g.A_hi || !g.A_lo || !g.B_hi || !g.B_lo || !g.C || g.lda % lda_align ||
         g.ldb % lda_align || g.ldc % 4 || !kqh::aligned(g.A_hi, 16) ||
         !kqh::aligned(g.A_lo, 16) || !kqh::aligned(g.B_hi, 16) || !kqh::aligned(g.B_lo, 16) ||
@@ -307,11 +325,11 @@ int kq_gemm_nt_tc(const kq::GemmNT* probs, int count, int32_t* info, cudaStream_
     if (g.lower && g.M != g.N) return KRONQ_ERR_INVALID_ARG;
     const int j = P.count;
     bool ok;
-    if (bf16)
-      ok = kqh::make_map_bf16(&maps.a_hi[j], g.A_hi, g.K, g.M, g.lda, KC, TM) &&
-           kqh::make_map_bf16(&maps.a_lo[j], g.A_lo, g.K, g.M, g.lda, KC, TM) &&
-           kqh::make_map_bf16(&maps.b_hi[j], g.B_hi, g.K, g.N, g.ldb, KC, TN) &&
-           kqh::make_map_bf16(&maps.b_lo[j], g.B_lo, g.K, g.N, g.ldb, KC, TN);
+    if (kind)
+      ok = kqh::make_map_bf16(&maps.a_hi[j], g.A_hi, g.K, g.M, g.lda, KC, TM, fp16) &&
+           kqh::make_map_bf16(&maps.a_lo[j], g.A_lo, g.K, g.M, g.lda, KC, TM, fp16) &&
+           kqh::make_map_bf16(&maps.b_hi[j], g.B_hi, g.K, g.N, g.ldb, KC, TN, fp16) &&
+           kqh::make_map_bf16(&maps.b_lo[j], g.B_lo, g.K, g.N, g.ldb, KC, TN, fp16);
     else
       ok = kqh::make_map_f32(&maps.a_hi[j], static_cast<const float*>(g.A_hi), g.K, g.M, g.lda, KC, TM) &&
            kqh::make_map_f32(&maps.a_lo[j], static_cast<const float*>(g.A_lo), g.K, g.M, g.lda, KC, TM) &&
@@ -320,6 +338,8 @@ int kq_gemm_nt_tc(const kq::GemmNT* probs, int count, int32_t* info, cudaStream_
     if (!ok || !kqh::make_map_f32(&maps.c[j], g.C, g.N, g.M, g.ldc, 32, 32)) return KRONQ_ERR_CUDA;
     Problem& q = P.p[j];
     q.C = g.C;
+    q.a_scale = g.a_scale;
+    q.b_scale = g.b_scale;
     q.ldc = g.ldc;
     q.M = g.M;
     q.N = g.N;
@@ -339,16 +359,19 @@ int kq_gemm_nt_tc(const kq::GemmNT* probs, int count, int32_t* info, cudaStream_
   }
   if (P.count == 0) return KRONQ_OK;
   if (P.count == 1) P.p[1] = P.p[0];
-  static kqh::PerDevice attr_tf32, attr_bf16;
-  if (bf16 ? kqh::smem_attr_once(attr_bf16, gemm_nt_tc_kernel<true>, SMEM_BYTES) <= 0
-           : kqh::smem_attr_once(attr_tf32, gemm_nt_tc_kernel<false>, SMEM_BYTES) <= 0)
-    return KRONQ_ERR_CUDA;
+  static kqh::PerDevice attr[3];
+  const int a_ok = kind == 2   ? kqh::smem_attr_once(attr[2], gemm_nt_tc_kernel<2>, SMEM_BYTES)
+                   : kind == 1 ? kqh::smem_attr_once(attr[1], gemm_nt_tc_kernel<1>, SMEM_BYTES)
+                               : kqh::smem_attr_once(attr[0], gemm_nt_tc_kernel<0>, SMEM_BYTES);
+  if (a_ok <= 0) return KRONQ_ERR_CUDA;
   int grid = P.total_tiles < kqh::num_sms() ? P.total_tiles : kqh::num_sms();
   if (max_ctas > 0 && grid > max_ctas) grid = max_ctas;
-  if (bf16)
-    gemm_nt_tc_kernel<true><<<grid, THREADS, SMEM_BYTES, st>>>(maps, P, info);
+  if (kind == 2)
+    gemm_nt_tc_kernel<2><<<grid, THREADS, SMEM_BYTES, st>>>(maps, P, info);
+  else if (kind == 1)
+    gemm_nt_tc_kernel<1><<<grid, THREADS, SMEM_BYTES, st>>>(maps, P, info);
   else
-    gemm_nt_tc_kernel<false><<<grid, THREADS, SMEM_BYTES, st>>>(maps, P, info);
+    gemm_nt_tc_kernel<0><<<grid, THREADS, SMEM_BYTES, st>>>(maps, P, info);
   KQ_CHECK_LAUNCH();
   return KRONQ_OK;
 }

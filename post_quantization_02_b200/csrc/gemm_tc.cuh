@@ -12,7 +12,11 @@ namespace kq {
 //   bf16 = 0: fp32 planes, A_hi exactly a tf32 value (the low 13 mantissa
 //             bits clear) and A_lo the fp32 remainder;
 //   bf16 = 1: bf16 planes, A_hi = RN_bf16(A) and A_lo = RN_bf16(A - A_hi)
-//             (A = A_hi + A_lo to about 2^-17 relative).
+//             (A = A_hi + A_lo to about 2^-17 relative);
+//   fp16 = 1: fp16 planes of rows scaled by exact powers of two (row i of A
+//             holds A[i][:] * 2^a_i in [2^13, 2^14) at its largest entry,
+//             split as fp16 hi / lo: about 2^-22 relative); a_scale[i] =
+//             2^-a_i and b_scale[j] = 2^-b_j undo the scaling in the epilogue.
 // lower = 1: M == N and only the lower triangle of C (tile by tile, the
 // diagonal tiles on and below the diagonal) is updated.  Pointers 16-byte
 // aligned, leading dimensions multiples of 16 bytes.
@@ -34,6 +38,9 @@ struct GemmNT {
   int tile_begin = 0;
   int tile_end = -1;
   int bf16 = 0;
+  int fp16 = 0;
+  const float* a_scale = nullptr;   // fp16 planes: per A row (M)
+  const float* b_scale = nullptr;   // fp16 planes: per B row (N)
 };
 
 }  // namespace kq

@@ -83,15 +83,18 @@ KQ_DEV void mma3(uint32_t d_tmem, uint32_t a_h, uint32_t a_l, uint32_t b_h, uint
 // K = 16 per instruction: a K step is again 32 bytes of the 128-byte row).
 constexpr uint32_t kIdescBf16_128 = idesc_f16(128, 128, /*bf16*/ 1, /*A K-major*/ 0, /*B K-major*/ 0);
 
-KQ_DEV void mma3_bf16(uint32_t d_tmem, uint32_t a_h, uint32_t a_l, uint32_t b_h, uint32_t b_l,
-                      int kk, uint32_t accumulate) {
+constexpr uint32_t kIdescFp16_128 = idesc_f16(128, 128, /*fp16*/ 0, /*A K-major*/ 0, /*B K-major*/ 0);
+
+// idesc: kIdescBf16_128 (bf16 planes) or kIdescFp16_128 (fp16 planes)
+KQ_DEV void mma3_16(uint32_t d_tmem, uint32_t a_h, uint32_t a_l, uint32_t b_h, uint32_t b_l, int kk,
+                    uint32_t accumulate, uint32_t idesc) {
   const uint64_t ah = smem_desc(a_h + kk * 32, 16, 1024, kLayoutSwizzle128B);
   const uint64_t al = smem_desc(a_l + kk * 32, 16, 1024, kLayoutSwizzle128B);
   const uint64_t bh = smem_desc(b_h + kk * 32, 16, 1024, kLayoutSwizzle128B);
   const uint64_t bl = smem_desc(b_l + kk * 32, 16, 1024, kLayoutSwizzle128B);
-  mma_f16(d_tmem, al, bh, kIdescBf16_128, accumulate);
-  mma_f16(d_tmem, ah, bl, kIdescBf16_128, 1u);
-  mma_f16(d_tmem, ah, bh, kIdescBf16_128, 1u);
+  mma_f16(d_tmem, al, bh, idesc, accumulate);
+  mma_f16(d_tmem, ah, bl, idesc, 1u);
+  mma_f16(d_tmem, ah, bh, idesc, 1u);
 }
 
 // Split x into bf16 hi = RN(x) and lo = RN(x - hi), as raw bits.
@@ -143,9 +146,9 @@ inline bool make_map_f32(CUtensorMap* map, const float* ptr, int64_t cols, int64
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// The same for a bf16 matrix (2-byte elements; ld in elements).
+// The same for a 2-byte matrix (bf16, or fp16 with fp16 = true; ld in elements).
 inline bool make_map_bf16(CUtensorMap* map, const void* ptr, int64_t cols, int64_t rows, int64_t ld,
-                          uint32_t box_cols, uint32_t box_rows) {
+                          uint32_t box_cols, uint32_t box_rows, bool fp16 = false) {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (!fn) {
     void* p = nullptr;
@@ -159,7 +162,8 @@ inline bool make_map_bf16(CUtensorMap* map, const void* ptr, int64_t cols, int64
   cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
   cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+  return fn(map, fp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+            const_cast<void*>(ptr), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }

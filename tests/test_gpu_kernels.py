@@ -214,7 +214,10 @@ def test_biip_alpha_half_exchanges_diagonal_and_norms_on_gpu(cuda):
 
 
 # ---------------------------------------------------------- inverse Cholesky
-@pytest.mark.parametrize("n", [64, 72, 200, 256, 1000])
+# n <= 1024 stays inside one 1024-wide super-block; 2304 and 3000 take outer
+# (K = 1024) updates on fp16 row-scaled planes, 3000 also padding and a ragged
+# last super-block
+@pytest.mark.parametrize("n", [64, 72, 200, 256, 1000, 2304, 3000])
 def test_cholesky_inv_matches_oracle(cuda, n):
     r = np.random.default_rng(n)
     H = spd(r, n, spread=1.5)
