@@ -368,8 +368,7 @@ def run_reference(args, rank, world):
 class Layer:
     """Device buffers of one sublayer for the timed steps (allocated once)."""
 
-    def __init__(self, cfg, sub, dev, seed_offset, host, act_order=False):
-        import numpy as np
+    def __init__(self, cfg, sub, dev, seed_offset, G, act_order=False):
         import torch
         import synth
         from post_quantization_02_b200 import abi
@@ -379,8 +378,7 @@ class Layer:
         su, sv = synth.make_signs(cfg, sub)
         self.su = torch.from_numpy(su).to(dev)
         self.sv = torch.from_numpy(sv).to(dev)
-        self.G_host = host["G"][sub.name]
-        self.G = torch.from_numpy(self.G_host.view(np.int16)).to(dev).view(torch.bfloat16)
+        self.G = G
         self.W = torch.empty_like(self.W0)
         self.HX = torch.empty((n, n), dtype=torch.float32, device=dev)
         self.HG = torch.empty((m, m), dtype=torch.float32, device=dev)
@@ -413,6 +411,23 @@ def packed_view(L, bits):
 def abi_packed_words(n, bits):
     from post_quantization_02_b200 import abi
     return abi.packed_words(n, bits)
+
+
+def draw_to_device(chunk_fn, tokens, width, dev, threads):
+    """A token-major bf16 input drawn chunk by chunk (synth's seeded chunks)
+    straight into device memory; at most `threads` chunks on the host at once."""
+    import numpy as np
+    import torch
+    import synth
+    from concurrent.futures import ThreadPoolExecutor
+    A = torch.empty((tokens, width), dtype=torch.bfloat16, device=dev)
+    nch = synth.n_chunks(tokens)
+    with ThreadPoolExecutor(threads) as ex:
+        for c0 in range(0, nch, threads):
+            for c, bits in zip(range(c0, nch), ex.map(chunk_fn, range(c0, min(nch, c0 + threads)))):
+                r0 = c * synth.CHUNK_TOKENS
+                A[r0:r0 + bits.shape[0]].copy_(torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16))
+    return A
 
 
 class StageMarks:
@@ -619,17 +634,40 @@ def stage_rooflines(cfg, layers, steps, stages, inner, peaks, peak_src, peak, pe
                     "lo*hi, ~2^-17 relative), so the algorithmic ceiling is 1/3 of the bf16 peak"}
     chol_ms = stages.get("inverse_cholesky", 0.0)
     chol_flops = sum(2 * L.sub.n ** 3 / 3 for L in layers)
+    # the panel kernels' own work: per 128-wide panel of the padded order np,
+    # the slice products (np rows x 128 x 128) and the diagonal block's factor
+    # and inverse (2 x 128^3 / 3); the update GEMMs carry the rest
+    panel_flops = sum((-(-L.sub.n // 128)) * (2 * 128 * 128 * (-(-L.sub.n // 128) * 128)
+                                              + 2 * 128 ** 3 / 3) for L in layers)
     if chol_ms > 0:
         ach = chol_flops / (chol_ms / 1e3) / 1e12
-        out["inverse_cholesky"] = {
-            "bound": "alu", "kernel": "panel_kernel + gemm_nt_tc_kernel (kronq_cholesky_inv)",
-            "achieved": ach, "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s",
-            "frac": ach / FP32_ALU_TFLOPS,
-            "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1965 MHz",
+        pan_ms, pan_cnt = inner["chol_panel"]
+        upd_ms, upd_cnt = inner["chol_update"]
+        entry = {
+            "bound": "tensor", "kernel": "panel_kernel + gemm_nt_tc_kernel (kronq_cholesky_inv)",
+            "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
+            "peak_source": f"{peak_src} {peak_kind}",
             "flops_per_step": chol_flops, "ms_per_step": chol_ms,
-            "panel_ms_per_step": inner["chol_panel"][0] / steps,
-            "update_ms_per_step": inner["chol_update"][0] / steps,
-            "panels_per_step": inner["chol_panel"][1] / steps}
+            "note": "2 n^3 / 3 per factorisation (Cholesky and triangular inverse); nearly all of it "
+                    "in the update GEMMs, whose products run as three tensor-core MMAs of hi / lo "
+                    "planes, so the algorithmic ceiling is 1/3 of the 16-bit peak"}
+        if pan_cnt and pan_ms > 0:
+            pa = panel_flops * steps / (pan_ms / 1e3) / 1e12
+            entry["panels"] = {
+                "bound": "alu", "achieved": pa, "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s",
+                "frac": pa / FP32_ALU_TFLOPS,
+                "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1965 MHz",
+                "flops_per_step": panel_flops, "ms_per_step": pan_ms / steps,
+                "launches_per_step": pan_cnt / steps,
+                "note": "latency-bound: 128 sequential pivots per diagonal block"}
+        if upd_cnt and upd_ms > 0:
+            ua = (chol_flops - panel_flops) * steps / (upd_ms / 1e3) / 1e12
+            entry["updates"] = {
+                "bound": "tensor", "achieved": ua, "peak": peak, "unit": "TFLOP/s",
+                "frac": ua / peak, "peak_source": f"{peak_src} {peak_kind}",
+                "flops_per_step": chol_flops - panel_flops, "ms_per_step": upd_ms / steps,
+                "launches_per_step": upd_cnt / steps}
+        out["inverse_cholesky"] = entry
     biip_ms = stages.get("biip_sensitivity", 0.0)
     biip_bytes = sum(16 * (L.sub.m * L.sub.n + L.sub.n ** 2 + L.sub.m ** 2) for L in layers)
     if biip_ms > 0:
@@ -896,16 +934,33 @@ def main():
         cfg0 = dataclasses.replace(cfg0, tokens=args.tokens)
     cfg = rank_config(cfg0, rank)   # each rank: its own layer (weak scaling)
 
-    # ---- seeded inputs on the host (pinned for the end-to-end leg), then HBM
+    # ---- seeded inputs on the host (pinned for the end-to-end leg), then HBM.
+    # When every rank's host copies (and their pinned twins) would not fit the
+    # host's memory, each rank draws its inputs chunk by chunk straight into
+    # device memory with its share of the host cores, and has no e2e leg.
+    in_bytes = sum(cfg.tokens * s_.width * 2 for s_ in cfg.sites) + \
+        sum(cfg.tokens * s_.m * 2 for s_ in cfg.sublayers)
+    ram = os.sysconf("SC_PAGE_SIZE") * os.sysconf("SC_PHYS_PAGES")
+    lean = world * in_bytes * (1 if args.no_e2e else 2) > 0.6 * ram
     t_gen = time.perf_counter()
     host = {"X": {}, "G": {}}
-    for site in cfg.sites:
-        host["X"][site.name] = synth.make_x(cfg, site)
-    for sub in cfg.sublayers:
-        host["G"][sub.name] = synth.make_g(cfg, sub)
+    if lean:
+        threads = max(1, (os.cpu_count() or 1) // world)
+        X = {s_.name: draw_to_device(lambda c, s_=s_: synth.x_chunk(cfg, s_, c), cfg.tokens,
+                                     s_.width, dev, threads) for s_ in cfg.sites}
+        Gd = {sub.name: draw_to_device(lambda c, sub=sub: synth.g_chunk(cfg, sub, c), cfg.tokens,
+                                       sub.m, dev, threads) for sub in cfg.sublayers}
+    else:
+        for site in cfg.sites:
+            host["X"][site.name] = synth.make_x(cfg, site)
+        for sub in cfg.sublayers:
+            host["G"][sub.name] = synth.make_g(cfg, sub)
+        X = {s_: torch.from_numpy(v.view(np.int16)).to(dev).view(torch.bfloat16)
+             for s_, v in host["X"].items()}
+        Gd = {s_: torch.from_numpy(v.view(np.int16)).to(dev).view(torch.bfloat16)
+              for s_, v in host["G"].items()}
     t_gen = time.perf_counter() - t_gen
-    X = {s: torch.from_numpy(v.view(np.int16)).to(dev).view(torch.bfloat16) for s, v in host["X"].items()}
-    layers = [Layer(cfg, sub, dev, rank, host, args.act_order) for sub in cfg.sublayers]
+    layers = [Layer(cfg, sub, dev, rank, Gd[sub.name], args.act_order) for sub in cfg.sublayers]
     mmax = max(s.m for s in cfg.sublayers)
     nmax = max(s.n for s in cfg.sublayers)
     ws = abi.workspace(mmax, nmax, device=dev)
@@ -954,7 +1009,11 @@ def main():
 
     # ---- end to end through the public API with pinned host buffers
     e2e = None
-    if not args.no_e2e:
+    e2e_skipped = None
+    if lean and not args.no_e2e:
+        e2e_skipped = (f"{world} ranks x {2 * in_bytes / 2 ** 30:.0f} GiB of host and pinned input "
+                       f"copies exceed 60 % of the host's {ram / 2 ** 30:.0f} GiB")
+    if not args.no_e2e and not lean:
         pin = {"X": {s: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).pin_memory()
                      for s, v in host["X"].items()},
                "G": {s: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -973,35 +1032,68 @@ def main():
             return gpipe.covariance_from_host(A_host, H, copy_stream=copy_stream, stream=stream,
                                               staging=staging[width])
 
+        solve_stream = torch.cuda.Stream(dev)
+
+        def finish_layer(L, st):
+            """BiIP, s, inverse Cholesky, solver, pack and the D2H copies of one
+            sublayer on stream st; returns the bytes copied back."""
+            abi.kronq_biip_rotate(L.W, L.HX, L.HG, L.su, L.sv, cfg.alpha, cfg.mode, 0, L.SX, L.SG,
+                                  ws, stream=st)
+            abi.kronq_sensitivity(L.HX, L.HG, L.sens, stream=st)
+            solve_layer(cfg, L, ws, st, args.act_order, args.w_clip)
+            pk, sc, zr = outs[L.sub.name]
+            n_out = 0
+            with torch.cuda.stream(st):
+                if L.bits in (2, 4):
+                    pv = packed_view(L, L.bits)
+                    abi.kronq_pack(L.codes, L.bits, pv, stream=st)
+                    pk[: pv.numel()].copy_(pv.view(-1), non_blocking=True)
+                    n_out += pv.numel() * 4
+                sc.copy_(L.scales, non_blocking=True)
+                zr.copy_(L.zeros, non_blocking=True)
+            return n_out + L.scales.numel() * 4 + L.zeros.numel()
+
         def e2e_step():
-            h2d = 0
+            """One step from pinned host buffers.  Fixed bit widths: sublayer by
+            sublayer, each sublayer's chain on a second stream as soon as its
+            covariances are done, while the next sublayer's inputs stream in
+            (the host-to-device copies bound the step).  A mixed 2/3/4-bit
+            allocation needs every score first, so it runs stage by stage."""
+            h2d = d2h = 0
             Hs = {}
-            for site in cfg.sites:
+
+            def site_cov(site):
+                nonlocal h2d
                 L0 = next(L for L in layers if L.sub.site == site.name)
                 h2d += cov_host(pin["X"][site.name], L0.HX, site.width)
                 Hs[site.name] = L0.HX
+                for L in layers:            # a shared input: every sublayer rotates its own copy
+                    if L.sub.site == site.name and L.HX is not L0.HX:
+                        L.HX.copy_(L0.HX)
+
+            if cfg.mixed_avg_bits:
+                for site in cfg.sites:
+                    site_cov(site)
+                for L in layers:
+                    h2d += cov_host(pin["G"][L.sub.name], L.HG, L.sub.m)
+                    L.W.copy_(pin["W"][L.sub.name], non_blocking=True)
+                    h2d += L.W.numel() * 4 + L.su.numel() + L.sv.numel()
+                for L in layers:
+                    d2h += finish_layer(L, stream)
+                return h2d, d2h
             for L in layers:
+                if L.sub.site not in Hs:
+                    site_cov(cfg.site(L.sub.site))
                 h2d += cov_host(pin["G"][L.sub.name], L.HG, L.sub.m)
-                if L.HX is not Hs[L.sub.site]:
-                    L.HX.copy_(Hs[L.sub.site])
                 L.W.copy_(pin["W"][L.sub.name], non_blocking=True)
                 h2d += L.W.numel() * 4 + L.su.numel() + L.sv.numel()
-            d2h = 0
-            for L in layers:
-                abi.kronq_biip_rotate(L.W, L.HX, L.HG, L.su, L.sv, cfg.alpha, cfg.mode, 0, L.SX, L.SG,
-                                      ws, stream=stream)
-                abi.kronq_sensitivity(L.HX, L.HG, L.sens, stream=stream)
-            for L in layers:
-                solve_layer(cfg, L, ws, stream, args.act_order, args.w_clip)
-                pk, sc, zr = outs[L.sub.name]
-                if L.bits in (2, 4):
-                    pv = packed_view(L, L.bits)
-                    abi.kronq_pack(L.codes, L.bits, pv, stream=stream)
-                    pk[: pv.numel()].copy_(pv.view(-1), non_blocking=True)
-                    d2h += pv.numel() * 4
-                sc.copy_(L.scales, non_blocking=True)
-                zr.copy_(L.zeros, non_blocking=True)
-                d2h += L.scales.numel() * 4 + L.zeros.numel()
+                ready = torch.cuda.Event()
+                ready.record(stream)
+                solve_stream.wait_event(ready)
+                d2h += finish_layer(L, solve_stream)
+            done = torch.cuda.Event()
+            done.record(solve_stream)
+            stream.wait_event(done)
             return h2d, d2h
 
         e2e_step()
@@ -1064,6 +1156,7 @@ def main():
                        "act_order": args.act_order, "w_clip": args.w_clip},
             "roofline": roofline, "rooflines": rooflines, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches,
+            **({"e2e_skipped": e2e_skipped} if e2e_skipped else {}),
             "clocks": clocks,
             "stages_ms": {k: round(v, 4) for k, v in stages.items()},
             # the solver alone, given H_X': inverse Cholesky + OBS loop

@@ -41,8 +41,8 @@ constexpr int SM_X = SM_D + NB * LDD;
 constexpr int SM_P = SM_X + NB * LDX;
 constexpr int SM_AS = SM_P + 32 * LDX;
 constexpr int SM_YT = SM_AS + 32 * LDA;
-constexpr int SM_LB = SM_YT + 32 * LDY;       // the leaf's broadcast buffers (2 x 32)
-constexpr int SM_P2 = SM_LB + 64;             // second slice buffer (double buffering)
+constexpr int SM_LB = SM_YT + 32 * LDY;       // the leaf's exchange buffers (6 x 32)
+constexpr int SM_P2 = SM_LB + 192;            // second slice buffer (double buffering)
 constexpr int SM_FLOATS = SM_P2 + 32 * LDX;
 static_assert(SM_LB % 4 == 0, "leaf buffers must allow 16-byte loads");
 
@@ -88,62 +88,107 @@ __global__ void reverse_damp_kernel(const float* __restrict__ H, int n, int np,
   }
 }
 
-// One warp factors the 32 x 32 diagonal block at offset o of D (lower part
-// valid, already updated) and inverts the factor: on return D holds L_oo,
-// X holds Y_oo = L_oo^-1 and YT its transpose.  Lane i keeps row i of the
-// block and row i of the accumulating inverse in registers; pivot step j:
+// Two warps factor the 32 x 32 diagonal block at offset o of D (lower part
+// valid, already updated) and invert the factor: on return D holds L_oo,
+// X holds Y_oo = L_oo^-1 and YT its transpose.  Pivot step j:
 //   L[i][j] = a_i[j] r,  r = 1 / sqrt(a_j[j]),   a_i[c] -= L[i][j] L[c][j]  (c > j)
 //   Y[j][:] = y_j[:] r,  y_i[:] -= L[i][j] Y[j][:]                          (i > j)
-// The pivot travels by one shuffle; the column L[:, j] and the finished row
-// Y[j][:] are broadcast through shared memory (lb: 2 x 32 floats), read by
-// every lane with 16-byte loads, which keeps the chain from one pivot to the
-// next short.  The arithmetic (and its order) is that of the plain update.
-__device__ __forceinline__ void warp_leaf32(float* D, float* X, float* YT, int o, int kb,
-                                            int* bad, float* lb) {
-  const int i = threadIdx.x & 31;
+// Warp 0 does the factorisation: lane i keeps row i of the block in
+// registers, shifted so that slot 0 is the current pivot column (slot c =
+// column j + c), stores L[i][j] into D and r into lb as it goes, and passes
+// the column L[j+1:, j] to its own lanes through lb.  Warp 1 carries the
+// inverse one pivot behind: lane i keeps row i of Y; the finished row Y[j][:]
+// travels through lb.  Warp 0 arrives on barrier FULL[j&1] after pivot j's
+// stores; warp 1 syncs on it, and arrives on EMPTY[j&1] when it is done with
+// pivot j, which warp 0 syncs on before pivot j+2 (so lb's double buffers and
+// the barriers are never reused early; every arrive has its sync).  The
+// pivot loop is not unrolled: the whole leaf is a few hundred instructions,
+// so its first pass does not stall on instruction fetch after the update
+// kernels ran.  The arithmetic (and its order) is that of the plain update.
+// lb: 192 floats, 16-byte aligned (colb 2 x 32 | rowb 2 x 32 | r 32).
+// Named barriers 1..4; called by the CTA's warps 0 and 1 together.
+KQ_DEV void named_sync64(int id) { asm volatile("bar.sync %0, 64;" ::"r"(id) : "memory"); }
+KQ_DEV void named_arrive64(int id) { asm volatile("bar.arrive %0, 64;" ::"r"(id) : "memory"); }
+
+__device__ __forceinline__ void leaf32(float* D, float* X, float* YT, int o, int kb, int* bad,
+                                       float* lb) {
+  const int i = threadIdx.x & 31, w = threadIdx.x >> 5;
   constexpr unsigned FULL = 0xffffffffu;
-  float* colb = lb;         // L[:, j] of the current pivot
-  float* rowb = lb + 32;    // Y[j][:] of the current pivot
-  float a[32], y[32];
+  float* rj = lb + 128;
+  if (w == 0) {
+    float a[32];
 #pragma unroll
-  for (int c = 0; c < 32; ++c) {
-    a[c] = (c <= i) ? D[(o + i) * LDD + o + c] : 0.f;
-    y[c] = (c == i) ? 1.f : 0.f;
-  }
-#pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    float d = __shfl_sync(FULL, a[j], j);
-    if (!(d > 0.f) || !isfinite(d)) {
-      if (i == 0 && o + j < kb) *bad = 1;
-      d = 1.f;
-    }
-    const float r = rsqrtf(d);
-    const float l = (i >= j) ? a[j] * r : 0.f;
-    a[j] = l;
-    colb[i] = l;
-    if (i == j) {
-#pragma unroll
-      for (int c = 0; c <= j; ++c) {
-        y[c] = y[c] * r;
-        rowb[c] = y[c];
+    for (int c = 0; c < 32; ++c) a[c] = (c <= i) ? D[(o + i) * LDD + o + c] : 0.f;
+    *reinterpret_cast<float2*>(lb + 2 * i) = make_float2(0.f, 0.f);
+    __syncwarp();
+#pragma unroll 1
+    for (int j = 0; j < 32; ++j) {
+      float* colb = lb + (j & 1) * 32;           // colb[c] = L[j+1+c][j]
+      float d = __shfl_sync(FULL, a[0], j);
+      if (!(d > 0.f) || !isfinite(d)) {
+        if (i == 0 && o + j < kb) *bad = 1;
+        d = 1.f;
       }
-    }
-    __syncwarp();
+      const float r = rsqrtf(d);
+      const float l = (i >= j) ? a[0] * r : 0.f;
+      if (j >= 2) named_sync64(3 + (j & 1));     // warp 1 is done with pivot j - 2
+      if (i >= j) D[(o + i) * LDD + o + j] = l;
+      if (i > j) colb[i - j - 1] = l;
+      if (i == j) rj[j] = r;
+      __syncwarp();
+      named_arrive64(1 + (j & 1));
+      // a_i[j+1+c] -= L[i][j] L[j+1+c][j], shifted down one slot; the slots
+      // past the row's last column hold values that are never used
 #pragma unroll
-    for (int c = j + 1; c < 32; ++c) a[c] = fmaf(-l, colb[c], a[c]);
-    if (i != j) {
+      for (int q = 0; q < 8; ++q) {
+        const float4 v = *reinterpret_cast<const float4*>(colb + 4 * q);
+        const float vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int c = 0; c <= j; ++c) y[c] = fmaf(-l, rowb[c], y[c]);
+        for (int u = 0; u < 4; ++u) {
+          const int c = 4 * q + u;
+          if (c < 31) a[c] = fmaf(-l, vv[u], a[c + 1]);
+        }
+      }
+      a[31] = 0.f;
     }
-    __syncwarp();
-  }
+  } else {
+    float y[32];
 #pragma unroll
-  for (int c = 0; c < 32; ++c) {
-    if (c <= i) {
-      D[(o + i) * LDD + o + c] = a[c];
-      X[(o + i) * LDX + o + c] = y[c];
+    for (int c = 0; c < 32; ++c) y[c] = (c == i) ? 1.f : 0.f;
+#pragma unroll 1
+    for (int j = 0; j < 32; ++j) {
+      float* rowb = lb + 64 + (j & 1) * 32;      // Y[j][:]
+      named_sync64(1 + (j & 1));
+      const float r = rj[j];
+      const float l = (i >= j) ? D[(o + i) * LDD + o + j] : 0.f;
+      if (i == j) {
+        // y_j[c] = 0 for c > j, so scaling the whole row changes nothing there
+#pragma unroll
+        for (int c = 0; c < 32; ++c) y[c] = y[c] * r;
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          *reinterpret_cast<float4*>(rowb + 4 * q) =
+              make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
+      }
+      __syncwarp();
+      if (i != j) {
+        // rowb[c] = 0 for c > j: those updates leave y (+0) as it is
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const float4 v = *reinterpret_cast<const float4*>(rowb + 4 * q);
+          y[4 * q + 0] = fmaf(-l, v.x, y[4 * q + 0]);
+          y[4 * q + 1] = fmaf(-l, v.y, y[4 * q + 1]);
+          y[4 * q + 2] = fmaf(-l, v.z, y[4 * q + 2]);
+          y[4 * q + 3] = fmaf(-l, v.w, y[4 * q + 3]);
+        }
+      }
+      if (j + 2 < 32) named_arrive64(3 + (j & 1));
     }
-    YT[c * LDY + i] = (c <= i) ? y[c] : 0.f;   // YT[c][i] = Y[i][c]
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+      if (c <= i) X[(o + i) * LDX + o + c] = y[c];
+      YT[c * LDY + i] = (c <= i) ? y[c] : 0.f;   // YT[c][i] = Y[i][c]
+    }
   }
 }
 
@@ -155,11 +200,11 @@ __device__ __forceinline__ void warp_leaf32(float* D, float* X, float* YT, int o
 // Right-looking over four 32-wide blocks b (o = 32 b), carrying L^-1 along
 // (block forward substitution of L Y = I, accumulators in X below the
 // diagonal blocks):
-//   1. warp 0: L_bb and Y_bb = L_bb^-1                          (warp_leaf32)
+//   1. warps 0-1: L_bb and Y_bb = L_bb^-1                       (leaf32)
 //   2. L_cb = D_cb Y_bb^T (c > b), also kept K-major in As;  Y_bj = Y_bb Acc_bj (j < b)
 //   3a. the next block column: D_{c,b+1} -= L_cb L_{b+1,b}^T
 //   3b. the rest: D_cd -= L_cb L_db^T (d > b+1);  Acc_cj -= L_cb Y_bj (j <= b)
-// with warp 0 factoring block b+1 (step 1 of the next round) while the other
+// with warps 0-1 factoring block b+1 (step 1 of the next round) while four other
 // warps do 3b.  Steps 2 and 3 are small register-tiled GEMMs out of shared
 // memory whose wide operands are read as contiguous rows (YT, As, rows of X).
 constexpr int PANEL_THREADS = 256;
@@ -169,7 +214,7 @@ __device__ void factor_and_invert(float* D, float* X, float* As, float* YT, floa
   const int tid = threadIdx.x;
   for (int e = tid; e < NB * LDX; e += blockDim.x) X[e] = 0.f;
   __syncthreads();
-  if (tid < 32) warp_leaf32(D, X, YT, 0, kb, bad, LB);
+  if (tid < 64) leaf32(D, X, YT, 0, kb, bad, LB);
   __syncthreads();
   for (int b = 0; b < NB / 32; ++b) {
     const int o = 32 * b;
@@ -254,13 +299,14 @@ __device__ void factor_and_invert(float* D, float* X, float* As, float* YT, floa
         }
     }
     __syncthreads();
-    // ---- step 3b on warps 1.., the next diagonal block on warp 0
-    if (tid < 32) {
-      warp_leaf32(D, X, YT, o2, kb, bad, LB);
-    } else {
+    // ---- step 3b on warps 2, 3, 6, 7, the next diagonal block on warps 0-1
+    if (tid < 64) {
+      leaf32(D, X, YT, o2, kb, bad, LB);
+    } else if (((tid >> 5) & 3) >= 2) {
+      // warps 2, 3, 6, 7: the leaf's warps share no scheduler with them
       // item = 4 rows x 8 columns; 12 column groups: 8 g < o2 (Acc), else past the next block
       const int items = (R1 / 4) * 12;
-      for (int it = tid - 32; it < items; it += PANEL_THREADS - 32) {
+      for (int it = (tid >> 5) < 4 ? tid - 64 : tid - 128; it < items; it += 128) {
         const int rg = it / 12, g = it % 12;
         const int c0 = (8 * g < o2) ? 8 * g : 8 * g + 32;
         const bool left = c0 < o2;
