@@ -202,11 +202,13 @@ __device__ __forceinline__ void leaf32(float* D, float* X, float* YT, int o, int
 // diagonal blocks):
 //   1. warps 0-1: L_bb and Y_bb = L_bb^-1                       (leaf32)
 //   2. L_cb = D_cb Y_bb^T (c > b), also kept K-major in As;  Y_bj = Y_bb Acc_bj (j < b)
+//      (together one 96 x 32 x 32 product whose B operand is Y_bb^T)
 //   3a. the next block column: D_{c,b+1} -= L_cb L_{b+1,b}^T
 //   3b. the rest: D_cd -= L_cb L_db^T (d > b+1);  Acc_cj -= L_cb Y_bj (j <= b)
 // with warps 0-1 factoring block b+1 (step 1 of the next round) while four other
 // warps do 3b.  Steps 2 and 3 are small register-tiled GEMMs out of shared
-// memory whose wide operands are read as contiguous rows (YT, As, rows of X).
+// memory (3 x 4 outputs per thread in steps 2 and 3a) whose wide operands are
+// read as contiguous rows (YT, As, rows of X).
 constexpr int PANEL_THREADS = 256;
 
 __device__ void factor_and_invert(float* D, float* X, float* As, float* YT, float* LB, int kb,
@@ -220,83 +222,81 @@ __device__ void factor_and_invert(float* D, float* X, float* As, float* YT, floa
     const int o = 32 * b;
     const int o2 = o + 32;
     const int R1 = NB - o2;                 // rows below the diagonal block
-    // ---- step 2: thread tid handles (tr, tc) = (tid / 16 + 16 u, tid % 16), u = 0, 1
+    // ---- step 2, one 96 x 32 x 32 product through YT (B[t][q] = Y_bb[q][t]):
+    //   rows m < R1:  L_cb[m][q]  = sum_t D[o2+m][o+t] Y_bb[q][t]   -> D, As
+    //   rows m >= R1: Y_bj[q][c'] = sum_t Acc[o+t][c'] Y_bb[q][t],  c' = m - R1 -> X
+    // thread (g, cg): rows g + 32 k (k < 3), columns 4 cg .. 4 cg + 3; each
+    // 32-row block lies on one side of R1 (a multiple of 32)
     {
-      const int tc = tid & 15;
-      const int nj = o >> 4;                // Y_bj columns per item: o / 16
-      float acc1[2][3][2], acc2[2][6];
+      const int cg = tid & 7, g = tid >> 3;
+      float acc[3][4];
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
+      for (int k = 0; k < 3; ++k)
 #pragma unroll
-        for (int s = 0; s < 3; ++s) acc1[u][s][0] = acc1[u][s][1] = 0.f;
-#pragma unroll
-        for (int q = 0; q < 6; ++q) acc2[u][q] = 0.f;
-      }
-#pragma unroll 2
+        for (int u = 0; u < 4; ++u) acc[k][u] = 0.f;
+#pragma unroll 4
       for (int t = 0; t < 32; ++t) {
-        const float2 bv = *reinterpret_cast<const float2*>(&YT[t * LDY + 2 * tc]);   // Y_bb[2tc+q][t]
+        const float4 bv = *reinterpret_cast<const float4*>(&YT[t * LDY + 4 * cg]);
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int tr = (tid >> 4) + 16 * u;
-#pragma unroll
-          for (int s = 0; s < 3; ++s) {
-            if (32 * s < R1) {
-              const float av = D[(o2 + tr + 32 * s) * LDD + o + t];
-              acc1[u][s][0] = fmaf(av, bv.x, acc1[u][s][0]);
-              acc1[u][s][1] = fmaf(av, bv.y, acc1[u][s][1]);
-            }
-          }
-          const float yv = X[(o + tr) * LDX + o + t];                          // Y_bb[tr][t]
-#pragma unroll
-          for (int q = 0; q < 6; ++q)
-            if (q < nj) acc2[u][q] = fmaf(yv, X[(o + t) * LDX + tc * nj + q], acc2[u][q]);  // Acc[t][c']
+        for (int k = 0; k < 3; ++k) {
+          const int m = g + 32 * k;
+          const float av = (32 * k < R1) ? D[(o2 + m) * LDD + o + t] : X[(o + t) * LDX + m - R1];
+          acc[k][0] = fmaf(av, bv.x, acc[k][0]);
+          acc[k][1] = fmaf(av, bv.y, acc[k][1]);
+          acc[k][2] = fmaf(av, bv.z, acc[k][2]);
+          acc[k][3] = fmaf(av, bv.w, acc[k][3]);
         }
       }
       __syncthreads();
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int tr = (tid >> 4) + 16 * u;
+      for (int k = 0; k < 3; ++k) {
+        const int m = g + 32 * k;
+        if (32 * k < R1) {
 #pragma unroll
-        for (int s = 0; s < 3; ++s)
-          if (32 * s < R1)
+          for (int u = 0; u < 4; ++u) {
+            D[(o2 + m) * LDD + o + 4 * cg + u] = acc[k][u];
+            As[(4 * cg + u) * LDA + m] = acc[k][u];
+          }
+        } else {
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-              D[(o2 + tr + 32 * s) * LDD + o + 2 * tc + q] = acc1[u][s][q];
-              As[(2 * tc + q) * LDA + tr + 32 * s] = acc1[u][s][q];
-            }
-#pragma unroll
-        for (int q = 0; q < 6; ++q)
-          if (q < nj) X[(o + tr) * LDX + tc * nj + q] = acc2[u][q];
+          for (int u = 0; u < 4; ++u) X[(o + 4 * cg + u) * LDX + m - R1] = acc[k][u];
+        }
       }
       __syncthreads();
     }
     if (R1 == 0) break;
-    // ---- step 3a: D[r][c] -= sum_t L[r][o+t] L[c][o+t], c in the next block column
-    for (int w = tid; w < 512; w += PANEL_THREADS) {
-      const int tr = w >> 4, tc = w & 15;          // rows tr + 32 s, columns 2 tc, 2 tc + 1
-      float acc[3][2];
+    // ---- step 3a: D[o2+m][o2+n] -= sum_t L[o2+m][o+t] L[o2+n][o+t] (n < 32, m >= n),
+    // both operands from the K-major copy As; thread (g, cg) as in step 2
+    {
+      const int cg = tid & 7, g = tid >> 3;
+      float acc[3][4];
 #pragma unroll
-      for (int s = 0; s < 3; ++s) acc[s][0] = acc[s][1] = 0.f;
+      for (int k = 0; k < 3; ++k)
+#pragma unroll
+        for (int u = 0; u < 4; ++u) acc[k][u] = 0.f;
 #pragma unroll 4
       for (int t = 0; t < 32; ++t) {
-        const float2 bv = *reinterpret_cast<const float2*>(&As[t * LDA + 2 * tc]);
+        const float4 bv = *reinterpret_cast<const float4*>(&As[t * LDA + 4 * cg]);
 #pragma unroll
-        for (int s = 0; s < 3; ++s) {
-          if (32 * s < R1) {
-            const float av = As[t * LDA + tr + 32 * s];
-            acc[s][0] = fmaf(av, bv.x, acc[s][0]);
-            acc[s][1] = fmaf(av, bv.y, acc[s][1]);
+        for (int k = 0; k < 3; ++k) {
+          if (32 * k < R1) {
+            const float av = As[t * LDA + g + 32 * k];
+            acc[k][0] = fmaf(av, bv.x, acc[k][0]);
+            acc[k][1] = fmaf(av, bv.y, acc[k][1]);
+            acc[k][2] = fmaf(av, bv.z, acc[k][2]);
+            acc[k][3] = fmaf(av, bv.w, acc[k][3]);
           }
         }
       }
 #pragma unroll
-      for (int s = 0; s < 3; ++s)
-        if (32 * s < R1) {
-          const int r = o2 + tr + 32 * s;
+      for (int k = 0; k < 3; ++k) {
+        const int m = g + 32 * k;
+        if (32 * k < R1) {
 #pragma unroll
-          for (int q = 0; q < 2; ++q)
-            if (o2 + 2 * tc + q <= r) D[r * LDD + o2 + 2 * tc + q] -= acc[s][q];
+          for (int u = 0; u < 4; ++u)
+            if (4 * cg + u <= m) D[(o2 + m) * LDD + o2 + 4 * cg + u] -= acc[k][u];
         }
+      }
     }
     __syncthreads();
     // ---- step 3b on warps 2, 3, 6, 7, the next diagonal block on warps 0-1
