@@ -126,6 +126,12 @@ class ClockSampler:
         self.proc = None
         self.lines = []
         self.thread = None
+        self.cut = None
+
+    def mark_end(self):
+        """The samples so far are the timed region's; later ones (the
+        end-to-end leg, the CPU baseline) stay out of the summary."""
+        self.cut = len(self.lines)
 
     def start(self):
         cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
@@ -156,7 +162,7 @@ class ClockSampler:
     def summary(self):
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for ln in self.lines[:self.cut]:
             p = [x.strip() for x in ln.split(",")]
             if len(p) < 8:
                 continue
@@ -997,6 +1003,7 @@ def main():
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
+    sampler.mark_end()
     launches = abi.kronq_launch_count() - launches0
     inner = {k: abi.kronq_timing_read(k) for k in abi.TIMERS}
     abi.kronq_timing_enable(False)

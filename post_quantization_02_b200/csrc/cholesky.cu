@@ -214,7 +214,9 @@ constexpr int PANEL_THREADS = 256;
 __device__ void factor_and_invert(float* D, float* X, float* As, float* YT, float* LB, int kb,
                                   int* bad) {
   const int tid = threadIdx.x;
-  for (int e = tid; e < NB * LDX; e += blockDim.x) X[e] = 0.f;
+  static_assert((NB * LDX) % 4 == 0 && SM_X % 4 == 0, "X is cleared in 16-byte stores");
+  for (int e = 4 * tid; e < NB * LDX; e += 4 * blockDim.x)
+    *reinterpret_cast<float4*>(X + e) = make_float4(0.f, 0.f, 0.f, 0.f);
   __syncthreads();
   if (tid < 64) leaf32(D, X, YT, 0, kb, bad, LB);
   __syncthreads();
@@ -411,22 +413,22 @@ __global__ void __launch_bounds__(PANEL_THREADS, 1) panel_kernel(const float* R,
   }
   __syncthreads();
   if (tid == 0 && (int)blockIdx.x < z_pp) fetch(blockIdx.x, 0);
-  // the diagonal block, lower triangle: 16-byte loads, a half of them
-  // requested before any is stored (one CTA per SM leaves few warps to hide
-  // the latency of one load at a time)
+  // the diagonal block, lower triangle: 16-byte loads, all requested before
+  // any is stored (one CTA per SM leaves few warps to hide the latency);
+  // the chunks wholly above the diagonal are not read
   static_assert(NB * NB / 4 == 16 * PANEL_THREADS, "diagonal block load assumes 256 threads");
+  {
+    float4 v[16];
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    float4 v[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int e4 = tid + PANEL_THREADS * (8 * h + u);
+    for (int u = 0; u < 16; ++u) {
+      const int e4 = tid + PANEL_THREADS * u;
       const int i = e4 >> 5, c = (e4 & 31) * 4;
-      v[u] = *reinterpret_cast<const float4*>(R + (int64_t)(k + i) * np + k + c);
+      v[u] = (c <= i) ? *reinterpret_cast<const float4*>(R + (int64_t)(k + i) * np + k + c)
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int e4 = tid + PANEL_THREADS * (8 * h + u);
+    for (int u = 0; u < 16; ++u) {
+      const int e4 = tid + PANEL_THREADS * u;
       const int i = e4 >> 5, c = (e4 & 31) * 4;
       float* d = D + i * LDD + c;
       d[0] = (c <= i) ? v[u].x : 0.f;
