@@ -419,6 +419,19 @@ def abi_packed_words(n, bits):
     return abi.packed_words(n, bits)
 
 
+def host_input_bytes(cfg) -> int:
+    """Bytes of one rank's host inputs: X per input site and G per sublayer
+    (bf16, every token)."""
+    return sum(cfg.tokens * s_.width * 2 for s_ in cfg.sites) + \
+        sum(cfg.tokens * s_.m * 2 for s_ in cfg.sublayers)
+
+
+def needs_lean_inputs(cfg, world: int, e2e: bool, ram: int) -> bool:
+    """True when every rank's host inputs (and, with the end-to-end leg, their
+    pinned copies) would take more than 60 % of the host's memory."""
+    return world * host_input_bytes(cfg) * (2 if e2e else 1) > 0.6 * ram
+
+
 def draw_to_device(chunk_fn, tokens, width, dev, threads):
     """A token-major bf16 input drawn chunk by chunk (synth's seeded chunks)
     straight into device memory; at most `threads` chunks on the host at once."""
@@ -944,10 +957,9 @@ def main():
     # When every rank's host copies (and their pinned twins) would not fit the
     # host's memory, each rank draws its inputs chunk by chunk straight into
     # device memory with its share of the host cores, and has no e2e leg.
-    in_bytes = sum(cfg.tokens * s_.width * 2 for s_ in cfg.sites) + \
-        sum(cfg.tokens * s_.m * 2 for s_ in cfg.sublayers)
+    in_bytes = host_input_bytes(cfg)
     ram = os.sysconf("SC_PAGE_SIZE") * os.sysconf("SC_PHYS_PAGES")
-    lean = world * in_bytes * (1 if args.no_e2e else 2) > 0.6 * ram
+    lean = needs_lean_inputs(cfg, world, not args.no_e2e, ram)
     t_gen = time.perf_counter()
     host = {"X": {}, "G": {}}
     if lean:

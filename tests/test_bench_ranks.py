@@ -72,3 +72,36 @@ def test_stage_marks_attribute_each_interval_to_the_stage_it_closes():
                 ("inverse_cholesky", Ev(12.0)), ("solver", Ev(12.5)), ("pack", Ev(12.75))]
     assert m.totals() == {"covariance": 7.0, "biip_sensitivity": 0.5, "inverse_cholesky": 3.0,
                           "solver": 1.75, "pack": 0.5}
+
+
+def test_draw_to_device_equals_the_host_generator():
+    """Ranks whose host copies would not fit draw their inputs chunk by chunk
+    straight into device memory; the result is the host generator's matrix
+    bit for bit (here into CPU memory with two threads, on a token count
+    whose last chunk is ragged)."""
+    sys.path.insert(0, str(ROOT))
+    import dataclasses
+    import torch
+    import bench
+    import synth
+    cfg = dataclasses.replace(synth.get_config("toy-256"), tokens=2 * synth.CHUNK_TOKENS + 100)
+    site, sub = cfg.sites[0], cfg.sublayers[0]
+    X = bench.draw_to_device(lambda c: synth.x_chunk(cfg, site, c), cfg.tokens, site.width, "cpu", 2)
+    G = bench.draw_to_device(lambda c: synth.g_chunk(cfg, sub, c), cfg.tokens, sub.m, "cpu", 2)
+    assert torch.equal(X.view(torch.int16), torch.from_numpy(synth.make_x(cfg, site).view(np.int16)))
+    assert torch.equal(G.view(torch.int16), torch.from_numpy(synth.make_g(cfg, sub).view(np.int16)))
+
+
+def test_lean_inputs_only_where_the_host_copies_would_not_fit():
+    """The Llama-3-70B MLP workload's inputs are 38.7 GB per rank: with their
+    pinned copies one rank fits a 196 GiB host, two do not."""
+    sys.path.insert(0, str(ROOT))
+    import bench
+    import synth
+    cfg = synth.get_config("llama3-70b-mlp")
+    assert bench.host_input_bytes(cfg) == 262144 * 2 * (8192 + 28672 + 28672 + 8192)
+    ram = 196 * 2 ** 30
+    assert not bench.needs_lean_inputs(cfg, 1, True, ram)
+    assert bench.needs_lean_inputs(cfg, 2, True, ram)
+    assert not bench.needs_lean_inputs(cfg, 2, False, ram)
+    assert bench.needs_lean_inputs(cfg, 4, False, ram)
