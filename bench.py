@@ -1074,10 +1074,11 @@ def main():
 
         def e2e_step():
             """One step from pinned host buffers.  Fixed bit widths: sublayer by
-            sublayer, each sublayer's chain on a second stream as soon as its
-            covariances are done, while the next sublayer's inputs stream in
-            (the host-to-device copies bound the step).  A mixed 2/3/4-bit
-            allocation needs every score first, so it runs stage by stage."""
+            sublayer (widest input first), each sublayer's chain on a second
+            stream as soon as its covariances are done, while the next
+            sublayer's inputs stream in (the host-to-device copies bound the
+            step).  A mixed 2/3/4-bit allocation needs every score first, so it
+            runs stage by stage."""
             h2d = d2h = 0
             Hs = {}
 
@@ -1100,7 +1101,9 @@ def main():
                 for L in layers:
                     d2h += finish_layer(L, stream)
                 return h2d, d2h
-            for L in layers:
+            # the widest input first: its inverse Cholesky (~n^3) is the
+            # longest chain, and it runs while the others' inputs stream in
+            for L in sorted(layers, key=lambda L_: -L_.sub.n):
                 if L.sub.site not in Hs:
                     site_cov(cfg.site(L.sub.site))
                 h2d += cov_host(pin["G"][L.sub.name], L.HG, L.sub.m)
