@@ -19,7 +19,7 @@ import pytest  # noqa: E402
 @pytest.fixture(scope="session")
 def cuda():
     """The CUDA device for -m gpu tests; libkronq must be built and loadable
-    (no skip on a GPU machine: a missing library is a failure)."""
+    (no skip where a GPU is present: a missing library is a failure)."""
     import torch
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")

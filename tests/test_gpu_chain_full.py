@@ -11,7 +11,7 @@ KronQ summary (hyper.ai), "Method" (Eq. 7 covariances, Eqs. 11-12 BiIP,
 Eq. 14 sensitivity, Prop. 1 column update); KronQ review (pith.science),
 appendix, Algorithms 1-2.
 
-Bars (north-star): H_X, H_G <= 1e-4 relative Frobenius; >= 99.9 % identical
+Bars: H_X, H_G <= 1e-4 relative Frobenius; >= 99.9 % identical
 codes; the layer loss tr(H_G' dW' H_X' dW'^T) within 1 %; packed words
 bit-exact where the codes are identical.  Intermediate stages carry the
 differences of the stages before them, so their bars are derived: a

@@ -42,7 +42,7 @@ from post_quantization_02_b200 import abi, alloc
 
 pytestmark = pytest.mark.gpu
 
-COV_TOL = 1e-4          # bf16 inputs, fp32 accumulation (spec bar)
+COV_TOL = 1e-4          # bf16 inputs, fp32 accumulation (the parity bar)
 ROT_TOL = 1e-5          # fp32 butterflies: ~log2(d) roundings of 2^-24 each
 CHOL_TOL = 1e-4         # fp32 factor of a 1 %-damped matrix
 PROP_TOL = 1e-2         # U^T U H_d = I residual on sampled columns (conditioning-bound)

@@ -1,7 +1,7 @@
 """Parity of every libkronq entry point with the fp64 oracle, through the C
 ABI, on seeded inputs sized to span several tiles with ragged tails.
 
-Tolerances (spec bar): covariances <= 1e-4 relative Frobenius
+Tolerances (the parity bar): covariances <= 1e-4 relative Frobenius
 (bf16 inputs, fp32 accumulation); packing bit-exact; codes >= 99.9 %
 identical with the row loss within 1 %.  Rotation and inverse Cholesky are
 intermediate fp32 stages: their bound (1e-5 and 1e-4 relative Frobenius)

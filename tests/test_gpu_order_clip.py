@@ -9,7 +9,7 @@ oracle/quantizer.py) with the fp64 oracle, through the C ABI.
   sides, so per-channel scales and zeros (and the first group's) are
   identical; later groups see weights that fp32 and fp64 error propagation
   round differently, so their grids are compared within 1e-4; codes
-  >= 99.9 % identical and the loss within 1 % (the spec bar), as for
+  >= 99.9 % identical and the loss within 1 % (the parity bar), as for
   the plain solver.
 * The full chain with both options on the toy layer: the rotated H_X'
   diagonal is nearly flat after BiIP, so near-equal entries may order
