@@ -58,7 +58,7 @@ enum kronq_incoh_mode {
 /* Human-readable name of a status code (static string, never NULL). */
 const char* kronq_status_string(int status);
 
-/* ABI version of this header (major * 100 + minor). */
+/* ABI version of this header (major * 100 + minor): 101. */
 int kronq_abi_version(void);
 
 /* Number of kernels this library has launched in this process (all devices,
@@ -398,6 +398,16 @@ int kronq_layer_loss(const float* W_ref, const float* W_hat, int64_t m, int64_t 
  * context stays usable.  Not part of the quantization path.
  */
 int kronq_selftest_wait(int32_t* info, int64_t limit_ns, void* stream);
+
+/*
+ * Waits for the work queued on `stream` and reports how it ended (a host
+ * convenience; the pages have no counterpart).  Returns KRONQ_ERR_CUDA when
+ * the stream's work raised a CUDA error; otherwise, when `info` is given
+ * (the device word passed to the earlier calls), its value: 0 (KRONQ_OK) or
+ * the first numerical failure those calls recorded (KRONQ_ERR_NOT_PD,
+ * KRONQ_ERR_TIMEOUT).  `info` is only read.  Blocks the calling thread.
+ */
+int kronq_sync_status(void* stream, const int32_t* info);
 
 #ifdef __cplusplus
 }

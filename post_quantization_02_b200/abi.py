@@ -63,6 +63,7 @@ def lib() -> ctypes.CDLL:
         "kronq_unpack": ([P, I64, I64, I32, P, P], I32),
         "kronq_layer_loss": ([P, P, I64, I64, P, P, P, P, SZ, P], I32),
         "kronq_selftest_wait": ([P, I64, P], I32),
+        "kronq_sync_status": ([P, P], I32),
         "kronq_gptaq_workspace_size": ([I64, I64], SZ),
         "kronq_drift_covariance": ([P, I64, I64, I64, P, P, P, P, SZ, P], I32),
         "kronq_biip_rotate_input": ([P, I64, P, P, I32, P, SZ, P], I32),
@@ -505,6 +506,14 @@ def kronq_selftest_wait(info, limit_ns: int, stream=None):
     _dev(info, torch.int32, "info")
     _on_current_device((info, "info"))
     _check("kronq_selftest_wait", lib().kronq_selftest_wait(_p(info), int(limit_ns), _s(stream)))
+
+
+def kronq_sync_status(stream=None, info=None) -> int:
+    """Wait for `stream` and return its status: KRONQ_ERR_CUDA (-4) after a
+    CUDA error, else the device word `info` (0 or the first numerical
+    failure), else 0.  Returns the code rather than raising."""
+    _dev(info, torch.int32, "info")
+    return int(lib().kronq_sync_status(_s(stream), _p(info)))
 
 
 def packed_words(n: int, bits: int) -> int:

@@ -155,7 +155,7 @@ const char* kronq_status_string(int st) {
   }
 }
 
-int kronq_abi_version(void) { return 100; }
+int kronq_abi_version(void) { return 101; }
 
 uint64_t kronq_launch_count(void) { return kqh::launches(); }
 
@@ -192,6 +192,20 @@ int kronq_selftest_wait(int32_t* info, int64_t limit_ns, void* stream) {
   if (!info || limit_ns <= 0 || limit_ns > 2000000000ll) return KRONQ_ERR_INVALID_ARG;
   selftest_wait_kernel<<<1, 32, 0, S(stream)>>>(info, (unsigned long long)limit_ns);
   return kqh::launch_status();
+}
+
+int kronq_sync_status(void* stream, const int32_t* info) {
+  if (cudaStreamSynchronize(S(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return KRONQ_ERR_CUDA;
+  }
+  if (!info) return KRONQ_OK;
+  int32_t v = 0;
+  if (cudaMemcpy(&v, info, sizeof(v), cudaMemcpyDefault) != cudaSuccess) {
+    cudaGetLastError();
+    return KRONQ_ERR_CUDA;
+  }
+  return v;
 }
 
 size_t kronq_workspace_size(int64_t m, int64_t n, int bits, int group, int block) {

@@ -42,7 +42,16 @@ def test_status_strings_and_version(L):
     assert L.kronq_status_string(0) == b"ok"
     assert L.kronq_status_string(-3) == b"matrix not positive definite"
     assert L.kronq_status_string(12345) == b"unknown status"
-    assert L.kronq_abi_version() == 100
+    assert L.kronq_abi_version() == 101
+
+
+def test_sync_status_reports_the_stream(L):
+    """kronq_sync_status waits for the stream: on a host without a usable
+    device that wait itself fails and is reported as KRONQ_ERR_CUDA (-4),
+    not raised; with a device and no work queued it is KRONQ_OK."""
+    import torch
+    expected = 0 if torch.cuda.is_available() else -4
+    assert L.kronq_sync_status(None, None) == expected
 
 
 def test_workspace_size(L):
