@@ -209,3 +209,12 @@ def test_binding_refuses_host_tensors_of_the_right_shape():
     t = _quant_tensors()
     with pytest.raises(ValueError, match="CUDA"):
         abi.kronq_quantize_layer(t["W"], t["U"], 4, -1, 128, t["codes"], t["scales"], t["zeros"])
+
+
+def test_sync_status_binding_checks_its_info_word():
+    """The binding passes an int32 info word through and rejects any other
+    dtype before calling the library."""
+    import torch
+    from post_quantization_02_b200 import abi
+    with pytest.raises(ValueError):
+        abi.kronq_sync_status(None, torch.zeros(1, dtype=torch.float32))
