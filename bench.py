@@ -221,10 +221,12 @@ def load_traffic(workload: str):
 # The fixed oracle sample both CPU legs time (the cpu_baseline of the GPU
 # run and every step of --impl reference): the same stages on the same
 # sample sizes, scaled to the whole layer the same way, so the two agree.
-SAMPLE_TOKENS = 512        # covariance rows, scaled by tokens
+SAMPLE_TOKENS = 2048       # covariance rows, scaled by tokens
+SAMPLE_COV_COLS = 4096     # covariance of the leading columns, scaled by (width / cols)^2
 SAMPLE_ROT_ROWS = 64       # rows through each rotation, scaled by rows
 SAMPLE_CHOL_N = 1024       # inverse Cholesky size, scaled by n^3
 SAMPLE_OBS_COLS = 4096     # column-loop width, scaled by cols^2 above it
+SAMPLE_OBS_ROWS = 32       # column-loop rows per host thread, scaled by rows
 
 
 def oracle_sample(cfg):
@@ -244,13 +246,20 @@ def oracle_sample(cfg):
     for sub in cfg.sublayers:
         site = cfg.site(sub.site)
         m, n = sub.m, sub.n
-        # covariances: tok tokens of X and G, scaled to all tokens
+        # covariances: tok tokens of the leading cx (cg) columns of X (G),
+        # scaled to all tokens and to the whole width by (width / cx)^2 -- the
+        # product's cost; the full d x d output of a small sample would be
+        # written at memory speed and, scaled by tokens, overstate it
         xb = synth.x_chunk(cfg, site, 0, tokens=tok)
         gb = synth.g_chunk(cfg, sub, 0, tokens=tok)
+        cx, cg = min(site.width, SAMPLE_COV_COLS), min(m, SAMPLE_COV_COLS)
         t0 = time.perf_counter()
-        ocov.covariance(synth.bf16_bits_to_f32(xb).astype(np.float64))
-        ocov.covariance(synth.bf16_bits_to_f32(gb).astype(np.float64))
-        t_cov = (time.perf_counter() - t0) * cfg.tokens / tok
+        ocov.covariance(synth.bf16_bits_to_f32(xb[:, :cx]).astype(np.float64))
+        t_x = time.perf_counter() - t0
+        t0 = time.perf_counter()
+        ocov.covariance(synth.bf16_bits_to_f32(gb[:, :cg]).astype(np.float64))
+        t_g = time.perf_counter() - t0
+        t_cov = (t_x * (site.width / cx) ** 2 + t_g * (m / cg) ** 2) * cfg.tokens / tok
         # BiIP: the transform on rows_rot rows of each width, scaled to the
         # row and column passes of W (m x n), H_X (n x n), H_G (m x m)
         su, sv = synth.make_signs(cfg, sub)
@@ -276,7 +285,7 @@ def oracle_sample(cfg):
         U = np.triu(r.standard_normal((nn, nn)) * 0.01) + np.eye(nn)
         bits = sub.bits or 3
         grp = sub.group if sub.group == -1 or nn % sub.group == 0 else -1
-        rows_obs = min(m, 64 * max(1, min(32, os.cpu_count() or 1)))
+        rows_obs = min(m, SAMPLE_OBS_ROWS * max(1, min(32, os.cpu_count() or 1)))
         Wr = r.standard_normal((rows_obs, nn)) * 0.02
         t0 = time.perf_counter()
         res = oq.obs_quantize_rows(Wr, U, bits, grp)
@@ -286,11 +295,12 @@ def oracle_sample(cfg):
             opack.pack(res["codes"], bits)
         t_pack = (time.perf_counter() - t0) * (m / rows_obs) * (n / nn)
         total += t_cov + t_rot + t_chol + t_obs + t_pack
-        parts.append(f"{sub.name}: cov {tok} of {cfg.tokens} tokens, rotation {rows_rot} rows, "
+        parts.append(f"{sub.name}: cov {tok} of {cfg.tokens} tokens x {cx} of {site.width} (X) and "
+                     f"{cg} of {m} (G) columns, rotation {rows_rot} rows, "
                      f"inverse Cholesky n={nc}, OBS {rows_obs} of {m} rows x {nn} cols")
     sample = ("fp64 oracle stages timed on a fixed sample and scaled to the whole layer (covariance "
-              "x tokens, rotation x rows, inverse Cholesky x n^3, OBS x rows, x cols^2 above "
-              f"{SAMPLE_OBS_COLS}): " + "; ".join(parts))
+              "x tokens x (width / columns)^2, rotation x rows, inverse Cholesky x n^3, OBS x rows, "
+              f"x cols^2 above {SAMPLE_OBS_COLS}): " + "; ".join(parts))
     return total, sample
 
 
